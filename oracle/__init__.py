@@ -1,0 +1,171 @@
+"""fp64 CPU oracle of the WKV7 recurrence.
+
+TEST INFRASTRUCTURE ONLY: imported by the test suite, by the smoke check and
+by the benchmark's CPU-baseline leg, never by the library's product path.  It
+shares no code with the CUDA library; the only thing both sides use is the
+seeded input generator, which holds none of the method's arithmetic.
+
+What it computes, per batch b and head h (S is N x N, row i = value index,
+column j = key index):
+
+    S_t = S_{t-1} (diag(w_t) + a_t b_t^T) + v_t k_t^T,    y_t = S_t r_t
+
+(the "diagonal plus rank one" generalised delta rule: Paper Review: RWKV-7
+"Goose" with Expressive Dynamic State Evolution, sections "Architecture" and
+"The approach"; vector decay, per-channel in-context learning rate and
+separate removal / write keys: Elamur Research summary of RWKV-7 "Goose",
+section "Summary").
+
+* ``forward`` / ``backward`` call the plain C loops in ``wkv7_oracle.c``
+  (fp64, one scalar loop per state row, OpenMP over heads).
+* ``step`` is ``forward`` with T = 1 (a decode step is one token of the same
+  recurrence: constant time and memory per token, RWKV-7 "Goose" abstract).
+* ``forward_chunked`` is the chunked (parallel-in-time) form, written with
+  numpy matrix products in fp64.  The pages only say that training stays
+  parallelisable (RWKV-7 "Goose" abstract) and cite chunk-wise delta-rule
+  parallelisation by title; the algebra here is our own derivation from the
+  recurrence, applied chunk by chunk in the order of its definition.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv7_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libwkv7_oracle.so")
+_lib = None
+
+_DP = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (fp64, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        i = ctypes.c_int
+        lib.oracle_forward.argtypes = [i, i, i, i] + [_DP] * 9
+        lib.oracle_forward.restype = None
+        lib.oracle_backward.argtypes = [i, i, i, i] + [_DP] * 16
+        lib.oracle_backward.restype = None
+        lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [i]
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def _f64(x):
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(x):
+    return None if x is None else x.ctypes.data_as(_DP)
+
+
+def forward(r, w, k, v, a, b, s0=None):
+    """y [B,T,H,N] and sT [B,H,N,N] in fp64 for inputs shaped [B,T,H,N]."""
+    lib = _load()
+    r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
+    B, T, H, N = r.shape
+    for x in (w, k, v, a, b):
+        assert x.shape == r.shape
+    s0 = None if s0 is None else _f64(s0)
+    if s0 is not None:
+        assert s0.shape == (B, H, N, N)
+    y = np.empty((B, T, H, N))
+    sT = np.empty((B, H, N, N))
+    lib.oracle_forward(B, T, H, N, *map(_ptr, (r, w, k, v, a, b, s0, y, sT)))
+    return y, sT
+
+
+def step(r, w, k, v, a, b, state):
+    """One decode token: inputs [B,H,N], state [B,H,N,N] -> (y [B,H,N], new state)."""
+    expand = [np.asarray(x)[:, None] for x in (r, w, k, v, a, b)]
+    y, sT = forward(*expand, s0=state)
+    return y[:, 0], sT
+
+
+def backward(r, w, k, v, a, b, s0, dy, dsT=None):
+    """Gradients (dr, dw, dk, dv, da, db, ds0) of sum(dy*y) + sum(dsT*sT)."""
+    lib = _load()
+    r, w, k, v, a, b, dy = (_f64(x) for x in (r, w, k, v, a, b, dy))
+    B, T, H, N = r.shape
+    s0 = None if s0 is None else _f64(s0)
+    dsT = None if dsT is None else _f64(dsT)
+    grads = [np.empty((B, T, H, N)) for _ in range(6)]
+    ds0 = np.empty((B, H, N, N))
+    lib.oracle_backward(B, T, H, N, *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT)),
+                        *map(_ptr, grads), _ptr(ds0))
+    return (*grads, ds0)
+
+
+def forward_chunked(r, w, k, v, a, b, s0=None, chunk_len=64):
+    """Chunked form of ``forward`` (fp64, w > 0), chunk by chunk.
+
+    Inside a chunk of L tokens (local index t = 0..L-1) starting from state
+    S_in, with gamma_t = prod_{m<=t} w_m (elementwise, gamma_{-1} = 1):
+
+      a~_t = a_t * gamma_{t-1},  r~_t = r_t * gamma_t,
+      b^_s = b_s / gamma_s,      k^_s = k_s / gamma_s
+      L_ab[t,s] = a~_t . b^_s,  L_ak[t,s] = a~_t . k^_s      (s <  t)
+      L_rb[t,s] = r~_t . b^_s,  L_rk[t,s] = r~_t . k^_s      (s <= t)
+      U = (I - L_ab)^{-1} (A~ S_in^T + L_ak V)     rows u_t = S_{t-1} a_t
+      Y = R~ S_in^T + L_rb U + L_rk V
+      S_out = S_in diag(gamma_{L-1}) + U^T B- + V^T K-,
+          B-_s = b_s * gamma_{L-1} / gamma_s,  K-_s = k_s * gamma_{L-1} / gamma_s
+
+    This follows from unrolling the recurrence inside the chunk:
+      S_t = S_in diag(gamma_t) + sum_{s<=t} (u_s b_s^T + v_s k_s^T) diag(gamma_t / gamma_s).
+    """
+    r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
+    B, T, H, N = r.shape
+    y = np.empty((B, T, H, N))
+    sT = np.empty((B, H, N, N))
+    for bb in range(B):
+        for h in range(H):
+            S = np.zeros((N, N)) if s0 is None else _f64(s0)[bb, h].copy()
+            for c0 in range(0, T, chunk_len):
+                c1 = min(T, c0 + chunk_len)
+                L = c1 - c0
+                R, W, K, V, A, Bm = (x[bb, c0:c1, h] for x in (r, w, k, v, a, b))
+                gam = np.cumprod(W, axis=0)
+                gam_prev = np.vstack([np.ones((1, N)), gam[:-1]])
+                At = A * gam_prev
+                Rt = R * gam
+                Bh = Bm / gam
+                Kh = K / gam
+                strict = np.tril(np.ones((L, L)), -1)
+                incl = np.tril(np.ones((L, L)), 0)
+                L_ab = (At @ Bh.T) * strict
+                L_ak = (At @ Kh.T) * strict
+                L_rb = (Rt @ Bh.T) * incl
+                L_rk = (Rt @ Kh.T) * incl
+                U = np.linalg.solve(np.eye(L) - L_ab, At @ S.T + L_ak @ V)
+                y[bb, c0:c1, h] = Rt @ S.T + L_rb @ U + L_rk @ V
+                Bbar = Bh * gam[-1]
+                Kbar = Kh * gam[-1]
+                S = S * gam[-1][None, :] + U.T @ Bbar + V.T @ Kbar
+            sT[bb, h] = S
+    return y, sT
