@@ -1,0 +1,151 @@
+/*
+ * wkv7.h - C ABI of the WKV7 recurrence library (libwkv7.so, CUDA sm_100a).
+ *
+ * The operation (per batch b, head h; the state S is an N x N fp32 matrix,
+ * row i = value index, column j = key index):
+ *
+ *     S_t = S_{t-1} (diag(w_t) + a_t b_t^T) + v_t k_t^T
+ *     y_t = S_t r_t                     (read after the write of token t)
+ *
+ * This is the RWKV-7 "generalized delta rule with vector-valued gating and
+ * in-context learning rates" (RWKV-7 "Goose" with Expressive Dynamic State
+ * Evolution, abstract): a "diagonal plus rank one" state transition with a
+ * vector-valued, data-dependent decay and separate removal / replacement
+ * keys (Paper Review: RWKV-7 "Goose", section "Architecture"), updated per
+ * head and read out by the receptance vector (same review, section "The
+ * approach").  w is the decay itself (0 < w <= 1 in the intended use), not its
+ * logarithm; a is the removal key, b the learning-rate-scaled replacement
+ * key; k, v the write key and value; r the receptance.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no memory; scratch comes from the caller through the
+ *    *_workspace_size queries.  Every pointer must be 16-byte aligned.
+ *  - Tensors are contiguous, row-major.  Per-token tensors (r, w, k, v, a, b,
+ *    y, dy and their gradients) are [B, T, H, N]; a decode step's tensors are
+ *    [B, H, N]; states (s0, sT, dsT, ds0, state) are [B, H, N, N] fp32 with
+ *    element S[b][h][i][j] (i = value row, j = key column).
+ *  - Calls are asynchronous on `stream`; they never synchronize (except
+ *    wkv7_get_device_status).  Launch errors are reported as WKV7_ERR_CUDA.
+ *  - Arguments are validated on the host before any launch; an invalid
+ *    argument returns WKV7_ERR_INVALID_ARG (N other than 64 returns
+ *    WKV7_ERR_UNSUPPORTED) and launches nothing.
+ *  - B, T, H may be 0 (nothing to do; with T = 0 the forward copies s0, or
+ *    zeros, to sT and the backward copies dsT, or zeros, to ds0).
+ *  - No exception crosses the ABI.  The library is safe to call from several
+ *    host threads as long as each call's buffers are its own.
+ */
+#ifndef WKV7_H
+#define WKV7_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define WKV7_API __attribute__((visibility("default")))
+#else
+#define WKV7_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WKV7_OK = 0,
+    WKV7_ERR_INVALID_ARG = 1,  /* bad pointer / size / dtype / alignment      */
+    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    WKV7_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed        */
+    WKV7_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up          */
+    WKV7_ERR_RANGE = 5         /* device-side: input outside the chunked
+                                  form's numeric domain (see wkv7_forward)   */
+} wkv7_status;
+
+typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1 } wkv7_dtype;
+
+typedef enum {
+    WKV7_ALGO_AUTO = 0,   /* library picks: CHUNK for bf16 inputs when T >= 2 * chunk, else SEQ */
+    WKV7_ALGO_SEQ = 1,    /* token-by-token scan, state kept on chip            */
+    WKV7_ALGO_CHUNK = 2   /* chunked (parallel-in-time) form on tensor cores    */
+} wkv7_algo;
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define WKV7_ABI_VERSION 1
+WKV7_API int wkv7_abi_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+WKV7_API const char *wkv7_status_string(wkv7_status status);
+
+/*
+ * Bytes of scratch wkv7_forward needs for these arguments (0 when the chosen
+ * algorithm needs none).  Same arguments as wkv7_forward's sizes and choice.
+ */
+WKV7_API size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                   wkv7_algo algo, int chunk_len);
+
+/*
+ * Forward over a whole sequence.
+ *   r, w, k, v, a, b : [B, T, H, N] of in_dtype (fp32 or bf16), read only
+ *   s0               : [B, H, N, N] fp32 initial state, or NULL for zeros
+ *   y                : [B, T, H, N] of y_dtype, written
+ *   sT               : [B, H, N, N] fp32 final state, or NULL to skip.
+ *                      sT may alias s0 (in-place continuation); no other
+ *                      output may alias an input.
+ *   algo, chunk_len  : algorithm choice; chunk_len 0 means 64 (the only
+ *                      length the chunked form implements).
+ *   workspace        : wkv7_forward_workspace_size() bytes, or NULL if 0.
+ * The chunked form needs the per-chunk decay product of every channel to stay
+ * in fp32's normal range (prod of 64 consecutive w >= 1e-30); a chunk outside
+ * it raises WKV7_ERR_RANGE in the device status word (wkv7_get_device_status)
+ * and its outputs are unspecified.  The SEQ form has no such limit.
+ */
+WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
+                         const void *r, const void *w, const void *k, const void *v,
+                         const void *a, const void *b, const float *s0, void *y, float *sT,
+                         wkv7_algo algo, int chunk_len, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
+ * One decode token (T = 1) for every (b, h), updating the state IN PLACE
+ * (constant memory and time per token: RWKV-7 "Goose" abstract).
+ *   r, w, k, v, a, b : [B, H, N] of in_dtype
+ *   state            : [B, H, N, N] fp32, read and overwritten with S_t
+ *   y                : [B, H, N] of y_dtype
+ */
+WKV7_API wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
+                      const void *r, const void *w, const void *k, const void *v,
+                      const void *a, const void *b, float *state, void *y, cudaStream_t stream);
+
+/* Bytes of scratch wkv7_backward needs (state checkpoints and recompute). */
+WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
+
+/*
+ * Backward: gradients of L = sum(dy * y) + sum(dsT * sT) with respect to every
+ * input and the initial state, by a reverse-time pass over recomputed states.
+ *   r..b, s0         : the forward's inputs (s0 NULL = zeros)
+ *   dy               : [B, T, H, N] of in_dtype
+ *   dsT              : [B, H, N, N] fp32, or NULL for zeros
+ *   dr, dw, dk, dv, da, db : [B, T, H, N] of grad_dtype, overwritten
+ *   ds0              : [B, H, N, N] fp32, overwritten (required)
+ *   workspace        : wkv7_backward_workspace_size() bytes
+ * dw is dL/dw for the decay value w itself.
+ */
+WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype grad_dtype,
+                          const void *r, const void *w, const void *k, const void *v,
+                          const void *a, const void *b, const float *s0, const void *dy,
+                          const float *dsT, void *dr, void *dw, void *dk, void *dv, void *da,
+                          void *db, float *ds0, void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
+/*
+ * Synchronizes `stream`, then returns and clears the sticky device-side status
+ * word of the current device (WKV7_OK, WKV7_ERR_TIMEOUT or WKV7_ERR_RANGE), or
+ * WKV7_ERR_CUDA if the synchronization itself failed.
+ */
+WKV7_API wkv7_status wkv7_get_device_status(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV7_H */

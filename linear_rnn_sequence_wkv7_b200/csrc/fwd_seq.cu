@@ -1,0 +1,238 @@
+// Sequential-scan WKV7 forward (token by token, state on chip).
+//
+// Per head, row i of the state evolves independently given the token's
+// shared vectors (the "diagonal plus rank one" transition of RWKV-7: Paper
+// Review: RWKV-7 "Goose", sections "Architecture" and "The approach"):
+//     p = S[i,:] . a_t ;  S[i,j] = S[i,j] w_t[j] + p b_t[j] + v_t[i] k_t[j] ;
+//     y_t[i] = S[i,:] . r_t
+//
+// Mapping: a CTA owns RB rows of one (b, h) state.  Four consecutive lanes
+// share a row group of RPT rows; lane q holds the 16 columns
+// j = 16 m + 4 q + e (m, e in 0..3) of each of its rows in registers, so the
+// two dot products per token are 16-term in-thread sums plus two xor-shuffle
+// steps, and the update is 3 FP32 instructions per element.  The token
+// vectors are streamed through shared memory in tiles of TT tokens with
+// double-buffered cp.async (16-byte, L2-only) and converted to fp32 once per
+// CTA; every lane reads them as broadcast float4s (the interleaved column
+// assignment keeps the 4 lanes of a row group on distinct banks).
+//
+// CKPT mode (used by the backward) writes the state before every CK-th token
+// to a checkpoint buffer instead of producing y.
+#include "common.cuh"
+
+namespace wkv7 {
+
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT>
+__global__ void __launch_bounds__((RB / RPT) * 4)
+fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
+               const InT *__restrict__ k, const InT *__restrict__ v, const InT *__restrict__ a,
+               const InT *__restrict__ b, const float *s0, OutT *__restrict__ y, float *sT,
+               float *__restrict__ ckpt, int CK) {
+    constexpr int NT = (RB / RPT) * 4;
+    constexpr int NTEN = 6;                          // r w k v a b
+    constexpr int VEC = 16 / sizeof(InT);            // elements per 16-byte chunk
+    constexpr int CHUNKS_PER_VEC = kN / VEC;         // 16-byte chunks per N-vector
+    constexpr int CHUNKS_PER_TILE = TT * NTEN * CHUNKS_PER_VEC;
+    constexpr bool kConvert = !std::is_same<InT, float>::value;
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    InT *raw = reinterpret_cast<InT *>(smem_raw);                 // [2][NTEN][TT][kN]
+    float *f32buf = kConvert ? reinterpret_cast<float *>(smem_raw + 2 * NTEN * TT * kN * sizeof(InT))
+                             : nullptr;                           // [NTEN][TT][kN]
+
+    const int tid = threadIdx.x;
+    const int q = tid & 3;
+    const int rg = tid >> 2;
+    const int blocks_per_head = kN / RB;
+    const int h = blockIdx.x / blocks_per_head;
+    const int row0 = (blockIdx.x % blocks_per_head) * RB + rg * RPT;
+    const int bb = blockIdx.y;
+    const size_t tok_stride = (size_t)H * kN;                     // between consecutive t
+    const size_t base = ((size_t)bb * T * H + h) * kN;            // (bb, t=0, h, 0)
+    const size_t st_base = ((size_t)bb * H + h) * kN * kN;
+
+    const InT *src[NTEN] = {r, w, k, v, a, b};
+
+    float S[RPT][16];
+#pragma unroll
+    for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s0) s4 = load4(s0 + st_base + (size_t)(row0 + rr) * kN + 16 * m + 4 * q);
+            S[rr][4 * m + 0] = s4.x;
+            S[rr][4 * m + 1] = s4.y;
+            S[rr][4 * m + 2] = s4.z;
+            S[rr][4 * m + 3] = s4.w;
+        }
+
+    const int ntiles = (T + TT - 1) / TT;
+    auto issue_tile = [&](int tile, int stage) {
+        const int t0 = tile * TT;
+        for (int c = tid; c < CHUNKS_PER_TILE; c += NT) {
+            const int ten = c / (TT * CHUNKS_PER_VEC);
+            const int rem = c % (TT * CHUNKS_PER_VEC);
+            const int tt = rem / CHUNKS_PER_VEC;
+            const int ch = rem % CHUNKS_PER_VEC;
+            if (t0 + tt < T) {
+                InT *dst = raw + (((size_t)stage * NTEN + ten) * TT + tt) * kN + ch * VEC;
+                cp_async16(dst, src[ten] + base + (size_t)(t0 + tt) * tok_stride + ch * VEC);
+            }
+        }
+        cp_async_commit();
+    };
+
+    if (ntiles > 0) issue_tile(0, 0);
+    for (int it = 0; it < ntiles; ++it) {
+        const int stage = it & 1;
+        const int t0 = it * TT;
+        cp_async_wait<0>();
+        __syncthreads();
+        const float *buf;
+        if constexpr (kConvert) {
+            const InT *rs = raw + (size_t)stage * NTEN * TT * kN;
+            for (int e = tid * 4; e < NTEN * TT * kN; e += NT * 4) store4(f32buf + e, load4(rs + e));
+            __syncthreads();
+            buf = f32buf;
+        } else {
+            buf = reinterpret_cast<const float *>(raw) + (size_t)stage * NTEN * TT * kN;
+        }
+        if (it + 1 < ntiles) issue_tile(it + 1, stage ^ 1);
+
+        if constexpr (CKPT) {
+            if (t0 % CK == 0) {
+                float *dst = ckpt + (((size_t)bb * H + h) * ((T + CK - 1) / CK) + t0 / CK) * kN * kN;
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        store4(dst + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                               make_float4(S[rr][4 * m], S[rr][4 * m + 1], S[rr][4 * m + 2], S[rr][4 * m + 3]));
+            }
+        }
+
+        const int tt_end = min(TT, T - t0);
+        for (int tt = 0; tt < tt_end; ++tt) {
+            const float *rv = buf + (0 * TT + tt) * kN;
+            const float *wv = buf + (1 * TT + tt) * kN;
+            const float *kv = buf + (2 * TT + tt) * kN;
+            const float *vv = buf + (3 * TT + tt) * kN;
+            const float *av = buf + (4 * TT + tt) * kN;
+            const float *bv = buf + (5 * TT + tt) * kN;
+
+            // p = S_{t-1}[i,:] . a_t
+            float p[RPT];
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) p[rr] = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(av + 16 * m + 4 * q);
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr) {
+                    p[rr] = fmaf(S[rr][4 * m + 0], a4.x, p[rr]);
+                    p[rr] = fmaf(S[rr][4 * m + 1], a4.y, p[rr]);
+                    p[rr] = fmaf(S[rr][4 * m + 2], a4.z, p[rr]);
+                    p[rr] = fmaf(S[rr][4 * m + 3], a4.w, p[rr]);
+                }
+            }
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) {
+                p[rr] += __shfl_xor_sync(0xffffffffu, p[rr], 1);
+                p[rr] += __shfl_xor_sync(0xffffffffu, p[rr], 2);
+            }
+            float vi[RPT];
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) vi[rr] = vv[row0 + rr];
+
+            // S = S * w + p b + v k ;  y = S . r
+            float yacc[RPT];
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) yacc[rr] = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(wv + 16 * m + 4 * q);
+                const float4 b4 = *reinterpret_cast<const float4 *>(bv + 16 * m + 4 * q);
+                const float4 k4 = *reinterpret_cast<const float4 *>(kv + 16 * m + 4 * q);
+                const float4 r4 = *reinterpret_cast<const float4 *>(rv + 16 * m + 4 * q);
+                const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
+                const float bj[4] = {b4.x, b4.y, b4.z, b4.w};
+                const float kj[4] = {k4.x, k4.y, k4.z, k4.w};
+                const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float s = S[rr][4 * m + e];
+                        s = fmaf(s, wj[e], fmaf(p[rr], bj[e], vi[rr] * kj[e]));
+                        S[rr][4 * m + e] = s;
+                        if constexpr (!CKPT) yacc[rr] = fmaf(s, rj[e], yacc[rr]);
+                    }
+            }
+            if constexpr (!CKPT) {
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr) {
+                    yacc[rr] += __shfl_xor_sync(0xffffffffu, yacc[rr], 1);
+                    yacc[rr] += __shfl_xor_sync(0xffffffffu, yacc[rr], 2);
+                }
+                OutT *yrow = y + base + (size_t)(t0 + tt) * tok_stride + row0;
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr)
+                    if (q == (rr & 3)) yrow[rr] = from_f32<OutT>(yacc[rr]);
+            }
+        }
+    }
+
+    if (sT) {
+        // Every CTA read its own rows of s0 before its first tile, so writing
+        // sT here is safe even when sT aliases s0.
+#pragma unroll
+        for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                store4(sT + st_base + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                       make_float4(S[rr][4 * m], S[rr][4 * m + 1], S[rr][4 * m + 2], S[rr][4 * m + 3]));
+    }
+}
+
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT>
+static cudaError_t launch_fwd_seq(int B, int T, int H, const void *r, const void *w, const void *k,
+                                  const void *v, const void *a, const void *b, const float *s0, void *y,
+                                  float *sT, float *ckpt, int CK, cudaStream_t st) {
+    constexpr int NT = (RB / RPT) * 4;
+    size_t smem = 2 * 6 * TT * kN * sizeof(InT);
+    if (!std::is_same<InT, float>::value) smem += 6 * TT * kN * sizeof(float);
+    auto kern = fwd_seq_kernel<InT, OutT, RPT, RB, TT, CKPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(H * (kN / RB), B);
+    kern<<<grid, NT, smem, st>>>(T, H, (const InT *)r, (const InT *)w, (const InT *)k, (const InT *)v,
+                                 (const InT *)a, (const InT *)b, s0, (OutT *)y, sT, ckpt, CK);
+    return cudaGetLastError();
+}
+
+// Host entry used by the API layer.
+cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                    const void *w, const void *k, const void *v, const void *a, const void *b,
+                    const float *s0, void *y, float *sT, cudaStream_t st) {
+    constexpr int RPT = 2, RB = 32, TT = 16;
+    if (in_dt == WKV7_F32 && y_dt == WKV7_F32)
+        return launch_fwd_seq<float, float, RPT, RB, TT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+    if (in_dt == WKV7_F32 && y_dt == WKV7_BF16)
+        return launch_fwd_seq<float, __nv_bfloat16, RPT, RB, TT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+    if (in_dt == WKV7_BF16 && y_dt == WKV7_F32)
+        return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+    return launch_fwd_seq<__nv_bfloat16, __nv_bfloat16, RPT, RB, TT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+}
+
+// State checkpoints every CK tokens (CK a multiple of 16): ckpt[b][h][c] holds
+// the state before token c * CK.  Used by the backward's first pass.
+cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
+                            const void *k, const void *v, const void *a, const void *b, const float *s0,
+                            float *ckpt, int CK, cudaStream_t st) {
+    constexpr int RPT = 2, RB = 32, TT = 16;
+    if (in_dt == WKV7_F32)
+        return launch_fwd_seq<float, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, nullptr, ckpt, CK, st);
+    return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, nullptr, ckpt, CK, st);
+}
+
+}  // namespace wkv7

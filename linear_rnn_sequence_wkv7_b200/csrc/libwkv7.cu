@@ -1,0 +1,7 @@
+// Single translation unit of libwkv7.so: the sticky device status word is one
+// __device__ variable shared by every kernel, so all kernels are compiled
+// together (no relocatable device code needed).
+#include "wkv7_api.cu"
+#include "fwd_seq.cu"
+#include "step.cu"
+#include "bwd_seq.cu"

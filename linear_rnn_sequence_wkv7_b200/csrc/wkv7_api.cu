@@ -1,0 +1,157 @@
+// extern "C" entry points of libwkv7.so: argument validation, workspace
+// layout and kernel dispatch.  Every check happens on the host before any
+// launch; nothing here allocates device memory or synchronizes (except
+// wkv7_get_device_status).
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace wkv7 {
+
+cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                    const void *w, const void *k, const void *v, const void *a, const void *b,
+                    const float *s0, void *y, float *sT, cudaStream_t st);
+cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
+                            const void *k, const void *v, const void *a, const void *b, const float *s0,
+                            float *ckpt, int CK, cudaStream_t st);
+cudaError_t step(int B, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
+                 const void *k, const void *v, const void *a, const void *b, float *state, void *y,
+                 cudaStream_t st);
+cudaError_t bwd_seq(int B, int T, int H, int CK, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
+                    const void *w, const void *k, const void *v, const void *a, const void *b,
+                    const void *dy, const float *dsT, const float *ckpt, float *hist, void *dr, void *dw,
+                    void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st);
+size_t bwd_hist_bytes(int B, int H, int CK);
+
+namespace {
+
+constexpr int kBwdChunk = 16;        // backward checkpoint interval (tokens)
+constexpr size_t kWsAlign = 256;
+
+bool dtype_ok(wkv7_dtype d) { return d == WKV7_F32 || d == WKV7_BF16; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
+bool opt_ptr_ok(const void *p) { return p == nullptr || aligned16(p); }
+size_t round_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+wkv7_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA; }
+
+// Shape checks common to every entry point.  Returns OK, INVALID_ARG or UNSUPPORTED.
+wkv7_status check_dims(int B, int T, int H, int N) {
+    if (B < 0 || T < 0 || H < 0 || N <= 0) return WKV7_ERR_INVALID_ARG;
+    if (B > 65535) return WKV7_ERR_UNSUPPORTED;             // grid.y limit of the scan kernels
+    if ((int64_t)B * H > (int64_t)INT32_MAX / 64) return WKV7_ERR_UNSUPPORTED;
+    if (N != kN) return WKV7_ERR_UNSUPPORTED;
+    return WKV7_OK;
+}
+
+// sT (or ds0) := src, or zeros when src is NULL; used for T = 0.
+wkv7_status copy_or_zero_state(float *dst, const float *src, int B, int H, cudaStream_t st) {
+    if (!dst) return WKV7_OK;
+    const size_t bytes = (size_t)B * H * kN * kN * sizeof(float);
+    if (bytes == 0 || dst == src) return WKV7_OK;
+    if (src) return from_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+    return from_cuda(cudaMemsetAsync(dst, 0, bytes, st));
+}
+
+size_t bwd_ckpt_bytes(int B, int T, int H) {
+    const size_t nck = ((size_t)T + kBwdChunk - 1) / kBwdChunk;
+    return (size_t)B * H * nck * kN * kN * sizeof(float);
+}
+
+}  // namespace
+}  // namespace wkv7
+
+using namespace wkv7;
+
+extern "C" {
+
+int wkv7_abi_version(void) { return WKV7_ABI_VERSION; }
+
+const char *wkv7_status_string(wkv7_status s) {
+    switch (s) {
+        case WKV7_OK: return "ok";
+        case WKV7_ERR_INVALID_ARG: return "invalid argument";
+        case WKV7_ERR_UNSUPPORTED: return "unsupported";
+        case WKV7_ERR_CUDA: return "CUDA error";
+        case WKV7_ERR_TIMEOUT: return "device wait timed out";
+        case WKV7_ERR_RANGE: return "input outside the chunked form's numeric domain";
+    }
+    return "unknown status";
+}
+
+size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_algo algo,
+                                   int chunk_len) {
+    (void)B; (void)T; (void)H; (void)N; (void)in_dtype; (void)algo; (void)chunk_len;
+    return 0;
+}
+
+wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                         const void *w, const void *k, const void *v, const void *a, const void *b,
+                         const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    (void)workspace; (void)workspace_bytes;
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
+    if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_SEQ && algo != WKV7_ALGO_CHUNK) return WKV7_ERR_INVALID_ARG;
+    if (chunk_len != 0 && chunk_len != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!opt_ptr_ok(s0) || !opt_ptr_ok(sT)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (T == 0) return copy_or_zero_state(sT, s0, B, H, stream);
+    for (const void *p : {r, w, k, v, a, b, (const void *)y})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    if (algo == WKV7_ALGO_CHUNK) return WKV7_ERR_UNSUPPORTED;
+    return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+}
+
+wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                      const void *w, const void *k, const void *v, const void *a, const void *b,
+                      float *state, void *y, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, 1, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    for (const void *p : {r, w, k, v, a, b, (const void *)state, (const void *)y})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    return from_cuda(wkv7::step(B, H, in_dt, y_dt, r, w, k, v, a, b, state, y, stream));
+}
+
+size_t wkv7_backward_workspace_size(int B, int T, int H, int N) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
+    return round_up(bwd_ckpt_bytes(B, T, H)) + round_up(bwd_hist_bytes(B, H, kBwdChunk));
+}
+
+wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
+                          const void *w, const void *k, const void *v, const void *a, const void *b,
+                          const float *s0, const void *dy, const float *dsT, void *dr, void *dw, void *dk,
+                          void *dv, void *da, void *db, float *ds0, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(g_dt)) return WKV7_ERR_INVALID_ARG;
+    if (!opt_ptr_ok(s0) || !opt_ptr_ok(dsT) || !ptr_ok(ds0)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (T == 0) return copy_or_zero_state(ds0, dsT, B, H, stream);
+    for (const void *p : {r, w, k, v, a, b, dy, (const void *)dr, (const void *)dw, (const void *)dk,
+                          (const void *)dv, (const void *)da, (const void *)db})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    const size_t need = wkv7_backward_workspace_size(B, T, H, N);
+    if (workspace_bytes < need || !ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
+    float *ckpt = static_cast<float *>(workspace);
+    float *hist = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(bwd_ckpt_bytes(B, T, H)));
+    cudaError_t e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, stream);
+    if (e != cudaSuccess) return WKV7_ERR_CUDA;
+    return from_cuda(bwd_seq(B, T, H, kBwdChunk, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, hist, dr, dw,
+                             dk, dv, da, db, ds0, stream));
+}
+
+wkv7_status wkv7_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV7_ERR_CUDA;
+    int h = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
+    if (h != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
+    return static_cast<wkv7_status>(h);
+}
+
+}  // extern "C"

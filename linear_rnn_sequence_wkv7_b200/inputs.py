@@ -16,6 +16,7 @@ Distributions (per head-token, an N-vector per tensor):
   a = -k_hat,  b = k_hat * lr
   s0 ~ N(0, 0.1) (standard deviation 0.1), dy ~ N(0, 1)
 
+All draws and the recipe are evaluated in float32, then stored.
 Random numbers come from numpy's Philox bit generator.  The flat stream of
 N-vectors of each tensor is cut into fixed blocks of ``BLOCK_VECS`` vectors,
 block ``c`` of stream ``s`` under seed ``seed`` is drawn from
@@ -63,8 +64,8 @@ def to_f64(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def _store(x64: np.ndarray, dtype: str) -> np.ndarray:
-    x32 = x64.astype(np.float32)
+def _store(x: np.ndarray, dtype: str) -> np.ndarray:
+    x32 = np.asarray(x, dtype=np.float32)
     if dtype == "bf16":
         return f32_to_bf16_bits(x32)
     if dtype == "f32":
@@ -103,18 +104,18 @@ def gen_vectors(nvec: int, N: int, *, seed: int, dtype: str = "bf16",
     def block(blk):
         c, lo, hi = blk
         n = hi - lo
-        buf = np.empty((n, N), dtype=np.float64)
+        buf = np.empty((n, N), dtype=np.float32)
         for name, stream in (("r", STREAM_R), ("k", STREAM_K), ("v", STREAM_V)):
-            _rng(seed, stream, c).standard_normal(out=buf)
+            _rng(seed, stream, c).standard_normal(out=buf, dtype=np.float32)
             out[name][lo:hi] = _store(buf, dtype)
-        _rng(seed, STREAM_W, c).standard_normal(out=buf)
-        buf += x_mean
-        out["w"][lo:hi] = _store(np.exp(-0.6065 / (1.0 + np.exp(-buf))), dtype)
-        _rng(seed, STREAM_KHAT, c).standard_normal(out=buf)
-        khat = buf / np.linalg.norm(buf, axis=1, keepdims=True)
-        lr = np.empty((n, N), dtype=np.float64)
-        _rng(seed, STREAM_LR, c).standard_normal(out=lr)
-        lr = 1.0 / (1.0 + np.exp(-lr))
+        _rng(seed, STREAM_W, c).standard_normal(out=buf, dtype=np.float32)
+        buf += np.float32(x_mean)
+        out["w"][lo:hi] = _store(np.exp(np.float32(-0.6065) / (np.float32(1.0) + np.exp(-buf))), dtype)
+        _rng(seed, STREAM_KHAT, c).standard_normal(out=buf, dtype=np.float32)
+        khat = buf / np.sqrt(np.einsum("ij,ij->i", buf, buf))[:, None]
+        lr = np.empty((n, N), dtype=np.float32)
+        _rng(seed, STREAM_LR, c).standard_normal(out=lr, dtype=np.float32)
+        lr = np.float32(1.0) / (np.float32(1.0) + np.exp(-lr))
         out["a"][lo:hi] = _store(-khat, dtype)
         out["b"][lo:hi] = _store(khat * lr, dtype)
 
@@ -129,9 +130,9 @@ def gen_normal(nvec: int, N: int, *, seed: int, stream: int, std: float = 1.0,
 
     def block(blk):
         c, lo, hi = blk
-        buf = np.empty((hi - lo, N), dtype=np.float64)
-        _rng(seed, stream, c).standard_normal(out=buf)
-        out[lo:hi] = _store(buf * std, dtype)
+        buf = np.empty((hi - lo, N), dtype=np.float32)
+        _rng(seed, stream, c).standard_normal(out=buf, dtype=np.float32)
+        out[lo:hi] = _store(buf * np.float32(std), dtype)
 
     _run(block, _blocks(nvec), threads)
     return out

@@ -1,0 +1,174 @@
+"""Python binding of libwkv7.so (ctypes): argument marshalling only.
+
+Each function takes torch CUDA tensors, checks dtype / shape / contiguity,
+and passes raw device pointers and the current CUDA stream to the C ABI
+declared in include/wkv7.h.  Every step of the computation runs in the
+library's kernels; there is no fallback of any kind.  If the shared library
+is missing or fails to load, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwkv7.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(6)
+F32, BF16 = 0, 1
+ALGO_AUTO, ALGO_SEQ, ALGO_CHUNK = 0, 1, 2
+ALGOS = {"auto": ALGO_AUTO, "seq": ALGO_SEQ, "chunk": ALGO_CHUNK}
+
+EXPORTED_SYMBOLS = (
+    "wkv7_abi_version", "wkv7_status_string", "wkv7_forward_workspace_size", "wkv7_forward",
+    "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
+)
+
+_lib = None
+
+
+class WKV7Error(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libwkv7.so and declare the C signatures (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libwkv7.so not built at {path}; run linear_rnn_sequence_wkv7_b200/build.py")
+    lib = ctypes.CDLL(path)
+    i, z, vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    lib.wkv7_abi_version.restype = i
+    lib.wkv7_status_string.argtypes = [i]
+    lib.wkv7_status_string.restype = ctypes.c_char_p
+    lib.wkv7_forward_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    lib.wkv7_forward_workspace_size.restype = z
+    lib.wkv7_forward.argtypes = [i, i, i, i, i, i] + [vp] * 9 + [i, i, vp, z, vp]
+    lib.wkv7_forward.restype = i
+    lib.wkv7_step.argtypes = [i, i, i, i, i] + [vp] * 8 + [vp]
+    lib.wkv7_step.restype = i
+    lib.wkv7_backward_workspace_size.argtypes = [i, i, i, i]
+    lib.wkv7_backward_workspace_size.restype = z
+    lib.wkv7_backward.argtypes = [i, i, i, i, i, i] + [vp] * 16 + [vp, z, vp]
+    lib.wkv7_backward.restype = i
+    lib.wkv7_get_device_status.argtypes = [vp]
+    lib.wkv7_get_device_status.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().wkv7_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != OK:
+        raise WKV7Error(fn, status)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _tdt(code: int) -> torch.dtype:
+    return torch.float32 if code == F32 else torch.bfloat16
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _same(ts, shape, dtype):
+    for t in ts:
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            raise ValueError(f"expected {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+
+
+def forward_workspace_size(B, T, H, N, in_dtype=torch.bfloat16, algo="auto", chunk_len=0) -> int:
+    code = F32 if in_dtype == torch.float32 else BF16
+    return load_library().wkv7_forward_workspace_size(B, T, H, N, code, ALGOS[algo], chunk_len)
+
+
+def forward(r, w, k, v, a, b, s0=None, *, y=None, sT=None, y_dtype=None, algo="auto",
+            chunk_len=0, workspace=None, return_state=True, stream=None):
+    """y [B,T,H,N] (and sT [B,H,N,N] fp32) for inputs [B,T,H,N] (fp32 or bf16)."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    ycode = _dt(r) if y_dtype is None else (F32 if y_dtype == torch.float32 else BF16)
+    if y is None:
+        y = torch.empty((B, T, H, N), dtype=_tdt(ycode), device=r.device)
+    if return_state and sT is None:
+        sT = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    if s0 is not None:
+        _same((s0,), (B, H, N, N), torch.float32)
+    ws_bytes = lib.wkv7_forward_workspace_size(B, T, H, N, _dt(r), ALGOS[algo], chunk_len)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=r.device)
+    st = lib.wkv7_forward(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s0, y, sT)),
+                          ALGOS[algo], chunk_len, _ptr(workspace),
+                          0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("wkv7_forward", st)
+    return (y, sT) if return_state else y
+
+
+def step(r, w, k, v, a, b, state, *, y=None, y_dtype=None, stream=None):
+    """One decode token: inputs [B,H,N]; the fp32 state [B,H,N,N] is updated in place."""
+    lib = load_library()
+    B, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    _same((state,), (B, H, N, N), torch.float32)
+    ycode = _dt(r) if y_dtype is None else (F32 if y_dtype == torch.float32 else BF16)
+    if y is None:
+        y = torch.empty((B, H, N), dtype=_tdt(ycode), device=r.device)
+    st = lib.wkv7_step(B, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, state, y)), _stream(stream))
+    _check("wkv7_step", st)
+    return y
+
+
+def backward_workspace_size(B, T, H, N) -> int:
+    return load_library().wkv7_backward_workspace_size(B, T, H, N)
+
+
+def backward(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.float32, workspace=None,
+             out=None, stream=None):
+    """(dr, dw, dk, dv, da, db, ds0) of L = sum(dy*y) + sum(dsT*sT)."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b, dy), r.shape, r.dtype)
+    gcode = F32 if grad_dtype == torch.float32 else BF16
+    if out is None:
+        out = [torch.empty((B, T, H, N), dtype=grad_dtype, device=r.device) for _ in range(6)]
+        out.append(torch.empty((B, H, N, N), dtype=torch.float32, device=r.device))
+    ws_bytes = lib.wkv7_backward_workspace_size(B, T, H, N)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=r.device)
+    st = lib.wkv7_backward(B, T, H, N, _dt(r), gcode,
+                           *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)),
+                           _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("wkv7_backward", st)
+    return tuple(out)
+
+
+def device_status(stream=None) -> int:
+    """Synchronize and read/clear the library's sticky device status word."""
+    return load_library().wkv7_get_device_status(_stream(stream))

@@ -1,0 +1,91 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every symbol that
+include/wkv7.h declares, and rejects invalid arguments on the host (these
+calls return before any CUDA call, so they run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_rnn_sequence_wkv7_b200 import build as libbuild
+from linear_rnn_sequence_wkv7_b200 import wkv7
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return wkv7.load_library()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"WKV7_API[^;(]*?\b(wkv7_\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_api():
+    assert set(wkv7.EXPORTED_SYMBOLS) <= declared_symbols()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in sorted(declared_symbols()):
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(lib):
+    assert lib.wkv7_abi_version() == 1
+    for code in range(6):
+        assert wkv7.status_string(code)
+    assert wkv7.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    assert lib.wkv7_forward_workspace_size(1, 64, 2, 64, wkv7.F32, wkv7.ALGO_SEQ, 0) == 0
+    ws = lib.wkv7_backward_workspace_size(8, 4096, 32, 64)
+    # checkpoints every 16 tokens plus a 16-token recompute history per head
+    assert ws >= 8 * 32 * (4096 // 16) * 64 * 64 * 4 + 8 * 32 * 16 * 64 * 64 * 4
+    assert lib.wkv7_backward_workspace_size(0, 10, 1, 64) == 0
+
+
+P = ctypes.c_void_p(16)   # aligned, never dereferenced: validation fails first
+
+
+def _fwd(lib, B=1, T=4, H=1, N=64, in_dt=0, y_dt=0, ptrs=None, algo=1, chunk=0):
+    ptrs = ptrs or [P] * 9
+    return lib.wkv7_forward(B, T, H, N, in_dt, y_dt, *ptrs, algo, chunk, None, 0, None)
+
+
+def test_forward_rejects_invalid_arguments(lib):
+    assert _fwd(lib, N=32) == wkv7.ERR_UNSUPPORTED
+    assert _fwd(lib, B=-1) == wkv7.ERR_INVALID_ARG
+    assert _fwd(lib, T=-3) == wkv7.ERR_INVALID_ARG
+    assert _fwd(lib, in_dt=7) == wkv7.ERR_INVALID_ARG
+    assert _fwd(lib, algo=9) == wkv7.ERR_INVALID_ARG
+    assert _fwd(lib, chunk=32) == wkv7.ERR_UNSUPPORTED
+    bad = [P] * 9
+    bad[0] = None                                    # r missing
+    assert _fwd(lib, ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 9
+    bad[2] = ctypes.c_void_p(18)                     # k misaligned
+    assert _fwd(lib, ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert _fwd(lib, B=0) == wkv7.OK                 # empty batch: nothing to do
+    assert _fwd(lib, H=0) == wkv7.OK
+
+
+def test_step_and_backward_reject_invalid_arguments(lib):
+    assert lib.wkv7_step(1, 1, 16, 0, 0, *([P] * 8), None) == wkv7.ERR_UNSUPPORTED
+    bad = [P] * 8
+    bad[6] = None                                    # state missing
+    assert lib.wkv7_step(1, 1, 64, 0, 0, *bad, None) == wkv7.ERR_INVALID_ARG
+    assert lib.wkv7_step(0, 4, 64, 0, 0, *([P] * 8), None) == wkv7.OK
+    ptrs = [P] * 16
+    # workspace too small
+    assert lib.wkv7_backward(1, 32, 1, 64, 0, 0, *ptrs, P, 16, None) == wkv7.ERR_INVALID_ARG
+    ptrs[15] = None                                  # ds0 is required
+    assert lib.wkv7_backward(1, 32, 1, 64, 0, 0, *ptrs, P, 1 << 40, None) == wkv7.ERR_INVALID_ARG

@@ -1,0 +1,114 @@
+"""GPU backward (through the C ABI) vs the fp64 oracle and finite differences."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_rnn_sequence_wkv7_b200 import inputs, wkv7
+from tests._dev import oracle_args, to_dev, to_f64
+from tests._tol import TAU_BF16, TAU_F32, assert_close
+
+pytestmark = pytest.mark.gpu
+
+GRAD_NAMES = ("dr", "dw", "dk", "dv", "da", "db", "ds0")
+
+
+def _case(B, T, H, seed, dtype, dsT=True):
+    N = 64
+    d = inputs.gen_sequence(B, T, H, N, seed=seed, dtype=dtype, s0_std=0.1)
+    d["dy"] = inputs.gen_dy(B, T, H, N, seed=seed, dtype=dtype)
+    d["dsT"] = (inputs.gen_normal(B * H * N, N, seed=seed, stream=inputs.STREAM_DST, std=0.1)
+                .reshape(B, H, N, N) if dsT else None)
+    return d
+
+
+def _gpu(d, grad_dtype=torch.float32, heads=None):
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    out = wkv7.backward(*args, to_dev(d["s0"]), to_dev(d["dy"]), to_dev(d["dsT"]), grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    if heads is not None:       # gather the sampled heads on the device first
+        out = [x[:, :, heads] for x in out[:6]] + [out[6][:, heads]]
+    return [to_f64(x) for x in out]
+
+
+def _ref(d, heads=None):
+    raw = [d[n] for n in inputs.INPUT_NAMES] + [d["dy"]]
+    s0, dsT = d["s0"], d["dsT"]
+    if heads is not None:       # slice before widening to fp64
+        raw = [x[:, :, heads] for x in raw]
+        s0 = s0[:, heads]
+        dsT = None if dsT is None else dsT[:, heads]
+    args = [inputs.to_f64(x) for x in raw]
+    return oracle.backward(*args[:6], s0.astype(np.float64), args[6],
+                           None if dsT is None else dsT.astype(np.float64))
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 48, 100])
+def test_fp32_small(cuda_device, T):
+    d = _case(2, T, 2, 300 + T, "f32")
+    for name, got, ref in zip(GRAD_NAMES, _gpu(d), _ref(d)):
+        assert_close(got, ref, TAU_F32, name)
+
+
+@pytest.mark.parametrize("T", [16, 77])
+def test_bf16_inputs(cuda_device, T):
+    d = _case(2, T, 3, 400 + T, "bf16", dsT=False)
+    ref = _ref(d)
+    for name, got, r in zip(GRAD_NAMES, _gpu(d), ref):
+        assert_close(got, r, TAU_BF16, name)
+    for name, got, r in zip(GRAD_NAMES[:6], _gpu(d, torch.bfloat16)[:6], ref[:6]):
+        assert_close(got, r, TAU_BF16, name + "(bf16 out)", bf16_out=True)
+
+
+def test_empty_sequence_copies_dsT(cuda_device):
+    e = torch.empty(1, 0, 2, 64, device="cuda")
+    dsT = torch.randn(1, 2, 64, 64, device="cuda")
+    out = wkv7.backward(e, e, e, e, e, e, None, e, dsT)
+    torch.cuda.synchronize()
+    assert torch.equal(out[-1], dsT)
+
+
+def test_central_differences_slice(cuda_device):
+    """B=1, T=16, H=1 (fp32): GPU gradients vs central differences of the fp64
+    forward, independent of the oracle's own backward."""
+    d = _case(1, 16, 1, 500, "f32")
+    got = _gpu(d)
+    args = oracle_args(d)
+    s0, dy, dsT = d["s0"].astype(np.float64), inputs.to_f64(d["dy"]), d["dsT"].astype(np.float64)
+    tensors = args + [s0]
+    rng = np.random.default_rng(0)
+    h = 1e-6
+
+    def loss():
+        y, sT = oracle.forward(*tensors[:6], s0=tensors[6])
+        return float(np.sum(dy * y) + np.sum(dsT * sT))
+
+    for x, g, name in zip(tensors, got, GRAD_NAMES):
+        flat = x.reshape(-1)
+        coords = rng.choice(flat.size, 64, replace=False)
+        fd = np.empty(len(coords))
+        for n, c in enumerate(coords):
+            old = flat[c]
+            flat[c] = old + h
+            lp = loss()
+            flat[c] = old - h
+            lm = loss()
+            flat[c] = old
+            fd[n] = (lp - lm) / (2 * h)
+        sel = g.reshape(-1)[coords]
+        scale = np.sqrt(np.mean(g ** 2))
+        assert np.max(np.abs(sel - fd)) <= 1e-5 * scale + 1e-7, name
+
+
+def test_training_workload_sampled_heads(cuda_device):
+    """B=8, T=4096, H=32 bf16 with dy ~ N(0,1) bf16 and dsT = 0: sampled heads."""
+    cfg = inputs.WORKLOADS["train_bwd_b8_t4096_h32"]
+    d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
+                            s0_std=cfg["s0_std"])
+    d["dy"] = inputs.gen_dy(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16")
+    d["dsT"] = None
+    heads = sorted(np.random.default_rng(4).choice(cfg["H"], 2, replace=False).tolist())
+    got = _gpu(d, heads=heads)
+    ref = _ref(d, heads)
+    for name, g, r in zip(GRAD_NAMES, got, ref):
+        assert_close(g, r, TAU_BF16, name)

@@ -1,0 +1,127 @@
+"""GPU forward (through the C ABI) vs the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_rnn_sequence_wkv7_b200 import inputs, wkv7
+from tests._dev import oracle_args, to_dev, to_f64
+from tests._tol import TAU_BF16, TAU_F32, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run_forward(d, y_dtype=None, algo="seq", s0=True):
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    s0_t = to_dev(d["s0"]) if (s0 and d["s0"] is not None) else None
+    y, sT = wkv7.forward(*args, s0=s0_t, y_dtype=y_dtype, algo=algo)
+    torch.cuda.synchronize()
+    return y, sT
+
+
+def oracle_forward(d, heads=None):
+    raw = [d[n] for n in inputs.INPUT_NAMES]
+    s0 = d["s0"]
+    if heads is not None:       # slice before widening to fp64
+        raw = [x[:, :, heads] for x in raw]
+        s0 = None if s0 is None else s0[:, heads]
+    args = [inputs.to_f64(x) for x in raw]
+    return oracle.forward(*args, s0=None if s0 is None else s0.astype(np.float64))
+
+
+def test_fp32_reference_workload(cuda_device):
+    """B=1, T=64, H=2, fp32 everywhere, zero s0: max err <= 1e-5 rms."""
+    cfg = inputs.WORKLOADS["fwd_b1_t64_h2_f32"]
+    d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="f32")
+    y, sT = run_forward(d)
+    yr, sr = oracle_forward(d)
+    assert_close(to_f64(y), yr, TAU_F32, "y")
+    assert_close(to_f64(sT), sr, TAU_F32, "sT")
+
+
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65, 200])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_small_shapes(cuda_device, T, dtype):
+    B, H, N = 2, 3, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=100 + T, dtype=dtype, s0_std=0.1)
+    yr, sr = oracle_forward(d)
+    tau = TAU_F32 if dtype == "f32" else TAU_BF16
+    y, sT = run_forward(d, y_dtype=torch.float32)
+    assert_close(to_f64(y), yr, tau, "y")
+    assert_close(to_f64(sT), sr, tau, "sT")
+    if dtype == "bf16":
+        yb, _ = run_forward(d, y_dtype=torch.bfloat16)
+        assert yb.dtype == torch.bfloat16
+        assert_close(to_f64(yb), yr, tau, "y(bf16 out)", bf16_out=True)
+
+
+def test_zero_initial_state_and_no_final_state(cuda_device):
+    B, T, H, N = 1, 33, 2, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=7, dtype="bf16")
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    y = wkv7.forward(*args, s0=None, y_dtype=torch.float32, algo="seq", return_state=False)
+    yr, _ = oracle_forward(d)
+    assert_close(to_f64(y), yr, TAU_BF16, "y")
+
+
+def test_state_passing_in_place(cuda_device):
+    """forward(T) == forward(T1) then forward(T - T1) continuing from sT (s0 aliasing sT)."""
+    B, T, H, N = 2, 100, 2, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=9, dtype="f32", s0_std=0.1)
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    s0 = to_dev(d["s0"])
+    y_full, s_full = wkv7.forward(*args, s0=s0, algo="seq")
+    state = s0.clone()
+    y1 = wkv7.forward(*(x[:, :37].contiguous() for x in args), s0=state, sT=state, algo="seq")[0]
+    y2 = wkv7.forward(*(x[:, 37:].contiguous() for x in args), s0=state, sT=state, algo="seq")[0]
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([y1, y2], dim=1), y_full)
+    assert torch.equal(state, s_full)
+
+
+def test_empty_sequence_copies_state(cuda_device):
+    s0 = torch.randn(2, 3, 64, 64, device="cuda")
+    e = torch.empty(2, 0, 3, 64, device="cuda")
+    y, sT = wkv7.forward(e, e, e, e, e, e, s0=s0, algo="seq")
+    torch.cuda.synchronize()
+    assert y.shape == (2, 0, 3, 64)
+    assert torch.equal(sT, s0)
+    y, sT = wkv7.forward(e, e, e, e, e, e, s0=None, algo="seq")
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(sT) == 0
+
+
+def test_invalid_arguments_raise(cuda_device):
+    x = torch.zeros(1, 4, 1, 32, device="cuda")
+    with pytest.raises(wkv7.WKV7Error) as ei:
+        wkv7.forward(x, x, x, x, x, x, algo="seq")
+    assert ei.value.status == wkv7.ERR_UNSUPPORTED
+
+
+def _sample_heads(H, n, seed):
+    return sorted(np.random.default_rng(seed).choice(H, size=min(n, H), replace=False).tolist())
+
+
+def test_prefill_workload_sampled_heads(cuda_device):
+    """B=8, T=4096, H=32 bf16 prefill (the benchmark's launch): y (bf16) and sT on
+    sampled heads of every batch row vs the oracle."""
+    cfg = inputs.WORKLOADS["prefill_b8_t4096_h32_bf16"]
+    d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
+                            s0_std=cfg["s0_std"])
+    y, sT = run_forward(d, algo="auto")
+    heads = _sample_heads(cfg["H"], 3, 0)
+    yr, sr = oracle_forward(d, heads)
+    assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y", bf16_out=True)
+    assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT")
+
+
+def test_long_context_workload_sampled_heads(cuda_device):
+    """B=1, T=65536, H=32 with w near 1 (long memory): sequential scan on sampled heads."""
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
+                            x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="seq")
+    heads = _sample_heads(cfg["H"], 2, 1)
+    yr, sr = oracle_forward(d, heads)
+    assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y")
+    assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT")
