@@ -90,6 +90,16 @@ def fwd_flops(B, T, H):
     return 9 * N * N * B * T * H
 
 
+def fwd_chunk_flops(B, T, H, L=32):
+    """Tensor-core flop the chunked form issues per call (bf16 passes counted):
+    per 32-token chunk 3-pass Gram 64x64x64, W^T 64x32x32 (3), U~^T (2),
+    M' 64x64x32 (3), Q'^T 64x32x32 (3), E 64x64x64 (3+2 over halves of K),
+    Y_loc^T 64x32x64 (3+2), state 64x96x64 (3)."""
+    per_chunk = 2 * (3 * 64 * 64 * 64 + 3 * 64 * 32 * 32 + 2 * 64 * 32 * 32 + 3 * 64 * 64 * 32
+                     + 3 * 64 * 32 * 32 + 5 * 64 * 64 * 32 + 5 * 64 * 32 * 32 + 3 * 64 * 96 * 64)
+    return per_chunk * B * H * ((T + L - 1) // L)
+
+
 def bwd_bytes(B, T, H, in_bytes=2, g_bytes=2):
     """Six inputs + dy read, six gradients written, s0 read, ds0 written."""
     return B * T * H * N * (7 * in_bytes + 6 * g_bytes) + 2 * B * H * N * N * 4
@@ -297,8 +307,7 @@ def bench_forward(args, dist, peaks, device):
     d2h = host_y.numel() * 2 + host_sT.numel() * 4
 
     head_tokens = B * T * H
-    kernel = "fwd_chunk" if (args.algo == "chunk" or (args.algo == "auto" and "fwd_chunk" in wkv7_kernels())) \
-        else "fwd_seq"
+    kernel = "fwd_" + wkv7.resolve_algo(T, torch.bfloat16, args.algo)
     per_launch = secs / args.steps
     nbytes = fwd_bytes(B, T, H)
     if kernel == "fwd_seq":
@@ -312,7 +321,8 @@ def bench_forward(args, dist, peaks, device):
         ach = nbytes / per_launch / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": pk, "unit": "GB/s", "frac": ach / pk,
                 "peak_source": peaks["source"], "per_unit": "896 B per head-token + 32 KiB state per head",
-                "units_per_launch": head_tokens}
+                "units_per_launch": head_tokens,
+                "tensor_tflops": fwd_chunk_flops(B, T, H) / per_launch / 1e12}
     src = {"fwd_seq": ("fwd_seq.cu", "common.cuh"), "fwd_chunk": ("fwd_chunk.cu", "common.cuh")}[kernel]
     roof["traffic"] = recorded_traffic(kernel, source_hash(*src))
     roof["kernel"] = kernel
@@ -327,15 +337,6 @@ def bench_forward(args, dist, peaks, device):
         "launches": args.steps,
         "sample": d,
     }
-
-
-def wkv7_kernels():
-    """Forward kernels this build implements (the chunked one is picked by AUTO
-    for bf16 inputs when present)."""
-    from linear_rnn_sequence_wkv7_b200 import wkv7
-    lib = wkv7.load_library()
-    return ("fwd_seq", "fwd_chunk") if getattr(lib, "wkv7_has_chunked", None) and lib.wkv7_has_chunked() \
-        else ("fwd_seq",)
 
 
 def bench_backward(args, dist, peaks, device, d):

@@ -106,6 +106,13 @@ WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dtyp
                          cudaStream_t stream);
 
 /*
+ * The algorithm wkv7_forward runs for these arguments (WKV7_ALGO_SEQ or
+ * WKV7_ALGO_CHUNK; AUTO picks CHUNK for bf16 inputs with T >= 64), or -1 for
+ * an invalid dtype / algorithm.  The chunked form takes bf16 inputs only.
+ */
+WKV7_API int wkv7_forward_resolve_algo(int T, wkv7_dtype in_dtype, wkv7_algo algo);
+
+/*
  * One decode token (T = 1) for every (b, h), updating the state IN PLACE
  * (constant memory and time per token: RWKV-7 "Goose" abstract).
  *   r, w, k, v, a, b : [B, H, N] of in_dtype

@@ -5,3 +5,4 @@
 #include "fwd_seq.cu"
 #include "step.cu"
 #include "bwd_seq.cu"
+#include "fwd_chunk.cu"

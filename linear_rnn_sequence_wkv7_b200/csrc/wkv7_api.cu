@@ -22,6 +22,9 @@ cudaError_t bwd_seq(int B, int T, int H, int CK, wkv7_dtype in_dt, wkv7_dtype g_
                     const void *dy, const float *dsT, const float *ckpt, float *hist, void *dr, void *dw,
                     void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st);
 size_t bwd_hist_bytes(int B, int H, int CK);
+cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
+                      const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
+                      cudaStream_t st);
 
 namespace {
 
@@ -52,6 +55,14 @@ wkv7_status copy_or_zero_state(float *dst, const float *src, int B, int H, cudaS
     if (bytes == 0 || dst == src) return WKV7_OK;
     if (src) return from_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
     return from_cuda(cudaMemsetAsync(dst, 0, bytes, st));
+}
+
+// The algorithm AUTO resolves to: the chunked tensor-core form for bf16 inputs
+// with at least two chunks of tokens, else the sequential scan (the only form
+// for fp32 inputs, whose 1e-5 tolerance the bf16-split products cannot meet).
+wkv7_algo resolve_algo(int T, wkv7_dtype in_dt, wkv7_algo algo) {
+    if (algo != WKV7_ALGO_AUTO) return algo;
+    return (in_dt == WKV7_BF16 && T >= 64) ? WKV7_ALGO_CHUNK : WKV7_ALGO_SEQ;
 }
 
 size_t bwd_ckpt_bytes(int B, int T, int H) {
@@ -101,8 +112,17 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
     if (T == 0) return copy_or_zero_state(sT, s0, B, H, stream);
     for (const void *p : {r, w, k, v, a, b, (const void *)y})
         if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
-    if (algo == WKV7_ALGO_CHUNK) return WKV7_ERR_UNSUPPORTED;
+    if (resolve_algo(T, in_dt, algo) == WKV7_ALGO_CHUNK) {
+        if (in_dt != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
+        return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+    }
     return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+}
+
+int wkv7_forward_resolve_algo(int T, wkv7_dtype in_dtype, wkv7_algo algo) {
+    if (!dtype_ok(in_dtype) || T < 0) return -1;
+    if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_SEQ && algo != WKV7_ALGO_CHUNK) return -1;
+    return (int)resolve_algo(T, in_dtype, algo);
 }
 
 wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,

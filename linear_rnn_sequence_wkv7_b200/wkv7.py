@@ -24,6 +24,7 @@ ALGOS = {"auto": ALGO_AUTO, "seq": ALGO_SEQ, "chunk": ALGO_CHUNK}
 EXPORTED_SYMBOLS = (
     "wkv7_abi_version", "wkv7_status_string", "wkv7_forward_workspace_size", "wkv7_forward",
     "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
+    "wkv7_forward_resolve_algo",
 )
 
 _lib = None
@@ -57,6 +58,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward_workspace_size.restype = z
     lib.wkv7_backward.argtypes = [i, i, i, i, i, i] + [vp] * 16 + [vp, z, vp]
     lib.wkv7_backward.restype = i
+    lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
+    lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_get_device_status.argtypes = [vp]
     lib.wkv7_get_device_status.restype = i
     _lib = lib
@@ -129,6 +132,14 @@ def forward(r, w, k, v, a, b, s0=None, *, y=None, sT=None, y_dtype=None, algo="a
                           0 if workspace is None else workspace.numel(), _stream(stream))
     _check("wkv7_forward", st)
     return (y, sT) if return_state else y
+
+
+def resolve_algo(T, in_dtype=torch.bfloat16, algo="auto") -> str:
+    """Which forward algorithm ("seq" or "chunk") the library runs for these arguments."""
+    code = load_library().wkv7_forward_resolve_algo(T, F32 if in_dtype == torch.float32 else BF16, ALGOS[algo])
+    if code < 0:
+        raise ValueError("invalid dtype or algorithm")
+    return {ALGO_SEQ: "seq", ALGO_CHUNK: "chunk"}[code]
 
 
 def step(r, w, k, v, a, b, state, *, y=None, y_dtype=None, stream=None):

@@ -108,7 +108,9 @@ def test_prefill_workload_sampled_heads(cuda_device):
     cfg = inputs.WORKLOADS["prefill_b8_t4096_h32_bf16"]
     d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
                             s0_std=cfg["s0_std"])
+    assert wkv7.resolve_algo(cfg["T"], torch.bfloat16, "auto") == "chunk"
     y, sT = run_forward(d, algo="auto")
+    assert wkv7.device_status() == wkv7.OK
     heads = _sample_heads(cfg["H"], 3, 0)
     yr, sr = oracle_forward(d, heads)
     assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y", bf16_out=True)
@@ -125,3 +127,79 @@ def test_long_context_workload_sampled_heads(cuda_device):
     yr, sr = oracle_forward(d, heads)
     assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y")
     assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT")
+
+
+# --- chunked tensor-core form ------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 15, 32, 33, 64, 65, 200])
+def test_chunked_small_shapes(cuda_device, T):
+    B, H, N = 2, 3, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=200 + T, dtype="bf16", s0_std=0.1)
+    yr, sr = oracle_forward(d)
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert_close(to_f64(y), yr, TAU_BF16, "y")
+    assert_close(to_f64(sT), sr, TAU_BF16, "sT")
+    yb, _ = run_forward(d, y_dtype=torch.bfloat16, algo="chunk")
+    assert_close(to_f64(yb), yr, TAU_BF16, "y(bf16 out)", bf16_out=True)
+    assert wkv7.device_status() == wkv7.OK
+
+
+def test_chunked_zero_state_and_in_place(cuda_device):
+    B, T, H, N = 2, 130, 2, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=301, dtype="bf16", s0_std=0.1)
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    y0 = wkv7.forward(*args, s0=None, y_dtype=torch.float32, algo="chunk", return_state=False)
+    d0 = dict(d, s0=None)
+    yr, _ = oracle_forward(d0)
+    assert_close(to_f64(y0), yr, TAU_BF16, "y (zero s0)")
+    state = to_dev(d["s0"])
+    y1, _ = wkv7.forward(*args, s0=state, sT=state, y_dtype=torch.float32, algo="chunk")
+    yr1, sr1 = oracle_forward(d)
+    assert_close(to_f64(y1), yr1, TAU_BF16, "y")
+    assert_close(to_f64(state), sr1, TAU_BF16, "sT in place")
+
+
+def test_auto_picks_chunked_for_bf16():
+    assert wkv7.resolve_algo(4096, torch.bfloat16, "auto") == "chunk"
+    assert wkv7.resolve_algo(4096, torch.float32, "auto") == "seq"
+    assert wkv7.resolve_algo(32, torch.bfloat16, "auto") == "seq"
+
+
+def test_chunked_rejects_fp32_inputs(cuda_device):
+    x = torch.zeros(1, 64, 1, 64, device="cuda")
+    with pytest.raises(wkv7.WKV7Error) as ei:
+        wkv7.forward(x, x, x, x, x, x, algo="chunk")
+    assert ei.value.status == wkv7.ERR_UNSUPPORTED
+
+
+def test_chunked_flags_out_of_domain_decay(cuda_device):
+    """A chunk whose decay product underflows the fp32 range raises the RANGE
+    status word (no fault); the sequential form handles the same input."""
+    B, T, H, N = 1, 64, 1, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=5, dtype="bf16")
+    d["w"] = inputs.f32_to_bf16_bits(np.full((B, T, H, N), 0.05, np.float32))
+    assert wkv7.device_status() == wkv7.OK
+    run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert wkv7.device_status() == wkv7.ERR_RANGE
+    assert wkv7.device_status() == wkv7.OK          # cleared by the read
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="seq")
+    yr, sr = oracle_forward(d)
+    assert_close(to_f64(y), yr, TAU_BF16, "y (seq)")
+
+
+def test_long_context_chunked_matches_oracle_and_sequential(cuda_device):
+    """B=1, T=65536, H=32, w near 1, chunked form: sampled heads vs the oracle,
+    and every head vs the sequential scan."""
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
+                            x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
+    yc, sc = run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert wkv7.device_status() == wkv7.OK
+    heads = _sample_heads(cfg["H"], 2, 2)
+    yr, sr = oracle_forward(d, heads)
+    assert_close(to_f64(yc[:, :, heads]), yr, TAU_BF16, "y vs oracle")
+    assert_close(to_f64(sc[:, heads]), sr, TAU_BF16, "sT vs oracle")
+    ys, ss = run_forward(d, y_dtype=torch.float32, algo="seq")
+    for h in range(cfg["H"]):
+        assert_close(to_f64(yc[:, :, h]), to_f64(ys[:, :, h]), TAU_BF16, f"y head {h} vs seq")
+    assert_close(to_f64(sc), to_f64(ss), TAU_BF16, "sT vs seq")
