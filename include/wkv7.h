@@ -57,8 +57,10 @@ typedef enum {
     WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
     WKV7_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed        */
     WKV7_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up          */
-    WKV7_ERR_RANGE = 5         /* device-side: input outside the chunked
+    WKV7_ERR_RANGE = 5,        /* device-side: input outside the chunked
                                   form's numeric domain (see wkv7_forward)   */
+    WKV7_ERR_TOO_LARGE = 6     /* problem needs more scratch than the fixed
+                                  array of wkv7_backward_noalloc holds       */
 } wkv7_status;
 
 typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1 } wkv7_dtype;
@@ -143,6 +145,30 @@ WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dty
                           const float *dsT, void *dr, void *dw, void *dk, void *dv, void *da,
                           void *db, float *ds0, void *workspace, size_t workspace_bytes,
                           cudaStream_t stream);
+
+/*
+ * wkv7_backward without workspace: the same computation, arguments and
+ * outputs, with its scratch taken from a fixed 32 MiB array in device memory
+ * that belongs to the library.  The pages have no counterpart of this call; it
+ * exists for callers that cannot allocate device memory where they run the
+ * backward (an engine plugin whose enqueue path must not call the allocator,
+ * or a framework whose memory pool already holds the device's memory).
+ *   - Every GPU that loads the library keeps the 32 MiB array until exit.
+ *   - Problems whose wkv7_backward_workspace_size() exceeds 32 MiB return
+ *     WKV7_ERR_TOO_LARGE and launch nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it: make that first call before any
+ *     stream capture.
+ *   - All calls share the array, which keeps the previous call's contents
+ *     (the backward overwrites every scratch byte before reading it).  Calls
+ *     that overlap on the GPU race on the array: do not run two at once.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ */
+WKV7_API wkv7_status wkv7_backward_noalloc(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                           wkv7_dtype grad_dtype, const void *r, const void *w, const void *k,
+                                           const void *v, const void *a, const void *b, const float *s0,
+                                           const void *dy, const float *dsT, void *dr, void *dw, void *dk,
+                                           void *dv, void *da, void *db, float *ds0, cudaStream_t stream);
 
 /*
  * Synchronizes `stream`, then returns and clears the sticky device-side status

@@ -6,3 +6,4 @@
 #include "step.cu"
 #include "bwd_seq.cu"
 #include "fwd_chunk.cu"
+#include "bwd_noalloc.cu"

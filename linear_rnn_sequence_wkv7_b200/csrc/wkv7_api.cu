@@ -87,6 +87,7 @@ const char *wkv7_status_string(wkv7_status s) {
         case WKV7_ERR_CUDA: return "CUDA error";
         case WKV7_ERR_TIMEOUT: return "device wait timed out";
         case WKV7_ERR_RANGE: return "input outside the chunked form's numeric domain";
+        case WKV7_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of wkv7_backward_noalloc";
     }
     return "unknown status";
 }

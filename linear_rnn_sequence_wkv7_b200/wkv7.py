@@ -16,7 +16,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libwkv7.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_TOO_LARGE = range(7)
 F32, BF16 = 0, 1
 ALGO_AUTO, ALGO_SEQ, ALGO_CHUNK = 0, 1, 2
 ALGOS = {"auto": ALGO_AUTO, "seq": ALGO_SEQ, "chunk": ALGO_CHUNK}
@@ -24,7 +24,7 @@ ALGOS = {"auto": ALGO_AUTO, "seq": ALGO_SEQ, "chunk": ALGO_CHUNK}
 EXPORTED_SYMBOLS = (
     "wkv7_abi_version", "wkv7_status_string", "wkv7_forward_workspace_size", "wkv7_forward",
     "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
-    "wkv7_forward_resolve_algo",
+    "wkv7_forward_resolve_algo", "wkv7_backward_noalloc",
 )
 
 _lib = None
@@ -58,6 +58,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward_workspace_size.restype = z
     lib.wkv7_backward.argtypes = [i, i, i, i, i, i] + [vp] * 16 + [vp, z, vp]
     lib.wkv7_backward.restype = i
+    lib.wkv7_backward_noalloc.argtypes = [i, i, i, i, i, i] + [vp] * 16 + [vp]
+    lib.wkv7_backward_noalloc.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_get_device_status.argtypes = [vp]
@@ -177,6 +179,24 @@ def backward(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.float32, wo
                            *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)),
                            _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check("wkv7_backward", st)
+    return tuple(out)
+
+
+def backward_noalloc(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.float32, out=None, stream=None):
+    """wkv7_backward_noalloc: the backward with the library's fixed 32 MiB device
+    scratch instead of a workspace, for callers that cannot allocate device
+    memory where they run it (see include/wkv7.h).  Output tensors are still the
+    caller's; pass ``out`` to avoid any allocation here as well."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b, dy), r.shape, r.dtype)
+    gcode = F32 if grad_dtype == torch.float32 else BF16
+    if out is None:
+        out = [torch.empty((B, T, H, N), dtype=grad_dtype, device=r.device) for _ in range(6)]
+        out.append(torch.empty((B, H, N, N), dtype=torch.float32, device=r.device))
+    st = lib.wkv7_backward_noalloc(B, T, H, N, _dt(r), gcode,
+                                   *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)), _stream(stream))
+    _check("wkv7_backward_noalloc", st)
     return tuple(out)
 
 
