@@ -75,6 +75,37 @@ __device__ __forceinline__ void gemm_split(uint32_t d_tmem, const Op &A, const O
             mma(d_tmem, sdesc(A.lo + ks * A.kstep, A.lbo, A.sbo), sdesc(B.hi + ks * B.kstep, B.lbo, B.sbo), idesc, 1u);
 }
 
+// Operand given by full base descriptors (hi copy, lo copy or 0 when the
+// operand is exact in bf16) and the start-address step between K=16 slices,
+// in 16-byte units.  Shared-memory addresses stay below 256 KB, so stepping
+// the 14-bit start field never carries into the other fields.
+struct OpD {
+    uint64_t hi, lo;
+    uint32_t kstep16;
+};
+
+__device__ __forceinline__ OpD opd_k(uint32_t hi, uint32_t lo, int cols) {
+    return OpD{sdesc(hi, 128u, (uint32_t)(cols >> 3) << 7), lo ? sdesc(lo, 128u, (uint32_t)(cols >> 3) << 7) : 0ull,
+               16u};
+}
+__device__ __forceinline__ OpD opd_mn(uint32_t hi, uint32_t lo, int cols) {
+    const uint32_t lbo = (uint32_t)(cols >> 3) << 7;
+    return OpD{sdesc(hi, lbo, 128u), lo ? sdesc(lo, lbo, 128u) : 0ull, (2u * lbo) >> 4};
+}
+
+__device__ __forceinline__ void gemm_split_d(uint32_t d_tmem, const OpD &A, const OpD &B, uint32_t idesc, int ksteps,
+                                             bool accumulate) {
+    uint32_t acc = accumulate ? 1u : 0u;
+    for (int ks = 0; ks < ksteps; ++ks) {
+        mma(d_tmem, A.hi + ks * A.kstep16, B.hi + ks * B.kstep16, idesc, acc);
+        acc = 1u;
+    }
+    if (B.lo)
+        for (int ks = 0; ks < ksteps; ++ks) mma(d_tmem, A.hi + ks * A.kstep16, B.lo + ks * B.kstep16, idesc, 1u);
+    if (A.lo)
+        for (int ks = 0; ks < ksteps; ++ks) mma(d_tmem, A.lo + ks * A.kstep16, B.hi + ks * B.kstep16, idesc, 1u);
+}
+
 __device__ __forceinline__ void commit(uint32_t mbar_saddr) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar_saddr)
                  : "memory");
@@ -92,6 +123,16 @@ __device__ __forceinline__ void tmem_alloc(uint32_t dst_saddr, uint32_t ncols) {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
+
+// 32 lanes x 16 consecutive 32-bit columns, without waiting (pair with tmem_wait)
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns; thread t of the warp gets lane (base + t)
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -138,16 +179,19 @@ __device__ __forceinline__ void split2(float x, __nv_bfloat16 &hi, __nv_bfloat16
 }
 
 // store 8 consecutive values (one core-matrix row) as hi and lo 16-byte vectors
+// (packed conversions: two values per cvt, the hi part re-expanded by bit ops)
 __device__ __forceinline__ void store8_split(unsigned char *hi_base, unsigned char *lo_base, uint32_t off,
                                              const float *x) {
     uint32_t h[4], l[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split2(x[2 * q], h0, l0);
-        split2(x[2 * q + 1], h1, l1);
-        h[q] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        l[q] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        const __nv_bfloat162 hp = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        const uint32_t hu = *reinterpret_cast<const uint32_t *>(&hp);
+        const float r0 = x[2 * q] - __uint_as_float(hu << 16);
+        const float r1 = x[2 * q + 1] - __uint_as_float(hu & 0xffff0000u);
+        const __nv_bfloat162 lp = __floats2bfloat162_rn(r0, r1);
+        h[q] = hu;
+        l[q] = *reinterpret_cast<const uint32_t *>(&lp);
     }
     *reinterpret_cast<uint4 *>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
     if (lo_base) *reinterpret_cast<uint4 *>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
