@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from linear_rnn_sequence_wkv7_b200 import inputs  # noqa: E402
+from linear_rnn_sequence_wkv7_b200.dist import Dist, aggregate_throughput, shard_seed  # noqa: E402
 
 METRIC = "WKV7 head-tokens/sec fwd/bwd + decode steps/sec; % of HBM/FP32/TC roofline"
 N = 64
@@ -211,40 +212,6 @@ def to_pinned(x):
     return t.pin_memory()
 
 
-class Dist:
-    def __init__(self):
-        self.world = int(os.environ.get("WORLD_SIZE", "1"))
-        self.rank = int(os.environ.get("RANK", "0"))
-        self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        self.pg = None
-
-    def init(self):
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(self.local)
-        if self.world > 1:
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
-            self.pg = dist
-
-    def barrier(self):
-        if self.pg:
-            self.pg.barrier()
-
-    def max(self, x):
-        if not self.pg:
-            return x
-        import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
-
-    def close(self):
-        if self.pg:
-            self.pg.destroy_process_group()
-
-
 def timed(fn, steps, warmup, dist, stream):
     """Device time of `steps` calls of fn (CUDA events on `stream`), max over ranks."""
     import torch
@@ -268,7 +235,7 @@ def bench_forward(args, dist, peaks, device):
     from linear_rnn_sequence_wkv7_b200 import wkv7
     cfg = FWD
     B, T, H = cfg["B"], cfg["T"], cfg["H"]
-    d = inputs.gen_sequence(B, T, H, N, seed=cfg["seed"] + 1000 * dist.rank, dtype="bf16",
+    d = inputs.gen_sequence(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16",
                             s0_std=cfg["s0_std"])
     dev = [to_dev(d[n], device) for n in inputs.INPUT_NAMES]
     s0 = to_dev(d["s0"], device)
@@ -328,11 +295,11 @@ def bench_forward(args, dist, peaks, device):
     roof["kernel"] = kernel
     roof["hbm_frac"] = nbytes / per_launch / 1e9 / peaks["hbm_gbs"]
     return {
-        "value": head_tokens * dist.world / secs * args.steps,
+        "value": aggregate_throughput(head_tokens * args.steps, secs, dist.world),
         "ms_per_step": secs / args.steps * 1e3,
         "roofline": roof,
         "clocks": clocks,
-        "e2e": {"value": head_tokens * dist.world / e2e_secs * e2e_steps, "unit": "head-tokens/s",
+        "e2e": {"value": aggregate_throughput(head_tokens * e2e_steps, e2e_secs, dist.world), "unit": "head-tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "launches": args.steps,
         "sample": d,
@@ -346,7 +313,7 @@ def bench_backward(args, dist, peaks, device, d):
     B, T, H = cfg["B"], cfg["T"], cfg["H"]
     dev = [to_dev(d[n], device) for n in inputs.INPUT_NAMES]
     s0 = to_dev(d["s0"], device)
-    dy = to_dev(inputs.gen_dy(B, T, H, N, seed=cfg["seed"] + 1000 * dist.rank, dtype="bf16"), device)
+    dy = to_dev(inputs.gen_dy(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16"), device)
     out = [torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device) for _ in range(6)]
     out.append(torch.empty(B, H, N, N, dtype=torch.float32, device=device))
     ws = torch.empty(wkv7.backward_workspace_size(B, T, H, N), dtype=torch.uint8, device=device)
@@ -360,7 +327,8 @@ def bench_backward(args, dist, peaks, device, d):
     per = secs / steps
     pk = fp32_peak_tflops(peaks["sm_max_mhz"])
     ach = bwd_flops(B, T, H) / per / 1e12
-    return {"value": B * T * H * dist.world / per, "unit": "head-tokens/s", "ms_per_step": per * 1e3,
+    return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
+            "ms_per_step": per * 1e3,
             "steps": steps, "launches": 2 * steps,
             "roofline": {"bound": "alu", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                          "per_unit": "28*N^2 flop per head-token",
@@ -395,9 +363,10 @@ def bench_decode(args, dist, peaks, device, steps_in):
     nbytes = step_bytes(B, H)
     ach = nbytes / per_step / 1e9
     del g
-    return {"value": dist.world / per_step, "unit": "steps/s", "us_per_step": per_step * 1e6,
+    return {"value": aggregate_throughput(1, per_step, dist.world), "unit": "steps/s",
+            "us_per_step": per_step * 1e6,
             "graph_replays": reps, "steps_per_replay": n, "launches": reps * n,
-            "head_tokens_per_s": B * H * dist.world / per_step,
+            "head_tokens_per_s": aggregate_throughput(B * H, per_step, dist.world),
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "per_unit": "32 KiB state RMW + 896 B per head",
                          "units_per_launch": B * H,
@@ -432,8 +401,7 @@ def cpu_baseline(d, budget_s=10.0):
 
 def run_ours(args):
     import torch
-    dist = Dist()
-    dist.init()
+    dist = Dist("nccl").init()
     device = torch.device("cuda", dist.local)
     from linear_rnn_sequence_wkv7_b200 import wkv7
     wkv7.load_library()
@@ -445,7 +413,7 @@ def run_ours(args):
     if "decode" in parts:
         def gen():
             steps_in.update(inputs.gen_steps(args.decode_steps, DEC["B"], DEC["H"], N,
-                                             seed=DEC["seed"] + 1000 * dist.rank, dtype="bf16"))
+                                             seed=shard_seed(DEC["seed"], dist.rank), dtype="bf16"))
         gen_thread = threading.Thread(target=gen)
         gen_thread.start()
 
