@@ -16,8 +16,9 @@
 //   Gram  = [a'; r'] [b-; k-]^T                        (64 x 64)
 //   L_ab, L_ak = strictly lower parts of the a' rows; L_rb, L_rk = lower
 //                parts of the r' rows (diagonal included)
-//   W' = (I - L_ab)^{-1} A',  U~ = (I - L_ab)^{-1} L_ak V
-//            (fp32 forward substitution on the CUDA cores; u_t = S G w'_t + u~_t)
+//   T = (I - L_ab)^{-1} (blocked: two 16x16 diagonal inverses by forward
+//       substitution, then T21 = T22 L21 T11),  P = T L_ak      (CUDA cores, fp32)
+//   W'^T = A'^T T^T,  U~^T = V^T P^T                   (u_t = S G w'_t + u~_t)
 //   M = G (I + W'^T B-),  Q^T = G (R'^T + W'^T L_rb^T)   (G scales rows)
 //   E = U~^T B- + V^T K-,  Y_loc^T = U~^T L_rb^T + V^T L_rk^T
 //   S_out = S M + E,  Y^T = S Q^T + Y_loc^T          (state-dependent part)
@@ -27,52 +28,64 @@
 // bf16 input such as v) with fp32 accumulation in TMEM.  A single tf32 or bf16
 // pass is not accurate enough for the 2e-3 rms bound on this workload.
 //
-// Mapping: one CTA (256 threads, 8 warps) per (b, h), two CTAs per SM;
-// chunks are processed in order.  Per chunk: P0 builds the decayed operands
-// from the token tile (suffix products by warp shuffles); R1 Gram; P1 masks
-// it; P1b solves W' and U~ by forward substitution; R3 M'', Q''^T, E,
-// Y_loc^T; P3 finishes M and Q; R4 accumulates the state product onto
-// [E | Y_loc^T]; P4 writes y and stages S_out as the next chunk's operand.
-// The rounds are software-pipelined across chunks: R4 of chunk c runs under
-// P0 of chunk c+1, and R1 of chunk c+1 under P4 of chunk c.  One thread issues
-// the MMAs; completion is tracked by an mbarrier with a bounded wait.  Token
-// tiles are fetched with cp.async two chunks ahead of use.
+// Mapping: one CTA per (b, h), two CTAs per SM.  Warps 0-7 (256 threads)
+// run the CUDA-core phases; warp 8 issues the tensor-core rounds.  Per chunk:
+// P0 builds the decayed operands from the token tile (suffix products by
+// warp shuffles); R1 Gram; P1 masks it and computes T and P; R2 W'^T, U~^T;
+// P2 stages them; R3 M'', Q''^T, E, Y_loc^T; P3 finishes M and Q; R4
+// accumulates the state product onto [E | Y_loc^T]; P4 writes y and stages
+// S_out as the next chunk's operand.  Each round has a "ready" mbarrier (the
+// 256 compute threads arrive after publishing their shared-memory writes) and
+// a "done" mbarrier (tcgen05.commit); every wait is bounded.  The compute
+// warps build chunk c+1's operands (P0) while R4 of chunk c runs, and R1 of
+// chunk c+1 runs while they finish chunk c (P4).  Token tiles arrive by
+// cp.async one chunk ahead.
 //
-// TMEM (256 columns; an M=64 accumulator occupies lanes 16q..16q+15 of warp
-// quadrant q):
-//   X: cols [0, 96)    Gram (64), then M'' (64) | Q''^T (32)
-//   Z: cols [128, 224) [E | Y_loc^T], then += S [M | Q^T]
+// TMEM (256 columns).  An M=64 accumulator occupies lanes 16q..16q+15 of warp
+// quadrant q; a second one at lane offset 16 fills lanes 16q+16..16q+31, so
+// paired results are read by all 32 lanes of a warp:
+//   X: cols [0, 96)     Gram (cols 0-63), then [M'' | Q''^T]
+//   Y: cols [96, 128)   W'^T (lane 0) and U~^T (lane 16)
+//   Z: cols [128, 224)  [E | Y_loc^T], then += S [M | Q^T] = [S_out | Y^T]
+// L_rb and L_rk are stored next to b- and k- (one [64][96] operand), and M
+// next to Q^T, so R3 and R4 run as N=96 products.
 #include "umma.cuh"
 
 namespace wkv7 {
 
 namespace chunk {
 
-constexpr int L = 32;          // tokens per chunk
-constexpr int NT = 256;        // threads per CTA
+constexpr int L = 32;              // tokens per chunk
+constexpr int NC = 256;            // compute threads (warps 0-7)
+constexpr int NT = NC + 32;        // + the MMA warp
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_X = 0, COL_Z = 128;
+constexpr uint32_t COL_X = 0, COL_Y = 96, COL_Z = 128;
+constexpr uint32_t LANE16 = 16u << 16;
 
 // shared memory map (bytes)
-constexpr uint32_t IN = 0;     // token tile: tensors w r k a b v, [32][128 B] each, 16-B chunks rotated by row
+constexpr uint32_t IN = 0;         // token tile: tensors w r k a b v, [32][128 B], 16-B chunks rotated by row
 constexpr uint32_t IN_W = 0, IN_R = 4096, IN_K = 8192, IN_A = 12288, IN_B = 16384, IN_V = 20480;
 constexpr uint32_t GA_HI = 24576, GA_LO = 32768;     // [64][64]: a' rows 0..31, r' rows 32..63
-constexpr uint32_t GBK_HI = 40960, GBK_LO = 49152;   // [64][64]: b- rows 0..31, k- rows 32..63
-constexpr uint32_t VB = 57344;                       // [32][64] exact bf16 v
-constexpr uint32_t LRB_HI = 61440, LRB_LO = 63488, LRK_HI = 65536, LRK_LO = 67584;   // [32][32]
+constexpr uint32_t BB_HI = 40960, BB_LO = 53248;     // [64][96]: rows s = [b-_s | L_rb[:, s]], rows 32+s = [k-_s | L_rk[:, s]]
+constexpr uint32_t VB = 65536;                       // [32][64] exact bf16 v
 constexpr uint32_t S_HI = 69632, S_LO = 77824;       // [64][64]
-constexpr uint32_t SCR = 86016;                      // 24 KB with three successive lives:
-constexpr uint32_t LABT = SCR, LAKT = SCR + 4096;    //  P1..P1b: fp32 [32][32] L_ab^T, L_ak^T
-constexpr uint32_t WT_HI = SCR + 8192, WT_LO = SCR + 12288, UT_HI = SCR + 16384, UT_LO = SCR + 20480;  // [64][32]
-constexpr uint32_t M_HI = SCR, M_LO = SCR + 8192, Q_HI = SCR + 16384, Q_LO = SCR + 20480;  //  P3..R4
-constexpr uint32_t YSM = SCR;                        //  P4: fp32 [32][64] y tile
+constexpr uint32_t R = 86016;                        // 24 KB, shared by short-lived buffers:
+constexpr uint32_t T_HI = R, T_LO = R + 2048, P_HI = R + 4096, P_LO = R + 6144;    //   P1..R2: [32][32]
+constexpr uint32_t ID32 = R;                         //   P2..R3: [32][32] bf16 identity
+constexpr uint32_t LABT = R + 8192;                  //   P1: fp32 L_ab^T [32][32]
+constexpr uint32_t LAK = R + 12288;                  //   P1: fp32 L_ak [32][33] (padded)
+constexpr uint32_t TSM = R + 16512;                  //   P1: fp32 T [32][32]
+constexpr uint32_t ZSM = R + 20608;                  //   P1: fp32 [16][16]
+constexpr uint32_t WT_HI = R + 8192, UT_HI = R + 12288, WT_LO = R + 16384, UT_LO = R + 20480;  // P2..R3: [64][32]
+constexpr uint32_t MQ_HI = R, MQ_LO = R + 12288;     //   P3..R4: [64][96] = [M | Q^T]
+constexpr uint32_t YSM = R;                          //   P4: fp32 [32][64]
 constexpr uint32_t GAML = 110592;                    // fp32 [64]: G per channel
-constexpr uint32_t MBAR = 110848;                    // u64
-constexpr uint32_t TMEM_SLOT = 110856;               // u32
-constexpr uint32_t FLAG = 110860;                    // u32 abort flag
-constexpr uint32_t SMEM_BYTES = 110864;
+constexpr uint32_t BAR = 110848;                     // 8 mbarriers: ready R1..R4, done R1..R4
+constexpr uint32_t TMEM_SLOT = 110912;
+constexpr uint32_t FLAG = 110916;
+constexpr uint32_t SMEM_BYTES = 110928;
 
-constexpr long long kWaitCycles = 2000000000LL;      // ~1 s: far above any legitimate MMA round
+constexpr long long kWaitCycles = 2000000000LL;      // ~1 s: far above any legitimate wait
 constexpr float kMinDecay = 1e-30f;                  // per-chunk decay floor (prod of 32 w)
 
 __device__ __forceinline__ uint32_t in_off(int t, int ch) { return (uint32_t)(t * 128 + (((ch + t) & 7) << 4)); }
@@ -90,6 +103,8 @@ __device__ __forceinline__ float bf_at(const unsigned char *p) {
     return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
 
+__device__ __forceinline__ void csync() { umma::named_sync(1, NC); }   // compute warps only
+
 }  // namespace chunk
 
 template <typename OutT>
@@ -103,19 +118,19 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
     extern __shared__ __align__(1024) unsigned char sm[];
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3, hc = warp >> 2;             // TMEM lane quadrant, column half
     const int h = blockIdx.x, bb = blockIdx.y;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
     const int nchunks = (T + L - 1) / L;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
-    const uint32_t mbar = sbase + MBAR;
+    auto ready_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };        // k = 0..3 (R1..R4)
+    auto done_bar = [&](int k) { return sbase + BAR + 32u + 8u * (uint32_t)k; };
 
-    auto issue_tile = [&](int c) {
+    auto issue_tile = [&](int c) {        // compute threads only
         const __nv_bfloat16 *src[6] = {w, r, k, a, b, v};
         const int t0 = c * L;
-        for (int x = tid; x < 6 * L * 8; x += NT) {
+        for (int x = tid; x < 6 * L * 8; x += NC) {
             const int ten = x >> 8, t = (x >> 3) & 31, ch = x & 7;
             if (t0 + t < T)
                 cp_async16(sm + IN + ten * 4096 + in_off(t, ch), src[ten] + base + (size_t)(t0 + t) * tok_stride + ch * 8);
@@ -125,12 +140,15 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
 
     // ---- set-up -------------------------------------------------------------------------
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        for (int kk = 0; kk < 4; ++kk) {
+            mbar_init(ready_bar(kk), NC);
+            mbar_init(done_bar(kk), 1);
+        }
         *abort_flag = 0;
     }
-    if (warp == 0) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
-    issue_tile(0);
-    {
+    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
+    if (tid < NC) {
+        issue_tile(0);
         const int i = tid >> 2, c0 = (tid & 3) * 16;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -146,310 +164,398 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
             store8_split(sm + S_HI, sm + S_LO, cm_off(i, c0 + 8 * g, 64), x);
         }
     }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + TMEM_SLOT);
-    const uint32_t quad = (uint32_t)(32 * q4) << 16;
-    uint32_t phase = 0;
 
-    auto round_wait = [&]() -> bool {
-        const bool ok = mbar_wait(mbar, phase, kWaitCycles);
-        phase ^= 1u;
-        if (!ok) *abort_flag = 1;
-        __syncthreads();
-        fence_after_sync();
-        return *abort_flag == 0;
-    };
-    auto issue_begin = [&]() {
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-    };
-
-    // ---- phases -------------------------------------------------------------------------
-    auto P0 = [&](int Lv) {                       // decayed operands of one chunk
-        const int g = warp, t = lane;             // channels 8g..8g+7, token t
-        const bool valid = t < Lv;
-        const uint32_t off = in_off(t, g);
-        float wv[8], rv[8], kv[8], av[8], bv[8];
-        bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_W + off), wv);
-        bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_R + off), rv);
-        bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_K + off), kv);
-        bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_A + off), av);
-        bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_B + off), bv);
-        const uint4 vraw = valid ? *reinterpret_cast<const uint4 *>(sm + IN_V + off) : make_uint4(0, 0, 0, 0);
-        float inc[8], nxt[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (!valid) { wv[e] = 1.f; rv[e] = 0.f; kv[e] = 0.f; av[e] = 0.f; bv[e] = 0.f; }
-            inc[e] = wv[e];
+    if (warp == 8) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            const uint32_t id_gram = idesc_bf16(64, 64, 0, 0), id_r2 = idesc_bf16(64, 32, 1, 0);
+            const uint32_t id_km96 = idesc_bf16(64, 96, 0, 1), id_mm96 = idesc_bf16(64, 96, 1, 1);
+            const OpD ga = opd_k(sbase + GA_HI, sbase + GA_LO, 64);
+            const OpD bbk = opd_k(sbase + BB_HI, sbase + BB_LO, 96);           // [b-; k-] rows, K = cols 0..63
+            const OpD at = opd_mn(sbase + GA_HI, sbase + GA_LO, 64);        // A'^T (rows 0..31 of GA)
+            const OpD vt = opd_mn(sbase + VB, 0, 64);                          // V^T, exact
+            const OpD tt = opd_k(sbase + T_HI, sbase + T_LO, L);
+            const OpD pp = opd_k(sbase + P_HI, sbase + P_LO, L);
+            const OpD wt = opd_k(sbase + WT_HI, sbase + WT_LO, L);
+            const OpD ut = opd_k(sbase + UT_HI, sbase + UT_LO, L);
+            const OpD bl = opd_mn(sbase + BB_HI, sbase + BB_LO, 96);          // [B- | L_rb^T]
+            const OpD kl = opd_mn(sbase + BB_HI + 6144, sbase + BB_LO + 6144, 96);   // [K- | L_rk^T]
+            const OpD ss = opd_k(sbase + S_HI, sbase + S_LO, 64);
+            const OpD mq = opd_mn(sbase + MQ_HI, sbase + MQ_LO, 96);          // [M | Q^T]
+            const OpD rt = opd_mn(sbase + GA_HI + 4096, sbase + GA_LO + 4096, 64);   // R'^T (rows 32..63 of GA)
+            const OpD id = opd_k(sbase + ID32, 0, L);                          // identity, exact
+            const uint32_t id_r = idesc_bf16(64, 32, 1, 0);
+            for (int c = 0; c < nchunks; ++c) {
+                const uint32_t par = (uint32_t)c & 1u;
+                // R1: Gram
+                if (!mbar_spin(ready_bar(0), par, kWaitCycles)) { *abort_flag = 1; break; }
+                fence_after_sync();
+                gemm_split_d(tmem + COL_X, ga, bbk, id_gram, 4, false);
+                commit(done_bar(0));
+                // R2: W'^T = A'^T T^T (lane 0), U~^T = V^T P^T (lane 16)
+                if (!mbar_spin(ready_bar(1), par, kWaitCycles)) { *abort_flag = 1; break; }
+                fence_after_sync();
+                gemm_split_d(tmem + COL_Y, at, tt, id_r2, 2, false);
+                gemm_split_d(tmem + COL_Y + LANE16, vt, pp, id_r2, 2, false);
+                commit(done_bar(1));
+                // R3: [M'' | Q''^T] = W'^T [B- | L_rb^T];  [E | Y_loc^T] = U~^T [B- | L_rb^T] + V^T [K- | L_rk^T]
+                if (!mbar_spin(ready_bar(2), par, kWaitCycles)) { *abort_flag = 1; break; }
+                fence_after_sync();
+                gemm_split_d(tmem + COL_X, wt, bl, id_km96, 2, false);
+                gemm_split_d(tmem + COL_X + 64, rt, id, id_r, 2, true);       // Q''^T += R'^T
+                gemm_split_d(tmem + COL_Z, ut, bl, id_km96, 2, false);
+                gemm_split_d(tmem + COL_Z, vt, kl, id_mm96, 2, true);
+                commit(done_bar(2));
+                // R4: [S_out | Y^T] += S [M | Q^T]
+                if (!mbar_spin(ready_bar(3), par, kWaitCycles)) { *abort_flag = 1; break; }
+                fence_after_sync();
+                gemm_split_d(tmem + COL_Z, ss, mq, id_km96, 4, true);
+                commit(done_bar(3));
+            }
         }
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1)
+        __syncwarp();
+    } else {
+        // ================= compute warps =================
+        const int q4 = warp & 3, hc = warp >> 2;     // TMEM lane quadrant, column half
+        const uint32_t quad = (uint32_t)(32 * q4) << 16;
+        const int sub = lane & 15;                   // row within the quadrant's 16
+        const bool upper = lane >= 16;               // lanes reading the lane-16 accumulator
+
+        auto done_wait = [&](int kk, int c) -> bool {   // one lane polls, the others park at the barrier
+            if (tid == 0 && !mbar_spin(done_bar(kk), (uint32_t)c & 1u, kWaitCycles)) *abort_flag = 1;
+            csync();
+            fence_after_sync();
+            return *abort_flag == 0;
+        };
+        auto ready_arrive = [&](int kk) {
+            fence_smem_to_async();
+            fence_before_sync();
+            mbar_arrive(ready_bar(kk));
+        };
+
+        auto P0 = [&](int Lv) {                   // decayed operands of one chunk
+            const int g = warp, t = lane;         // channels 8g..8g+7, token t
+            const bool valid = t < Lv;
+            const uint32_t off = in_off(t, g);
+            float wv[8], rv[8], kv[8], av[8], bv[8];
+            bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_W + off), wv);
+            bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_R + off), rv);
+            bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_K + off), kv);
+            bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_A + off), av);
+            bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_B + off), bv);
+            const uint4 vraw = valid ? *reinterpret_cast<const uint4 *>(sm + IN_V + off) : make_uint4(0, 0, 0, 0);
+            float inc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float up = __shfl_down_sync(0xffffffffu, inc[e], o);
-                if (lane + o < 32) inc[e] *= up;
+                if (!valid) { wv[e] = 1.f; rv[e] = 0.f; kv[e] = 0.f; av[e] = 0.f; bv[e] = 0.f; }
+                inc[e] = wv[e];
             }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float n1 = __shfl_down_sync(0xffffffffu, inc[e], 1);
-            nxt[e] = lane == 31 ? 1.f : n1;
-            const float G = __shfl_sync(0xffffffffu, inc[e], 0);
-            if (lane == 0) {
-                reinterpret_cast<float *>(sm + GAML)[8 * g + e] = G;
-                if (G < kMinDecay) raise_status(WKV7_ERR_RANGE);
-            }
-        }
-        float xa[8], xr[8], xb[8], xk[8];
+            for (int o = 1; o < 32; o <<= 1)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            xa[e] = __fdividef(av[e], inc[e]);
-            xr[e] = __fdividef(rv[e], nxt[e]);
-            xb[e] = bv[e] * nxt[e];
-            xk[e] = kv[e] * nxt[e];
-        }
-        store8_split(sm + GA_HI, sm + GA_LO, cm_off(t, 8 * g, 64), xa);
-        store8_split(sm + GA_HI, sm + GA_LO, cm_off(L + t, 8 * g, 64), xr);
-        store8_split(sm + GBK_HI, sm + GBK_LO, cm_off(t, 8 * g, 64), xb);
-        store8_split(sm + GBK_HI, sm + GBK_LO, cm_off(L + t, 8 * g, 64), xk);
-        *reinterpret_cast<uint4 *>(sm + VB + cm_off(t, 8 * g, 64)) = vraw;
-    };
-
-    auto issue_R1 = [&]() {
-        fence_after_sync();
-        gemm_split_d(tmem + COL_X, opd_k(sbase + GA_HI, sbase + GA_LO, 64), opd_k(sbase + GBK_HI, sbase + GBK_LO, 64),
-                     idesc_bf16(64, 64, 0, 0), 4, false);
-        commit(mbar);
-    };
-
-    auto P1 = [&]() {                             // mask the Gram into L_ab^T, L_ak^T (fp32), L_rb, L_rk (split)
-        uint32_t r0[16], r1[16];
-        tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc, r0);
-        tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc + 16, r1);
-        tmem_wait();
-        if (lane < 16) {
-            const int rho = 16 * q4 + lane;
-            float g[32];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                g[e] = __uint_as_float(r0[e]);
-                g[16 + e] = __uint_as_float(r1[e]);
-            }
-            if (rho < L) {
-                const int t = rho;
-                float *dst = reinterpret_cast<float *>(sm + (hc == 0 ? LABT : LAKT));
-#pragma unroll
-                for (int s = 0; s < L; ++s) dst[s * L + t] = s < t ? g[s] : 0.f;
-            } else {
-                const int t = rho - L;
-                unsigned char *hi = sm + (hc == 0 ? LRB_HI : LRK_HI);
-                unsigned char *lo = sm + (hc == 0 ? LRB_LO : LRK_LO);
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = (8 * qq + e <= t) ? g[8 * qq + e] : 0.f;
-                    store8_split(hi, lo, cm_off(t, 8 * qq, L), x);
+                for (int e = 0; e < 8; ++e) {
+                    const float up = __shfl_down_sync(0xffffffffu, inc[e], o);
+                    if (lane + o < 32) inc[e] *= up;
                 }
+            float xa[8], xr[8], xb[8], xk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float n1 = __shfl_down_sync(0xffffffffu, inc[e], 1);
+                const float nxt = lane == 31 ? 1.f : n1;
+                const float G = __shfl_sync(0xffffffffu, inc[e], 0);
+                if (lane == 0) {
+                    reinterpret_cast<float *>(sm + GAML)[8 * g + e] = G;
+                    if (G < kMinDecay) raise_status(WKV7_ERR_RANGE);
+                }
+                xa[e] = __fdividef(av[e], inc[e]);
+                xr[e] = __fdividef(rv[e], nxt);
+                xb[e] = bv[e] * nxt;
+                xk[e] = kv[e] * nxt;
             }
-        }
-    };
+            store8_split(sm + GA_HI, sm + GA_LO, cm_off(t, 8 * g, 64), xa);
+            store8_split(sm + GA_HI, sm + GA_LO, cm_off(L + t, 8 * g, 64), xr);
+            store8_split(sm + BB_HI, sm + BB_LO, cm_off(t, 8 * g, 96), xb);
+            store8_split(sm + BB_HI, sm + BB_LO, cm_off(L + t, 8 * g, 96), xk);
+            *reinterpret_cast<uint4 *>(sm + VB + cm_off(t, 8 * g, 64)) = vraw;
+        };
 
-    auto P1b = [&]() {                            // forward substitution for W' and U~ (column per thread)
-        if (tid < 2 * kN) {
-            const bool is_w = tid < kN;
-            const int col = tid & 63;
-            const float *labt = reinterpret_cast<const float *>(sm + LABT);
-            const float *lakt = reinterpret_cast<const float *>(sm + LAKT);
-            float acc[L];
+        auto P1 = [&]() {                         // Gram -> L's; T = (I - L_ab)^{-1}; P = T L_ak
+            {
+                uint32_t r0[16], r1[16];
+                tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc, r0);
+                tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc + 16, r1);
+                tmem_wait();
+                if (!upper) {
+                    const int rho = 16 * q4 + sub;
+                    float g[32];
 #pragma unroll
-            for (int t = 0; t < L; ++t) {
-                const uint32_t o = cm_off(t, col, 64);
-                acc[t] = is_w ? bf_at(sm + GA_HI + o) + bf_at(sm + GA_LO + o) : 0.f;
-            }
+                    for (int e = 0; e < 16; ++e) {
+                        g[e] = __uint_as_float(r0[e]);
+                        g[16 + e] = __uint_as_float(r1[e]);
+                    }
+                    if (rho < L) {                // a' row t
+                        const int t = rho;
+                        if (hc == 0) {            // L_ab^T[s][t] (fp32)
+                            float *dst = reinterpret_cast<float *>(sm + LABT);
 #pragma unroll
-            for (int m = 0; m < L; ++m) {
-                const float x = acc[m];
-                const float vm = is_w ? 0.f : bf_at(sm + VB + cm_off(m, col, 64));
+                            for (int s = 0; s < L; ++s) dst[s * L + t] = s < t ? g[s] : 0.f;
+                        } else {                  // L_ak[t][s] (fp32, rows padded to 33)
+                            float *dst = reinterpret_cast<float *>(sm + LAK) + t * 33;
 #pragma unroll
-                for (int c4 = (m + 1) / 4; c4 < L / 4; ++c4) {
-                    const float4 lab = *reinterpret_cast<const float4 *>(labt + m * L + 4 * c4);
-                    const float4 lak = *reinterpret_cast<const float4 *>(lakt + m * L + 4 * c4);
-                    const float la[4] = {lab.x, lab.y, lab.z, lab.w};
-                    const float lk[4] = {lak.x, lak.y, lak.z, lak.w};
+                            for (int s = 0; s < L; ++s) dst[s] = s < t ? g[s] : 0.f;
+                        }
+                    } else {                      // r' row t: L_rb / L_rk into columns 64 + t of the b- / k- rows
+                        const int t = rho - L;
+                        const int row0 = hc == 0 ? 0 : L;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int t = 4 * c4 + e;
-                        if (t > m) acc[t] = fmaf(la[e], x, fmaf(lk[e], vm, acc[t]));
+                        for (int s = 0; s < L; ++s) {
+                            const float x = s <= t ? g[s] : 0.f;
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+                            const uint32_t o = cm_off(row0 + s, 64 + t, 96);
+                            *reinterpret_cast<__nv_bfloat16 *>(sm + BB_HI + o) = hi;
+                            *reinterpret_cast<__nv_bfloat16 *>(sm + BB_LO + o) = lo;
+                        }
                     }
                 }
             }
-            unsigned char *hi = sm + (is_w ? WT_HI : UT_HI);
-            unsigned char *lo = sm + (is_w ? WT_LO : UT_LO);
+            fence_before_sync();
+            csync();
+            const float *labt = reinterpret_cast<const float *>(sm + LABT);
+            float *tsm = reinterpret_cast<float *>(sm + TSM);
+            if (warp == 0) {                      // diagonal 16x16 blocks of T, one column per lane
+                const int blk = lane >> 4, s = 16 * blk + sub;
+                float acc[16];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) store8_split(hi, lo, cm_off(col, 8 * qq, L), acc + 8 * qq);
-        }
-    };
-
-    auto issue_R3 = [&]() {
-        fence_after_sync();
-        const OpD wt = opd_k(sbase + WT_HI, sbase + WT_LO, L);
-        const OpD ut = opd_k(sbase + UT_HI, sbase + UT_LO, L);
-        const OpD vt = opd_mn(sbase + VB, 0, 64);
-        const OpD bbar = opd_mn(sbase + GBK_HI, sbase + GBK_LO, 64);
-        const OpD kbar = opd_mn(sbase + GBK_HI + 4096, sbase + GBK_LO + 4096, 64);
-        const OpD lrb = opd_k(sbase + LRB_HI, sbase + LRB_LO, L);
-        const OpD lrk = opd_k(sbase + LRK_HI, sbase + LRK_LO, L);
-        gemm_split_d(tmem + COL_X, wt, bbar, idesc_bf16(64, 64, 0, 1), 2, false);
-        gemm_split_d(tmem + COL_X + 64, wt, lrb, idesc_bf16(64, 32, 0, 0), 2, false);
-        gemm_split_d(tmem + COL_Z, ut, bbar, idesc_bf16(64, 64, 0, 1), 2, false);
-        gemm_split_d(tmem + COL_Z, vt, kbar, idesc_bf16(64, 64, 1, 1), 2, true);
-        gemm_split_d(tmem + COL_Z + 64, ut, lrb, idesc_bf16(64, 32, 0, 0), 2, false);
-        gemm_split_d(tmem + COL_Z + 64, vt, lrk, idesc_bf16(64, 32, 1, 0), 2, true);
-        commit(mbar);
-    };
-
-    auto P3 = [&]() {                             // M = G (I + M''), Q^T = G (R'^T + Q''^T)
-        uint32_t r0[16], r1[16], r2[16];
-        tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc, r0);
-        tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc + 16, r1);
-        tmem_ld16_nowait(tmem + quad + COL_X + 64 + 16 * hc, r2);
-        tmem_wait();
-        if (lane < 16) {
-            const int j = 16 * q4 + lane;
-            const float G = reinterpret_cast<const float *>(sm + GAML)[j];
-            float m[32];
+                for (int e = 0; e < 16; ++e) acc[e] = (e == sub) ? 1.f : 0.f;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                m[e] = G * (__uint_as_float(r0[e]) + (32 * hc + e == j ? 1.f : 0.f));
-                m[16 + e] = G * (__uint_as_float(r1[e]) + (32 * hc + 16 + e == j ? 1.f : 0.f));
+                for (int m = 0; m < 15; ++m) {
+                    const float x = acc[m];
+                    const float *row = labt + (16 * blk + m) * L + 16 * blk;
+#pragma unroll
+                    for (int e4 = (m + 1) / 4; e4 < 4; ++e4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(row + 4 * e4);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            if (4 * e4 + c4 > m) acc[4 * e4 + c4] = fmaf(lv[c4], x, acc[4 * e4 + c4]);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) tsm[(16 * blk + e) * L + s] = acc[e];
+            } else if (warp == 1) {               // upper-right block of T is zero
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int x = lane + 32 * e;
+                    tsm[(x >> 4) * L + 16 + (x & 15)] = 0.f;
+                }
             }
+            csync();
+            float *zsm = reinterpret_cast<float *>(sm + ZSM);
+            {                                     // Z = L21 T11 (16 x 16), one entry per thread
+                const int t = tid >> 4, s = tid & 15;
+                float acc = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) store8_split(sm + M_HI, sm + M_LO, cm_off(j, 32 * hc + 8 * qq, 64), m + 8 * qq);
-            float qv[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const uint32_t o = cm_off(L + 16 * hc + e, j, 64);
-                qv[e] = G * (__uint_as_float(r2[e]) + bf_at(sm + GA_HI + o) + bf_at(sm + GA_LO + o));
+                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * L + 16 + t], tsm[m * L + s], acc);
+                zsm[t * 16 + s] = acc;
             }
+            csync();
+            {                                     // T21 = T22 Z
+                const int t = tid >> 4, s = tid & 15;
+                float acc = 0.f;
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) store8_split(sm + Q_HI, sm + Q_LO, cm_off(j, 16 * hc + 8 * qq, L), qv + 8 * qq);
-        }
-    };
+                for (int m = 0; m < 16; ++m) acc = fmaf(tsm[(16 + t) * L + 16 + m], zsm[m * 16 + s], acc);
+                tsm[(16 + t) * L + s] = acc;
+            }
+            csync();
+            {                                     // P = T L_ak and T, 4 rows per warp, one column per lane
+                const float *lak = reinterpret_cast<const float *>(sm + LAK);
+                const int s = lane;
+                float pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < L / 4; ++m4) {
+                    float4 tr[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) tr[i] = *reinterpret_cast<const float4 *>(tsm + (4 * warp + i) * L + 4 * m4);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float lv = lak[(4 * m4 + c4) * 33 + s];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float tv = c4 == 0 ? tr[i].x : c4 == 1 ? tr[i].y : c4 == 2 ? tr[i].z : tr[i].w;
+                            pv[i] = fmaf(tv, lv, pv[i]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = 4 * warp + i;
+                    const uint32_t o = cm_off(t, s, L);
+                    const float tv = tsm[t * L + s];
+                    __nv_bfloat16 hi = __float2bfloat16_rn(pv[i]);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_HI + o) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_LO + o) = __float2bfloat16_rn(pv[i] - __bfloat162float(hi));
+                    hi = __float2bfloat16_rn(tv);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + T_HI + o) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + T_LO + o) = __float2bfloat16_rn(tv - __bfloat162float(hi));
+                }
+            }
+        };
 
-    auto issue_R4 = [&]() {
-        fence_after_sync();
-        const OpD s = opd_k(sbase + S_HI, sbase + S_LO, 64);
-        gemm_split_d(tmem + COL_Z, s, opd_mn(sbase + M_HI, sbase + M_LO, 64), idesc_bf16(64, 64, 0, 1), 4, true);
-        gemm_split_d(tmem + COL_Z + 64, s, opd_mn(sbase + Q_HI, sbase + Q_LO, L), idesc_bf16(64, 32, 0, 1), 4, true);
-        commit(mbar);
-    };
+        auto P2 = [&]() {                         // stage W'^T (lanes 0-15) and U~^T (lanes 16-31)
+            uint32_t r0[16];
+            tmem_ld16_nowait(tmem + quad + COL_Y + 16 * hc, r0);
+            tmem_wait();
+            float x[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r0[e]);
+            const int row = 16 * q4 + sub;
+            unsigned char *hi = sm + (upper ? UT_HI : WT_HI);
+            unsigned char *lo = sm + (upper ? UT_LO : WT_LO);
+            store8_split(hi, lo, cm_off(row, 16 * hc, L), x);
+            store8_split(hi, lo, cm_off(row, 16 * hc + 8, L), x + 8);
+            {   // identity operand for R3 (the T/P space is free once R2 is done)
+                const int rr = tid >> 3, cc = 4 * (tid & 7);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + ID32 + cm_off(rr, cc + e, L)) =
+                        __float2bfloat16_rn(rr == cc + e ? 1.f : 0.f);
+            }
+        };
 
-    auto P4 = [&](int c, int Lv) {                // y, next S operand, final state
-        uint32_t r0[16], r1[16], r2[16];
-        tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc, r0);
-        tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc + 16, r1);
-        tmem_ld16_nowait(tmem + quad + COL_Z + 64 + 16 * hc, r2);
-        tmem_wait();
-        if (lane < 16) {
-            const int i = 16 * q4 + lane;
-            float sv[32];
+        auto P3 = [&]() {                         // [M | Q^T] rows j: M = G (I + M''), Q^T = G (R'^T + Q''^T) (R'^T added by R3)
+            uint32_t r0[16], r1[16], r2[16];
+            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc, r0);
+            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc + 16, r1);
+            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc + 32, r2);
+            tmem_wait();
+            if (!upper) {
+                const int j = 16 * q4 + sub;
+                const float G = reinterpret_cast<const float *>(sm + GAML)[j];
+                float x[48];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                sv[e] = __uint_as_float(r0[e]);
-                sv[16 + e] = __uint_as_float(r1[e]);
+                for (int e = 0; e < 16; ++e) {
+                    x[e] = __uint_as_float(r0[e]);
+                    x[16 + e] = __uint_as_float(r1[e]);
+                    x[32 + e] = __uint_as_float(r2[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 48; ++e) {
+                    const int col = 48 * hc + e;
+                    x[e] = G * (x[e] + (col == j ? 1.f : 0.f));   // Q columns (col >= 64) never match j
+                }
+#pragma unroll
+                for (int qq = 0; qq < 6; ++qq)
+                    store8_split(sm + MQ_HI, sm + MQ_LO, cm_off(j, 48 * hc + 8 * qq, 96), x + 8 * qq);
             }
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) store8_split(sm + S_HI, sm + S_LO, cm_off(i, 32 * hc + 8 * qq, 64), sv + 8 * qq);
-            if (c == nchunks - 1 && sT) {
-#pragma unroll
-                for (int qq = 0; qq < 8; ++qq)
-                    store4(sT + st_base + (size_t)i * kN + 32 * hc + 4 * qq,
-                           make_float4(sv[4 * qq], sv[4 * qq + 1], sv[4 * qq + 2], sv[4 * qq + 3]));
-            }
-            float *ysm = reinterpret_cast<float *>(sm + YSM);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ysm[(16 * hc + e) * kN + i] = __uint_as_float(r2[e]);
-        }
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-        {   // coalesced y rows: thread -> (token, 8 channels)
-            const int t = tid >> 3, c8 = tid & 7;
-            if (t < Lv) {
-                const float *ysm = reinterpret_cast<const float *>(sm + YSM) + t * kN + 8 * c8;
-                OutT *dst = y + base + (size_t)(c * L + t) * tok_stride + 8 * c8;
-                store4(dst, *reinterpret_cast<const float4 *>(ysm));
-                store4(dst + 4, *reinterpret_cast<const float4 *>(ysm + 4));
-            }
-        }
-        __syncthreads();
-    };
+        };
 
-    // ---- software-pipelined chunk loop ----------------------------------------------------
-    auto run = [&]() {
+        auto P4 = [&](int c, int Lv) {            // rows i of [S_out | Y^T]: next S operand, y, final state
+            uint32_t r0[16], r1[16], r2[16];
+            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc, r0);
+            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc + 16, r1);
+            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc + 32, r2);
+            tmem_wait();
+            if (!upper) {
+                const int i = 16 * q4 + sub;
+                float x[48];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    x[e] = __uint_as_float(r0[e]);
+                    x[16 + e] = __uint_as_float(r1[e]);
+                    x[32 + e] = __uint_as_float(r2[e]);
+                }
+                const bool last = c == nchunks - 1 && sT != nullptr;
+                if (hc == 0) {                    // S columns 0..47
+#pragma unroll
+                    for (int qq = 0; qq < 6; ++qq) store8_split(sm + S_HI, sm + S_LO, cm_off(i, 8 * qq, 64), x + 8 * qq);
+                    if (last) {
+#pragma unroll
+                        for (int qq = 0; qq < 12; ++qq)
+                            store4(sT + st_base + (size_t)i * kN + 4 * qq,
+                                   make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
+                    }
+                } else {                          // S columns 48..63, then y^T columns 0..31
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq)
+                        store8_split(sm + S_HI, sm + S_LO, cm_off(i, 48 + 8 * qq, 64), x + 8 * qq);
+                    if (last) {
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq)
+                            store4(sT + st_base + (size_t)i * kN + 48 + 4 * qq,
+                                   make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
+                    }
+                    float *ysm = reinterpret_cast<float *>(sm + YSM);
+#pragma unroll
+                    for (int e = 0; e < L; ++e) ysm[e * kN + i] = x[16 + e];
+                }
+            }
+            fence_before_sync();
+            csync();
+            {   // coalesced y rows: thread -> (token, 8 channels)
+                const int t = tid >> 3, c8 = tid & 7;
+                if (t < Lv) {
+                    const float *ysm = reinterpret_cast<const float *>(sm + YSM) + t * kN + 8 * c8;
+                    OutT *dst = y + base + (size_t)(c * L + t) * tok_stride + 8 * c8;
+                    store4(dst, *reinterpret_cast<const float4 *>(ysm));
+                    store4(dst + 4, *reinterpret_cast<const float4 *>(ysm + 4));
+                }
+            }
+            csync();
+        };
+
+        // ---- compute schedule ----
         cp_async_wait<0>();
-        __syncthreads();
+        csync();
         P0(min(L, T));
-        __syncthreads();
+        csync();
+        ready_arrive(0);                                   // R1(0)
         if (nchunks > 1) issue_tile(1);
-        issue_begin();
-        if (tid == 0) issue_R1();
-        if (!round_wait()) return;
-        P1();
-        __syncthreads();
-        P1b();
-        issue_begin();
-        if (tid == 0) issue_R3();
-        if (!round_wait()) return;
-        P3();
-        issue_begin();
-        if (tid == 0) issue_R4();
         for (int c = 0; c < nchunks; ++c) {
-            const bool has_next = c + 1 < nchunks;
-            if (has_next) {
+            if (!done_wait(0, c)) break;                   // Gram(c)
+            P1();
+            ready_arrive(1);                               // R2(c)
+            if (!done_wait(1, c)) break;
+            P2();
+            ready_arrive(2);                               // R3(c)
+            if (!done_wait(2, c)) break;
+            P3();
+            ready_arrive(3);                               // R4(c)
+            if (c + 1 < nchunks) {                         // next chunk's operands under R4(c)
                 cp_async_wait<0>();
-                __syncthreads();
+                csync();
                 P0(min(L, T - (c + 1) * L));
-                __syncthreads();
+                csync();
+                ready_arrive(0);                           // R1(c+1), under P4(c)
                 if (c + 2 < nchunks) issue_tile(c + 2);
             }
-            if (!round_wait()) return;                       // R4(c)
-            if (has_next) {
-                issue_begin();
-                if (tid == 0) issue_R1();                    // R1(c+1), overlapped with P4(c)
-            }
+            if (!done_wait(3, c)) break;                   // R4(c)
             P4(c, min(L, T - c * L));
-            if (has_next) {
-                if (!round_wait()) return;                   // R1(c+1)
-                P1();
-                __syncthreads();
-                P1b();
-                issue_begin();
-                if (tid == 0) issue_R3();
-                if (!round_wait()) return;
-                P3();
-                issue_begin();
-                if (tid == 0) issue_R4();                    // R4(c+1), overlapped with P0(c+2)
-            }
         }
-    };
-    run();
+        cp_async_wait<0>();
+    }
 
     // ---- tear-down ----------------------------------------------------------------------
-    cp_async_wait<0>();
     __syncthreads();
     if (*abort_flag) {
-        // a tensor-core round did not complete in time: report it, give the
-        // in-flight work one more bounded wait, then release TMEM
+        // a wait gave up: report it, give in-flight tensor-core work one more
+        // bounded wait, then release TMEM
         if (tid == 0) raise_status(WKV7_ERR_TIMEOUT);
-        mbar_wait(mbar, phase ^ 1u, kWaitCycles);
+        if (tid == NC) {
+            for (int kk = 0; kk < 4; ++kk) {
+                mbar_wait(done_bar(kk), 0u, kWaitCycles / 8);
+                mbar_wait(done_bar(kk), 1u, kWaitCycles / 8);
+            }
+        }
         __syncthreads();
     }
     fence_after_sync();
-    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,

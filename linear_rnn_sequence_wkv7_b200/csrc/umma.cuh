@@ -170,6 +170,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, long 
     }
 }
 
+// Same, polling with the non-suspending test_wait (prompt wake-up; for a single
+// thread that has nothing else to do).
+__device__ __forceinline__ bool mbar_spin(uint32_t saddr, uint32_t parity, long long limit_cycles) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(saddr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > limit_cycles) return false;
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(saddr) : "memory");
+}
+
+// named barrier among `count` threads (a multiple of 32)
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---- bf16 hi/lo split --------------------------------------------------------
 
 // x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi): 16 significant bits.
