@@ -13,9 +13,9 @@
 //   k-_t = k_t p_{t+1}                                (p_32 = 1)
 // so that a'_t . b-_s = sum_j a_t b_s prod_{s<m<t} w_m, the decayed
 // interaction of token t's removal read with token s's write, etc.
-//   Gram  = [a'; r'] [b-; k-]^T                        (64 x 64)
-//   L_ab, L_ak = strictly lower parts of the a' rows; L_rb, L_rk = lower
-//                parts of the r' rows (diagonal included)
+//   Gram^T = [b-; k-] [a'; r']^T                       (64 x 64; row s of b-
+//            holds column s of L_ab and L_rb, row s of k- those of L_ak, L_rk)
+//   L_ab, L_ak = strictly lower parts (t > s); L_rb, L_rk = lower parts (t >= s)
 //   T = (I - L_ab)^{-1} (blocked: two 16x16 diagonal inverses by forward
 //       substitution, then T21 = T22 L21 T11),  P = T L_ak      (CUDA cores, fp32)
 //   W'^T = A'^T T^T,  U~^T = V^T P^T                   (u_t = S G w'_t + u~_t)
@@ -72,10 +72,11 @@ constexpr uint32_t S_HI = 69632, S_LO = 77824;       // [64][64]
 constexpr uint32_t R = 86016;                        // 24 KB, shared by short-lived buffers:
 constexpr uint32_t T_HI = R, T_LO = R + 2048, P_HI = R + 4096, P_LO = R + 6144;    //   P1..R2: [32][32]
 constexpr uint32_t ID32 = R;                         //   P2..R3: [32][32] bf16 identity
-constexpr uint32_t LABT = R + 8192;                  //   P1: fp32 L_ab^T [32][32]
-constexpr uint32_t LAK = R + 12288;                  //   P1: fp32 L_ak [32][33] (padded)
-constexpr uint32_t TSM = R + 16512;                  //   P1: fp32 T [32][32]
-constexpr uint32_t ZSM = R + 20608;                  //   P1: fp32 [16][16]
+constexpr int LDT = 36;                              //   row pitch of L_ab^T (floats; bank spread)
+constexpr uint32_t LABT = R + 8192;                  //   P1: fp32 L_ab^T [32][36]
+constexpr uint32_t LAK = R + 12800;                  //   P1: fp32 L_ak [32][33] (padded)
+constexpr uint32_t TSM = R + 17024;                  //   P1: fp32 T [32][32]
+constexpr uint32_t ZSM = R + 21120;                  //   P1: fp32 [16][16]
 constexpr uint32_t WT_HI = R + 8192, UT_HI = R + 12288, WT_LO = R + 16384, UT_LO = R + 20480;  // P2..R3: [64][32]
 constexpr uint32_t MQ_HI = R, MQ_LO = R + 12288;     //   P3..R4: [64][96] = [M | Q^T]
 constexpr uint32_t YSM = R;                          //   P4: fp32 [32][64]
@@ -195,7 +196,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
                 // R1: Gram
                 if (!mbar_spin(ready_bar(0), par, kWaitCycles)) { *abort_flag = 1; break; }
                 fence_after_sync();
-                gemm_split_d(tmem + COL_X, ga, bbk, id_gram, 4, false);
+                gemm_split_d(tmem + COL_X, bbk, ga, id_gram, 4, false);       // Gram^T
                 commit(done_bar(0));
                 // R2: W'^T = A'^T T^T (lane 0), U~^T = V^T P^T (lane 16)
                 if (!mbar_spin(ready_bar(1), par, kWaitCycles)) { *abort_flag = 1; break; }
@@ -298,28 +299,29 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
                         g[e] = __uint_as_float(r0[e]);
                         g[16 + e] = __uint_as_float(r1[e]);
                     }
-                    if (rho < L) {                // a' row t
-                        const int t = rho;
-                        if (hc == 0) {            // L_ab^T[s][t] (fp32)
-                            float *dst = reinterpret_cast<float *>(sm + LABT);
+                    const int s = rho & 31;
+                    if (rho < L && hc == 0) {         // column s of L_ab -> row s of L_ab^T
+                        float *dst = reinterpret_cast<float *>(sm + LABT) + s * LDT;
 #pragma unroll
-                            for (int s = 0; s < L; ++s) dst[s * L + t] = s < t ? g[s] : 0.f;
-                        } else {                  // L_ak[t][s] (fp32, rows padded to 33)
-                            float *dst = reinterpret_cast<float *>(sm + LAK) + t * 33;
-#pragma unroll
-                            for (int s = 0; s < L; ++s) dst[s] = s < t ? g[s] : 0.f;
+                        for (int t4 = 0; t4 < 8; ++t4) {
+                            float4 o;
+                            o.x = 4 * t4 + 0 > s ? g[4 * t4 + 0] : 0.f;
+                            o.y = 4 * t4 + 1 > s ? g[4 * t4 + 1] : 0.f;
+                            o.z = 4 * t4 + 2 > s ? g[4 * t4 + 2] : 0.f;
+                            o.w = 4 * t4 + 3 > s ? g[4 * t4 + 3] : 0.f;
+                            *reinterpret_cast<float4 *>(dst + 4 * t4) = o;
                         }
-                    } else {                      // r' row t: L_rb / L_rk into columns 64 + t of the b- / k- rows
-                        const int t = rho - L;
-                        const int row0 = hc == 0 ? 0 : L;
+                    } else if (rho >= L && hc == 0) { // column s of L_ak (rows padded to 33)
+                        float *dst = reinterpret_cast<float *>(sm + LAK) + s;
 #pragma unroll
-                        for (int s = 0; s < L; ++s) {
-                            const float x = s <= t ? g[s] : 0.f;
-                            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-                            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-                            const uint32_t o = cm_off(row0 + s, 64 + t, 96);
-                            *reinterpret_cast<__nv_bfloat16 *>(sm + BB_HI + o) = hi;
-                            *reinterpret_cast<__nv_bfloat16 *>(sm + BB_LO + o) = lo;
+                        for (int t = 0; t < L; ++t) dst[t * 33] = t > s ? g[t] : 0.f;
+                    } else {                          // column s of L_rb / L_rk -> columns 64.. of row s / 32+s
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] = (8 * qq + e >= s) ? g[8 * qq + e] : 0.f;
+                            store8_split(sm + BB_HI, sm + BB_LO, cm_off(rho, 64 + 8 * qq, 96), x);
                         }
                     }
                 }
@@ -336,7 +338,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
 #pragma unroll
                 for (int m = 0; m < 15; ++m) {
                     const float x = acc[m];
-                    const float *row = labt + (16 * blk + m) * L + 16 * blk;
+                    const float *row = labt + (16 * blk + m) * LDT + 16 * blk;
 #pragma unroll
                     for (int e4 = (m + 1) / 4; e4 < 4; ++e4) {
                         const float4 l4 = *reinterpret_cast<const float4 *>(row + 4 * e4);
@@ -361,7 +363,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
                 const int t = tid >> 4, s = tid & 15;
                 float acc = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * L + 16 + t], tsm[m * L + s], acc);
+                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * LDT + 16 + t], tsm[m * L + s], acc);
                 zsm[t * 16 + s] = acc;
             }
             csync();
