@@ -171,6 +171,16 @@ WKV7_API wkv7_status wkv7_backward_noalloc(int B, int T, int H, int N, wkv7_dtyp
                                            void *dv, void *da, void *db, float *ds0, cudaStream_t stream);
 
 /*
+ * Bound, in SM clock cycles, on every device-side wait of kernels launched
+ * afterwards from this process (the chunked forward's tensor-core round
+ * handshakes).  A wait that runs out sets WKV7_ERR_TIMEOUT in the device status
+ * word, lets already-committed tensor-core work finish, frees its tensor
+ * memory and returns; the context stays usable.  0 restores the default
+ * (about one second).  Meant for testing that path.
+ */
+WKV7_API void wkv7_set_wait_limit(long long cycles);
+
+/*
  * Synchronizes `stream`, then returns and clears the sticky device-side status
  * word of the current device (WKV7_OK, WKV7_ERR_TIMEOUT or WKV7_ERR_RANGE), or
  * WKV7_ERR_CUDA if the synchronization itself failed.

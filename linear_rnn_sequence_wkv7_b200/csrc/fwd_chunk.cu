@@ -83,10 +83,11 @@ constexpr uint32_t YSM = R;                          //   P4: fp32 [32][64]
 constexpr uint32_t GAML = 110592;                    // fp32 [64]: G per channel
 constexpr uint32_t BAR = 110848;                     // 8 mbarriers: ready R1..R4, done R1..R4
 constexpr uint32_t TMEM_SLOT = 110912;
-constexpr uint32_t FLAG = 110916;
+constexpr uint32_t FLAG = 110916;                    // set by whichever role gives up first
+constexpr uint32_t CFLAG = 110920;                   // compute warps' copy, written by thread 0 only
 constexpr uint32_t SMEM_BYTES = 110928;
 
-constexpr long long kWaitCycles = 2000000000LL;      // ~1 s: far above any legitimate wait
+constexpr long long kDrainCycles = 200000000LL;      // ~0.1 s to let committed tensor-core work finish
 constexpr float kMinDecay = 1e-30f;                  // per-chunk decay floor (prod of 32 w)
 
 __device__ __forceinline__ uint32_t in_off(int t, int ch) { return (uint32_t)(t * 128 + (((ch + t) & 7) << 4)); }
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(chunk::NT, 2)
 fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_bfloat16 *__restrict__ w,
                  const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
                  const __nv_bfloat16 *__restrict__ a, const __nv_bfloat16 *__restrict__ b,
-                 const float *s0, OutT *__restrict__ y, float *sT) {
+                 const float *s0, OutT *__restrict__ y, float *sT, long long wait_limit) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -125,6 +126,9 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
     const int nchunks = (T + L - 1) / L;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
+    volatile uint32_t *compute_flag = reinterpret_cast<volatile uint32_t *>(sm + CFLAG);
+    int last_k = -1;                                 // issuer: last committed round and its parity
+    uint32_t last_par = 0;
     auto ready_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };        // k = 0..3 (R1..R4)
     auto done_bar = [&](int k) { return sbase + BAR + 32u + 8u * (uint32_t)k; };
 
@@ -146,6 +150,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
             mbar_init(done_bar(kk), 1);
         }
         *abort_flag = 0;
+        *compute_flag = 0;
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if (tid < NC) {
@@ -194,29 +199,37 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
             for (int c = 0; c < nchunks; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
                 // R1: Gram
-                if (!mbar_spin(ready_bar(0), par, kWaitCycles)) { *abort_flag = 1; break; }
+                if (!mbar_spin(ready_bar(0), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_X, bbk, ga, id_gram, 4, false);       // Gram^T
                 commit(done_bar(0));
+                last_k = 0;
+                last_par = par;
                 // R2: W'^T = A'^T T^T (lane 0), U~^T = V^T P^T (lane 16)
-                if (!mbar_spin(ready_bar(1), par, kWaitCycles)) { *abort_flag = 1; break; }
+                if (!mbar_spin(ready_bar(1), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_Y, at, tt, id_r2, 2, false);
                 gemm_split_d(tmem + COL_Y + LANE16, vt, pp, id_r2, 2, false);
                 commit(done_bar(1));
+                last_k = 1;
+                last_par = par;
                 // R3: [M'' | Q''^T] = W'^T [B- | L_rb^T];  [E | Y_loc^T] = U~^T [B- | L_rb^T] + V^T [K- | L_rk^T]
-                if (!mbar_spin(ready_bar(2), par, kWaitCycles)) { *abort_flag = 1; break; }
+                if (!mbar_spin(ready_bar(2), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_X, wt, bl, id_km96, 2, false);
                 gemm_split_d(tmem + COL_X + 64, rt, id, id_r, 2, true);       // Q''^T += R'^T
                 gemm_split_d(tmem + COL_Z, ut, bl, id_km96, 2, false);
                 gemm_split_d(tmem + COL_Z, vt, kl, id_mm96, 2, true);
                 commit(done_bar(2));
+                last_k = 2;
+                last_par = par;
                 // R4: [S_out | Y^T] += S [M | Q^T]
-                if (!mbar_spin(ready_bar(3), par, kWaitCycles)) { *abort_flag = 1; break; }
+                if (!mbar_spin(ready_bar(3), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_Z, ss, mq, id_km96, 4, true);
                 commit(done_bar(3));
+                last_k = 3;
+                last_par = par;
             }
         }
         __syncwarp();
@@ -227,11 +240,19 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
         const int sub = lane & 15;                   // row within the quadrant's 16
         const bool upper = lane >= 16;               // lanes reading the lane-16 accumulator
 
-        auto done_wait = [&](int kk, int c) -> bool {   // one lane polls, the others park at the barrier
-            if (tid == 0 && !mbar_spin(done_bar(kk), (uint32_t)c & 1u, kWaitCycles)) *abort_flag = 1;
+        // One lane polls, the others park at the barrier.  Only thread 0 reads
+        // the shared abort flag (the issuer may set it at any time) and it
+        // publishes its decision before the barrier, so all 256 threads take
+        // the same branch afterwards.
+        auto done_wait = [&](int kk, int c) -> bool {
+            if (tid == 0) {
+                const bool ok = mbar_spin(done_bar(kk), (uint32_t)c & 1u, wait_limit);
+                if (!ok) *abort_flag = 1;
+                *compute_flag = (!ok || *abort_flag) ? 1u : 0u;
+            }
             csync();
             fence_after_sync();
-            return *abort_flag == 0;
+            return *compute_flag == 0;
         };
         auto ready_arrive = [&](int kk) {
             fence_smem_to_async();
@@ -545,15 +566,11 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
     // ---- tear-down ----------------------------------------------------------------------
     __syncthreads();
     if (*abort_flag) {
-        // a wait gave up: report it, give in-flight tensor-core work one more
-        // bounded wait, then release TMEM
+        // a wait gave up: report it, let the tensor-core work already
+        // committed finish (rounds complete in order, so the last commit
+        // covers all), then release TMEM
         if (tid == 0) raise_status(WKV7_ERR_TIMEOUT);
-        if (tid == NC) {
-            for (int kk = 0; kk < 4; ++kk) {
-                mbar_wait(done_bar(kk), 0u, kWaitCycles / 8);
-                mbar_wait(done_bar(kk), 1u, kWaitCycles / 8);
-            }
-        }
+        if (tid == NC && last_k >= 0) mbar_wait(done_bar(last_k), last_par, kDrainCycles);
         __syncthreads();
     }
     fence_after_sync();
@@ -562,7 +579,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      cudaStream_t st) {
+                      long long wait_limit, cudaStream_t st) {
     dim3 grid(H, B);
     const size_t smem = chunk::SMEM_BYTES;
 #define WKV7_CHUNK_LAUNCH(O)                                                                                 \
@@ -572,7 +589,8 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
         if (e != cudaSuccess) return e;                                                                      \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w,        \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,              \
-                                            (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, (O *)y, sT); \
+                                            (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, (O *)y, sT, \
+                                            wait_limit);                                                    \
     } while (0)
     if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
     else WKV7_CHUNK_LAUNCH(__nv_bfloat16);

@@ -4,6 +4,8 @@
 // wkv7_get_device_status).
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace wkv7 {
@@ -24,11 +26,13 @@ cudaError_t bwd_seq(int B, int T, int H, int CK, wkv7_dtype in_dt, wkv7_dtype g_
 size_t bwd_hist_bytes(int B, int H, int CK);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      cudaStream_t st);
+                      long long wait_limit, cudaStream_t st);
 
 namespace {
 
 constexpr int kBwdChunk = 16;        // backward checkpoint interval (tokens)
+constexpr long long kDefaultWaitCycles = 2000000000LL;   // ~1 s of SM clock
+std::atomic<long long> g_wait_limit{0};                  // 0 = default
 constexpr size_t kWsAlign = 256;
 
 bool dtype_ok(wkv7_dtype d) { return d == WKV7_F32 || d == WKV7_BF16; }
@@ -115,7 +119,9 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
         if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
     if (resolve_algo(T, in_dt, algo) == WKV7_ALGO_CHUNK) {
         if (in_dt != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
-        return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+        const long long lim = g_wait_limit.load();
+        return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT,
+                                   lim > 0 ? lim : kDefaultWaitCycles, stream));
     }
     return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
 }
@@ -166,6 +172,8 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     return from_cuda(bwd_seq(B, T, H, kBwdChunk, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, hist, dr, dw,
                              dk, dv, da, db, ds0, stream));
 }
+
+void wkv7_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }
 
 wkv7_status wkv7_get_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV7_ERR_CUDA;

@@ -24,7 +24,7 @@ ALGOS = {"auto": ALGO_AUTO, "seq": ALGO_SEQ, "chunk": ALGO_CHUNK}
 EXPORTED_SYMBOLS = (
     "wkv7_abi_version", "wkv7_status_string", "wkv7_forward_workspace_size", "wkv7_forward",
     "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
-    "wkv7_forward_resolve_algo", "wkv7_backward_noalloc",
+    "wkv7_forward_resolve_algo", "wkv7_backward_noalloc", "wkv7_set_wait_limit",
 )
 
 _lib = None
@@ -62,6 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward_noalloc.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
+    lib.wkv7_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.wkv7_set_wait_limit.restype = None
     lib.wkv7_get_device_status.argtypes = [vp]
     lib.wkv7_get_device_status.restype = i
     _lib = lib
@@ -198,6 +200,11 @@ def backward_noalloc(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.flo
                                    *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)), _stream(stream))
     _check("wkv7_backward_noalloc", st)
     return tuple(out)
+
+
+def set_wait_limit(cycles: int = 0) -> None:
+    """Bound (SM cycles) on device-side waits of later launches; 0 = default (~1 s)."""
+    load_library().wkv7_set_wait_limit(int(cycles))
 
 
 def device_status(stream=None) -> int:

@@ -203,3 +203,24 @@ def test_long_context_chunked_matches_oracle_and_sequential(cuda_device):
     for h in range(cfg["H"]):
         assert_close(to_f64(yc[:, :, h]), to_f64(ys[:, :, h]), TAU_BF16, f"y head {h} vs seq")
     assert_close(to_f64(sc), to_f64(ss), TAU_BF16, "sT vs seq")
+
+
+def test_chunked_wait_timeout_reports_and_recovers(cuda_device):
+    """A device-side wait that runs out (limit forced to 1 cycle) makes the
+    chunked kernel give up cleanly: WKV7_ERR_TIMEOUT in the status word, no
+    fault, and the next launch with the default limit is correct."""
+    B, T, H, N = 1, 96, 2, 64
+    d = inputs.gen_sequence(B, T, H, N, seed=77, dtype="bf16", s0_std=0.1)
+    assert wkv7.device_status() == wkv7.OK
+    wkv7.set_wait_limit(1)
+    try:
+        run_forward(d, y_dtype=torch.float32, algo="chunk")
+        status = wkv7.device_status()
+    finally:
+        wkv7.set_wait_limit(0)
+    assert status == wkv7.ERR_TIMEOUT
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert wkv7.device_status() == wkv7.OK
+    yr, sr = oracle_forward(d)
+    assert_close(to_f64(y), yr, TAU_BF16, "y after recovery")
+    assert_close(to_f64(sT), sr, TAU_BF16, "sT after recovery")
