@@ -8,7 +8,9 @@ B=8, T=4096, H=32, N=64 bf16 workload (fp32 state, s0 ~ N(0, 0.1)); one step
 is one ``wkv7_forward`` call over the whole batch with inputs resident in
 HBM.  The same run also measures, under ``parts``, the training backward on
 the same shape (dy ~ N(0,1) bf16, dsT = 0) and the decode step (B=256, H=40,
-1000 consecutive steps replayed from a CUDA graph).
+1000 consecutive steps replayed from a CUDA graph) and the long-context
+chunked forward (B=1, T=65536, H=32, decays near 1), where 32 heads cannot
+fill the GPU and the sequence runs as parallel segments.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
 (weak scaling, no collective on the data path); times are the max over
@@ -43,6 +45,7 @@ N = 64
 FWD = inputs.WORKLOADS["prefill_b8_t4096_h32_bf16"]
 BWD = inputs.WORKLOADS["train_bwd_b8_t4096_h32"]
 DEC = inputs.WORKLOADS["decode_b256_h40_x1000"]
+LONG = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
@@ -55,7 +58,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--algo", default="auto", choices=["auto", "seq", "chunk"])
-    p.add_argument("--parts", default="fwd,bwd,decode")
+    p.add_argument("--parts", default="fwd,bwd,decode,long")
     p.add_argument("--decode-steps", type=int, default=DEC["steps"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -375,6 +378,42 @@ def bench_decode(args, dist, peaks, device, steps_in):
                        "l2": "state 168 MB > 126 MB L2; inputs pre-staged, 7.9 GB"}}
 
 
+def bench_long(args, dist, peaks, device):
+    import torch
+    from linear_rnn_sequence_wkv7_b200 import wkv7
+    cfg = LONG
+    B, T, H = cfg["B"], cfg["T"], cfg["H"]
+    d = inputs.gen_sequence(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16",
+                            x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
+    dev = [to_dev(d[n], device) for n in inputs.INPUT_NAMES]
+    s0 = to_dev(d["s0"], device)
+    y = torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device)
+    sT = torch.empty(B, H, N, N, dtype=torch.float32, device=device)
+    ws_n = wkv7.forward_workspace_size(B, T, H, N, torch.bfloat16, "chunk")
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        wkv7.forward(*dev, s0=s0, y=y, sT=sT, algo="chunk", workspace=ws, stream=stream)
+
+    steps = max(3, min(args.steps // 20, 10))
+    secs = timed(step, steps, 2, dist, stream)
+    per = secs / steps
+    nbytes = fwd_bytes(B, T, H)
+    ach = nbytes / per / 1e9
+    # launches per call: one pass, or summary pass + entry-state scan + output pass
+    per_call = 3 if ws_n else 1
+    return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
+            "ms_per_step": per * 1e3, "steps": steps, "launches": per_call * steps,
+            "workspace_bytes": ws_n,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "per_unit": "896 B per head-token + 32 KiB state per head",
+                         "units_per_launch": B * T * H},
+            "config": {"workload": "long_b1_t65536_h32", "B": B, "T": T, "H": H, "N": N, "algo": "chunk",
+                       "w": "exp(-0.6065 sigmoid(x)), x ~ N(-2, 1)",
+                       "l2": "no flush: each step reads 1.6 GB of inputs (> 126 MB L2)"}}
+
+
 def cpu_baseline(d, budget_s=10.0):
     """The oracle as it stands on this host's cores: forward over the first
     heads of the prefill workload (all T tokens), repeated up to budget_s."""
@@ -425,6 +464,8 @@ def run_ours(args):
     if gen_thread is not None:
         gen_thread.join()
         out_parts["decode"] = bench_decode(args, dist, peaks, device, steps_in)
+    if "long" in parts:
+        out_parts["long_context"] = bench_long(args, dist, peaks, device)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(fwd["sample"])

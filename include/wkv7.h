@@ -79,14 +79,19 @@ WKV7_API int wkv7_abi_version(void);
 WKV7_API const char *wkv7_status_string(wkv7_status status);
 
 /*
- * Bytes of scratch wkv7_forward needs for these arguments (0 when the chosen
- * algorithm needs none).  Same arguments as wkv7_forward's sizes and choice.
+ * Bytes of scratch wkv7_forward can use for these arguments on the current
+ * device (0 when the chosen algorithm needs none).  The chunked form uses it to
+ * split long sequences into segments that run in parallel when B*H heads are
+ * too few to fill the GPU (a per-segment summary S -> S M + E, a scan of the
+ * entry states, then every segment from its entry state).  Without it (NULL
+ * or too small) the chunked form runs in one pass; the results are the same.
  */
 WKV7_API size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype,
                                    wkv7_algo algo, int chunk_len);
 
 /*
- * Forward over a whole sequence.
+ * Forward over a whole sequence (when the chunked form splits the sequence into
+ * segments, the state crosses segment boundaries through the summary scan).
  *   r, w, k, v, a, b : [B, T, H, N] of in_dtype (fp32 or bf16), read only
  *   s0               : [B, H, N, N] fp32 initial state, or NULL for zeros
  *   y                : [B, T, H, N] of y_dtype, written

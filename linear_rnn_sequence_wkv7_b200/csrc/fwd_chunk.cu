@@ -49,6 +49,8 @@
 //   Z: cols [128, 224)  [E | Y_loc^T], then += S [M | Q^T] = [S_out | Y^T]
 // L_rb and L_rk are stored next to b- and k- (one [64][96] operand), and M
 // next to Q^T, so R3 and R4 run as N=96 products.
+#include <algorithm>
+
 #include "umma.cuh"
 
 namespace wkv7 {
@@ -111,19 +113,30 @@ __device__ __forceinline__ void csync() { umma::named_sync(1, NC); }   // comput
 
 template <typename OutT>
 __global__ void __launch_bounds__(chunk::NT, 2)
-fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_bfloat16 *__restrict__ w,
-                 const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-                 const __nv_bfloat16 *__restrict__ a, const __nv_bfloat16 *__restrict__ b,
-                 const float *s0, OutT *__restrict__ y, float *sT, long long wait_limit) {
+fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *__restrict__ r,
+                 const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
+                 const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
+                 const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
+                 float *sT, long long sT_zstride, int st_only_z, long long wait_limit) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, bb = blockIdx.y;
+    const int h = blockIdx.x, bb = blockIdx.y, z = blockIdx.z;
+    // blockIdx.z selects a segment of the sequence; z >= nseg marks a
+    // "transition" run of segment z - nseg (state starts at I, v taken as 0),
+    // whose final state is the segment's linear map S -> S M_seg.
+    const int seg = z % nseg;
+    const bool transition = z >= nseg;
+    const int t_begin = seg * t_seg;
+    const int T = min(t_seg, T_total - t_begin);     // tokens of this segment
     const size_t tok_stride = (size_t)H * kN;
-    const size_t base = ((size_t)bb * T * H + h) * kN;
+    const size_t base = (((size_t)bb * T_total + t_begin) * H + h) * kN;
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
+    const float *s0p = s0 ? s0 + (size_t)z * s0_zstride + st_base : nullptr;
+    float *sTp = (sT && (st_only_z < 0 || st_only_z == z)) ? sT + (st_only_z < 0 ? (size_t)z * sT_zstride : 0) + st_base
+                                                            : nullptr;
     const int nchunks = (T + L - 1) / L;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
     volatile uint32_t *compute_flag = reinterpret_cast<volatile uint32_t *>(sm + CFLAG);
@@ -159,9 +172,12 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             float x[8];
-            if (s0) {
-                const float4 u0 = load4(s0 + st_base + (size_t)i * kN + c0 + 8 * g);
-                const float4 u1 = load4(s0 + st_base + (size_t)i * kN + c0 + 8 * g + 4);
+            if (transition) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = (c0 + 8 * g + e == i) ? 1.f : 0.f;
+            } else if (s0p) {
+                const float4 u0 = load4(s0p + (size_t)i * kN + c0 + 8 * g);
+                const float4 u1 = load4(s0p + (size_t)i * kN + c0 + 8 * g + 4);
                 x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w; x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
             } else {
 #pragma unroll
@@ -270,7 +286,8 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_K + off), kv);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_A + off), av);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_B + off), bv);
-            const uint4 vraw = valid ? *reinterpret_cast<const uint4 *>(sm + IN_V + off) : make_uint4(0, 0, 0, 0);
+            const uint4 vraw = (valid && !transition) ? *reinterpret_cast<const uint4 *>(sm + IN_V + off)
+                                                      : make_uint4(0, 0, 0, 0);
             float inc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -493,14 +510,14 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
                     x[16 + e] = __uint_as_float(r1[e]);
                     x[32 + e] = __uint_as_float(r2[e]);
                 }
-                const bool last = c == nchunks - 1 && sT != nullptr;
+                const bool last = c == nchunks - 1 && sTp != nullptr;
                 if (hc == 0) {                    // S columns 0..47
 #pragma unroll
                     for (int qq = 0; qq < 6; ++qq) store8_split(sm + S_HI, sm + S_LO, cm_off(i, 8 * qq, 64), x + 8 * qq);
                     if (last) {
 #pragma unroll
                         for (int qq = 0; qq < 12; ++qq)
-                            store4(sT + st_base + (size_t)i * kN + 4 * qq,
+                            store4(sTp + (size_t)i * kN + 4 * qq,
                                    make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
                     }
                 } else {                          // S columns 48..63, then y^T columns 0..31
@@ -510,7 +527,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
                     if (last) {
 #pragma unroll
                         for (int qq = 0; qq < 4; ++qq)
-                            store4(sT + st_base + (size_t)i * kN + 48 + 4 * qq,
+                            store4(sTp + (size_t)i * kN + 48 + 4 * qq,
                                    make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
                     }
                     float *ysm = reinterpret_cast<float *>(sm + YSM);
@@ -520,7 +537,7 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
             }
             fence_before_sync();
             csync();
-            {   // coalesced y rows: thread -> (token, 8 channels)
+            if (y) {   // coalesced y rows: thread -> (token, 8 channels)
                 const int t = tid >> 3, c8 = tid & 7;
                 if (t < Lv) {
                     const float *ysm = reinterpret_cast<const float *>(sm + YSM) + t * kN + 8 * c8;
@@ -577,25 +594,134 @@ fwd_chunk_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __nv_b
     if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
-                      const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      long long wait_limit, cudaStream_t st) {
-    dim3 grid(H, B);
+// One launch of the chunked kernel over nz = gridDim.z segment runs.
+static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz, wkv7_dtype y_dt, const void *r,
+                                const void *w, const void *k, const void *v, const void *a, const void *b,
+                                const float *s0, long long s0_zstride, void *y, float *sT, long long sT_zstride,
+                                int st_only_z, long long wait_limit, cudaStream_t st) {
+    dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES;
-#define WKV7_CHUNK_LAUNCH(O)                                                                                 \
-    do {                                                                                                     \
-        auto kern = fwd_chunk_kernel<O>;                                                                     \
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);  \
-        if (e != cudaSuccess) return e;                                                                      \
-        kern<<<grid, chunk::NT, smem, st>>>(T, H, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w,        \
-                                            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,              \
-                                            (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, (O *)y, sT, \
-                                            wait_limit);                                                    \
+#define WKV7_CHUNK_LAUNCH(O)                                                                                  \
+    do {                                                                                                      \
+        auto kern = fwd_chunk_kernel<O>;                                                                      \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
+        if (e != cudaSuccess) return e;                                                                       \
+        kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
+                                            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
+                                            (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
+                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit);                   \
     } while (0)
     if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
     else WKV7_CHUNK_LAUNCH(__nv_bfloat16);
 #undef WKV7_CHUNK_LAUNCH
     return cudaGetLastError();
+}
+
+// Segments combine: per head, S_in(0) = s0 (or 0) and
+// S_in(k+1) = S_in(k) M_k + E_k, where E_k / M_k are the final states of the
+// segment's plain and transition runs.  Writes S_in(k) for k < nseg.  One CTA
+// (256 threads) per head, fp32 on the CUDA cores; thread -> row i, 16 columns.
+__global__ void __launch_bounds__(256)
+seg_combine_kernel(int BH, int nseg, const float *__restrict__ s0, const float *__restrict__ em,
+                   float *__restrict__ sin_out) {
+    __shared__ __align__(16) float Ssm[kN * kN];
+    __shared__ __align__(16) float Msm[kN * kN];
+    const int head = blockIdx.x, tid = threadIdx.x;
+    const int i = tid >> 2, j0 = (tid & 3) * 16;
+    const size_t hoff = (size_t)head * kN * kN;
+    const size_t zstride = (size_t)BH * kN * kN;
+    float cur[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) cur[e] = s0 ? s0[hoff + (size_t)i * kN + j0 + e] : 0.f;
+    for (int kk = 0; kk < nseg; ++kk) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            sin_out[(size_t)kk * zstride + hoff + (size_t)i * kN + j0 + e] = cur[e];
+            Ssm[i * kN + j0 + e] = cur[e];
+        }
+        if (kk + 1 == nseg) break;
+        const float *E = em + (size_t)kk * zstride + hoff;
+        const float *M = em + (size_t)(nseg - 1 + kk) * zstride + hoff;
+        for (int x = tid; x < kN * kN; x += 256) Msm[x] = M[x];
+        __syncthreads();
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = E[(size_t)i * kN + j0 + e];
+        for (int m = 0; m < kN; ++m) {
+            const float sm_ = Ssm[i * kN + m];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = fmaf(sm_, Msm[m * kN + j0 + e], acc[e]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cur[e] = acc[e];
+    }
+}
+
+// Relative time of one launch of n chunk CTAs that each run the same number
+// of chunks, on sms SMs holding two CTAs each: a CTA alone on its SM runs at
+// speed 1, two co-resident CTAs each take 1.46 times as long (measured on the
+// prefill and long-context shapes); CTAs beyond the resident ones run in later
+// rounds.
+static double launch_rounds(long long n, int sms) {
+    double t = 0.0;
+    while (n > 0) {
+        t += n > sms ? 1.46 : 1.0;
+        n -= 2LL * sms;
+    }
+    return t;
+}
+
+// Number of sequence segments for a chunked forward over B*H heads.  The
+// segmented form runs 2 (nseg - 1) summary runs and nseg output runs of T/nseg
+// tokens each, i.e. about 3x the work of one pass, so it only pays when B*H
+// CTAs leave most of the GPU idle.  Picks the nseg (segments of at least 4
+// chunks) with the lowest estimated time, if that is below 95% of one pass;
+// among near-ties (within 3%) the fewest segments, which need the least scratch.
+int chunk_segments(int B, int T, int H, int sm_count) {
+    static_assert(2 * chunk::SMEM_BYTES <= 228 * 1024, "two chunk CTAs per SM");
+    const long long heads = (long long)B * H;
+    const long long chunks = (T + chunk::L - 1) / chunk::L;
+    if (sm_count <= 0 || heads <= 0) return 1;
+    const long long max_n = std::min<long long>(64, chunks / 4);
+    auto cost = [&](long long n) {
+        return (launch_rounds(2 * (n - 1) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
+    };
+    double best = 0.95 * launch_rounds(heads, sm_count);
+    for (long long n = 2; n <= max_n; ++n) best = std::min(best, cost(n));
+    for (long long n = 2; n <= max_n; ++n)
+        if (cost(n) <= 1.03 * best) return (int)n;
+    return 1;
+}
+
+size_t chunk_workspace_bytes(int B, int T, int H, int nseg) {
+    if (nseg <= 1) return 0;
+    // E_k, M_k for segments 0..nseg-2 and S_in(k) for k < nseg
+    return (size_t)(2 * (nseg - 1) + nseg) * B * H * kN * kN * sizeof(float);
+}
+
+cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
+                      const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st) {
+    if (nseg <= 1)
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
+    const int chunks = (T + chunk::L - 1) / chunk::L;
+    const int t_seg = ((chunks + nseg - 1) / nseg) * chunk::L;
+    nseg = (T + t_seg - 1) / t_seg;
+    const long long zst = (long long)B * H * kN * kN;
+    float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
+    float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg][B][H][64][64]
+    // pass 1: E_k (s0 = 0) and M_k (s0 = I, v = 0) for segments 0..nseg-2, no y
+    cudaError_t e = launch_chunk(B, T, H, t_seg, nseg - 1, 2 * (nseg - 1), y_dt, r, w, k, v, a, b, nullptr, 0,
+                                 nullptr, em, zst, -1, wait_limit, st);
+    if (e != cudaSuccess) return e;
+    // pass 2: entry state of every segment
+    seg_combine_kernel<<<B * H, 256, 0, st>>>(B * H, nseg, s0, em, sin);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // pass 3: every segment from its true entry state; the last one writes sT
+    return launch_chunk(B, T, H, t_seg, nseg, nseg, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 1,
+                        wait_limit, st);
 }
 
 }  // namespace wkv7

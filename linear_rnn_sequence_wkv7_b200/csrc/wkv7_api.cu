@@ -4,6 +4,7 @@
 // wkv7_get_device_status).
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -26,7 +27,9 @@ cudaError_t bwd_seq(int B, int T, int H, int CK, wkv7_dtype in_dt, wkv7_dtype g_
 size_t bwd_hist_bytes(int B, int H, int CK);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      long long wait_limit, cudaStream_t st);
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st);
+int chunk_segments(int B, int T, int H, int sm_count);
+size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
 
 namespace {
 
@@ -69,6 +72,13 @@ wkv7_algo resolve_algo(int T, wkv7_dtype in_dt, wkv7_algo algo) {
     return (in_dt == WKV7_BF16 && T >= 64) ? WKV7_ALGO_CHUNK : WKV7_ALGO_SEQ;
 }
 
+int current_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 size_t bwd_ckpt_bytes(int B, int T, int H) {
     const size_t nck = ((size_t)T + kBwdChunk - 1) / kBwdChunk;
     return (size_t)B * H * nck * kN * kN * sizeof(float);
@@ -98,15 +108,18 @@ const char *wkv7_status_string(wkv7_status s) {
 
 size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_algo algo,
                                    int chunk_len) {
-    (void)B; (void)T; (void)H; (void)N; (void)in_dtype; (void)algo; (void)chunk_len;
-    return 0;
+    (void)chunk_len;
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN || !dtype_ok(in_dtype)) return 0;
+    if (resolve_algo(T, in_dtype, algo) != WKV7_ALGO_CHUNK || in_dtype != WKV7_BF16) return 0;
+    const int sms = current_sm_count();
+    if (sms <= 0) return 0;
+    return chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms));
 }
 
 wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
                          const void *w, const void *k, const void *v, const void *a, const void *b,
                          const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    (void)workspace; (void)workspace_bytes;
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
@@ -120,7 +133,17 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
     if (resolve_algo(T, in_dt, algo) == WKV7_ALGO_CHUNK) {
         if (in_dt != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
         const long long lim = g_wait_limit.load();
-        return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT,
+        // sequence segments run in parallel when there are too few heads to
+        // fill the GPU and the caller provided the workspace they need
+        int nseg = 1;
+        const int sms = current_sm_count();
+        if (sms > 0) {
+            const int want = chunk_segments(B, T, H, sms);
+            if (want > 1 && workspace != nullptr && aligned16(workspace) &&
+                workspace_bytes >= chunk_workspace_bytes(B, T, H, want))
+                nseg = want;
+        }
+        return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
                                    lim > 0 ? lim : kDefaultWaitCycles, stream));
     }
     return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));

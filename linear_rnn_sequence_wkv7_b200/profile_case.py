@@ -48,7 +48,9 @@ def main():
     if a.op == "fwd":
         y = torch.empty(a.B, T, a.H, N, dtype=torch.bfloat16, device="cuda")
         sT = torch.empty_like(s0)
-        run = lambda: wkv7.forward(*x, s0=s0, y=y, sT=sT, algo=a.algo)
+        nws = wkv7.forward_workspace_size(a.B, T, a.H, N, torch.bfloat16, a.algo)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
+        run = lambda: wkv7.forward(*x, s0=s0, y=y, sT=sT, algo=a.algo, workspace=ws)
     elif a.op == "step":
         xs = [t[:, 0].contiguous() for t in x]
         y = torch.empty(a.B, a.H, N, dtype=torch.bfloat16, device="cuda")

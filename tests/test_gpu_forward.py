@@ -224,3 +224,54 @@ def test_chunked_wait_timeout_reports_and_recovers(cuda_device):
     yr, sr = oracle_forward(d)
     assert_close(to_f64(y), yr, TAU_BF16, "y after recovery")
     assert_close(to_f64(sT), sr, TAU_BF16, "sT after recovery")
+
+
+# --- chunked form over sequence segments (few heads, long sequences) -----------------
+
+@pytest.mark.parametrize("T", [512, 700, 2000, 4097])
+def test_chunked_segments_match_oracle_and_single_pass(cuda_device, T):
+    """With B*H heads too few to fill the GPU the chunked form splits the
+    sequence into segments (summary pass, entry-state scan, output pass).
+    Ragged last segment, nonzero s0: y and sT vs the oracle, and vs the same
+    call run in one pass (workspace too small)."""
+    B, H, N = 1, 2, 64
+    assert wkv7.forward_workspace_size(B, T, H, N, torch.bfloat16, "chunk") > 0
+    d = inputs.gen_sequence(B, T, H, N, seed=400 + T, dtype="bf16", s0_std=0.1)
+    yr, sr = oracle_forward(d)
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert wkv7.device_status() == wkv7.OK
+    assert_close(to_f64(y), yr, TAU_BF16, "y")
+    assert_close(to_f64(sT), sr, TAU_BF16, "sT")
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    tiny = torch.empty(16, dtype=torch.uint8, device="cuda")
+    y1, s1 = wkv7.forward(*args, s0=to_dev(d["s0"]), y_dtype=torch.float32, algo="chunk", workspace=tiny)
+    torch.cuda.synchronize()
+    assert_close(to_f64(y), to_f64(y1), TAU_BF16, "y segmented vs one pass")
+    assert_close(to_f64(sT), to_f64(s1), TAU_BF16, "sT segmented vs one pass")
+
+
+def test_chunked_segments_zero_state_in_place_and_bf16_out(cuda_device):
+    B, T, H, N = 2, 1500, 1, 64
+    assert wkv7.forward_workspace_size(B, T, H, N, torch.bfloat16, "chunk") > 0
+    d = inputs.gen_sequence(B, T, H, N, seed=451, dtype="bf16", s0_std=0.1)
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    y0 = wkv7.forward(*args, s0=None, y_dtype=torch.bfloat16, algo="chunk", return_state=False)
+    torch.cuda.synchronize()
+    yr0, _ = oracle_forward(dict(d, s0=None))
+    assert_close(to_f64(y0), yr0, TAU_BF16, "y (zero s0, bf16 out)", bf16_out=True)
+    state = to_dev(d["s0"])
+    y1, _ = wkv7.forward(*args, s0=state, sT=state, y_dtype=torch.float32, algo="chunk")
+    torch.cuda.synchronize()
+    yr1, sr1 = oracle_forward(d)
+    assert_close(to_f64(y1), yr1, TAU_BF16, "y")
+    assert_close(to_f64(state), sr1, TAU_BF16, "sT in place")
+    assert wkv7.device_status() == wkv7.OK
+
+
+def test_forward_workspace_size_rules(cuda_device):
+    """Scratch only for the chunked form with too few heads for the GPU."""
+    assert wkv7.forward_workspace_size(8, 4096, 32, 64, torch.bfloat16, "chunk") == 0
+    assert wkv7.forward_workspace_size(1, 65536, 32, 64, torch.bfloat16, "chunk") > 0
+    assert wkv7.forward_workspace_size(1, 65536, 32, 64, torch.bfloat16, "seq") == 0
+    assert wkv7.forward_workspace_size(1, 65536, 32, 64, torch.float32, "auto") == 0
+    assert wkv7.forward_workspace_size(1, 200, 1, 64, torch.bfloat16, "chunk") == 0
