@@ -28,27 +28,35 @@
 // bf16 input such as v) with fp32 accumulation in TMEM.  A single tf32 or bf16
 // pass is not accurate enough for the 2e-3 rms bound on this workload.
 //
-// Mapping: one CTA per (b, h), two CTAs per SM.  Warps 0-7 (256 threads)
-// run the CUDA-core phases; warp 8 issues the tensor-core rounds.  Per chunk:
-// P0 builds the decayed operands from the token tile (suffix products by
-// warp shuffles); R1 Gram; P1 masks it and computes T and P; R2 W'^T, U~^T;
-// P2 stages them; R3 M'', Q''^T, E, Y_loc^T; P3 finishes M and Q; R4
-// accumulates the state product onto [E | Y_loc^T]; P4 writes y and stages
-// S_out as the next chunk's operand.  Each round has a "ready" mbarrier (the
-// 256 compute threads arrive after publishing their shared-memory writes) and
-// a "done" mbarrier (tcgen05.commit); every wait is bounded.  The compute
-// warps build chunk c+1's operands (P0) while R4 of chunk c runs, and R1 of
-// chunk c+1 runs while they finish chunk c (P4).  Token tiles arrive by
-// cp.async one chunk ahead.
+// The state-dependent products run transposed so that they are M=128 tensor-core
+// products with one output row per TMEM lane:
+//   [M''^T; Q''] = [B-^T; L_rb] W',   [E^T; Y_loc] = [B-^T; L_rb] U~ + [K-^T; L_rk] V
+//   [S_out^T; Y] = [M^T; Q] S^T + [E^T; Y_loc]
+// (96 rows used: 64 key rows j, then 32 tokens t).  W'^T and U~^T come from one
+// stacked product [A'^T; V^T] [T^T | P^T] (the off-diagonal blocks are unused).
 //
-// TMEM (256 columns).  An M=64 accumulator occupies lanes 16q..16q+15 of warp
-// quadrant q; a second one at lane offset 16 fills lanes 16q+16..16q+31, so
-// paired results are read by all 32 lanes of a warp:
-//   X: cols [0, 96)     Gram (cols 0-63), then [M'' | Q''^T]
-//   Y: cols [96, 128)   W'^T (lane 0) and U~^T (lane 16)
-//   Z: cols [128, 224)  [E | Y_loc^T], then += S [M | Q^T] = [S_out | Y^T]
-// L_rb and L_rk are stored next to b- and k- (one [64][96] operand), and M
-// next to Q^T, so R3 and R4 run as N=96 products.
+// Mapping: one CTA per (b, h), two CTAs per SM.  Warps 0-7 (256 threads) run
+// the CUDA-core phases; warp 8 issues the tensor-core rounds.  Per chunk:
+//   P0  decayed operands from the token tile (suffix products by shuffles)
+//   R1  Gram^T = [b-; k-] [a'; r']^T                     (M=64, N=64)
+//   P1  masks -> L's; T = (I - L_ab)^-1 and P = T L_ak on the CUDA cores
+//   R2  [A'^T; V^T] [T^T | P^T] -> W'^T, U~^T             (M=128, N=64)
+//   P2  stages [W' | U~] as the next B operand
+//   R3  [M''^T; Q'' | E^T; Y_loc]                         (M=128, N=128 + 64)
+//   P3  M^T = (I + M''^T) G, Q = (R' + Q'') G (G scales columns), written to
+//       TMEM as the A operand of R4 (bf16 hi/lo pairs)
+//   R4  += [M^T; Q] S^T, A from TMEM                      (M=128, N=64)
+//   P4  S_out^T -> next S^T operand (and sT at the end); Y rows -> y directly
+// Each round has a "ready" mbarrier (the 256 compute threads arrive after
+// publishing their writes) and a "done" mbarrier (tcgen05.commit); every wait
+// is bounded.  P0 of chunk c+1 overlaps R4 of chunk c, R1 of chunk c+1
+// overlaps P4 of chunk c.  Token tiles (w r k a b) arrive by cp.async one chunk
+// ahead into a staging tile; v goes by cp.async straight into its operand.
+//
+// TMEM (256 columns):
+//   X: cols [0, 64)     Gram^T (M=64 layout: lanes 16q..16q+15), then W'^T | U~^T
+//   Z: cols [64, 192)   [M''^T; Q''] (0-63), [E^T; Y_loc] -> [S_out^T; Y] (64-127)
+//   MQ: cols [192, 256) [M^T; Q] as bf16 pairs: hi 192-223, lo 224-255
 #include <algorithm>
 
 #include "umma.cuh"
@@ -61,38 +69,37 @@ constexpr int L = 32;              // tokens per chunk
 constexpr int NC = 256;            // compute threads (warps 0-7)
 constexpr int NT = NC + 32;        // + the MMA warp
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_X = 0, COL_Y = 96, COL_Z = 128;
-constexpr uint32_t LANE16 = 16u << 16;
+constexpr uint32_t COL_X = 0, COL_Z = 64, COL_MQ = 192;
 
 // shared memory map (bytes)
-constexpr uint32_t IN = 0;         // token tile: tensors w r k a b v, [32][128 B], 16-B chunks rotated by row
-constexpr uint32_t IN_W = 0, IN_R = 4096, IN_K = 8192, IN_A = 12288, IN_B = 16384, IN_V = 20480;
-constexpr uint32_t GA_HI = 24576, GA_LO = 32768;     // [64][64]: a' rows 0..31, r' rows 32..63
-constexpr uint32_t BB_HI = 40960, BB_LO = 53248;     // [64][96]: rows s = [b-_s | L_rb[:, s]], rows 32+s = [k-_s | L_rk[:, s]]
-constexpr uint32_t VB = 65536;                       // [32][64] exact bf16 v
-constexpr uint32_t S_HI = 69632, S_LO = 77824;       // [64][64]
-constexpr uint32_t R = 86016;                        // 24 KB, shared by short-lived buffers:
-constexpr uint32_t T_HI = R, T_LO = R + 2048, P_HI = R + 4096, P_LO = R + 6144;    //   P1..R2: [32][32]
-constexpr uint32_t ID32 = R;                         //   P2..R3: [32][32] bf16 identity
-constexpr int LDT = 36;                              //   row pitch of L_ab^T (floats; bank spread)
-constexpr uint32_t LABT = R + 8192;                  //   P1: fp32 L_ab^T [32][36]
-constexpr uint32_t LAK = R + 12800;                  //   P1: fp32 L_ak [32][33] (padded)
-constexpr uint32_t TSM = R + 17024;                  //   P1: fp32 T [32][32]
-constexpr uint32_t ZSM = R + 21120;                  //   P1: fp32 [16][16]
-constexpr uint32_t WT_HI = R + 8192, UT_HI = R + 12288, WT_LO = R + 16384, UT_LO = R + 20480;  // P2..R3: [64][32]
-constexpr uint32_t MQ_HI = R, MQ_LO = R + 12288;     //   P3..R4: [64][96] = [M | Q^T]
-constexpr uint32_t YSM = R;                          //   P4: fp32 [32][64]
-constexpr uint32_t GAML = 110592;                    // fp32 [64]: G per channel
-constexpr uint32_t BAR = 110848;                     // 8 mbarriers: ready R1..R4, done R1..R4
-constexpr uint32_t TMEM_SLOT = 110912;
-constexpr uint32_t FLAG = 110916;                    // set by whichever role gives up first
-constexpr uint32_t CFLAG = 110920;                   // compute warps' copy, written by thread 0 only
-constexpr uint32_t SMEM_BYTES = 110928;
+constexpr uint32_t IN_W = 0, IN_R = 4096, IN_K = 8192, IN_A = 12288, IN_B = 16384;   // [32][128 B], rotated
+// [32 tokens][128]: a' (cols 0-63) | v (cols 64-127); R2's A and R1's B rows 0-31.
+// RZ follows AV so that R1's B rows 32-63 are r'; RZ cols 64-127 are free space.
+constexpr uint32_t AV_HI = 20480, RZ_HI = 28672, AV_LO = 36864, RZ_LO = 45056;
+// [64][96]: rows s = [b-_s | L_rb[:, s]], rows 32+s = [k-_s | L_rk[:, s]]
+constexpr uint32_t BB_HI = 53248, BB_LO = 65536;
+constexpr uint32_t S_HI = 77824, S_LO = 86016;      // S^T [64 j][64 i]
+constexpr uint32_t R = 94208;                       // short-lived buffers:
+constexpr uint32_t TP_HI = R, TP_LO = R + 4096;     //   P1..R2: [64][32] = T rows 0-31, P rows 32-63
+constexpr int LDT = 36;                             //   row pitch of L_ab^T (floats; bank spread)
+constexpr uint32_t LABT = R + 8192;                 //   P1: fp32 L_ab^T [32][36]
+constexpr uint32_t LAK = R + 12800;                 //   P1: fp32 L_ak [32][33] (padded)
+constexpr uint32_t WU_HI = R, WU_LO = R + 8192;     //   P2..R3: [128][32] = W'^T rows, U~^T rows
+constexpr uint32_t SMEM_BYTES = R + 17024;
+// in the free halves of RZ (bytes [1024, 2048) of each 2 KB group)
+constexpr uint32_t TSM = RZ_HI + 1024;              // fp32 T, row t at TSM + (t/8)*2048 + (t%8)*128
+constexpr uint32_t ZSM = RZ_LO + 1024;              // fp32 [16][16]
+constexpr uint32_t GAML = RZ_LO + 3072;             // fp32 [64]: G per channel
+constexpr uint32_t BAR = GAML + 256;                // 8 mbarriers: ready R1..R4, done R1..R4
+constexpr uint32_t TMEM_SLOT = BAR + 64;
+constexpr uint32_t FLAG = BAR + 68;                 // set by whichever role gives up first
+constexpr uint32_t CFLAG = BAR + 72;                // compute warps' copy, written by thread 0 only
 
-constexpr long long kDrainCycles = 200000000LL;      // ~0.1 s to let committed tensor-core work finish
-constexpr float kMinDecay = 1e-30f;                  // per-chunk decay floor (prod of 32 w)
+constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
+constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (prod of 32 w)
 
 __device__ __forceinline__ uint32_t in_off(int t, int ch) { return (uint32_t)(t * 128 + (((ch + t) & 7) << 4)); }
+__device__ __forceinline__ uint32_t tsm_row(int t) { return TSM + (uint32_t)((t >> 3) * 2048 + (t & 7) * 128); }
 
 __device__ __forceinline__ void bf8_to_f32(uint4 u, float *o) {
     const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
@@ -101,10 +108,6 @@ __device__ __forceinline__ void bf8_to_f32(uint4 u, float *o) {
         o[2 * q] = __uint_as_float(uu[q] << 16);
         o[2 * q + 1] = __uint_as_float(uu[q] & 0xffff0000u);
     }
-}
-
-__device__ __forceinline__ float bf_at(const unsigned char *p) {
-    return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
 
 __device__ __forceinline__ void csync() { umma::named_sync(1, NC); }   // compute warps only
@@ -145,13 +148,27 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     auto ready_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };        // k = 0..3 (R1..R4)
     auto done_bar = [&](int k) { return sbase + BAR + 32u + 8u * (uint32_t)k; };
 
-    auto issue_tile = [&](int c) {        // compute threads only
-        const __nv_bfloat16 *src[6] = {w, r, k, a, b, v};
-        const int t0 = c * L;
-        for (int x = tid; x < 6 * L * 8; x += NC) {
-            const int ten = x >> 8, t = (x >> 3) & 31, ch = x & 7;
+    // token tile of chunk c (w r k a b) into the staging area; compute threads only
+    auto issue_in = [&](int c) {
+        if (c < nchunks) {
+            const __nv_bfloat16 *src[5] = {w, r, k, a, b};
+            const int t0 = c * L;
+            for (int x = tid; x < 5 * L * 8; x += NC) {
+                const int ten = x >> 8, t = (x >> 3) & 31, ch = x & 7;
+                if (t0 + t < T)
+                    cp_async16(sm + IN_W + ten * 4096 + in_off(t, ch), src[ten] + base + (size_t)(t0 + t) * tok_stride + ch * 8);
+            }
+        }
+        cp_async_commit();
+    };
+    // v of chunk c straight into its operand (AV columns 64-127); rows past the
+    // end keep the zeros P0 writes.  Transition runs keep v = 0.
+    auto issue_v = [&](int c) {
+        if (c < nchunks && !transition) {
+            const int t0 = c * L;
+            const int t = tid >> 3, ch = tid & 7;
             if (t0 + t < T)
-                cp_async16(sm + IN + ten * 4096 + in_off(t, ch), src[ten] + base + (size_t)(t0 + t) * tok_stride + ch * 8);
+                cp_async16(sm + AV_HI + cm_off(t, 64 + 8 * ch, 128), v + base + (size_t)(t0 + t) * tok_stride + ch * 8);
         }
         cp_async_commit();
     };
@@ -167,24 +184,23 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if (tid < NC) {
-        issue_tile(0);
-        const int i = tid >> 2, c0 = (tid & 3) * 16;
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            float x[8];
-            if (transition) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = (c0 + 8 * g + e == i) ? 1.f : 0.f;
-            } else if (s0p) {
-                const float4 u0 = load4(s0p + (size_t)i * kN + c0 + 8 * g);
-                const float4 u1 = load4(s0p + (size_t)i * kN + c0 + 8 * g + 4);
-                x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w; x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
-            }
-            store8_split(sm + S_HI, sm + S_LO, cm_off(i, c0 + 8 * g, 64), x);
+        {   // v columns of AV: lo always zero (v is exact), hi zero in transition runs
+            const int t = tid >> 3, ch = tid & 7;
+            if (transition) *reinterpret_cast<uint4 *>(sm + AV_HI + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sm + AV_LO + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
         }
+        issue_in(0);
+        issue_v(0);
+        // S^T operand: thread -> key column j of S, 16 value rows i
+        const int j = tid & 63, part = tid >> 6;
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int i = 16 * part + e;
+            x[e] = transition ? (i == j ? 1.f : 0.f) : (s0p ? s0p[(size_t)i * kN + j] : 0.f);
+        }
+        store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part, 64), x);
+        store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part + 8, 64), x + 8);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_before_sync();
@@ -195,54 +211,48 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     if (warp == 8) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            const uint32_t id_gram = idesc_bf16(64, 64, 0, 0), id_r2 = idesc_bf16(64, 32, 1, 0);
-            const uint32_t id_km96 = idesc_bf16(64, 96, 0, 1), id_mm96 = idesc_bf16(64, 96, 1, 1);
-            const OpD ga = opd_k(sbase + GA_HI, sbase + GA_LO, 64);
-            const OpD bbk = opd_k(sbase + BB_HI, sbase + BB_LO, 96);           // [b-; k-] rows, K = cols 0..63
-            const OpD at = opd_mn(sbase + GA_HI, sbase + GA_LO, 64);        // A'^T (rows 0..31 of GA)
-            const OpD vt = opd_mn(sbase + VB, 0, 64);                          // V^T, exact
-            const OpD tt = opd_k(sbase + T_HI, sbase + T_LO, L);
-            const OpD pp = opd_k(sbase + P_HI, sbase + P_LO, L);
-            const OpD wt = opd_k(sbase + WT_HI, sbase + WT_LO, L);
-            const OpD ut = opd_k(sbase + UT_HI, sbase + UT_LO, L);
-            const OpD bl = opd_mn(sbase + BB_HI, sbase + BB_LO, 96);          // [B- | L_rb^T]
-            const OpD kl = opd_mn(sbase + BB_HI + 6144, sbase + BB_LO + 6144, 96);   // [K- | L_rk^T]
-            const OpD ss = opd_k(sbase + S_HI, sbase + S_LO, 64);
-            const OpD mq = opd_mn(sbase + MQ_HI, sbase + MQ_LO, 96);          // [M | Q^T]
-            const OpD rt = opd_mn(sbase + GA_HI + 4096, sbase + GA_LO + 4096, 64);   // R'^T (rows 32..63 of GA)
-            const OpD id = opd_k(sbase + ID32, 0, L);                          // identity, exact
-            const uint32_t id_r = idesc_bf16(64, 32, 1, 0);
+            const uint32_t id_gram = idesc_bf16(64, 64, 0, 0);
+            const uint32_t id_r2 = idesc_bf16(128, 64, 1, 0);
+            const uint32_t id_r3a = idesc_bf16(128, 128, 1, 0);
+            const uint32_t id_r3b = idesc_bf16(128, 64, 1, 1);
+            const uint32_t id_r4 = idesc_bf16(128, 64, 0, 1);
+            const OpD bbk = opd_k(sbase + BB_HI, sbase + BB_LO, 96);          // [b-; k-] rows, K = cols 0..63
+            const OpD avk = opd_k(sbase + AV_HI, sbase + AV_LO, 128);         // [a'; r'] rows, K = cols 0..63
+            const OpD avm = opd_mn(sbase + AV_HI, sbase + AV_LO, 128);        // [A'^T; V^T], K = tokens
+            const OpD tp = opd_k(sbase + TP_HI, sbase + TP_LO, L);            // [T; P] rows, K = tokens
+            const OpD a1 = opd_mn(sbase + BB_HI, sbase + BB_LO, 96);          // [B-^T; L_rb], K = tokens
+            const OpD a2 = opd_mn(sbase + BB_HI + 6144, sbase + BB_LO + 6144, 96);   // [K-^T; L_rk]
+            const OpD wu = opd_k(sbase + WU_HI, sbase + WU_LO, L);            // [W' | U~], K = tokens
+            const OpD vv = opd_mn(sbase + AV_HI + 1024, 0, 128);              // V, exact
+            const OpD ss = opd_mn(sbase + S_HI, sbase + S_LO, 64);            // S^T, K = key j
             for (int c = 0; c < nchunks; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
-                // R1: Gram
+                // R1: Gram^T
                 if (!mbar_spin(ready_bar(0), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
-                gemm_split_d(tmem + COL_X, bbk, ga, id_gram, 4, false);       // Gram^T
+                gemm_split_d(tmem + COL_X, bbk, avk, id_gram, 4, false);
                 commit(done_bar(0));
                 last_k = 0;
                 last_par = par;
-                // R2: W'^T = A'^T T^T (lane 0), U~^T = V^T P^T (lane 16)
+                // R2: [A'^T; V^T] [T^T | P^T]
                 if (!mbar_spin(ready_bar(1), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
-                gemm_split_d(tmem + COL_Y, at, tt, id_r2, 2, false);
-                gemm_split_d(tmem + COL_Y + LANE16, vt, pp, id_r2, 2, false);
+                gemm_split_d(tmem + COL_X, avm, tp, id_r2, 2, false);
                 commit(done_bar(1));
                 last_k = 1;
                 last_par = par;
-                // R3: [M'' | Q''^T] = W'^T [B- | L_rb^T];  [E | Y_loc^T] = U~^T [B- | L_rb^T] + V^T [K- | L_rk^T]
+                // R3: [B-^T; L_rb] [W' | U~] + [K-^T; L_rk] [0 | V]
                 if (!mbar_spin(ready_bar(2), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
-                gemm_split_d(tmem + COL_X, wt, bl, id_km96, 2, false);
-                gemm_split_d(tmem + COL_X + 64, rt, id, id_r, 2, true);       // Q''^T += R'^T
-                gemm_split_d(tmem + COL_Z, ut, bl, id_km96, 2, false);
-                gemm_split_d(tmem + COL_Z, vt, kl, id_mm96, 2, true);
+                gemm_split_d(tmem + COL_Z, a1, wu, id_r3a, 2, false);
+                gemm_split_d(tmem + COL_Z + 64, a2, vv, id_r3b, 2, true);
                 commit(done_bar(2));
                 last_k = 2;
                 last_par = par;
-                // R4: [S_out | Y^T] += S [M | Q^T]
+                // R4: [S_out^T; Y] += [M^T; Q] S^T
                 if (!mbar_spin(ready_bar(3), par, wait_limit)) { *abort_flag = 1; break; }
                 fence_after_sync();
-                gemm_split_d(tmem + COL_Z, ss, mq, id_km96, 4, true);
+                gemm_split_ts(tmem + COL_Z + 64, tmem + COL_MQ, tmem + COL_MQ + 32, ss, id_r4, 4, true);
                 commit(done_bar(3));
                 last_k = 3;
                 last_par = par;
@@ -253,8 +263,9 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         // ================= compute warps =================
         const int q4 = warp & 3, hc = warp >> 2;     // TMEM lane quadrant, column half
         const uint32_t quad = (uint32_t)(32 * q4) << 16;
-        const int sub = lane & 15;                   // row within the quadrant's 16
-        const bool upper = lane >= 16;               // lanes reading the lane-16 accumulator
+        const int sub = lane & 15;                   // row within the quadrant's 16 (M=64 layout)
+        const bool upper = lane >= 16;
+        const int rho = 32 * q4 + lane;              // row of an M=128 accumulator
 
         // One lane polls, the others park at the barrier.  Only thread 0 reads
         // the shared abort flag (the issuer may set it at any time) and it
@@ -286,14 +297,14 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_K + off), kv);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_A + off), av);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_B + off), bv);
-            const uint4 vraw = (valid && !transition) ? *reinterpret_cast<const uint4 *>(sm + IN_V + off)
-                                                      : make_uint4(0, 0, 0, 0);
             float inc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 if (!valid) { wv[e] = 1.f; rv[e] = 0.f; kv[e] = 0.f; av[e] = 0.f; bv[e] = 0.f; }
                 inc[e] = wv[e];
             }
+            if (!valid)                           // rows past the end of the sequence: v = 0
+                *reinterpret_cast<uint4 *>(sm + AV_HI + cm_off(t, 64 + 8 * g, 128)) = make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1)
 #pragma unroll
@@ -316,11 +327,10 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 xb[e] = bv[e] * nxt;
                 xk[e] = kv[e] * nxt;
             }
-            store8_split(sm + GA_HI, sm + GA_LO, cm_off(t, 8 * g, 64), xa);
-            store8_split(sm + GA_HI, sm + GA_LO, cm_off(L + t, 8 * g, 64), xr);
+            store8_split(sm + AV_HI, sm + AV_LO, cm_off(t, 8 * g, 128), xa);
+            store8_split(sm + AV_HI, sm + AV_LO, cm_off(L + t, 8 * g, 128), xr);     // RZ rows
             store8_split(sm + BB_HI, sm + BB_LO, cm_off(t, 8 * g, 96), xb);
             store8_split(sm + BB_HI, sm + BB_LO, cm_off(L + t, 8 * g, 96), xk);
-            *reinterpret_cast<uint4 *>(sm + VB + cm_off(t, 8 * g, 64)) = vraw;
         };
 
         auto P1 = [&]() {                         // Gram -> L's; T = (I - L_ab)^{-1}; P = T L_ak
@@ -330,15 +340,15 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc + 16, r1);
                 tmem_wait();
                 if (!upper) {
-                    const int rho = 16 * q4 + sub;
+                    const int row = 16 * q4 + sub;
                     float g[32];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         g[e] = __uint_as_float(r0[e]);
                         g[16 + e] = __uint_as_float(r1[e]);
                     }
-                    const int s = rho & 31;
-                    if (rho < L && hc == 0) {         // column s of L_ab -> row s of L_ab^T
+                    const int s = row & 31;
+                    if (row < L && hc == 0) {         // column s of L_ab -> row s of L_ab^T
                         float *dst = reinterpret_cast<float *>(sm + LABT) + s * LDT;
 #pragma unroll
                         for (int t4 = 0; t4 < 8; ++t4) {
@@ -349,7 +359,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                             o.w = 4 * t4 + 3 > s ? g[4 * t4 + 3] : 0.f;
                             *reinterpret_cast<float4 *>(dst + 4 * t4) = o;
                         }
-                    } else if (rho >= L && hc == 0) { // column s of L_ak (rows padded to 33)
+                    } else if (row >= L && hc == 0) { // column s of L_ak (rows padded to 33)
                         float *dst = reinterpret_cast<float *>(sm + LAK) + s;
 #pragma unroll
                         for (int t = 0; t < L; ++t) dst[t * 33] = t > s ? g[t] : 0.f;
@@ -359,7 +369,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                             float x[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) x[e] = (8 * qq + e >= s) ? g[8 * qq + e] : 0.f;
-                            store8_split(sm + BB_HI, sm + BB_LO, cm_off(rho, 64 + 8 * qq, 96), x);
+                            store8_split(sm + BB_HI, sm + BB_LO, cm_off(row, 64 + 8 * qq, 96), x);
                         }
                     }
                 }
@@ -367,7 +377,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             fence_before_sync();
             csync();
             const float *labt = reinterpret_cast<const float *>(sm + LABT);
-            float *tsm = reinterpret_cast<float *>(sm + TSM);
+            auto trow = [&](int t) { return reinterpret_cast<float *>(sm + tsm_row(t)); };
             if (warp == 0) {                      // diagonal 16x16 blocks of T, one column per lane
                 const int blk = lane >> 4, s = 16 * blk + sub;
                 float acc[16];
@@ -387,12 +397,12 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) tsm[(16 * blk + e) * L + s] = acc[e];
+                for (int e = 0; e < 16; ++e) trow(16 * blk + e)[s] = acc[e];
             } else if (warp == 1) {               // upper-right block of T is zero
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int x = lane + 32 * e;
-                    tsm[(x >> 4) * L + 16 + (x & 15)] = 0.f;
+                    trow(x >> 4)[16 + (x & 15)] = 0.f;
                 }
             }
             csync();
@@ -401,7 +411,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 const int t = tid >> 4, s = tid & 15;
                 float acc = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * LDT + 16 + t], tsm[m * L + s], acc);
+                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * LDT + 16 + t], trow(m)[s], acc);
                 zsm[t * 16 + s] = acc;
             }
             csync();
@@ -409,8 +419,8 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 const int t = tid >> 4, s = tid & 15;
                 float acc = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(tsm[(16 + t) * L + 16 + m], zsm[m * 16 + s], acc);
-                tsm[(16 + t) * L + s] = acc;
+                for (int m = 0; m < 16; ++m) acc = fmaf(trow(16 + t)[16 + m], zsm[m * 16 + s], acc);
+                trow(16 + t)[s] = acc;
             }
             csync();
             {                                     // P = T L_ak and T, 4 rows per warp, one column per lane
@@ -421,7 +431,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 for (int m4 = 0; m4 < L / 4; ++m4) {
                     float4 tr[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) tr[i] = *reinterpret_cast<const float4 *>(tsm + (4 * warp + i) * L + 4 * m4);
+                    for (int i = 0; i < 4; ++i) tr[i] = *reinterpret_cast<const float4 *>(trow(4 * warp + i) + 4 * m4);
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const float lv = lak[(4 * m4 + c4) * 33 + s];
@@ -435,144 +445,139 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int t = 4 * warp + i;
-                    const uint32_t o = cm_off(t, s, L);
-                    const float tv = tsm[t * L + s];
-                    __nv_bfloat16 hi = __float2bfloat16_rn(pv[i]);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_HI + o) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_LO + o) = __float2bfloat16_rn(pv[i] - __bfloat162float(hi));
-                    hi = __float2bfloat16_rn(tv);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + T_HI + o) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + T_LO + o) = __float2bfloat16_rn(tv - __bfloat162float(hi));
+                    const float tv = trow(t)[s];
+                    const uint32_t ot = cm_off(t, s, L), op = cm_off(L + t, s, L);
+                    __nv_bfloat16 hi = __float2bfloat16_rn(tv);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_HI + ot) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_LO + ot) = __float2bfloat16_rn(tv - __bfloat162float(hi));
+                    hi = __float2bfloat16_rn(pv[i]);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_HI + op) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_LO + op) = __float2bfloat16_rn(pv[i] - __bfloat162float(hi));
                 }
             }
         };
 
-        auto P2 = [&]() {                         // stage W'^T (lanes 0-15) and U~^T (lanes 16-31)
+        auto P2 = [&]() {                         // rows of W'^T (quadrants 0-1) and U~^T (2-3) -> [W' | U~]
             uint32_t r0[16];
-            tmem_ld16_nowait(tmem + quad + COL_Y + 16 * hc, r0);
+            const uint32_t col = (q4 < 2 ? 0u : 32u) + 16u * (uint32_t)hc;
+            tmem_ld16_nowait(tmem + quad + COL_X + col, r0);
             tmem_wait();
             float x[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r0[e]);
-            const int row = 16 * q4 + sub;
-            unsigned char *hi = sm + (upper ? UT_HI : WT_HI);
-            unsigned char *lo = sm + (upper ? UT_LO : WT_LO);
-            store8_split(hi, lo, cm_off(row, 16 * hc, L), x);
-            store8_split(hi, lo, cm_off(row, 16 * hc + 8, L), x + 8);
-            {   // identity operand for R3 (the T/P space is free once R2 is done)
-                const int rr = tid >> 3, cc = 4 * (tid & 7);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + ID32 + cm_off(rr, cc + e, L)) =
-                        __float2bfloat16_rn(rr == cc + e ? 1.f : 0.f);
-            }
+            store8_split(sm + WU_HI, sm + WU_LO, cm_off(rho, 16 * hc, L), x);
+            store8_split(sm + WU_HI, sm + WU_LO, cm_off(rho, 16 * hc + 8, L), x + 8);
         };
 
-        auto P3 = [&]() {                         // [M | Q^T] rows j: M = G (I + M''), Q^T = G (R'^T + Q''^T) (R'^T added by R3)
-            uint32_t r0[16], r1[16], r2[16];
-            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc, r0);
-            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc + 16, r1);
-            tmem_ld16_nowait(tmem + quad + COL_X + 48 * hc + 32, r2);
-            tmem_wait();
-            if (!upper) {
-                const int j = 16 * q4 + sub;
-                const float G = reinterpret_cast<const float *>(sm + GAML)[j];
-                float x[48];
+        auto P3 = [&]() {                         // rows of [M^T; Q] -> TMEM A operand of R4
+            if (q4 == 3) return;
+            uint32_t r0[16], r1[16];
+            tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc, r0);
+            tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc + 16, r1);
+            float gv[32];
+            const float4 *g4 = reinterpret_cast<const float4 *>(sm + GAML) + 8 * hc;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    x[e] = __uint_as_float(r0[e]);
-                    x[16 + e] = __uint_as_float(r1[e]);
-                    x[32 + e] = __uint_as_float(r2[e]);
-                }
-#pragma unroll
-                for (int e = 0; e < 48; ++e) {
-                    const int col = 48 * hc + e;
-                    x[e] = G * (x[e] + (col == j ? 1.f : 0.f));   // Q columns (col >= 64) never match j
-                }
-#pragma unroll
-                for (int qq = 0; qq < 6; ++qq)
-                    store8_split(sm + MQ_HI, sm + MQ_LO, cm_off(j, 48 * hc + 8 * qq, 96), x + 8 * qq);
+            for (int u = 0; u < 8; ++u) {
+                const float4 q = g4[u];
+                gv[4 * u] = q.x; gv[4 * u + 1] = q.y; gv[4 * u + 2] = q.z; gv[4 * u + 3] = q.w;
             }
+            float add[32];
+            if (q4 < 2) {                         // M^T row j' = rho: + identity
+#pragma unroll
+                for (int e = 0; e < 32; ++e) add[e] = (32 * hc + e == rho) ? 1.f : 0.f;
+            } else {                              // Q row t: + r'_t (hi + lo)
+                const int t = rho - 64;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float hv[8], lv[8];
+                    bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + AV_HI + cm_off(L + t, 32 * hc + 8 * u, 128)), hv);
+                    bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + AV_LO + cm_off(L + t, 32 * hc + 8 * u, 128)), lv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) add[8 * u + e] = hv[e] + lv[e];
+                }
+            }
+            tmem_wait();
+            float xv[32];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                xv[e] = gv[e] * (__uint_as_float(r0[e]) + add[e]);
+                xv[16 + e] = gv[16 + e] * (__uint_as_float(r1[e]) + add[16 + e]);
+            }
+            uint32_t ph[16], pl[16];
+#pragma unroll
+            for (int e2 = 0; e2 < 16; ++e2) {
+                const float x0 = xv[2 * e2], x1 = xv[2 * e2 + 1];
+                const __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
+                const uint32_t hu = *reinterpret_cast<const uint32_t *>(&hp);
+                const __nv_bfloat162 lp = __floats2bfloat162_rn(x0 - __uint_as_float(hu << 16),
+                                                                x1 - __uint_as_float(hu & 0xffff0000u));
+                ph[e2] = hu;
+                pl[e2] = *reinterpret_cast<const uint32_t *>(&lp);
+            }
+            tmem_st16(tmem + quad + COL_MQ + 16 * hc, ph);
+            tmem_st16(tmem + quad + COL_MQ + 32 + 16 * hc, pl);
+            tmem_st_wait();
         };
 
-        auto P4 = [&](int c, int Lv) {            // rows i of [S_out | Y^T]: next S operand, y, final state
-            uint32_t r0[16], r1[16], r2[16];
-            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc, r0);
-            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc + 16, r1);
-            tmem_ld16_nowait(tmem + quad + COL_Z + 48 * hc + 32, r2);
+        auto P4 = [&](int c, int Lv) {            // rows of [S_out^T; Y]
+            if (q4 == 3) return;
+            uint32_t r0[16], r1[16];
+            tmem_ld16_nowait(tmem + quad + COL_Z + 64 + 32 * hc, r0);
+            tmem_ld16_nowait(tmem + quad + COL_Z + 64 + 32 * hc + 16, r1);
             tmem_wait();
-            if (!upper) {
-                const int i = 16 * q4 + sub;
-                float x[48];
+            float x[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    x[e] = __uint_as_float(r0[e]);
-                    x[16 + e] = __uint_as_float(r1[e]);
-                    x[32 + e] = __uint_as_float(r2[e]);
-                }
-                const bool last = c == nchunks - 1 && sTp != nullptr;
-                if (hc == 0) {                    // S columns 0..47
-#pragma unroll
-                    for (int qq = 0; qq < 6; ++qq) store8_split(sm + S_HI, sm + S_LO, cm_off(i, 8 * qq, 64), x + 8 * qq);
-                    if (last) {
-#pragma unroll
-                        for (int qq = 0; qq < 12; ++qq)
-                            store4(sTp + (size_t)i * kN + 4 * qq,
-                                   make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
-                    }
-                } else {                          // S columns 48..63, then y^T columns 0..31
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq)
-                        store8_split(sm + S_HI, sm + S_LO, cm_off(i, 48 + 8 * qq, 64), x + 8 * qq);
-                    if (last) {
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq)
-                            store4(sTp + (size_t)i * kN + 48 + 4 * qq,
-                                   make_float4(x[4 * qq], x[4 * qq + 1], x[4 * qq + 2], x[4 * qq + 3]));
-                    }
-                    float *ysm = reinterpret_cast<float *>(sm + YSM);
-#pragma unroll
-                    for (int e = 0; e < L; ++e) ysm[e * kN + i] = x[16 + e];
-                }
+            for (int e = 0; e < 16; ++e) {
+                x[e] = __uint_as_float(r0[e]);
+                x[16 + e] = __uint_as_float(r1[e]);
             }
-            fence_before_sync();
-            csync();
-            if (y) {   // coalesced y rows: thread -> (token, 8 channels)
-                const int t = tid >> 3, c8 = tid & 7;
+            if (q4 < 2) {                         // column j = rho of S_out, rows i = 32 hc + e
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    store8_split(sm + S_HI, sm + S_LO, cm_off(rho, 32 * hc + 8 * u, 64), x + 8 * u);
+                if (c == nchunks - 1 && sTp != nullptr) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sTp[(size_t)(32 * hc + e) * kN + rho] = x[e];
+                }
+            } else if (y) {                       // y row t, channels 32 hc .. 32 hc + 31
+                const int t = rho - 64;
                 if (t < Lv) {
-                    const float *ysm = reinterpret_cast<const float *>(sm + YSM) + t * kN + 8 * c8;
-                    OutT *dst = y + base + (size_t)(c * L + t) * tok_stride + 8 * c8;
-                    store4(dst, *reinterpret_cast<const float4 *>(ysm));
-                    store4(dst + 4, *reinterpret_cast<const float4 *>(ysm + 4));
+                    OutT *dst = y + base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        store4(dst + 4 * u, make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
                 }
             }
-            csync();
         };
 
         // ---- compute schedule ----
+        // cp.async groups are committed in a fixed order: [w r k a b](c) after
+        // P0(c-1), [v](c) in chunk c-1's P3 (both possibly empty).
         cp_async_wait<0>();
         csync();
         P0(min(L, T));
         csync();
         ready_arrive(0);                                   // R1(0)
-        if (nchunks > 1) issue_tile(1);
+        issue_in(1);
         for (int c = 0; c < nchunks; ++c) {
             if (!done_wait(0, c)) break;                   // Gram(c)
             P1();
+            cp_async_wait<1>();                            // v(c) is in place
             ready_arrive(1);                               // R2(c)
             if (!done_wait(1, c)) break;
             P2();
             ready_arrive(2);                               // R3(c)
             if (!done_wait(2, c)) break;
+            issue_v(c + 1);                                // v(c) is no longer read
             P3();
             ready_arrive(3);                               // R4(c)
             if (c + 1 < nchunks) {                         // next chunk's operands under R4(c)
-                cp_async_wait<0>();
+                cp_async_wait<1>();
                 csync();
                 P0(min(L, T - (c + 1) * L));
                 csync();
                 ready_arrive(0);                           // R1(c+1), under P4(c)
-                if (c + 2 < nchunks) issue_tile(c + 2);
+                issue_in(c + 2);
             }
             if (!done_wait(3, c)) break;                   // R4(c)
             P4(c, min(L, T - c * L));
@@ -679,7 +684,7 @@ static double launch_rounds(long long n, int sms) {
 // chunks) with the lowest estimated time, if that is below 95% of one pass;
 // among near-ties (within 3%) the fewest segments, which need the least scratch.
 int chunk_segments(int B, int T, int H, int sm_count) {
-    static_assert(2 * chunk::SMEM_BYTES <= 228 * 1024, "two chunk CTAs per SM");
+    static_assert(2 * (chunk::SMEM_BYTES + 1024) <= 228 * 1024, "two chunk CTAs per SM");
     const long long heads = (long long)B * H;
     const long long chunks = (T + chunk::L - 1) / chunk::L;
     if (sm_count <= 0 || heads <= 0) return 1;

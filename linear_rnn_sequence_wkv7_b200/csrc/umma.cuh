@@ -106,6 +106,27 @@ __device__ __forceinline__ void gemm_split_d(uint32_t d_tmem, const OpD &A, cons
         for (int ks = 0; ks < ksteps; ++ks) mma(d_tmem, A.lo + ks * A.kstep16, B.hi + ks * B.kstep16, idesc, 1u);
 }
 
+// D (+)= A * B with A read from tensor memory (M lanes; bf16 pairs packed per
+// 32-bit column, the lower half holding the even K index) and B from shared
+// memory.  Split passes: Ahi*Bhi + Ahi*Blo + Alo*Bhi; one K=16 step is 8 columns.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void gemm_split_ts(uint32_t d_tmem, uint32_t a_hi, uint32_t a_lo, const OpD &B,
+                                              uint32_t idesc, int ksteps, bool accumulate) {
+    uint32_t acc = accumulate ? 1u : 0u;
+    for (int ks = 0; ks < ksteps; ++ks) {
+        mma_ts(d_tmem, a_hi + 8u * ks, B.hi + ks * B.kstep16, idesc, acc);
+        acc = 1u;
+    }
+    for (int ks = 0; ks < ksteps; ++ks) mma_ts(d_tmem, a_hi + 8u * ks, B.lo + ks * B.kstep16, idesc, 1u);
+    for (int ks = 0; ks < ksteps; ++ks) mma_ts(d_tmem, a_lo + 8u * ks, B.hi + ks * B.kstep16, idesc, 1u);
+}
+
 __device__ __forceinline__ void commit(uint32_t mbar_saddr) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar_saddr)
                  : "memory");
@@ -133,6 +154,17 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[1
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns from registers (thread t -> lane base + t)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns; thread t of the warp gets lane (base + t)
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
