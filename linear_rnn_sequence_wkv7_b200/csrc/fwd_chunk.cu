@@ -47,9 +47,9 @@
 //       TMEM as the A operand of R4 (bf16 hi/lo pairs)
 //   R4  += [M^T; Q] S^T, A from TMEM                      (M=128, N=64)
 //   P4  S_out^T -> next S^T operand (and sT at the end); Y rows -> y directly
-// Each round has a "ready" mbarrier (the 256 compute threads arrive after
-// publishing their writes) and a "done" mbarrier (tcgen05.commit); every wait
-// is bounded.  P0 of chunk c+1 overlaps R4 of chunk c, R1 of chunk c+1
+// Each round has a "ready" mbarrier (each compute warp arrives once its threads
+// have published their writes) and a "done" mbarrier (tcgen05.commit); every
+// wait is bounded.  P0 of chunk c+1 overlaps R4 of chunk c, R1 of chunk c+1
 // overlaps P4 of chunk c.  Token tiles (w r k a b) arrive by cp.async one chunk
 // ahead into a staging tile; v goes by cp.async straight into its operand.
 //
@@ -93,7 +93,6 @@ constexpr uint32_t GAML = RZ_LO + 3072;             // fp32 [64]: G per channel
 constexpr uint32_t BAR = GAML + 256;                // 8 mbarriers: ready R1..R4, done R1..R4
 constexpr uint32_t TMEM_SLOT = BAR + 64;
 constexpr uint32_t FLAG = BAR + 68;                 // set by whichever role gives up first
-constexpr uint32_t CFLAG = BAR + 72;                // compute warps' copy, written by thread 0 only
 
 constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
 constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (prod of 32 w)
@@ -142,22 +141,23 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                                                             : nullptr;
     const int nchunks = (T + L - 1) / L;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
-    volatile uint32_t *compute_flag = reinterpret_cast<volatile uint32_t *>(sm + CFLAG);
     int last_k = -1;                                 // issuer: last committed round and its parity
     uint32_t last_par = 0;
     auto ready_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };        // k = 0..3 (R1..R4)
     auto done_bar = [&](int k) { return sbase + BAR + 32u + 8u * (uint32_t)k; };
 
-    // token tile of chunk c (w r k a b) into the staging area; compute threads only
+    // token tile of chunk c (w r k a b) into the staging area; compute threads
+    // only, thread -> (token, 16-byte chunk) of each tensor
     auto issue_in = [&](int c) {
-        if (c < nchunks) {
-            const __nv_bfloat16 *src[5] = {w, r, k, a, b};
-            const int t0 = c * L;
-            for (int x = tid; x < 5 * L * 8; x += NC) {
-                const int ten = x >> 8, t = (x >> 3) & 31, ch = x & 7;
-                if (t0 + t < T)
-                    cp_async16(sm + IN_W + ten * 4096 + in_off(t, ch), src[ten] + base + (size_t)(t0 + t) * tok_stride + ch * 8);
-            }
+        const int t = tid >> 3, ch = tid & 7;
+        if (c < nchunks && c * L + t < T) {
+            const size_t g = base + (size_t)(c * L + t) * tok_stride + ch * 8;
+            const uint32_t o = in_off(t, ch);
+            cp_async16(sm + IN_W + o, w + g);
+            cp_async16(sm + IN_R + o, r + g);
+            cp_async16(sm + IN_K + o, k + g);
+            cp_async16(sm + IN_A + o, a + g);
+            cp_async16(sm + IN_B + o, b + g);
         }
         cp_async_commit();
     };
@@ -176,11 +176,10 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     // ---- set-up -------------------------------------------------------------------------
     if (tid == 0) {
         for (int kk = 0; kk < 4; ++kk) {
-            mbar_init(ready_bar(kk), NC);
+            mbar_init(ready_bar(kk), NC / 32);            // one arrival per compute warp
             mbar_init(done_bar(kk), 1);
         }
         *abort_flag = 0;
-        *compute_flag = 0;
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if (tid < NC) {
@@ -228,21 +227,21 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             for (int c = 0; c < nchunks; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
                 // R1: Gram^T
-                if (!mbar_spin(ready_bar(0), par, wait_limit)) { *abort_flag = 1; break; }
+                if (!mbar_poll(ready_bar(0), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_X, bbk, avk, id_gram, 4, false);
                 commit(done_bar(0));
                 last_k = 0;
                 last_par = par;
                 // R2: [A'^T; V^T] [T^T | P^T]
-                if (!mbar_spin(ready_bar(1), par, wait_limit)) { *abort_flag = 1; break; }
+                if (!mbar_poll(ready_bar(1), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_X, avm, tp, id_r2, 2, false);
                 commit(done_bar(1));
                 last_k = 1;
                 last_par = par;
                 // R3: [B-^T; L_rb] [W' | U~] + [K-^T; L_rk] [0 | V]
-                if (!mbar_spin(ready_bar(2), par, wait_limit)) { *abort_flag = 1; break; }
+                if (!mbar_poll(ready_bar(2), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_d(tmem + COL_Z, a1, wu, id_r3a, 2, false);
                 gemm_split_d(tmem + COL_Z + 64, a2, vv, id_r3b, 2, true);
@@ -250,7 +249,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 last_k = 2;
                 last_par = par;
                 // R4: [S_out^T; Y] += [M^T; Q] S^T
-                if (!mbar_spin(ready_bar(3), par, wait_limit)) { *abort_flag = 1; break; }
+                if (!mbar_poll(ready_bar(3), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
                 fence_after_sync();
                 gemm_split_ts(tmem + COL_Z + 64, tmem + COL_MQ, tmem + COL_MQ + 32, ss, id_r4, 4, true);
                 commit(done_bar(3));
@@ -267,24 +266,27 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         const bool upper = lane >= 16;
         const int rho = 32 * q4 + lane;              // row of an M=128 accumulator
 
-        // One lane polls, the others park at the barrier.  Only thread 0 reads
-        // the shared abort flag (the issuer may set it at any time) and it
-        // publishes its decision before the barrier, so all 256 threads take
-        // the same branch afterwards.
-        auto done_wait = [&](int kk, int c) -> bool {
-            if (tid == 0) {
-                const bool ok = mbar_spin(done_bar(kk), (uint32_t)c & 1u, wait_limit);
-                if (!ok) *abort_flag = 1;
-                *compute_flag = (!ok || *abort_flag) ? 1u : 0u;
+        // One thread polls for a tensor-core round, the other compute threads
+        // park at the named barrier (parked warps take no issue slots from the
+        // other CTA on the SM).  All compute warps run the same schedule of
+        // barriers whatever happens: a wait that gives up sets the abort flag,
+        // later waits return at once, and the remaining chunks run through on
+        // garbage (the status word reports the timeout), so that no warp is
+        // ever left at a barrier.
+        auto done_wait = [&](int kk, int c) {
+            if (tid == 0 && *abort_flag == 0u) {
+                if (!mbar_spin_abortable(done_bar(kk), (uint32_t)c & 1u, wait_limit, abort_flag)) *abort_flag = 1;
             }
             csync();
             fence_after_sync();
-            return *compute_flag == 0;
         };
+        // every thread publishes its own writes (shared memory to the async
+        // proxy, TMEM stores); the warp converges and lane 0 arrives for it
         auto ready_arrive = [&](int kk) {
             fence_smem_to_async();
             fence_before_sync();
-            mbar_arrive(ready_bar(kk));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ready_bar(kk));
         };
 
         auto P0 = [&](int Lv) {                   // decayed operands of one chunk
@@ -423,37 +425,51 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 trow(16 + t)[s] = acc;
             }
             csync();
-            {                                     // P = T L_ak and T, 4 rows per warp, one column per lane
+            {   // P = T L_ak, skipping the zero 16x16 blocks: P11 = T11 L11,
+                // P21 = T21 L11 + T22 L21, P22 = T22 L22, P12 = 0.  Half-warp
+                // kk (0..15), lane column s: row kk (cols < 16, m < 16), row
+                // 16 + kk (cols < 16, all m; cols >= 16, m >= 16).
                 const float *lak = reinterpret_cast<const float *>(sm + LAK);
-                const int s = lane;
-                float pv[4] = {0.f, 0.f, 0.f, 0.f};
+                const int kk = 2 * warp + (lane >> 4), s = lane & 15;
+                const float *ta = trow(kk), *tb = trow(16 + kk);
+                float pa = 0.f, pb = 0.f, pc = 0.f;
 #pragma unroll
-                for (int m4 = 0; m4 < L / 4; ++m4) {
-                    float4 tr[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) tr[i] = *reinterpret_cast<const float4 *>(trow(4 * warp + i) + 4 * m4);
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    const float4 xa = *reinterpret_cast<const float4 *>(ta + 4 * m4);
+                    const float4 xb = *reinterpret_cast<const float4 *>(tb + 4 * m4);
+                    const float va[4] = {xa.x, xa.y, xa.z, xa.w}, vb[4] = {xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const float lv = lak[(4 * m4 + c4) * 33 + s];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float tv = c4 == 0 ? tr[i].x : c4 == 1 ? tr[i].y : c4 == 2 ? tr[i].z : tr[i].w;
-                            pv[i] = fmaf(tv, lv, pv[i]);
-                        }
+                        pa = fmaf(va[c4], lv, pa);
+                        pb = fmaf(vb[c4], lv, pb);
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 4 * warp + i;
-                    const float tv = trow(t)[s];
-                    const uint32_t ot = cm_off(t, s, L), op = cm_off(L + t, s, L);
-                    __nv_bfloat16 hi = __float2bfloat16_rn(tv);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_HI + ot) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_LO + ot) = __float2bfloat16_rn(tv - __bfloat162float(hi));
-                    hi = __float2bfloat16_rn(pv[i]);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_HI + op) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + TP_LO + op) = __float2bfloat16_rn(pv[i] - __bfloat162float(hi));
+                for (int m4 = 4; m4 < 8; ++m4) {
+                    const float4 xb = *reinterpret_cast<const float4 *>(tb + 4 * m4);
+                    const float vb[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float* lrow = lak + (4 * m4 + c4) * 33;
+                        pb = fmaf(vb[c4], lrow[s], pb);
+                        pc = fmaf(vb[c4], lrow[16 + s], pc);
+                    }
                 }
+                auto put = [&](uint32_t hi_base, uint32_t lo_base, int row, int col, float x) {
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                    const uint32_t o = cm_off(row, col, L);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + hi_base + o) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + lo_base + o) = __float2bfloat16_rn(x - __bfloat162float(hi));
+                };
+                put(TP_HI, TP_LO, kk, s, ta[s]);
+                put(TP_HI, TP_LO, kk, 16 + s, ta[16 + s]);
+                put(TP_HI, TP_LO, 16 + kk, s, tb[s]);
+                put(TP_HI, TP_LO, 16 + kk, 16 + s, tb[16 + s]);
+                put(TP_HI, TP_LO, L + kk, s, pa);
+                put(TP_HI, TP_LO, L + kk, 16 + s, 0.f);
+                put(TP_HI, TP_LO, L + 16 + kk, s, pb);
+                put(TP_HI, TP_LO, L + 16 + kk, 16 + s, pc);
             }
         };
 
@@ -551,35 +567,34 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         };
 
         // ---- compute schedule ----
-        // cp.async groups are committed in a fixed order: [w r k a b](c) after
-        // P0(c-1), [v](c) in chunk c-1's P3 (both possibly empty).
+        // cp.async groups are committed in a fixed order: [w r k a b](c+1) at
+        // the start of P1(c), [v](c+1) at the start of P3(c) (both possibly
+        // empty).  Gram(c) done means every warp has finished P0(c), so the
+        // staging tile is free for the next chunk.
         cp_async_wait<0>();
         csync();
         P0(min(L, T));
-        csync();
         ready_arrive(0);                                   // R1(0)
-        issue_in(1);
         for (int c = 0; c < nchunks; ++c) {
-            if (!done_wait(0, c)) break;                   // Gram(c)
+            done_wait(0, c);                               // Gram(c)
+            issue_in(c + 1);
             P1();
             cp_async_wait<1>();                            // v(c) is in place
             ready_arrive(1);                               // R2(c)
-            if (!done_wait(1, c)) break;
+            done_wait(1, c);
             P2();
             ready_arrive(2);                               // R3(c)
-            if (!done_wait(2, c)) break;
+            done_wait(2, c);
             issue_v(c + 1);                                // v(c) is no longer read
             P3();
             ready_arrive(3);                               // R4(c)
             if (c + 1 < nchunks) {                         // next chunk's operands under R4(c)
-                cp_async_wait<1>();
-                csync();
+                cp_async_wait<1>();                        // tile c+1 is in place
+                csync();                                   // ... for all threads; P3(c) reads are done
                 P0(min(L, T - (c + 1) * L));
-                csync();
                 ready_arrive(0);                           // R1(c+1), under P4(c)
-                issue_in(c + 2);
             }
-            if (!done_wait(3, c)) break;                   // R4(c)
+            done_wait(3, c);                               // R4(c)
             P4(c, min(L, T - c * L));
         }
         cp_async_wait<0>();

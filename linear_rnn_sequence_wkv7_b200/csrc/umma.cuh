@@ -219,6 +219,43 @@ __device__ __forceinline__ bool mbar_spin(uint32_t saddr, uint32_t parity, long 
     }
 }
 
+// test_wait polling that also gives up as soon as *abort (a shared flag set by
+// another warp that gave up) becomes nonzero.
+__device__ __forceinline__ bool mbar_spin_abortable(uint32_t saddr, uint32_t parity, long long limit_cycles,
+                                                    const volatile uint32_t *abort) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(saddr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit_cycles) return false;
+    }
+}
+
+// Same, for a thread that only polls: the clock and the flag are read once
+// every 16 polls, which keeps the loop short.
+__device__ __forceinline__ bool mbar_poll(uint32_t saddr, uint32_t parity, long long limit_cycles,
+                                         const volatile uint32_t *abort) {
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(saddr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((it & 15u) == 0u && (*abort || clock64() - t0 > limit_cycles)) return false;
+    }
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(saddr) : "memory");
 }
