@@ -299,14 +299,14 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_K + off), kv);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_A + off), av);
             bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + IN_B + off), bv);
+            if (Lv < L && !valid) {               // rows past the end of the sequence: no-op tokens, v = 0
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { wv[e] = 1.f; rv[e] = 0.f; kv[e] = 0.f; av[e] = 0.f; bv[e] = 0.f; }
+                *reinterpret_cast<uint4 *>(sm + AV_HI + cm_off(t, 64 + 8 * g, 128)) = make_uint4(0, 0, 0, 0);
+            }
             float inc[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (!valid) { wv[e] = 1.f; rv[e] = 0.f; kv[e] = 0.f; av[e] = 0.f; bv[e] = 0.f; }
-                inc[e] = wv[e];
-            }
-            if (!valid)                           // rows past the end of the sequence: v = 0
-                *reinterpret_cast<uint4 *>(sm + AV_HI + cm_off(t, 64 + 8 * g, 128)) = make_uint4(0, 0, 0, 0);
+            for (int e = 0; e < 8; ++e) inc[e] = wv[e];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1)
 #pragma unroll
