@@ -639,42 +639,42 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
 
 // Segments combine: per head, S_in(0) = s0 (or 0) and
 // S_in(k+1) = S_in(k) M_k + E_k, where E_k / M_k are the final states of the
-// segment's plain and transition runs.  Writes S_in(k) for k < nseg.  One CTA
-// (256 threads) per head, fp32 on the CUDA cores; thread -> row i, 16 columns.
+// segment's plain and transition runs.  Writes S_in(k) for k < nseg.  The
+// rows of S are independent: CTA (head, rb) owns rows 8 rb .. 8 rb + 7, thread
+// -> (row, two columns); M_k is staged in shared memory.  fp32 on CUDA cores.
+constexpr int kCombineRows = 8;
+
 __global__ void __launch_bounds__(256)
 seg_combine_kernel(int BH, int nseg, const float *__restrict__ s0, const float *__restrict__ em,
                    float *__restrict__ sin_out) {
-    __shared__ __align__(16) float Ssm[kN * kN];
     __shared__ __align__(16) float Msm[kN * kN];
+    __shared__ float Ssm[kCombineRows][kN];
     const int head = blockIdx.x, tid = threadIdx.x;
-    const int i = tid >> 2, j0 = (tid & 3) * 16;
+    const int rr = tid >> 5, c2 = 2 * (tid & 31);
+    const int i = kCombineRows * blockIdx.y + rr;
     const size_t hoff = (size_t)head * kN * kN;
     const size_t zstride = (size_t)BH * kN * kN;
-    float cur[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) cur[e] = s0 ? s0[hoff + (size_t)i * kN + j0 + e] : 0.f;
+    float2 cur = s0 ? *reinterpret_cast<const float2 *>(s0 + hoff + (size_t)i * kN + c2) : make_float2(0.f, 0.f);
     for (int kk = 0; kk < nseg; ++kk) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            sin_out[(size_t)kk * zstride + hoff + (size_t)i * kN + j0 + e] = cur[e];
-            Ssm[i * kN + j0 + e] = cur[e];
-        }
+        *reinterpret_cast<float2 *>(sin_out + (size_t)kk * zstride + hoff + (size_t)i * kN + c2) = cur;
         if (kk + 1 == nseg) break;
         const float *E = em + (size_t)kk * zstride + hoff;
         const float *M = em + (size_t)(nseg - 1 + kk) * zstride + hoff;
-        for (int x = tid; x < kN * kN; x += 256) Msm[x] = M[x];
+        Ssm[rr][c2] = cur.x;
+        Ssm[rr][c2 + 1] = cur.y;
+        for (int x = tid; x < kN * kN / 4; x += 256)
+            reinterpret_cast<float4 *>(Msm)[x] = reinterpret_cast<const float4 *>(M)[x];
         __syncthreads();
-        float acc[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = E[(size_t)i * kN + j0 + e];
+        float2 acc = *reinterpret_cast<const float2 *>(E + (size_t)i * kN + c2);
+#pragma unroll 16
         for (int m = 0; m < kN; ++m) {
-            const float sm_ = Ssm[i * kN + m];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = fmaf(sm_, Msm[m * kN + j0 + e], acc[e]);
+            const float sv = Ssm[rr][m];
+            const float2 mv = *reinterpret_cast<const float2 *>(Msm + m * kN + c2);
+            acc.x = fmaf(sv, mv.x, acc.x);
+            acc.y = fmaf(sv, mv.y, acc.y);
         }
         __syncthreads();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) cur[e] = acc[e];
+        cur = acc;
     }
 }
 
@@ -736,7 +736,7 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
                                  nullptr, em, zst, -1, wait_limit, st);
     if (e != cudaSuccess) return e;
     // pass 2: entry state of every segment
-    seg_combine_kernel<<<B * H, 256, 0, st>>>(B * H, nseg, s0, em, sin);
+    seg_combine_kernel<<<dim3(B * H, kN / kCombineRows), 256, 0, st>>>(B * H, nseg, s0, em, sin);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // pass 3: every segment from its true entry state; the last one writes sT
