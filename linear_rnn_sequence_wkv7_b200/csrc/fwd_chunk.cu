@@ -90,7 +90,7 @@ constexpr uint32_t SMEM_BYTES = R + 17024;
 constexpr uint32_t TSM = RZ_HI + 1024;              // fp32 T, row t at TSM + (t/8)*2048 + (t%8)*128
 constexpr uint32_t ZSM = RZ_LO + 1024;              // fp32 [16][16]
 constexpr uint32_t GAML = RZ_LO + 3072;             // fp32 [64]: G per channel
-constexpr uint32_t BAR = GAML + 256;                // 8 mbarriers: ready R1..R4, done R1..R4
+constexpr uint32_t BAR = GAML + 256;                // 4 mbarriers: tcgen05.commit of R1..R4
 constexpr uint32_t TMEM_SLOT = BAR + 64;
 constexpr uint32_t FLAG = BAR + 68;                 // set by whichever role gives up first
 
@@ -110,6 +110,9 @@ __device__ __forceinline__ void bf8_to_f32(uint4 u, float *o) {
 }
 
 __device__ __forceinline__ void csync() { umma::named_sync(1, NC); }   // compute warps only
+// hand-off of round k (0..3 = R1..R4) between the compute warps and the issuer:
+// named barriers over all NT threads
+constexpr uint32_t BAR_READY = 2, BAR_DONE = 6;
 
 }  // namespace chunk
 
@@ -143,8 +146,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
     int last_k = -1;                                 // issuer: last committed round and its parity
     uint32_t last_par = 0;
-    auto ready_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };        // k = 0..3 (R1..R4)
-    auto done_bar = [&](int k) { return sbase + BAR + 32u + 8u * (uint32_t)k; };
+    auto done_bar = [&](int k) { return sbase + BAR + 8u * (uint32_t)k; };         // k = 0..3 (R1..R4)
 
     // token tile of chunk c (w r k a b) into the staging area; compute threads
     // only, thread -> (token, 16-byte chunk) of each tensor
@@ -176,7 +178,6 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     // ---- set-up -------------------------------------------------------------------------
     if (tid == 0) {
         for (int kk = 0; kk < 4; ++kk) {
-            mbar_init(ready_bar(kk), NC / 32);            // one arrival per compute warp
             mbar_init(done_bar(kk), 1);
         }
         *abort_flag = 0;
@@ -209,7 +210,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 
     if (warp == 8) {
         // ================= MMA issuer =================
-        if (lane == 0) {
+        {
             const uint32_t id_gram = idesc_bf16(64, 64, 0, 0);
             const uint32_t id_r2 = idesc_bf16(128, 64, 1, 0);
             const uint32_t id_r3a = idesc_bf16(128, 128, 1, 0);
@@ -224,37 +225,38 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             const OpD wu = opd_k(sbase + WU_HI, sbase + WU_LO, L);            // [W' | U~], K = tokens
             const OpD vv = opd_mn(sbase + AV_HI + 1024, 0, 128);              // V, exact
             const OpD ss = opd_mn(sbase + S_HI, sbase + S_LO, 64);            // S^T, K = key j
+            // One tensor-core round: wait until the compute warps hand it over
+            // (bar.arrive on its ready barrier), issue and commit it, wait for
+            // the commit, and release the compute warps (bar.sync on its done
+            // barrier).  The whole warp passes every barrier once per chunk
+            // whatever happens; after a wait gives up nothing more is issued.
+            auto round = [&](int rd, uint32_t par, auto &&issue) {
+                named_sync(BAR_READY + rd, NT);
+                fence_after_sync();
+                if (lane == 0 && *abort_flag == 0u) {
+                    issue();
+                    commit(done_bar(rd));
+                    last_k = rd;
+                    last_par = par;
+                    if (!mbar_spin_abortable(done_bar(rd), par, wait_limit, abort_flag)) *abort_flag = 1;
+                }
+                __syncwarp();
+                fence_before_sync();
+                named_arrive(BAR_DONE + rd, NT);
+            };
             for (int c = 0; c < nchunks; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
-                // R1: Gram^T
-                if (!mbar_poll(ready_bar(0), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
-                fence_after_sync();
-                gemm_split_d(tmem + COL_X, bbk, avk, id_gram, 4, false);
-                commit(done_bar(0));
-                last_k = 0;
-                last_par = par;
-                // R2: [A'^T; V^T] [T^T | P^T]
-                if (!mbar_poll(ready_bar(1), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
-                fence_after_sync();
-                gemm_split_d(tmem + COL_X, avm, tp, id_r2, 2, false);
-                commit(done_bar(1));
-                last_k = 1;
-                last_par = par;
-                // R3: [B-^T; L_rb] [W' | U~] + [K-^T; L_rk] [0 | V]
-                if (!mbar_poll(ready_bar(2), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
-                fence_after_sync();
-                gemm_split_d(tmem + COL_Z, a1, wu, id_r3a, 2, false);
-                gemm_split_d(tmem + COL_Z + 64, a2, vv, id_r3b, 2, true);
-                commit(done_bar(2));
-                last_k = 2;
-                last_par = par;
-                // R4: [S_out^T; Y] += [M^T; Q] S^T
-                if (!mbar_poll(ready_bar(3), par, wait_limit, abort_flag)) { *abort_flag = 1; break; }
-                fence_after_sync();
-                gemm_split_ts(tmem + COL_Z + 64, tmem + COL_MQ, tmem + COL_MQ + 32, ss, id_r4, 4, true);
-                commit(done_bar(3));
-                last_k = 3;
-                last_par = par;
+                round(0, par, [&] { gemm_split_d(tmem + COL_X, bbk, avk, id_gram, 4, false); });   // Gram^T
+                round(1, par, [&] {                                                              // [W'^T; U~^T]
+                    gemm_split_d(tmem + COL_X, avm, tp, id_r2, 2, false);
+                });
+                round(2, par, [&] {                         // [B-^T; L_rb] [W' | U~] + [K-^T; L_rk] [0 | V]
+                    gemm_split_d(tmem + COL_Z, a1, wu, id_r3a, 2, false);
+                    gemm_split_d(tmem + COL_Z + 64, a2, vv, id_r3b, 2, true);
+                });
+                round(3, par, [&] {                         // [S_out^T; Y] += [M^T; Q] S^T
+                    gemm_split_ts(tmem + COL_Z + 64, tmem + COL_MQ, tmem + COL_MQ + 32, ss, id_r4, 4, true);
+                });
             }
         }
         __syncwarp();
@@ -266,27 +268,22 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         const bool upper = lane >= 16;
         const int rho = 32 * q4 + lane;              // row of an M=128 accumulator
 
-        // One thread polls for a tensor-core round, the other compute threads
-        // park at the named barrier (parked warps take no issue slots from the
-        // other CTA on the SM).  All compute warps run the same schedule of
-        // barriers whatever happens: a wait that gives up sets the abort flag,
-        // later waits return at once, and the remaining chunks run through on
-        // garbage (the status word reports the timeout), so that no warp is
-        // ever left at a barrier.
-        auto done_wait = [&](int kk, int c) {
-            if (tid == 0 && *abort_flag == 0u) {
-                if (!mbar_spin_abortable(done_bar(kk), (uint32_t)c & 1u, wait_limit, abort_flag)) *abort_flag = 1;
-            }
-            csync();
+        // Hand-offs with the issuer warp.  Waiting warps park at a hardware
+        // barrier (no issue slots taken from the other CTA on the SM).  The
+        // compute warps run one fixed schedule of barriers whatever happens;
+        // after a wait gives up (abort flag, status word WKV7_ERR_TIMEOUT) the
+        // remaining chunks run through on garbage so no warp is ever left at
+        // a barrier.
+        auto done_wait = [&](int kk, int) {
+            named_sync(BAR_DONE + kk, NT);
             fence_after_sync();
         };
         // every thread publishes its own writes (shared memory to the async
-        // proxy, TMEM stores); the warp converges and lane 0 arrives for it
+        // proxy, TMEM stores) before it arrives
         auto ready_arrive = [&](int kk) {
             fence_smem_to_async();
             fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ready_bar(kk));
+            named_arrive(BAR_READY + kk, NT);
         };
 
         auto P0 = [&](int Lv) {                   // decayed operands of one chunk

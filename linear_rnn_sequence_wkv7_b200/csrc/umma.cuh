@@ -220,7 +220,9 @@ __device__ __forceinline__ bool mbar_spin(uint32_t saddr, uint32_t parity, long 
 }
 
 // test_wait polling that also gives up as soon as *abort (a shared flag set by
-// another warp that gave up) becomes nonzero.
+// another warp that gave up) becomes nonzero.  The phase must be observed
+// within limit_cycles of the start of the wait: a poll that sees it complete
+// after the limit still counts as a timeout.
 __device__ __forceinline__ bool mbar_spin_abortable(uint32_t saddr, uint32_t parity, long long limit_cycles,
                                                     const volatile uint32_t *abort) {
     const long long t0 = clock64();
@@ -232,27 +234,9 @@ __device__ __forceinline__ bool mbar_spin_abortable(uint32_t saddr, uint32_t par
             : "=r"(done)
             : "r"(saddr), "r"(parity)
             : "memory");
+        if (clock64() - t0 > limit_cycles) return false;
         if (done) return true;
         if (*abort) return false;
-        if (clock64() - t0 > limit_cycles) return false;
-    }
-}
-
-// Same, for a thread that only polls: the clock and the flag are read once
-// every 16 polls, which keeps the loop short.
-__device__ __forceinline__ bool mbar_poll(uint32_t saddr, uint32_t parity, long long limit_cycles,
-                                         const volatile uint32_t *abort) {
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(saddr), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if ((it & 15u) == 0u && (*abort || clock64() - t0 > limit_cycles)) return false;
     }
 }
 
@@ -263,6 +247,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
 // named barrier among `count` threads (a multiple of 32)
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// arrive at a named barrier without waiting (producer side)
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---- bf16 hi/lo split --------------------------------------------------------
