@@ -25,6 +25,9 @@ section "Summary").
   parallelisable (RWKV-7 "Goose" abstract) and cite chunk-wise delta-rule
   parallelisation by title; the algebra here is our own derivation from the
   recurrence, applied chunk by chunk in the order of its definition.
+* ``backward_chunked`` is the reverse-mode derivative of ``forward_chunked``,
+  chunk by chunk (last chunk first), each line the adjoint of one line of the
+  forward definition; pinned against ``backward``.
 """
 from __future__ import annotations
 
@@ -169,3 +172,102 @@ def forward_chunked(r, w, k, v, a, b, s0=None, chunk_len=64):
                 S = S * gam[-1][None, :] + U.T @ Bbar + V.T @ Kbar
             sT[bb, h] = S
     return y, sT
+
+
+def backward_chunked(r, w, k, v, a, b, s0, dy, dsT=None, chunk_len=64):
+    """Chunked form of ``backward`` (fp64, w > 0): the reverse-mode derivative
+    of ``forward_chunked``, taken chunk by chunk, last chunk first.
+
+    With the chunk quantities of ``forward_chunked`` (S = S_in, M = I - L_ab,
+    Z = A~ S^T + L_ak V, U = M^{-1} Z, X = S + U^T B^ + V^T K^, S_out =
+    X diag(gamma_{L-1})) and the upstream gradients dY (rows t) and dS_out:
+
+      dX  = dS_out diag(gamma_{L-1});   dgamma_{L-1} += sum_i X * dS_out
+      dS  = dX + dY^T R~ + dZ^T A~;     dU  = B^ dX^T + L_rb^T dY
+      dZ  = M^{-T} dU
+      dV  = K^ dX^T + L_rk^T dY + L_ak^T dZ
+      dL_ab = (dZ U^T) strict,  dL_ak = (dZ V^T) strict,
+      dL_rb = (dY U^T) incl,    dL_rk = (dY V^T) incl
+      dA~ = dZ S + dL_ab B^ + dL_ak K^;    dR~ = dY S + dL_rb B^ + dL_rk K^
+      dB^ = U dX + dL_ab^T A~ + dL_rb^T R~;  dK^ = V dX + dL_ak^T A~ + dL_rk^T R~
+
+    then through the decay scalings (a~ = a gamma_{t-1}, r~ = r gamma_t,
+    b^ = b / gamma_s, k^ = k / gamma_s) and gamma_t = prod_{m<=t} w_m.
+    dS becomes dS_out of the previous chunk; at the start it is ds0.  Every
+    line is the adjoint of one line of the forward definition.
+    """
+    r, w, k, v, a, b, dy = (_f64(x) for x in (r, w, k, v, a, b, dy))
+    B, T, H, N = r.shape
+    grads = [np.zeros((B, T, H, N)) for _ in range(6)]   # dr dw dk dv da db
+    ds0 = np.zeros((B, H, N, N))
+    for bb in range(B):
+        for h in range(H):
+            # forward pass, keeping the state entering each chunk
+            S = np.zeros((N, N)) if s0 is None else _f64(s0)[bb, h].copy()
+            starts = list(range(0, T, chunk_len))
+            s_in = []
+            for c0 in starts:
+                c1 = min(T, c0 + chunk_len)
+                s_in.append(S.copy())
+                R, W, K, V, A, Bm = (x[bb, c0:c1, h] for x in (r, w, k, v, a, b))
+                gam = np.cumprod(W, axis=0)
+                gam_prev = np.vstack([np.ones((1, N)), gam[:-1]])
+                L = c1 - c0
+                strict = np.tril(np.ones((L, L)), -1)
+                At, Bh, Kh = A * gam_prev, Bm / gam, K / gam
+                L_ab = (At @ Bh.T) * strict
+                L_ak = (At @ Kh.T) * strict
+                U = np.linalg.solve(np.eye(L) - L_ab, At @ S.T + L_ak @ V)
+                S = (S + U.T @ Bh + V.T @ Kh) * gam[-1][None, :]
+            dS = np.zeros((N, N)) if dsT is None else _f64(dsT)[bb, h].copy()
+            for ci in range(len(starts) - 1, -1, -1):
+                c0 = starts[ci]
+                c1 = min(T, c0 + chunk_len)
+                L = c1 - c0
+                S = s_in[ci]
+                R, W, K, V, A, Bm = (x[bb, c0:c1, h] for x in (r, w, k, v, a, b))
+                dY = dy[bb, c0:c1, h]
+                # recompute the chunk
+                gam = np.cumprod(W, axis=0)
+                gam_prev = np.vstack([np.ones((1, N)), gam[:-1]])
+                strict = np.tril(np.ones((L, L)), -1)
+                incl = np.tril(np.ones((L, L)), 0)
+                At, Rt, Bh, Kh = A * gam_prev, R * gam, Bm / gam, K / gam
+                L_ab = (At @ Bh.T) * strict
+                L_ak = (At @ Kh.T) * strict
+                L_rb = (Rt @ Bh.T) * incl
+                L_rk = (Rt @ Kh.T) * incl
+                Mt = np.eye(L) - L_ab
+                U = np.linalg.solve(Mt, At @ S.T + L_ak @ V)
+                X = S + U.T @ Bh + V.T @ Kh
+                # adjoints
+                gL = gam[-1]
+                dX = dS * gL[None, :]
+                dgam = np.zeros((L, N))
+                dgam[-1] += (X * dS).sum(axis=0)
+                dU = Bh @ dX.T + L_rb.T @ dY
+                dZ = np.linalg.solve(Mt.T, dU)
+                dSin = dX + dY.T @ Rt + dZ.T @ At
+                dV = Kh @ dX.T + L_rk.T @ dY + L_ak.T @ dZ
+                dL_ab = (dZ @ U.T) * strict
+                dL_ak = (dZ @ V.T) * strict
+                dL_rb = (dY @ U.T) * incl
+                dL_rk = (dY @ V.T) * incl
+                dAt = dZ @ S + dL_ab @ Bh + dL_ak @ Kh
+                dRt = dY @ S + dL_rb @ Bh + dL_rk @ Kh
+                dBh = U @ dX + dL_ab.T @ At + dL_rb.T @ Rt
+                dKh = V @ dX + dL_ak.T @ At + dL_rk.T @ Rt
+                # decay scalings
+                da = dAt * gam_prev
+                dr = dRt * gam
+                db = dBh / gam
+                dk = dKh / gam
+                dgam += dRt * R - dBh * Bh / gam - dKh * Kh / gam
+                dgam[:-1] += (dAt * A)[1:]
+                # gamma_t = prod_{m<=t} w_m: dw_m = sum_{t>=m} dgamma_t gamma_t / w_m
+                dw = np.cumsum((dgam * gam)[::-1], axis=0)[::-1] / W
+                for g, x in zip(grads, (dr, dw, dk, dV, da, db)):
+                    g[bb, c0:c1, h] = x
+                dS = dSin
+            ds0[bb, h] = dS
+    return (*grads, ds0)

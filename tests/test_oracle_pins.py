@@ -194,6 +194,48 @@ def test_chunked_equals_sequential_full_width_long_memory():
     assert rel_err(sTc, sT) < 1e-11
 
 
+@pytest.mark.parametrize("L", [1, 5, 16, 64])
+def test_chunked_backward_equals_sequential(L):
+    """The chunk-level backward (adjoint of the chunked form, matrix products
+    per chunk) against the sequential C backward, which the central-difference
+    pins below hold to the definition.  Ragged tails, nonzero s0 and dsT."""
+    B, T, H, N = 1, 83, 2, 16
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=29)
+    rng = np.random.default_rng(31)
+    dy = rng.standard_normal((B, T, H, N))
+    dsT = rng.standard_normal((B, H, N, N))
+    ref = oracle.backward(r, w, k, v, a, b, s0, dy, dsT)
+    got = oracle.backward_chunked(r, w, k, v, a, b, s0, dy, dsT, chunk_len=L)
+    for name, g, x in zip(("dr", "dw", "dk", "dv", "da", "db", "ds0"), got, ref):
+        assert rel_err(g, x) < 1e-11, name
+
+
+CHUNKED_BWD_MUTANTS = {
+    "drop_removal_path_into_ds": ("dSin = dX + dY.T @ Rt + dZ.T @ At", "dSin = dX + dY.T @ Rt"),
+    "untransposed_solve": ("dZ = np.linalg.solve(Mt.T, dU)", "dZ = np.linalg.solve(Mt, dU)"),
+    "decay_index_shift": ("dgam[:-1] += (dAt * A)[1:]", "dgam += dAt * A"),
+    "inclusive_removal_mask": ("dL_ab = (dZ @ U.T) * strict", "dL_ab = (dZ @ U.T) * incl"),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(CHUNKED_BWD_MUTANTS))
+def test_chunked_backward_mutants_are_caught(mutant):
+    import inspect
+    src = inspect.getsource(oracle.backward_chunked)
+    old, new = CHUNKED_BWD_MUTANTS[mutant]
+    assert src.count(old) == 1, "mutation anchor not found"
+    ns = dict(np=np, _f64=oracle._f64)
+    exec(src.replace(old, new), ns)
+    B, T, H, N = 1, 19, 1, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=37)
+    rng = np.random.default_rng(41)
+    dy = rng.standard_normal((B, T, H, N))
+    dsT = rng.standard_normal((B, H, N, N))
+    ref = oracle.backward(r, w, k, v, a, b, s0, dy, dsT)
+    got = ns["backward_chunked"](r, w, k, v, a, b, s0, dy, dsT, chunk_len=8)
+    assert max(rel_err(g, x) for g, x in zip(got, ref)) > 1e-6, f"mutant {mutant} slipped through"
+
+
 def test_state_passing_split():
     B, T, H, N = 2, 37, 3, 8
     (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=23)
