@@ -130,12 +130,17 @@ WKV7_API wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dtype, wkv7_dt
                       const void *r, const void *w, const void *k, const void *v,
                       const void *a, const void *b, float *state, void *y, cudaStream_t stream);
 
-/* Bytes of scratch wkv7_backward needs (state checkpoints and recompute). */
+/* Bytes of scratch wkv7_backward needs: per (b, h), the state before every
+ * 32-token chunk, dL/dS at the end of every chunk, and the final state
+ * (fp32, 16 KiB each). */
 WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
 
 /*
  * Backward: gradients of L = sum(dy * y) + sum(dsT * sT) with respect to every
- * input and the initial state, by a reverse-time pass over recomputed states.
+ * input and the initial state.  Three launches: state checkpoints every 32
+ * tokens, a reverse sweep of the state gradient that records dL/dS at every
+ * chunk end (and ds0), then the input gradients of every chunk independently
+ * (the adjoint of the chunked form of the recurrence, in fp32).
  *   r..b, s0         : the forward's inputs (s0 NULL = zeros)
  *   dy               : [B, T, H, N] of in_dtype
  *   dsT              : [B, H, N, N] fp32, or NULL for zeros

@@ -1,0 +1,615 @@
+// Chunked WKV7 backward.
+//
+// Gradient of L = sum(dy * y) + sum(dsT * sT) for the recurrence
+//     S_t = S_{t-1} (diag(w_t) + a_t b_t^T) + v_t k_t^T,   y_t = S_t r_t
+// (RWKV-7 "Goose" with Expressive Dynamic State Evolution: the generalised
+// delta rule with vector decay; the pages give no backward, this is our own
+// reverse-mode derivation of the chunked form).
+//
+// Three launches:
+//  1. state checkpoints S_in(c) before every chunk of L = 32 tokens and the
+//     final state (the sequential forward in checkpoint mode, fwd_seq.cu);
+//  2. bwd_dstate_kernel: dS_out(c) = dL/dS at the end of every chunk, through
+//     the chunk's own outputs excluded, by a reverse sweep of the state
+//     gradient alone (per row i: g += dy_t[i] r_t; g = g w_t + (g . b_t) a_t);
+//     it needs no state and no column sums, and ends with ds0;
+//  3. bwd_chunk_kernel: one CTA per chunk, all chunks independent given
+//     S_in(c) and dS_out(c): the chunk's six input gradients by fp32 matrix
+//     products in shared memory.
+//
+// Per chunk (local t, s in [0, L), suffix decay products p_t = prod_{m>=t} w_m,
+// p_L = 1, G = p_0; all decay ratios that appear are <= 1):
+//   a'_t = a_t / p_t,  r'_t = r_t / p_{t+1},  b-_s = b_s p_{s+1},  k-_s = k_s p_{s+1}
+//   [L_ab L_ak; L_rb L_rk] = [a'; r'] [b-; k-]^T  (ab, ak strictly lower; rb, rk lower)
+//   T = (I - L_ab)^{-1},  SG = S_in diag(G)
+//   U   = T (a' SG^T + L_ak V)                        (rows u_t = S_{t-1} a_t)
+//   dU  = b- dS^T + L_rb^T dY,   dZ = T^T dU
+//   dV  = k- dS^T + L_rk^T dY + L_ak^T dZ
+//   [dL_ab dL_ak; dL_rb dL_rk] = [dZ; dY] [U; V]^T  (same masks)
+//   da = (dZ SG + dL_ab b- + dL_ak k-) / p_t
+//   dr = (dY SG + dL_rb b- + dL_rk k-) / p_{t+1}
+//   db = (U dS + dL_ab^T a' + dL_rb^T r') p_{s+1}
+//   dk = (V dS + dL_ak^T a' + dL_rk^T r') p_{s+1}
+//   q_t = dr_t r_t - db_t b_t - dk_t k_t + da_{t+1} a_{t+1} (t+1 < L)
+//         + [t = L-1] sum_i S_out[i,:] dS[i,:]
+//   dw_m = (sum_{t>=m} q_t) / w_m
+// with dS = dS_out(c).  (q_t is the derivative through the prefix decay
+// gamma_t = prod_{m<=t} w_m times gamma_t; dw_m = sum_{t>=m} dL/dgamma_t
+// gamma_t / w_m.)
+#include "common.cuh"
+
+namespace wkv7 {
+
+namespace bwdc {
+
+constexpr int L = 32;          // tokens per chunk (the checkpoint interval)
+constexpr int NT = 256;        // threads of the gradient kernel
+constexpr int LD = 68;         // row pitch (floats) of 64-wide fp32 tiles
+constexpr int LDS = 36;        // row pitch of 32-wide fp32 tiles
+constexpr float kMinDecay = 1e-30f;
+
+}  // namespace bwdc
+
+// ---------------------------------------------------------------------------
+// dS_out(c) for every chunk and ds0: reverse sweep of the state gradient.
+// One CTA of 128 threads per (b, h); thread -> 2 rows, 16 columns (four lanes
+// per row); token tiles of r w a b dy are prefetched by cp.async, 32 tokens
+// ahead.
+// ---------------------------------------------------------------------------
+template <typename InT>
+__global__ void __launch_bounds__(128)
+bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
+                  const InT *__restrict__ a, const InT *__restrict__ b, const InT *__restrict__ dy,
+                  const float *__restrict__ dsT, float *__restrict__ dS_out, float *__restrict__ ds0) {
+    constexpr int L = bwdc::L, NTEN = 5, VEC = 16 / sizeof(InT), CPV = kN / VEC;
+    extern __shared__ __align__(16) unsigned char dsmem[];
+    auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
+    const int tid = threadIdx.x, q = tid & 3, row0 = 2 * (tid >> 2);
+    const int head = blockIdx.x, bb = head / H, h = head % H;
+    const size_t tok_stride = (size_t)H * kN;
+    const size_t base = ((size_t)bb * T * H + h) * kN;
+    const int nck = (T + L - 1) / L;
+    const InT *src[NTEN] = {r, w, a, b, dy};
+
+    auto issue = [&](int c, int stage) {
+        const int t0 = c * L, Lc = min(L, T - t0);
+#pragma unroll
+        for (int ten = 0; ten < NTEN; ++ten)
+            for (int x = tid; x < L * CPV; x += 128) {
+                const int tt = x / CPV, ch = x % CPV;
+                if (tt < Lc)
+                    cp_async16(&tile[stage][ten][tt][ch * VEC], src[ten] + base + (size_t)(t0 + tt) * tok_stride + ch * VEC);
+            }
+        cp_async_commit();
+    };
+
+    float g[2][16];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q);
+            g[rr][4 * m] = d4.x; g[rr][4 * m + 1] = d4.y; g[rr][4 * m + 2] = d4.z; g[rr][4 * m + 3] = d4.w;
+        }
+    issue(nck - 1, 0);
+    for (int c = nck - 1; c >= 0; --c) {
+        const int stage = (nck - 1 - c) & 1;
+        const int t0 = c * L, Lc = min(L, T - t0);
+        cp_async_wait<0>();
+        __syncthreads();
+        if (c > 0) issue(c - 1, stage ^ 1);
+        {   // dL/dS after the chunk's last token, before its own output is added
+            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    store4(dst + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                           make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
+        }
+        for (int tt = Lc - 1; tt >= 0; --tt) {
+            const InT *rv = tile[stage][0][tt], *wv = tile[stage][1][tt], *av = tile[stage][2][tt];
+            const InT *bv = tile[stage][3][tt], *dv = tile[stage][4][tt];
+            const float dyi[2] = {to_f32(dv[row0]), to_f32(dv[row0 + 1])};
+            float dp[2] = {0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 r4 = load4(rv + 16 * m + 4 * q), b4 = load4(bv + 16 * m + 4 * q);
+                const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float gg = fmaf(dyi[rr], rj[e], g[rr][4 * m + e]);
+                        g[rr][4 * m + e] = gg;
+                        dp[rr] = fmaf(gg, bj[e], dp[rr]);
+                    }
+            }
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 1);
+                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 2);
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 w4 = load4(wv + 16 * m + 4 * q), a4 = load4(av + 16 * m + 4 * q);
+                const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        g[rr][4 * m + e] = fmaf(g[rr][4 * m + e], wj[e], dp[rr] * aj[e]);
+            }
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            store4(ds0 + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                   make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
+}
+
+// ---------------------------------------------------------------------------
+// fp32 products in shared memory for the gradient kernel (256 threads).
+// C is M x 64 (M = 64 or 32); thread tid owns rows m0 .. m0 + RM - 1
+// (RM = 4 or 2, m0 = RM * (tid >> 4)) and columns n0 .. n0 + 3 (n0 = 4 (tid & 15)).
+// B(k, n) is read row-major, B[k * ldb + n]; A(m, k) either row-major
+// (A[m * lda + k]) or column-major (A[k * lda + m], vector loads).
+// ---------------------------------------------------------------------------
+namespace bwdc {
+
+template <int M>
+struct Acc {
+    static constexpr int RM = M == 64 ? 4 : 2;
+    float c[RM][4];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < RM; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c[i][j] = 0.f;
+    }
+};
+
+template <int M, bool A_COL>
+__device__ __forceinline__ void load_a(float (&av)[Acc<M>::RM], const float *A, int lda, int k, int m0) {
+    constexpr int RM = Acc<M>::RM;
+    if constexpr (A_COL) {
+        if constexpr (RM == 4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(A + (size_t)k * lda + m0);
+            av[0] = a4.x; av[1] = a4.y; av[2] = a4.z; av[3] = a4.w;
+        } else {
+            const float2 a2 = *reinterpret_cast<const float2 *>(A + (size_t)k * lda + m0);
+            av[0] = a2.x; av[1] = a2.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < RM; ++i) av[i] = A[(size_t)(m0 + i) * lda + k];
+    }
+}
+
+// K is a multiple of 4; the operands of step k + 1 are loaded while step k
+// is multiplied
+template <int M, bool A_COL>
+__device__ __forceinline__ void mm(Acc<M> &acc, const float *A, int lda, const float *B, int ldb, int K) {
+    constexpr int RM = Acc<M>::RM;
+    const int tid = threadIdx.x;
+    const int m0 = RM * (tid >> 4), n0 = 4 * (tid & 15);
+    float4 bn = *reinterpret_cast<const float4 *>(B + n0);
+    float an[RM];
+    load_a<M, A_COL>(an, A, lda, 0, m0);
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        const float4 b4 = bn;
+        float av[RM];
+#pragma unroll
+        for (int i = 0; i < RM; ++i) av[i] = an[i];
+        if (k + 1 < K) {
+            bn = *reinterpret_cast<const float4 *>(B + (size_t)(k + 1) * ldb + n0);
+            load_a<M, A_COL>(an, A, lda, k + 1, m0);
+        }
+#pragma unroll
+        for (int i = 0; i < RM; ++i) {
+            acc.c[i][0] = fmaf(av[i], b4.x, acc.c[i][0]);
+            acc.c[i][1] = fmaf(av[i], b4.y, acc.c[i][1]);
+            acc.c[i][2] = fmaf(av[i], b4.z, acc.c[i][2]);
+            acc.c[i][3] = fmaf(av[i], b4.w, acc.c[i][3]);
+        }
+    }
+}
+
+// store the accumulator row-major (C[m * ldc + n]) or transposed (C[n * ldc + m])
+template <int M>
+__device__ __forceinline__ void put(const Acc<M> &acc, float *C, int ldc, bool transposed) {
+    constexpr int RM = Acc<M>::RM;
+    const int tid = threadIdx.x;
+    const int m0 = RM * (tid >> 4), n0 = 4 * (tid & 15);
+#pragma unroll
+    for (int i = 0; i < RM; ++i) {
+        if (!transposed) {
+            *reinterpret_cast<float4 *>(C + (size_t)(m0 + i) * ldc + n0) =
+                make_float4(acc.c[i][0], acc.c[i][1], acc.c[i][2], acc.c[i][3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) C[(size_t)(n0 + j) * ldc + m0 + i] = acc.c[i][j];
+        }
+    }
+}
+
+// shared-memory map of the gradient kernel (floats)
+constexpr int SZ64 = 64 * LD, SZ32 = 32 * LD;
+constexpr int O_AR = 0;                 // [64][LD] a' rows 0-31, r' rows 32-63 (token-major)
+constexpr int O_BKT = O_AR + SZ64;      // [64 j][LD] b- (cols 0-31), k- (cols 32-63) (channel-major)
+constexpr int O_X1 = O_BKT + SZ64;      // SG^T [j][i], then dS^T, then [b-; k-] token-major
+constexpr int O_DZY = O_X1 + SZ64;      // [64][LD] dZ rows 0-31, dY rows 32-63
+constexpr int O_UVT = O_DZY + SZ64;     // [64 i][LD] U (cols 0-31), V (cols 32-63) (channel-major)
+constexpr int O_LB = O_UVT + SZ64;      // [L_ab L_ak; L_rb L_rk], then the dL block
+constexpr int O_X2 = O_LB + SZ64;       // SG [i][j], then dS [i][j]
+constexpr int O_V = O_X2 + SZ64;        // V [s][i], then dU
+constexpr int O_Z = O_V + SZ32;         // Z, then da_{t} a_t for q
+constexpr int O_T = O_Z + SZ32;         // T [32][LDS]
+constexpr int O_ZS = O_T + 32 * LDS;    // [16][16] scratch of the inverse
+constexpr int O_P = O_ZS + 256;         // p [33][64]
+constexpr int O_RAW = O_P + 33 * kN;    // r w k a b, [5][32][64]
+constexpr int O_Q = O_RAW + 5 * L * kN; // q [32][64]
+constexpr int SMEM_FLOATS = O_Q + L * kN;
+constexpr size_t SMEM_BYTES = (size_t)SMEM_FLOATS * sizeof(float);
+
+}  // namespace bwdc
+
+// ---------------------------------------------------------------------------
+// Gradients of one chunk (one CTA per chunk, 256 threads), from S_in(c),
+// S_out(c) (the next checkpoint, or the final state) and dS_out(c).
+// ---------------------------------------------------------------------------
+template <typename InT, typename GradT>
+__global__ void __launch_bounds__(bwdc::NT, 1)
+bwd_chunk_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w, const InT *__restrict__ k,
+                 const InT *__restrict__ v, const InT *__restrict__ a, const InT *__restrict__ b,
+                 const InT *__restrict__ dy, const float *__restrict__ ckpt, const float *__restrict__ sfin,
+                 const float *__restrict__ dS_out, GradT *__restrict__ dr, GradT *__restrict__ dw,
+                 GradT *__restrict__ dk, GradT *__restrict__ dv, GradT *__restrict__ da,
+                 GradT *__restrict__ db) {
+    using namespace bwdc;
+    extern __shared__ __align__(16) unsigned char dsmem[];
+    float *sm = reinterpret_cast<float *>(dsmem);
+    const int tid = threadIdx.x;
+    const int nck = (T + L - 1) / L;
+    const int head = blockIdx.x / nck, c = blockIdx.x % nck;     // chunk-major within a head
+    const int bb = head / H, h = head % H;
+    const int t0 = c * L, Lc = min(L, T - t0);
+    const size_t tok_stride = (size_t)H * kN;
+    const size_t base = (((size_t)bb * T + t0) * H + h) * kN;       // token t0 of this head
+    const float *S_in = ckpt + ((size_t)head * nck + c) * kN * kN;
+    const float *S_out = c + 1 < nck ? ckpt + ((size_t)head * nck + c + 1) * kN * kN : sfin + (size_t)head * kN * kN;
+    const float *dSo = dS_out + ((size_t)head * nck + c) * kN * kN;
+    float *AR = sm + O_AR, *BKT = sm + O_BKT, *X1 = sm + O_X1, *DZY = sm + O_DZY, *UVT = sm + O_UVT;
+    float *LB = sm + O_LB, *X2 = sm + O_X2, *VB = sm + O_V, *ZB = sm + O_Z, *TB = sm + O_T, *ZS = sm + O_ZS;
+    float *P = sm + O_P, *RAW = sm + O_RAW, *Q = sm + O_Q;
+    auto raw = [&](int ten, int t, int j) -> float & { return RAW[(ten * L + t) * kN + j]; };   // r w k a b
+    const int m0_64 = 4 * (tid >> 4), m0_32 = 2 * (tid >> 4), n0 = 4 * (tid & 15);
+
+    // 1. every global read of the chunk is issued here: the states (thread ->
+    //    float4 u of element 4 (tid + 256 u)) stay in registers until used
+    float4 s_in[4], ds_o[4], s_ou[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int x = 4 * (tid + NT * u);
+        s_in[u] = __ldcg(reinterpret_cast<const float4 *>(S_in + x));
+        ds_o[u] = __ldcg(reinterpret_cast<const float4 *>(dSo + x));
+        s_ou[u] = __ldcg(reinterpret_cast<const float4 *>(S_out + x));
+    }
+    //    inputs of the chunk (rows past the end: no-op tokens, w = 1), four
+    //    consecutive channels per thread and pass
+    for (int x = 4 * tid; x < L * kN; x += 4 * NT) {
+        const int t = x >> 6, j = x & 63;
+        const bool ok = t < Lc;
+        const size_t g = base + (size_t)t * tok_stride + j;
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 r4 = ok ? load4(r + g) : z4, w4 = ok ? load4(w + g) : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 k4 = ok ? load4(k + g) : z4, a4 = ok ? load4(a + g) : z4, b4 = ok ? load4(b + g) : z4;
+        const float4 v4 = ok ? load4(v + g) : z4, y4 = ok ? load4(dy + g) : z4;
+        *reinterpret_cast<float4 *>(&raw(0, t, j)) = r4;
+        *reinterpret_cast<float4 *>(&raw(1, t, j)) = w4;
+        *reinterpret_cast<float4 *>(&raw(2, t, j)) = k4;
+        *reinterpret_cast<float4 *>(&raw(3, t, j)) = a4;
+        *reinterpret_cast<float4 *>(&raw(4, t, j)) = b4;
+        *reinterpret_cast<float4 *>(VB + t * LD + j) = v4;
+        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) UVT[(j + e) * LD + 32 + t] = vv[e];
+        *reinterpret_cast<float4 *>(DZY + (32 + t) * LD + j) = y4;
+    }
+    __syncthreads();
+    // 2. suffix decay products, one thread per channel
+    if (tid < kN) {
+        float pp = 1.f;
+        P[L * kN + tid] = 1.f;
+        for (int t = L - 1; t >= 0; --t) {
+            pp *= raw(1, t, tid);
+            P[t * kN + tid] = pp;
+        }
+        if (pp < kMinDecay) raise_status(WKV7_ERR_RANGE);
+    }
+    __syncthreads();
+    // 3. scaled operands, and SG^T = (S_in diag(G))^T
+    for (int x = tid; x < L * kN; x += NT) {
+        const int t = x >> 6, j = x & 63;
+        const float pt = P[t * kN + j], pn = P[(t + 1) * kN + j];
+        AR[t * LD + j] = raw(3, t, j) / pt;
+        AR[(32 + t) * LD + j] = raw(0, t, j) / pn;
+        BKT[j * LD + t] = raw(4, t, j) * pn;
+        BKT[j * LD + 32 + t] = raw(2, t, j) * pn;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int x = 4 * (tid + NT * u), i = x >> 6, j = x & 63;
+        const float sv[4] = {s_in[u].x * P[j], s_in[u].y * P[j + 1], s_in[u].z * P[j + 2], s_in[u].w * P[j + 3]};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) X1[(j + e) * LD + i] = sv[e];
+        *reinterpret_cast<float4 *>(X2 + i * LD + j) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+    }
+    __syncthreads();
+    // 4. [L_ab L_ak; L_rb L_rk] = [a'; r'] [b-; k-]^T, masked
+    {
+        Acc<64> acc;
+        acc.zero();
+        mm<64, false>(acc, AR, LD, BKT, LD, kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int m = m0_64 + i, n = n0 + jj, t = m & 31, s = n & 31;
+                if (m < 32 ? s >= t : s > t) acc.c[i][jj] = 0.f;
+            }
+        put(acc, LB, LD, false);
+    }
+    __syncthreads();
+    // 5. T = (I - L_ab)^{-1}: two 16x16 diagonal blocks by forward substitution
+    //    (one column per lane of warp 0), then T21 = T22 L21 T11
+    if (tid < 32) {
+        const int blk = tid >> 4, s = tid & 15, o = 16 * blk;
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = e == s ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+            const float x = acc[m];
+#pragma unroll
+            for (int e = m + 1; e < 16; ++e) acc[e] = fmaf(LB[(o + e) * LD + o + m], x, acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) TB[(o + e) * LDS + o + s] = acc[e];
+    } else if (tid < 64) {
+        const int s = tid & 31;
+        if (s < 16)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) TB[e * LDS + 16 + s] = 0.f;
+    }
+    __syncthreads();
+    {
+        const int t = tid >> 4, s = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = fmaf(LB[(16 + t) * LD + m], TB[m * LDS + s], acc);
+        ZS[t * 16 + s] = acc;
+    }
+    __syncthreads();
+    {
+        const int t = tid >> 4, s = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = fmaf(TB[(16 + t) * LDS + 16 + m], ZS[m * 16 + s], acc);
+        TB[(16 + t) * LDS + s] = acc;
+    }
+    __syncthreads();
+    // 6. Z = a' SG^T + L_ak V
+    {
+        Acc<32> acc;
+        acc.zero();
+        mm<32, false>(acc, AR, LD, X1, LD, kN);
+        mm<32, false>(acc, LB + 32, LD, VB, LD, L);
+        put(acc, ZB, LD, false);
+    }
+    __syncthreads();
+    // 7. U = T Z, stored channel-major next to V;  dS^T replaces SG^T
+    {
+        Acc<32> acc;
+        acc.zero();
+        mm<32, false>(acc, TB, LDS, ZB, LD, L);
+        put(acc, UVT, LD, true);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int x = 4 * (tid + NT * u), i = x >> 6, j = x & 63;
+        X1[j * LD + i] = ds_o[u].x;
+        X1[(j + 1) * LD + i] = ds_o[u].y;
+        X1[(j + 2) * LD + i] = ds_o[u].z;
+        X1[(j + 3) * LD + i] = ds_o[u].w;
+    }
+    __syncthreads();
+    // 8. dU = b- dS^T + L_rb^T dY  (into VB)
+    {
+        Acc<32> acc;
+        acc.zero();
+        mm<32, true>(acc, BKT, LD, X1, LD, kN);
+        mm<32, true>(acc, LB + 32 * LD, LD, DZY + 32 * LD, LD, L);
+        put(acc, VB, LD, false);
+    }
+    __syncthreads();
+    // 9. dZ = T^T dU  (into DZY rows 0-31)
+    {
+        Acc<32> acc;
+        acc.zero();
+        mm<32, true>(acc, TB, LDS, VB, LD, L);
+        put(acc, DZY, LD, false);
+    }
+    __syncthreads();
+    // 10. dV = k- dS^T + L_rk^T dY + L_ak^T dZ  -> dv
+    {
+        Acc<32> acc;
+        acc.zero();
+        mm<32, true>(acc, BKT + 32, LD, X1, LD, kN);
+        mm<32, true>(acc, LB + 32 * LD + 32, LD, DZY + 32 * LD, LD, L);
+        mm<32, true>(acc, LB + 32, LD, DZY, LD, L);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int s = m0_32 + i;
+            if (s < Lc)
+                store4(dv + base + (size_t)s * tok_stride + n0,
+                       make_float4(acc.c[i][0], acc.c[i][1], acc.c[i][2], acc.c[i][3]));
+        }
+    }
+    __syncthreads();
+    // 11. [dL_ab dL_ak; dL_rb dL_rk] = [dZ; dY] [U; V]^T, masked (into LB)
+    {
+        Acc<64> acc;
+        acc.zero();
+        mm<64, false>(acc, DZY, LD, UVT, LD, kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int m = m0_64 + i, n = n0 + jj, t = m & 31, s = n & 31;
+                if (m < 32 ? s >= t : s > t) acc.c[i][jj] = 0.f;
+            }
+        put(acc, LB, LD, false);   // the L block was last read in step 10
+    }
+    // 12. [b-; k-] token-major (X1); SG is already in X2
+    for (int x = tid; x < kN * kN; x += NT) {
+        const int i = x >> 6, j = x & 63;
+        X1[i * LD + j] = BKT[j * LD + i];
+    }
+    __syncthreads();
+    // 13. da, dr: [dZ; dY] SG + dL [b-; k-], then the decay factors; q terms
+    {
+        Acc<64> acc;
+        acc.zero();
+        mm<64, false>(acc, DZY, LD, X2, LD, kN);
+        mm<64, false>(acc, LB, LD, X1, LD, kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = m0_64 + i, t = m & 31;
+            float o[4];
+            if (m < 32) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    o[jj] = acc.c[i][jj] / P[t * kN + n0 + jj];
+                    ZB[t * LD + n0 + jj] = o[jj] * raw(3, t, n0 + jj);
+                }
+                if (t < Lc) store4(da + base + (size_t)t * tok_stride + n0, make_float4(o[0], o[1], o[2], o[3]));
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    o[jj] = acc.c[i][jj] / P[(t + 1) * kN + n0 + jj];
+                    Q[t * kN + n0 + jj] = o[jj] * raw(0, t, n0 + jj);
+                }
+                if (t < Lc) store4(dr + base + (size_t)t * tok_stride + n0, make_float4(o[0], o[1], o[2], o[3]));
+            }
+        }
+    }
+    __syncthreads();
+    // 14. dS row-major (X2)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int x = 4 * (tid + NT * u), i = x >> 6, j = x & 63;
+        *reinterpret_cast<float4 *>(X2 + i * LD + j) = ds_o[u];
+    }
+    __syncthreads();
+    // 15. db, dk: [U; V] dS + dL^T [a'; r'], times p_{s+1}; q terms
+    {
+        Acc<64> acc;
+        acc.zero();
+        mm<64, true>(acc, UVT, LD, X2, LD, kN);
+        mm<64, true>(acc, LB, LD, AR, LD, kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = m0_64 + i, s = m & 31;
+            const int ten = m < 32 ? 4 : 2;   // b or k
+            float o[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                o[jj] = acc.c[i][jj] * P[(s + 1) * kN + n0 + jj];
+                atomicAdd(&Q[s * kN + n0 + jj], -o[jj] * raw(ten, s, n0 + jj));
+            }
+            if (s < Lc) store4((m < 32 ? db : dk) + base + (size_t)s * tok_stride + n0, make_float4(o[0], o[1], o[2], o[3]));
+        }
+    }
+    // 16. the last token's decay also scales S_out: q_{Lc-1} += sum_i S_out dS.
+    //     A thread's four float4 share columns 4 (tid & 15) .. +3; lanes l and
+    //     l + 16 too: sum those first, then one atomic per column and warp.
+    {
+        float cs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            cs[0] = fmaf(s_ou[u].x, ds_o[u].x, cs[0]);
+            cs[1] = fmaf(s_ou[u].y, ds_o[u].y, cs[1]);
+            cs[2] = fmaf(s_ou[u].z, ds_o[u].z, cs[2]);
+            cs[3] = fmaf(s_ou[u].w, ds_o[u].w, cs[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 16);
+        if ((tid & 31) < 16) {
+            float *qr = Q + (Lc - 1) * kN + 4 * (tid & 15);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) atomicAdd(qr + e, cs[e]);
+        }
+    }
+    __syncthreads();
+    // 17. dw_m = sum_{t >= m} q_t / w_m,  q_t = Q_t + da_{t+1} a_{t+1}
+    if (tid < kN) {
+        const int j = tid;
+        float run = 0.f;
+        for (int t = Lc - 1; t >= 0; --t) {
+            run += Q[t * kN + j] + (t + 1 < Lc ? ZB[(t + 1) * LD + j] : 0.f);
+            dw[base + (size_t)t * tok_stride + j] = from_f32<GradT>(run / raw(1, t, j));
+        }
+    }
+}
+
+size_t bwd_chunk_ckpt_bytes(int B, int T, int H) {
+    const size_t nck = ((size_t)T + bwdc::L - 1) / bwdc::L;
+    return (size_t)B * H * nck * kN * kN * sizeof(float);
+}
+
+cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
+                        const void *k, const void *v, const void *a, const void *b, const void *dy,
+                        const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st) {
+    using namespace bwdc;
+    const int heads = B * H, nck = (T + L - 1) / L;
+    {   // dS at every chunk end, and ds0
+        const size_t smem = 2 * 5 * L * kN * (in_dt == WKV7_F32 ? 4 : 2);
+#define WKV7_DSTATE(I)                                                                                    \
+    do {                                                                                                  \
+        auto kern = bwd_dstate_kernel<I>;                                                                 \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+        if (e != cudaSuccess) return e;                                                                   \
+        kern<<<heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a, (const I *)b,     \
+                                       (const I *)dy, dsT, dS_out, ds0);                                 \
+    } while (0)
+        if (in_dt == WKV7_F32) WKV7_DSTATE(float);
+        else WKV7_DSTATE(__nv_bfloat16);
+#undef WKV7_DSTATE
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const dim3 grid((unsigned)((size_t)heads * nck));
+#define WKV7_CHUNK_BWD(I, G)                                                                                 \
+    do {                                                                                                     \
+        auto kern = bwd_chunk_kernel<I, G>;                                                                  \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES); \
+        if (e != cudaSuccess) return e;                                                                      \
+        kern<<<grid, NT, SMEM_BYTES, st>>>(T, H, (const I *)r, (const I *)w, (const I *)k, (const I *)v,    \
+                                           (const I *)a, (const I *)b, (const I *)dy, ckpt, sfin, dS_out,  \
+                                           (G *)dr, (G *)dw, (G *)dk, (G *)dv, (G *)da, (G *)db);           \
+    } while (0)
+    if (in_dt == WKV7_F32 && g_dt == WKV7_F32) WKV7_CHUNK_BWD(float, float);
+    else if (in_dt == WKV7_F32) WKV7_CHUNK_BWD(float, __nv_bfloat16);
+    else if (g_dt == WKV7_F32) WKV7_CHUNK_BWD(__nv_bfloat16, float);
+    else WKV7_CHUNK_BWD(__nv_bfloat16, __nv_bfloat16);
+#undef WKV7_CHUNK_BWD
+    return cudaGetLastError();
+}
+
+}  // namespace wkv7

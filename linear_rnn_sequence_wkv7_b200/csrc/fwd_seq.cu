@@ -224,15 +224,16 @@ cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, cons
     return launch_fwd_seq<__nv_bfloat16, __nv_bfloat16, RPT, RB, TT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
 }
 
-// State checkpoints every CK tokens (CK a multiple of 16): ckpt[b][h][c] holds
+// State checkpoints every CK tokens (CK a multiple of 16), and the final state
+// when sT is given: ckpt[b][h][c] holds
 // the state before token c * CK.  Used by the backward's first pass.
 cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
                             const void *k, const void *v, const void *a, const void *b, const float *s0,
-                            float *ckpt, int CK, cudaStream_t st) {
+                            float *ckpt, int CK, float *sT, cudaStream_t st) {
     constexpr int RPT = 2, RB = 32, TT = 16;
     if (in_dt == WKV7_F32)
-        return launch_fwd_seq<float, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, nullptr, ckpt, CK, st);
-    return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, nullptr, ckpt, CK, st);
+        return launch_fwd_seq<float, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
+    return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
 }
 
 }  // namespace wkv7

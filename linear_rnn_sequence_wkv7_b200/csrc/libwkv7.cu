@@ -4,6 +4,6 @@
 #include "wkv7_api.cu"
 #include "fwd_seq.cu"
 #include "step.cu"
-#include "bwd_seq.cu"
+#include "bwd_chunk.cu"
 #include "fwd_chunk.cu"
 #include "bwd_noalloc.cu"

@@ -16,15 +16,15 @@ cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, cons
                     const float *s0, void *y, float *sT, cudaStream_t st);
 cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
                             const void *k, const void *v, const void *a, const void *b, const float *s0,
-                            float *ckpt, int CK, cudaStream_t st);
+                            float *ckpt, int CK, float *sT, cudaStream_t st);
 cudaError_t step(int B, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                  const void *k, const void *v, const void *a, const void *b, float *state, void *y,
                  cudaStream_t st);
-cudaError_t bwd_seq(int B, int T, int H, int CK, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
-                    const void *w, const void *k, const void *v, const void *a, const void *b,
-                    const void *dy, const float *dsT, const float *ckpt, float *hist, void *dr, void *dw,
-                    void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st);
-size_t bwd_hist_bytes(int B, int H, int CK);
+cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
+                        const void *k, const void *v, const void *a, const void *b, const void *dy,
+                        const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st);
+size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st);
@@ -33,7 +33,7 @@ size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
 
 namespace {
 
-constexpr int kBwdChunk = 16;        // backward checkpoint interval (tokens)
+constexpr int kBwdChunk = 32;        // backward chunk (= checkpoint interval, tokens)
 constexpr long long kDefaultWaitCycles = 2000000000LL;   // ~1 s of SM clock
 std::atomic<long long> g_wait_limit{0};                  // 0 = default
 constexpr size_t kWsAlign = 256;
@@ -79,10 +79,8 @@ int current_sm_count() {
     return n;
 }
 
-size_t bwd_ckpt_bytes(int B, int T, int H) {
-    const size_t nck = ((size_t)T + kBwdChunk - 1) / kBwdChunk;
-    return (size_t)B * H * nck * kN * kN * sizeof(float);
-}
+size_t bwd_ckpt_bytes(int B, int T, int H) { return bwd_chunk_ckpt_bytes(B, T, H); }
+size_t state_bytes(int B, int H) { return (size_t)B * H * kN * kN * sizeof(float); }
 
 }  // namespace
 }  // namespace wkv7
@@ -169,7 +167,8 @@ wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, co
 
 size_t wkv7_backward_workspace_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
-    return round_up(bwd_ckpt_bytes(B, T, H)) + round_up(bwd_hist_bytes(B, H, kBwdChunk));
+    // state before every chunk, the final state, dL/dS at every chunk end
+    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
 }
 
 wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
@@ -188,12 +187,14 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
         if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
     const size_t need = wkv7_backward_workspace_size(B, T, H, N);
     if (workspace_bytes < need || !ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
-    float *ckpt = static_cast<float *>(workspace);
-    float *hist = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(bwd_ckpt_bytes(B, T, H)));
-    cudaError_t e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, stream);
+    char *ws = static_cast<char *>(workspace);
+    float *ckpt = reinterpret_cast<float *>(ws);
+    float *dSo = reinterpret_cast<float *>(ws + round_up(bwd_ckpt_bytes(B, T, H)));
+    float *sfin = reinterpret_cast<float *>(ws + 2 * round_up(bwd_ckpt_bytes(B, T, H)));
+    cudaError_t e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
-    return from_cuda(bwd_seq(B, T, H, kBwdChunk, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, hist, dr, dw,
-                             dk, dv, da, db, ds0, stream));
+    return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
+                                 dv, da, db, ds0, stream));
 }
 
 void wkv7_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }

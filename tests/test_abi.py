@@ -48,8 +48,8 @@ def test_version_and_status_strings(lib):
 def test_workspace_sizes(lib):
     assert lib.wkv7_forward_workspace_size(1, 64, 2, 64, wkv7.F32, wkv7.ALGO_SEQ, 0) == 0
     ws = lib.wkv7_backward_workspace_size(8, 4096, 32, 64)
-    # checkpoints every 16 tokens plus a 16-token recompute history per head
-    assert ws >= 8 * 32 * (4096 // 16) * 64 * 64 * 4 + 8 * 32 * 16 * 64 * 64 * 4
+    # per head: the state before every 32-token chunk, dL/dS at every chunk end, the final state
+    assert ws >= 8 * 32 * (2 * (4096 // 32) + 1) * 64 * 64 * 4
     assert lib.wkv7_backward_workspace_size(0, 10, 1, 64) == 0
 
 
