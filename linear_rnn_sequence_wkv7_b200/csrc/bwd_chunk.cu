@@ -12,7 +12,8 @@
 //  2. bwd_dstate_kernel: dS_out(c) = dL/dS at the end of every chunk, through
 //     the chunk's own outputs excluded, by a reverse sweep of the state
 //     gradient alone (per row i: g += dy_t[i] r_t; g = g w_t + (g . b_t) a_t);
-//     it needs no state and no column sums, and ends with ds0;
+//     it needs no state and no column sums (rows are independent, two CTAs
+//     per head), and ends with ds0;
 //  3. bwd_chunk_kernel: one CTA per chunk, all chunks independent given
 //     S_in(c) and dS_out(c): the chunk's six input gradients by fp32 matrix
 //     products in shared memory.
@@ -52,9 +53,10 @@ constexpr float kMinDecay = 1e-30f;
 
 // ---------------------------------------------------------------------------
 // dS_out(c) for every chunk and ds0: reverse sweep of the state gradient.
-// One CTA of 128 threads per (b, h); thread -> 2 rows, 16 columns (four lanes
-// per row); token tiles of r w a b dy are prefetched by cp.async, 32 tokens
-// ahead.
+// The rows of dS evolve independently, so two CTAs of 128 threads share a
+// (b, h): CTA half q owns rows 32 q .. 32 q + 31, thread -> 1 row, 16 columns
+// (four lanes per row).  Token tiles of r w a b dy are prefetched by
+// cp.async, 32 tokens ahead.
 // ---------------------------------------------------------------------------
 template <typename InT>
 __global__ void __launch_bounds__(128)
@@ -64,8 +66,9 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
     constexpr int L = bwdc::L, NTEN = 5, VEC = 16 / sizeof(InT), CPV = kN / VEC;
     extern __shared__ __align__(16) unsigned char dsmem[];
     auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
-    const int tid = threadIdx.x, q = tid & 3, row0 = 2 * (tid >> 2);
-    const int head = blockIdx.x, bb = head / H, h = head % H;
+    const int tid = threadIdx.x, q = tid & 3;
+    const int head = blockIdx.x >> 1, row = 32 * (blockIdx.x & 1) + (tid >> 2);
+    const int bb = head / H, h = head % H;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
     const int nck = (T + L - 1) / L;
@@ -83,15 +86,13 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         cp_async_commit();
     };
 
-    float g[2][16];
+    float g[16];
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q);
-            g[rr][4 * m] = d4.x; g[rr][4 * m + 1] = d4.y; g[rr][4 * m + 2] = d4.z; g[rr][4 * m + 3] = d4.w;
-        }
+    for (int m = 0; m < 4; ++m) {
+        float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)row * kN + 16 * m + 4 * q);
+        g[4 * m] = d4.x; g[4 * m + 1] = d4.y; g[4 * m + 2] = d4.z; g[4 * m + 3] = d4.w;
+    }
     issue(nck - 1, 0);
     for (int c = nck - 1; c >= 0; --c) {
         const int stage = (nck - 1 - c) & 1;
@@ -100,55 +101,43 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         __syncthreads();
         if (c > 0) issue(c - 1, stage ^ 1);
         {   // dL/dS after the chunk's last token, before its own output is added
-            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN;
+            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN + (size_t)row * kN + 4 * q;
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    store4(dst + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
-                           make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
+            for (int m = 0; m < 4; ++m)
+                store4(dst + 16 * m, make_float4(g[4 * m], g[4 * m + 1], g[4 * m + 2], g[4 * m + 3]));
         }
         for (int tt = Lc - 1; tt >= 0; --tt) {
             const InT *rv = tile[stage][0][tt], *wv = tile[stage][1][tt], *av = tile[stage][2][tt];
-            const InT *bv = tile[stage][3][tt], *dv = tile[stage][4][tt];
-            const float dyi[2] = {to_f32(dv[row0]), to_f32(dv[row0 + 1])};
-            float dp[2] = {0.f, 0.f};
+            const InT *bv = tile[stage][3][tt];
+            const float dyi = to_f32(tile[stage][4][tt][row]);
+            float dp4[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums: a shorter dependency chain
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 r4 = load4(rv + 16 * m + 4 * q), b4 = load4(bv + 16 * m + 4 * q);
                 const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float gg = fmaf(dyi[rr], rj[e], g[rr][4 * m + e]);
-                        g[rr][4 * m + e] = gg;
-                        dp[rr] = fmaf(gg, bj[e], dp[rr]);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float gg = fmaf(dyi, rj[e], g[4 * m + e]);
+                    g[4 * m + e] = gg;
+                    dp4[e] = fmaf(gg, bj[e], dp4[e]);
+                }
             }
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 1);
-                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 2);
-            }
+            float dp = (dp4[0] + dp4[1]) + (dp4[2] + dp4[3]);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 2);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 w4 = load4(wv + 16 * m + 4 * q), a4 = load4(av + 16 * m + 4 * q);
                 const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        g[rr][4 * m + e] = fmaf(g[rr][4 * m + e], wj[e], dp[rr] * aj[e]);
+                for (int e = 0; e < 4; ++e) g[4 * m + e] = fmaf(g[4 * m + e], wj[e], dp * aj[e]);
             }
         }
     }
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            store4(ds0 + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
-                   make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
+    for (int m = 0; m < 4; ++m)
+        store4(ds0 + (size_t)head * kN * kN + (size_t)row * kN + 16 * m + 4 * q,
+               make_float4(g[4 * m], g[4 * m + 1], g[4 * m + 2], g[4 * m + 3]));
 }
 
 // ---------------------------------------------------------------------------
@@ -585,7 +574,7 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
         auto kern = bwd_dstate_kernel<I>;                                                                 \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         if (e != cudaSuccess) return e;                                                                   \
-        kern<<<heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a, (const I *)b,     \
+        kern<<<2 * heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a, (const I *)b, \
                                        (const I *)dy, dsT, dS_out, ds0);                                 \
     } while (0)
         if (in_dt == WKV7_F32) WKV7_DSTATE(float);

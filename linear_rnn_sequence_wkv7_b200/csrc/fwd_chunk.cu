@@ -122,7 +122,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                  const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
-                 float *sT, long long sT_zstride, int st_only_z, long long wait_limit) {
+                 float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -143,6 +143,9 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     float *sTp = (sT && (st_only_z < 0 || st_only_z == z)) ? sT + (st_only_z < 0 ? (size_t)z * sT_zstride : 0) + st_base
                                                             : nullptr;
     const int nchunks = (T + L - 1) / L;
+    // optional state checkpoints (one-segment runs): the state before every
+    // chunk, [B][H][nchunks][64][64]
+    float *ckp = ckpt ? ckpt + ((size_t)bb * H + h) * nchunks * kN * kN : nullptr;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
     int last_k = -1;                                 // issuer: last committed round and its parity
     uint32_t last_par = 0;
@@ -201,6 +204,10 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         }
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part, 64), x);
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part + 8, 64), x + 8);
+        if (ckp) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ckp[(size_t)(16 * part + e) * kN + j] = x[e];
+        }
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_before_sync();
@@ -552,6 +559,11 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
                     for (int e = 0; e < 32; ++e) sTp[(size_t)(32 * hc + e) * kN + rho] = x[e];
                 }
+                if (ckp != nullptr && c + 1 < nchunks) {
+                    float *dst = ckp + (size_t)(c + 1) * kN * kN + rho;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dst[(size_t)(32 * hc + e) * kN] = x[e];
+                }
             } else if (y) {                       // y row t, channels 32 hc .. 32 hc + 31
                 const int t = rho - 64;
                 if (t < Lv) {
@@ -615,7 +627,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz, wkv7_dtype y_dt, const void *r,
                                 const void *w, const void *k, const void *v, const void *a, const void *b,
                                 const float *s0, long long s0_zstride, void *y, float *sT, long long sT_zstride,
-                                int st_only_z, long long wait_limit, cudaStream_t st) {
+                                int st_only_z, long long wait_limit, cudaStream_t st, float *ckpt = nullptr) {
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES;
 #define WKV7_CHUNK_LAUNCH(O)                                                                                  \
@@ -626,7 +638,7 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
-                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit);                   \
+                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt);             \
     } while (0)
     if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
     else WKV7_CHUNK_LAUNCH(__nv_bfloat16);
@@ -715,6 +727,15 @@ size_t chunk_workspace_bytes(int B, int T, int H, int nseg) {
     if (nseg <= 1) return 0;
     // E_k, M_k for segments 0..nseg-2 and S_in(k) for k < nseg
     return (size_t)(2 * (nseg - 1) + nseg) * B * H * kN * kN * sizeof(float);
+}
+
+// State checkpoints before every 32-token chunk (and the final state) for the
+// backward: one pass of the chunked kernel without y.
+cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
+                                  const void *a, const void *b, const float *s0, float *ckpt, float *sT,
+                                  long long wait_limit, cudaStream_t st) {
+    return launch_chunk(B, T, H, T, 1, 1, WKV7_BF16, r, w, k, v, a, b, s0, 0, nullptr, sT, 0, -1, wait_limit, st,
+                        ckpt);
 }
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,

@@ -29,6 +29,9 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st);
 int chunk_segments(int B, int T, int H, int sm_count);
+cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
+                                  const void *a, const void *b, const float *s0, float *ckpt, float *sT,
+                                  long long wait_limit, cudaStream_t st);
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
 
 namespace {
@@ -191,7 +194,13 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     float *ckpt = reinterpret_cast<float *>(ws);
     float *dSo = reinterpret_cast<float *>(ws + round_up(bwd_ckpt_bytes(B, T, H)));
     float *sfin = reinterpret_cast<float *>(ws + 2 * round_up(bwd_ckpt_bytes(B, T, H)));
-    cudaError_t e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
+    // checkpoints: the chunked tensor-core forward for bf16 inputs (its chunk
+    // is the backward's), the sequential scan for fp32 inputs
+    const long long lim = g_wait_limit.load();
+    cudaError_t e = in_dt == WKV7_BF16
+                        ? fwd_chunk_checkpoints(B, T, H, r, w, k, v, a, b, s0, ckpt, sfin,
+                                                lim > 0 ? lim : kDefaultWaitCycles, stream)
+                        : fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
                                  dv, da, db, ds0, stream));
