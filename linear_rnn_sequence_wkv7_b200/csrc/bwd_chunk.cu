@@ -53,12 +53,13 @@ constexpr float kMinDecay = 1e-30f;
 
 // ---------------------------------------------------------------------------
 // dS_out(c) for every chunk and ds0: reverse sweep of the state gradient.
-// The rows of dS evolve independently, so two CTAs of 128 threads share a
-// (b, h): CTA half q owns rows 32 q .. 32 q + 31, thread -> 1 row, 16 columns
-// (four lanes per row).  Token tiles of r w a b dy are prefetched by
-// cp.async, 32 tokens ahead.
+// The rows of dS evolve independently.  CTAs of 128 threads, four lanes per
+// row (16 columns each) and RPT rows per thread: RPT = 2 covers a (b, h) with
+// one CTA; RPT = 1 splits it over two CTAs (rows 32 q .. 32 q + 31), for
+// problems with too few heads to fill the GPU.  Token tiles of r w a b dy are
+// prefetched by cp.async, 32 tokens ahead.
 // ---------------------------------------------------------------------------
-template <typename InT>
+template <typename InT, int RPT>
 __global__ void __launch_bounds__(128)
 bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
                   const InT *__restrict__ a, const InT *__restrict__ b, const InT *__restrict__ dy,
@@ -66,8 +67,10 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
     constexpr int L = bwdc::L, NTEN = 5, VEC = 16 / sizeof(InT), CPV = kN / VEC;
     extern __shared__ __align__(16) unsigned char dsmem[];
     auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
+    constexpr int SPLIT = 2 / RPT;     // CTAs per head
     const int tid = threadIdx.x, q = tid & 3;
-    const int head = blockIdx.x >> 1, row = 32 * (blockIdx.x & 1) + (tid >> 2);
+    const int head = blockIdx.x / SPLIT;
+    const int row0 = 32 * (blockIdx.x % SPLIT) * (SPLIT - 1) + RPT * (tid >> 2);
     const int bb = head / H, h = head % H;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
@@ -86,13 +89,15 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         cp_async_commit();
     };
 
-    float g[16];
+    float g[RPT][16];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)row * kN + 16 * m + 4 * q);
-        g[4 * m] = d4.x; g[4 * m + 1] = d4.y; g[4 * m + 2] = d4.z; g[4 * m + 3] = d4.w;
-    }
+    for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q);
+            g[rr][4 * m] = d4.x; g[rr][4 * m + 1] = d4.y; g[rr][4 * m + 2] = d4.z; g[rr][4 * m + 3] = d4.w;
+        }
     issue(nck - 1, 0);
     for (int c = nck - 1; c >= 0; --c) {
         const int stage = (nck - 1 - c) & 1;
@@ -101,43 +106,61 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         __syncthreads();
         if (c > 0) issue(c - 1, stage ^ 1);
         {   // dL/dS after the chunk's last token, before its own output is added
-            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN + (size_t)row * kN + 4 * q;
+            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN + (size_t)row0 * kN + 4 * q;
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-                store4(dst + 16 * m, make_float4(g[4 * m], g[4 * m + 1], g[4 * m + 2], g[4 * m + 3]));
+            for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    store4(dst + (size_t)rr * kN + 16 * m,
+                           make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
         }
         for (int tt = Lc - 1; tt >= 0; --tt) {
             const InT *rv = tile[stage][0][tt], *wv = tile[stage][1][tt], *av = tile[stage][2][tt];
             const InT *bv = tile[stage][3][tt];
-            const float dyi = to_f32(tile[stage][4][tt][row]);
-            float dp4[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums: a shorter dependency chain
+            float dyi[RPT], dp4[RPT][4];   // four partial sums per row: a shorter dependency chain
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) {
+                dyi[rr] = to_f32(tile[stage][4][tt][row0 + rr]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dp4[rr][e] = 0.f;
+            }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 r4 = load4(rv + 16 * m + 4 * q), b4 = load4(bv + 16 * m + 4 * q);
                 const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float gg = fmaf(dyi, rj[e], g[4 * m + e]);
-                    g[4 * m + e] = gg;
-                    dp4[e] = fmaf(gg, bj[e], dp4[e]);
-                }
+                for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float gg = fmaf(dyi[rr], rj[e], g[rr][4 * m + e]);
+                        g[rr][4 * m + e] = gg;
+                        dp4[rr][e] = fmaf(gg, bj[e], dp4[rr][e]);
+                    }
             }
-            float dp = (dp4[0] + dp4[1]) + (dp4[2] + dp4[3]);
-            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
-            dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+            float dp[RPT];
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) {
+                dp[rr] = (dp4[rr][0] + dp4[rr][1]) + (dp4[rr][2] + dp4[rr][3]);
+                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 1);
+                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 2);
+            }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 w4 = load4(wv + 16 * m + 4 * q), a4 = load4(av + 16 * m + 4 * q);
                 const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) g[4 * m + e] = fmaf(g[4 * m + e], wj[e], dp * aj[e]);
+                for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) g[rr][4 * m + e] = fmaf(g[rr][4 * m + e], wj[e], dp[rr] * aj[e]);
             }
         }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-        store4(ds0 + (size_t)head * kN * kN + (size_t)row * kN + 16 * m + 4 * q,
-               make_float4(g[4 * m], g[4 * m + 1], g[4 * m + 2], g[4 * m + 3]));
+    for (int rr = 0; rr < RPT; ++rr)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            store4(ds0 + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                   make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
 }
 
 // ---------------------------------------------------------------------------
@@ -567,18 +590,25 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
                         void *dw, void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st) {
     using namespace bwdc;
     const int heads = B * H, nck = (T + L - 1) / L;
-    {   // dS at every chunk end, and ds0
+    {   // dS at every chunk end, and ds0; split rows over two CTAs when the
+        // heads alone leave SMs idle (measured: 1.45 vs 1.67 ms at 256 heads)
         const size_t smem = 2 * 5 * L * kN * (in_dt == WKV7_F32 ? 4 : 2);
-#define WKV7_DSTATE(I)                                                                                    \
+        const bool split = heads <= 148;
+#define WKV7_DSTATE(I, R)                                                                                 \
     do {                                                                                                  \
-        auto kern = bwd_dstate_kernel<I>;                                                                 \
+        auto kern = bwd_dstate_kernel<I, R>;                                                              \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         if (e != cudaSuccess) return e;                                                                   \
-        kern<<<2 * heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a, (const I *)b, \
-                                       (const I *)dy, dsT, dS_out, ds0);                                 \
+        kern<<<(2 / R) * heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a,          \
+                                                 (const I *)b, (const I *)dy, dsT, dS_out, ds0);          \
     } while (0)
-        if (in_dt == WKV7_F32) WKV7_DSTATE(float);
-        else WKV7_DSTATE(__nv_bfloat16);
+        if (in_dt == WKV7_F32) {
+            if (split) WKV7_DSTATE(float, 1);
+            else WKV7_DSTATE(float, 2);
+        } else {
+            if (split) WKV7_DSTATE(__nv_bfloat16, 1);
+            else WKV7_DSTATE(__nv_bfloat16, 2);
+        }
 #undef WKV7_DSTATE
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
