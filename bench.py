@@ -332,9 +332,10 @@ def bench_backward(args, dist, peaks, device, d):
     ach = bwd_flops(B, T, H) / per / 1e12
     return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
             "ms_per_step": per * 1e3,
-            "steps": steps, "launches": 2 * steps,
+            "steps": steps, "launches": 3 * steps,
             "roofline": {"bound": "alu", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                          "per_unit": "28*N^2 flop per head-token",
+                         "kernels": "checkpoints (chunked forward), dS chain, per-chunk gradients (fp32)",
                          "hbm_frac": bwd_bytes(B, T, H) / per / 1e9 / peaks["hbm_gbs"]},
             "config": {"workload": "train_bwd_b8_t4096_h32", "B": B, "T": T, "H": H, "N": N,
                        "grad_dtype": "bf16", "dsT": "zero"}}
