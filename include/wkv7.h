@@ -66,7 +66,7 @@ typedef enum {
 typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1 } wkv7_dtype;
 
 typedef enum {
-    WKV7_ALGO_AUTO = 0,   /* library picks: CHUNK for bf16 inputs when T >= 2 * chunk, else SEQ */
+    WKV7_ALGO_AUTO = 0,   /* library picks: CHUNK for bf16 inputs when T >= 64, else SEQ */
     WKV7_ALGO_SEQ = 1,    /* token-by-token scan, state kept on chip            */
     WKV7_ALGO_CHUNK = 2   /* chunked (parallel-in-time) form on tensor cores    */
 } wkv7_algo;
@@ -98,11 +98,11 @@ WKV7_API size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dty
  *   sT               : [B, H, N, N] fp32 final state, or NULL to skip.
  *                      sT may alias s0 (in-place continuation); no other
  *                      output may alias an input.
- *   algo, chunk_len  : algorithm choice; chunk_len 0 means 64 (the only
+ *   algo, chunk_len  : algorithm choice; chunk_len 0 means 32 (the only
  *                      length the chunked form implements).
  *   workspace        : wkv7_forward_workspace_size() bytes, or NULL if 0.
  * The chunked form needs the per-chunk decay product of every channel to stay
- * in fp32's normal range (prod of 64 consecutive w >= 1e-30); a chunk outside
+ * in fp32's normal range (prod of 32 consecutive w >= 1e-30); a chunk outside
  * it raises WKV7_ERR_RANGE in the device status word (wkv7_get_device_status)
  * and its outputs are unspecified.  The SEQ form has no such limit.
  */

@@ -125,7 +125,7 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
     if (algo != WKV7_ALGO_AUTO && algo != WKV7_ALGO_SEQ && algo != WKV7_ALGO_CHUNK) return WKV7_ERR_INVALID_ARG;
-    if (chunk_len != 0 && chunk_len != 64) return WKV7_ERR_UNSUPPORTED;
+    if (chunk_len != 0 && chunk_len != 32) return WKV7_ERR_UNSUPPORTED;   // the chunked form's chunk
     if (!opt_ptr_ok(s0) || !opt_ptr_ok(sT)) return WKV7_ERR_INVALID_ARG;
     if ((size_t)B * H == 0) return WKV7_OK;
     if (T == 0) return copy_or_zero_state(sT, s0, B, H, stream);

@@ -67,7 +67,7 @@ def test_forward_rejects_invalid_arguments(lib):
     assert _fwd(lib, T=-3) == wkv7.ERR_INVALID_ARG
     assert _fwd(lib, in_dt=7) == wkv7.ERR_INVALID_ARG
     assert _fwd(lib, algo=9) == wkv7.ERR_INVALID_ARG
-    assert _fwd(lib, chunk=32) == wkv7.ERR_UNSUPPORTED
+    assert _fwd(lib, chunk=64) == wkv7.ERR_UNSUPPORTED     # the chunked form's chunk is 32
     bad = [P] * 9
     bad[0] = None                                    # r missing
     assert _fwd(lib, ptrs=bad) == wkv7.ERR_INVALID_ARG
