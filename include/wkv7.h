@@ -113,6 +113,75 @@ WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dtyp
                          cudaStream_t stream);
 
 /*
+ * Sequence (context) parallel forward, in three calls around an exchange.
+ * The recurrence is affine in the state (the transition diag(w_t) + a_t b_t^T
+ * does not depend on S: RWKV-7 "Goose" paper review, section "Architecture"),
+ * so a stretch of T tokens maps its entry state to its final state as
+ *     S_out = S_in M + E,
+ *     M = prod_t (diag(w_t) + a_t b_t^T)      (t in order, right-multiplied)
+ *     E = the final state of the stretch started from S = 0.
+ * A sequence split over P devices in order runs, on device i with stretch i:
+ *   wkv7_forward_summary   -> [E_i; M_i]
+ *   (exchange the P summaries: an all-gather)
+ *   wkv7_compose_states    -> the entry state of every stretch
+ *   wkv7_forward_continue  -> y of stretch i from its entry state
+ * which gives the same y and final state as one wkv7_forward over the whole
+ * sequence.  All three take bf16 inputs (the chunked form); fp32 inputs return
+ * WKV7_ERR_UNSUPPORTED.
+ */
+
+/* Bytes of scratch that lets wkv7_forward_summary / wkv7_forward_continue
+ * split a stretch into segments that run in parallel (0 when one pass fills
+ * the GPU).  Both calls of a pair must get the same workspace. */
+WKV7_API size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N);
+
+/*
+ * Summary of one stretch.
+ *   r, w, k, v, a, b : [B, T, H, N] bf16
+ *   summary          : [2, B, H, N, N] fp32, written: summary[0] = E,
+ *                      summary[1] = M.  T = 0 gives E = 0, M = I.
+ *   workspace        : wkv7_forward_summary_workspace_size() bytes, or NULL.
+ *                      With it the stretch runs as segments whose summaries
+ *                      are chained into E and M and stay in the workspace for
+ *                      wkv7_forward_continue; without it, one launch of the
+ *                      two runs (from S = 0, and from S = I with v read as 0).
+ * Shares the chunked form's numeric domain (see wkv7_forward).
+ */
+WKV7_API wkv7_status wkv7_forward_summary(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                          const void *r, const void *w, const void *k, const void *v,
+                                          const void *a, const void *b, float *summary, void *workspace,
+                                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Forward of one stretch from its entry state s_in (NULL = zeros), after
+ * wkv7_forward_summary ran on the SAME inputs with the SAME workspace pointer
+ * and size, and nothing wrote the workspace in between (the segment summaries
+ * it left there are reused; the results are unspecified otherwise).  With a
+ * NULL workspace it is a plain one-pass chunked forward from s_in.
+ *   y  : [B, T, H, N] of y_dtype, written
+ *   sT : [B, H, N, N] fp32 final state of the stretch, or NULL
+ */
+WKV7_API wkv7_status wkv7_forward_continue(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                           wkv7_dtype y_dtype, const void *r, const void *w, const void *k,
+                                           const void *v, const void *a, const void *b, const float *s_in,
+                                           void *y, float *sT, void *workspace, size_t workspace_bytes,
+                                           cudaStream_t stream);
+
+/*
+ * Entry states of nseg consecutive stretches from their summaries:
+ *     states[0] = s0 (or zeros when s0 is NULL)
+ *     states[k + 1] = states[k] M_k + E_k,  k = 0 .. nseg - 1
+ *   summaries : [nseg, 2, B, H, N, N] fp32, summaries[k] as written by
+ *               wkv7_forward_summary for stretch k (may be NULL if nseg = 0)
+ *   states    : [nseg + 1, B, H, N, N] fp32, written; states[k] is the state
+ *               before stretch k and states[nseg] the final state.  states
+ *               must not overlap s0 or summaries.
+ * fp32 on CUDA cores, one launch; nseg >= 0.
+ */
+WKV7_API wkv7_status wkv7_compose_states(int nseg, int B, int H, int N, const float *s0,
+                                         const float *summaries, float *states, cudaStream_t stream);
+
+/*
  * The algorithm wkv7_forward runs for these arguments (WKV7_ALGO_SEQ or
  * WKV7_ALGO_CHUNK; AUTO picks CHUNK for bf16 inputs with T >= 64), or -1 for
  * an invalid dtype / algorithm.  The chunked form takes bf16 inputs only.

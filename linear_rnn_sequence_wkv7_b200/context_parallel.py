@@ -1,0 +1,102 @@
+"""Sequence (context) parallel forward of the WKV7 recurrence over a process group.
+
+One long sequence is cut into contiguous stretches, stretch i on rank i (rank
+order = time order).  The recurrence S_t = S_{t-1} (diag(w_t) + a_t b_t^T) +
+v_t k_t^T is affine in the state, because the transition does not depend on S
+(RWKV-7 "Goose" paper review, section "Architecture"): a stretch maps its entry
+state to its final state as S_out = S_in M + E.  So each rank
+
+  1. computes the summary [E; M] of its own stretch (wkv7_forward_summary: the
+     stretch's segments run side by side from S = 0 and from S = I with v read
+     as 0, and their summaries are chained into E and M);
+  2. all-gathers the summaries (2 B H N^2 fp32 per rank: 1 MiB for B = 1,
+     H = 32, N = 64);
+  3. composes the entry state of every stretch (wkv7_compose_states), which
+     also yields the final state of the whole sequence on every rank;
+  4. runs its stretch from that entry state (wkv7_forward_continue, which
+     reuses the segment summaries of step 1 kept in the workspace).
+
+The exchange is one small all-gather, latency-bound whatever carries it, so it
+goes through the process group's collective (NCCL over NVLink on GPUs, gloo on
+CPU in tests).  The per-rank compute is injectable (``ops``) so the host
+logic can be tested on CPU against a reference implementation.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, Optional
+
+import torch
+import torch.distributed as dist
+
+
+@dataclass
+class StretchOps:
+    """The three per-rank computations the orchestration needs.
+
+    summary(r, w, k, v, a, b) -> ([2, B, H, N, N] fp32 [E; M], ctx)
+    compose(summaries [n, 2, B, H, N, N], s0 or None) -> states [n + 1, B, H, N, N]
+    forward(r, w, k, v, a, b, s_in, ctx) -> y [B, T, H, N]
+
+    ``ctx`` is whatever summary() keeps for forward() (the CUDA path's
+    workspace with the segment summaries).
+    """
+    summary: Callable
+    compose: Callable
+    forward: Callable
+
+
+def cuda_ops(y_dtype: Optional[torch.dtype] = None, stream=None) -> StretchOps:
+    """The library's kernels (through the C ABI) on the current CUDA device."""
+    from . import wkv7
+
+    def summary(r, w, k, v, a, b):
+        B, T, H, N = r.shape
+        nbytes = wkv7.forward_summary_workspace_size(B, T, H, N)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=r.device) if nbytes else None
+        return wkv7.forward_summary(r, w, k, v, a, b, workspace=ws, stream=stream), ws
+
+    def forward(r, w, k, v, a, b, s_in, ws):
+        return wkv7.forward_continue(r, w, k, v, a, b, s_in, workspace=ws, y_dtype=y_dtype, stream=stream)
+
+    return StretchOps(summary=summary, compose=lambda sums, s0: wkv7.compose_states(sums, s0, stream=stream),
+                      forward=forward)
+
+
+def forward_context_parallel(r, w, k, v, a, b, s0=None, *, ops: Optional[StretchOps] = None, group=None):
+    """Forward of this rank's stretch [B, T_i, H, N] of a sequence split over the
+    ranks of ``group`` in rank order.
+
+    ``s0`` is the state before the first token of the whole sequence; pass the
+    same tensor (or None for zeros) on every rank.  Stretch lengths may differ
+    between ranks, including 0.  Returns (y of this stretch, the entry state of
+    this stretch, the final state of the whole sequence).
+    """
+    ops = ops or cuda_ops()
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    summary, ctx = ops.summary(r, w, k, v, a, b)
+    summary = summary.contiguous()
+    if world > 1:
+        gathered = [torch.empty_like(summary) for _ in range(world)]
+        dist.all_gather(gathered, summary, group=group)
+        summaries = torch.stack(gathered)
+    else:
+        summaries = summary[None]
+    states = ops.compose(summaries, s0)
+    s_in = states[rank].contiguous()
+    y = ops.forward(r, w, k, v, a, b, s_in, ctx)
+    return y, s_in, states[world]
+
+
+def split_lengths(T: int, world: int, chunk: int = 32) -> list:
+    """Stretch lengths for ``world`` ranks: whole chunks of ``chunk`` tokens,
+    as even as possible (earlier ranks take the extra chunks), with the ragged
+    tail in the last non-empty stretch."""
+    chunks = -(-T // chunk)
+    base, extra = divmod(chunks, world)
+    ends, c = [], 0
+    for i in range(world):
+        c += base + (1 if i < extra else 0)
+        ends.append(min(T, c * chunk))
+    return [e - s for s, e in zip([0] + ends[:-1], ends)]

@@ -646,35 +646,37 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
     return cudaGetLastError();
 }
 
-// Segments combine: per head, S_in(0) = s0 (or 0) and
-// S_in(k+1) = S_in(k) M_k + E_k, where E_k / M_k are the final states of the
-// segment's plain and transition runs.  Writes S_in(k) for k < nseg.  The
-// rows of S are independent: CTA (head, rb) owns rows 8 rb .. 8 rb + 7, thread
-// -> (row, two columns); M_k is staged in shared memory.  fp32 on CUDA cores.
+// Chain of affine state maps, per head: X_0 = s0 (I when s0_eye, zeros when
+// s0 is null), X_{k+1} = X_k M_k + E_k for k < nsteps, with M_k at
+// m_base + k m_stride and E_k at e_base + k e_stride ([B*H][64][64] each; E
+// read as zeros when e_base is null).  With out_stride != 0 writes every X_k,
+// k <= nsteps, at out + k out_stride; else only X_nsteps at out.  The rows of
+// X are independent: CTA (head, rb) owns rows 8 rb .. 8 rb + 7, thread ->
+// (row, two columns); M_k is staged in shared memory.  fp32 on CUDA cores.
 constexpr int kCombineRows = 8;
 
 __global__ void __launch_bounds__(256)
-seg_combine_kernel(int BH, int nseg, const float *__restrict__ s0, const float *__restrict__ em,
-                   float *__restrict__ sin_out) {
+seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const float *__restrict__ e_base,
+                   long long e_stride, const float *__restrict__ m_base, long long m_stride,
+                   float *__restrict__ out, long long out_stride) {
     __shared__ __align__(16) float Msm[kN * kN];
     __shared__ float Ssm[kCombineRows][kN];
     const int head = blockIdx.x, tid = threadIdx.x;
     const int rr = tid >> 5, c2 = 2 * (tid & 31);
     const int i = kCombineRows * blockIdx.y + rr;
-    const size_t hoff = (size_t)head * kN * kN;
-    const size_t zstride = (size_t)BH * kN * kN;
-    float2 cur = s0 ? *reinterpret_cast<const float2 *>(s0 + hoff + (size_t)i * kN + c2) : make_float2(0.f, 0.f);
-    for (int kk = 0; kk < nseg; ++kk) {
-        *reinterpret_cast<float2 *>(sin_out + (size_t)kk * zstride + hoff + (size_t)i * kN + c2) = cur;
-        if (kk + 1 == nseg) break;
-        const float *E = em + (size_t)kk * zstride + hoff;
-        const float *M = em + (size_t)(nseg - 1 + kk) * zstride + hoff;
+    const size_t hoff = (size_t)head * kN * kN, eoff = hoff + (size_t)i * kN + c2;
+    float2 cur = s0 ? *reinterpret_cast<const float2 *>(s0 + eoff)
+                    : (s0_eye ? make_float2(i == c2 ? 1.f : 0.f, i == c2 + 1 ? 1.f : 0.f) : make_float2(0.f, 0.f));
+    for (int kk = 0;; ++kk) {
+        if (out_stride != 0 || kk == nsteps) *reinterpret_cast<float2 *>(out + kk * out_stride + eoff) = cur;
+        if (kk == nsteps) break;
+        const float *M = m_base + kk * m_stride + hoff;
         Ssm[rr][c2] = cur.x;
         Ssm[rr][c2 + 1] = cur.y;
         for (int x = tid; x < kN * kN / 4; x += 256)
             reinterpret_cast<float4 *>(Msm)[x] = reinterpret_cast<const float4 *>(M)[x];
         __syncthreads();
-        float2 acc = *reinterpret_cast<const float2 *>(E + (size_t)i * kN + c2);
+        float2 acc = e_base ? *reinterpret_cast<const float2 *>(e_base + kk * e_stride + eoff) : make_float2(0.f, 0.f);
 #pragma unroll 16
         for (int m = 0; m < kN; ++m) {
             const float sv = Ssm[rr][m];
@@ -685,6 +687,14 @@ seg_combine_kernel(int BH, int nseg, const float *__restrict__ s0, const float *
         __syncthreads();
         cur = acc;
     }
+}
+
+static cudaError_t launch_combine(int B, int H, int nsteps, const float *s0, bool s0_eye, const float *e_base,
+                                  long long e_stride, const float *m_base, long long m_stride, float *out,
+                                  long long out_stride, cudaStream_t st) {
+    seg_combine_kernel<<<dim3(B * H, kN / kCombineRows), 256, 0, st>>>(nsteps, s0, s0_eye ? 1 : 0, e_base, e_stride,
+                                                                       m_base, m_stride, out, out_stride);
+    return cudaGetLastError();
 }
 
 // Relative time of one launch of n chunk CTAs that each run the same number
@@ -707,26 +717,107 @@ static double launch_rounds(long long n, int sms) {
 // CTAs leave most of the GPU idle.  Picks the nseg (segments of at least 4
 // chunks) with the lowest estimated time, if that is below 95% of one pass;
 // among near-ties (within 3%) the fewest segments, which need the least scratch.
-int chunk_segments(int B, int T, int H, int sm_count) {
+// With summarize_last (the summary / continue pair) the last segment's summary
+// runs too and one segment means two launches (summary, then output), so the
+// cost model counts 2 nseg summary runs and n = 1 competes on equal terms.
+int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last) {
     static_assert(2 * (chunk::SMEM_BYTES + 1024) <= 228 * 1024, "two chunk CTAs per SM");
     const long long heads = (long long)B * H;
     const long long chunks = (T + chunk::L - 1) / chunk::L;
     if (sm_count <= 0 || heads <= 0) return 1;
     const long long max_n = std::min<long long>(64, chunks / 4);
+    const long long extra = summarize_last ? 0 : 1;
     auto cost = [&](long long n) {
-        return (launch_rounds(2 * (n - 1) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
+        return (launch_rounds(2 * (n - extra) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
     };
-    double best = 0.95 * launch_rounds(heads, sm_count);
+    double best = summarize_last ? cost(1) : 0.95 * launch_rounds(heads, sm_count);
     for (long long n = 2; n <= max_n; ++n) best = std::min(best, cost(n));
     for (long long n = 2; n <= max_n; ++n)
         if (cost(n) <= 1.03 * best) return (int)n;
     return 1;
 }
 
+// Segment length (whole chunks) and the number of non-empty segments for a
+// request of nseg segments over T tokens.
+static void seg_split(int T, int nseg, int &t_seg, int &n) {
+    const int chunks = (T + chunk::L - 1) / chunk::L;
+    t_seg = ((chunks + nseg - 1) / nseg) * chunk::L;
+    n = (T + t_seg - 1) / t_seg;
+}
+
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg) {
     if (nseg <= 1) return 0;
     // E_k, M_k for segments 0..nseg-2 and S_in(k) for k < nseg
     return (size_t)(2 * (nseg - 1) + nseg) * B * H * kN * kN * sizeof(float);
+}
+
+size_t summary_workspace_bytes(int B, int T, int H, int nseg) {
+    if (nseg <= 1) return 0;
+    // E_k, M_k and S_in(k) for every segment
+    return (size_t)3 * nseg * B * H * kN * kN * sizeof(float);
+}
+
+// The summary of an empty sequence: E = 0, M = I (one thread per element of both).
+__global__ void summary_empty_kernel(long long zst, float *summary) {
+    const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= 2 * zst) return;
+    const int e = (int)(x % (kN * kN));
+    summary[x] = (x >= zst && e / kN == e % kN) ? 1.f : 0.f;
+}
+
+// Affine summary of a whole sequence, S_out = S_in M + E, E to summary[0] and
+// M to summary[1] ([B][H][64][64] each).  One segment: one launch of two runs,
+// E from S_in = 0 and M from S_in = I with v read as 0.  nseg segments: the
+// same two runs for every segment in one launch (their summaries stay in the
+// workspace for fwd_chunk_continue), then E and M of the whole sequence by
+// chaining them: E from 0 through every (E_k, M_k), M from I through the M_k.
+cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
+                              const void *a, const void *b, float *summary, int nseg, void *workspace,
+                              long long wait_limit, cudaStream_t st) {
+    const long long zst = (long long)B * H * kN * kN;
+    if (T == 0) {
+        summary_empty_kernel<<<(unsigned)((2 * zst + 255) / 256), 256, 0, st>>>(zst, summary);
+        return cudaGetLastError();
+    }
+    if (nseg <= 1)
+        return launch_chunk(B, T, H, T, 1, 2, WKV7_BF16, r, w, k, v, a, b, nullptr, 0, nullptr, summary, zst, -1,
+                            wait_limit, st);
+    int t_seg, n;
+    seg_split(T, nseg, t_seg, n);
+    float *em = static_cast<float *>(workspace);                // E_0..E_{n-1}, M_0..M_{n-1}
+    cudaError_t e = launch_chunk(B, T, H, t_seg, n, 2 * n, WKV7_BF16, r, w, k, v, a, b, nullptr, 0, nullptr, em,
+                                 zst, -1, wait_limit, st);
+    if (e != cudaSuccess) return e;
+    e = launch_combine(B, H, n, nullptr, false, em, zst, em + n * zst, zst, summary, 0, st);
+    if (e != cudaSuccess) return e;
+    return launch_combine(B, H, n, nullptr, true, nullptr, 0, em + n * zst, zst, summary + zst, 0, st);
+}
+
+// The forward of a sequence from its entry state s_in after fwd_chunk_summary
+// ran on the same inputs, segment count and workspace: the entry state of
+// every segment from the kept (E_k, M_k), then every segment's output run.
+cudaError_t fwd_chunk_continue(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
+                               const void *v, const void *a, const void *b, const float *s_in, void *y, float *sT,
+                               int nseg, void *workspace, long long wait_limit, cudaStream_t st) {
+    if (nseg <= 1)
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s_in, 0, y, sT, 0, -1, wait_limit, st);
+    const long long zst = (long long)B * H * kN * kN;
+    int t_seg, n;
+    seg_split(T, nseg, t_seg, n);
+    float *em = static_cast<float *>(workspace);
+    float *sin = em + 2 * n * zst;
+    cudaError_t e = launch_combine(B, H, n - 1, s_in, false, em, zst, em + n * zst, zst, sin, zst, st);
+    if (e != cudaSuccess) return e;
+    return launch_chunk(B, T, H, t_seg, n, n, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, n - 1, wait_limit, st);
+}
+
+// Entry states of nseg consecutive segments and the state after the last:
+// out[0] = s0 (or 0), out[k+1] = out[k] M_k + E_k, with summary[k] = [E_k; M_k].
+cudaError_t compose_states(int B, int H, int nseg, const float *s0, const float *summary, float *out,
+                           cudaStream_t st) {
+    const long long zst = (long long)B * H * kN * kN;
+    const float *m0 = summary ? summary + zst : nullptr;     // nseg = 0 reads no summary
+    return launch_combine(B, H, nseg, s0, false, summary, 2 * zst, m0, 2 * zst, out, zst, st);
 }
 
 // State checkpoints before every 32-token chunk (and the final state) for the
@@ -743,9 +834,10 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st) {
     if (nseg <= 1)
         return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
-    const int chunks = (T + chunk::L - 1) / chunk::L;
-    const int t_seg = ((chunks + nseg - 1) / nseg) * chunk::L;
-    nseg = (T + t_seg - 1) / t_seg;
+    int t_seg;
+    seg_split(T, nseg, t_seg, nseg);
+    if (nseg <= 1)
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
     float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg][B][H][64][64]
@@ -754,8 +846,7 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
                                  nullptr, em, zst, -1, wait_limit, st);
     if (e != cudaSuccess) return e;
     // pass 2: entry state of every segment
-    seg_combine_kernel<<<dim3(B * H, kN / kCombineRows), 256, 0, st>>>(B * H, nseg, s0, em, sin);
-    e = cudaGetLastError();
+    e = launch_combine(B, H, nseg - 1, s0, false, em, zst, em + (size_t)(nseg - 1) * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
     // pass 3: every segment from its true entry state; the last one writes sT
     return launch_chunk(B, T, H, t_seg, nseg, nseg, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 1,

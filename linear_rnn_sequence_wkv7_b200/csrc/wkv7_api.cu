@@ -28,11 +28,20 @@ size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st);
-int chunk_segments(int B, int T, int H, int sm_count);
+int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last);
 cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
                                   const void *a, const void *b, const float *s0, float *ckpt, float *sT,
                                   long long wait_limit, cudaStream_t st);
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
+cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
+                              const void *a, const void *b, float *summary, int nseg, void *workspace,
+                              long long wait_limit, cudaStream_t st);
+cudaError_t fwd_chunk_continue(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
+                               const void *v, const void *a, const void *b, const float *s_in, void *y, float *sT,
+                               int nseg, void *workspace, long long wait_limit, cudaStream_t st);
+size_t summary_workspace_bytes(int B, int T, int H, int nseg);
+cudaError_t compose_states(int B, int H, int nseg, const float *s0, const float *summary, float *out,
+                           cudaStream_t st);
 
 namespace {
 
@@ -82,6 +91,16 @@ int current_sm_count() {
     return n;
 }
 
+// Segments of the summary / continue pair: the cost model's choice when the
+// workspace holds their scratch, else 1 (both calls of a pair must get the
+// same workspace size, so they agree).
+int summary_segments(int B, int T, int H, const void *workspace, size_t workspace_bytes) {
+    const int sms = current_sm_count();
+    if (sms <= 0 || T <= 0 || workspace == nullptr || !aligned16(workspace)) return 1;
+    const int want = chunk_segments(B, T, H, sms, true);
+    return (want > 1 && workspace_bytes >= summary_workspace_bytes(B, T, H, want)) ? want : 1;
+}
+
 size_t bwd_ckpt_bytes(int B, int T, int H) { return bwd_chunk_ckpt_bytes(B, T, H); }
 size_t state_bytes(int B, int H) { return (size_t)B * H * kN * kN * sizeof(float); }
 
@@ -114,7 +133,7 @@ size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dty
     if (resolve_algo(T, in_dtype, algo) != WKV7_ALGO_CHUNK || in_dtype != WKV7_BF16) return 0;
     const int sms = current_sm_count();
     if (sms <= 0) return 0;
-    return chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms));
+    return chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms, false));
 }
 
 wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
@@ -139,7 +158,7 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
         int nseg = 1;
         const int sms = current_sm_count();
         if (sms > 0) {
-            const int want = chunk_segments(B, T, H, sms);
+            const int want = chunk_segments(B, T, H, sms, false);
             if (want > 1 && workspace != nullptr && aligned16(workspace) &&
                 workspace_bytes >= chunk_workspace_bytes(B, T, H, want))
                 nseg = want;
@@ -148,6 +167,61 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
                                    lim > 0 ? lim : kDefaultWaitCycles, stream));
     }
     return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+}
+
+size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
+    const int sms = current_sm_count();
+    if (sms <= 0) return 0;
+    return summary_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms, true));
+}
+
+wkv7_status wkv7_forward_summary(int B, int T, int H, int N, wkv7_dtype in_dt, const void *r, const void *w,
+                                 const void *k, const void *v, const void *a, const void *b, float *summary,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt)) return WKV7_ERR_INVALID_ARG;
+    if (in_dt != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;                // computed by the chunked form
+    if (!opt_ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (!ptr_ok(summary)) return WKV7_ERR_INVALID_ARG;
+    if (T > 0)
+        for (const void *p : {r, w, k, v, a, b})
+            if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    const long long lim = g_wait_limit.load();
+    const int nseg = summary_segments(B, T, H, workspace, workspace_bytes);
+    return from_cuda(fwd_chunk_summary(B, T, H, r, w, k, v, a, b, summary, nseg, workspace,
+                                       lim > 0 ? lim : kDefaultWaitCycles, stream));
+}
+
+wkv7_status wkv7_forward_continue(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                                  const void *w, const void *k, const void *v, const void *a, const void *b,
+                                  const float *s_in, void *y, float *sT, void *workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
+    if (in_dt != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
+    if (!opt_ptr_ok(s_in) || !opt_ptr_ok(sT) || !opt_ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (T == 0) return copy_or_zero_state(sT, s_in, B, H, stream);
+    for (const void *p : {r, w, k, v, a, b, (const void *)y})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    const long long lim = g_wait_limit.load();
+    const int nseg = summary_segments(B, T, H, workspace, workspace_bytes);
+    return from_cuda(fwd_chunk_continue(B, T, H, y_dt, r, w, k, v, a, b, s_in, y, sT, nseg, workspace,
+                                        lim > 0 ? lim : kDefaultWaitCycles, stream));
+}
+
+wkv7_status wkv7_compose_states(int nseg, int B, int H, int N, const float *s0, const float *summaries,
+                                float *states, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, 0, H, N);
+    if (s != WKV7_OK) return s;
+    if (nseg < 0 || !opt_ptr_ok(s0)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (!ptr_ok(states) || (nseg > 0 && !ptr_ok(summaries))) return WKV7_ERR_INVALID_ARG;
+    return from_cuda(compose_states(B, H, nseg, s0, summaries, states, stream));
 }
 
 int wkv7_forward_resolve_algo(int T, wkv7_dtype in_dtype, wkv7_algo algo) {

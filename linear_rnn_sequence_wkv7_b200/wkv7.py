@@ -25,6 +25,8 @@ EXPORTED_SYMBOLS = (
     "wkv7_abi_version", "wkv7_status_string", "wkv7_forward_workspace_size", "wkv7_forward",
     "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
     "wkv7_forward_resolve_algo", "wkv7_backward_noalloc", "wkv7_set_wait_limit",
+    "wkv7_forward_summary", "wkv7_compose_states", "wkv7_forward_summary_workspace_size",
+    "wkv7_forward_continue",
 )
 
 _lib = None
@@ -60,6 +62,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward.restype = i
     lib.wkv7_backward_noalloc.argtypes = [i, i, i, i, i, i] + [vp] * 16 + [vp]
     lib.wkv7_backward_noalloc.restype = i
+    lib.wkv7_forward_summary_workspace_size.argtypes = [i, i, i, i]
+    lib.wkv7_forward_summary_workspace_size.restype = z
+    lib.wkv7_forward_summary.argtypes = [i, i, i, i, i] + [vp] * 8 + [z, vp]
+    lib.wkv7_forward_summary.restype = i
+    lib.wkv7_forward_continue.argtypes = [i, i, i, i, i, i] + [vp] * 10 + [z, vp]
+    lib.wkv7_forward_continue.restype = i
+    lib.wkv7_compose_states.argtypes = [i, i, i, i, vp, vp, vp, vp]
+    lib.wkv7_compose_states.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_set_wait_limit.argtypes = [ctypes.c_longlong]
@@ -136,6 +146,65 @@ def forward(r, w, k, v, a, b, s0=None, *, y=None, sT=None, y_dtype=None, algo="a
                           0 if workspace is None else workspace.numel(), _stream(stream))
     _check("wkv7_forward", st)
     return (y, sT) if return_state else y
+
+
+def forward_summary_workspace_size(B, T, H, N) -> int:
+    return load_library().wkv7_forward_summary_workspace_size(B, T, H, N)
+
+
+def forward_summary(r, w, k, v, a, b, *, out=None, workspace=None, stream=None):
+    """[2,B,H,N,N] fp32 summary [E; M] of a bf16 stretch [B,T,H,N]: its final
+    state is S_in @ M + E for entry state S_in.  Pass the same ``workspace``
+    (or None) to the ``forward_continue`` of this stretch."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    if out is None:
+        out = torch.empty((2, B, H, N, N), dtype=torch.float32, device=r.device)
+    _same((out,), (2, B, H, N, N), torch.float32)
+    st = lib.wkv7_forward_summary(B, T, H, N, _dt(r), *map(_ptr, (r, w, k, v, a, b, out)), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("wkv7_forward_summary", st)
+    return out
+
+
+def forward_continue(r, w, k, v, a, b, s_in=None, *, workspace=None, y=None, sT=None, y_dtype=None,
+                     return_state=False, stream=None):
+    """y [B,T,H,N] of a bf16 stretch from entry state ``s_in``, reusing what
+    ``forward_summary`` left in ``workspace`` (same inputs, same workspace)."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    ycode = _dt(r) if y_dtype is None else (F32 if y_dtype == torch.float32 else BF16)
+    if y is None:
+        y = torch.empty((B, T, H, N), dtype=_tdt(ycode), device=r.device)
+    if return_state and sT is None:
+        sT = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    if s_in is not None:
+        _same((s_in,), (B, H, N, N), torch.float32)
+    st = lib.wkv7_forward_continue(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s_in, y, sT)),
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                   _stream(stream))
+    _check("wkv7_forward_continue", st)
+    return (y, sT) if return_state else y
+
+
+def compose_states(summaries, s0=None, *, out=None, stream=None):
+    """states [nseg+1,B,H,N,N]: states[0] = s0 (or 0), states[k+1] = states[k] @ M_k + E_k
+    for summaries [nseg,2,B,H,N,N]."""
+    lib = load_library()
+    nseg, two, B, H, N, _ = summaries.shape
+    if two != 2:
+        raise ValueError("summaries must be [nseg, 2, B, H, N, N]")
+    _same((summaries,), summaries.shape, torch.float32)
+    if s0 is not None:
+        _same((s0,), (B, H, N, N), torch.float32)
+    if out is None:
+        out = torch.empty((nseg + 1, B, H, N, N), dtype=torch.float32, device=summaries.device)
+    _same((out,), (nseg + 1, B, H, N, N), torch.float32)
+    st = lib.wkv7_compose_states(nseg, B, H, N, _ptr(s0), _ptr(summaries), _ptr(out), _stream(stream))
+    _check("wkv7_compose_states", st)
+    return out
 
 
 def resolve_algo(T, in_dtype=torch.bfloat16, algo="auto") -> str:

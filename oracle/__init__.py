@@ -28,6 +28,12 @@ section "Summary").
 * ``backward_chunked`` is the reverse-mode derivative of ``forward_chunked``,
   chunk by chunk (last chunk first), each line the adjoint of one line of the
   forward definition; pinned against ``backward``.
+* ``forward_summary`` / ``compose_states``: the recurrence is affine in the
+  state (the transition diag(w_t) + a_t b_t^T does not depend on S: paper
+  review, section "Architecture"), so a stretch of tokens maps S_in to
+  S_in M + E with M the ordered product of its transitions and E its final
+  state from S = 0.  Both are written as those definitions: the product taken
+  token by token, E from ``forward``.
 """
 from __future__ import annotations
 
@@ -271,3 +277,35 @@ def backward_chunked(r, w, k, v, a, b, s0, dy, dsT=None, chunk_len=64):
                 dS = dSin
             ds0[bb, h] = dS
     return (*grads, ds0)
+
+
+def forward_summary(r, w, k, v, a, b):
+    """(E, M), each [B,H,N,N] fp64, of a stretch shaped [B,T,H,N]:
+    M = (diag(w_1) + a_1 b_1^T)(diag(w_2) + a_2 b_2^T)...(diag(w_T) + a_T b_T^T)
+    (right-multiplied in token order, as S_t = S_{t-1} A_t applies them), and
+    E = the final state of ``forward`` from S = 0.  T = 0 gives E = 0, M = I."""
+    r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
+    B, T, H, N = r.shape
+    M = np.empty((B, H, N, N))
+    for bb in range(B):
+        for h in range(H):
+            P = np.eye(N)
+            for t in range(T):
+                P = P @ (np.diag(w[bb, t, h]) + np.outer(a[bb, t, h], b[bb, t, h]))
+            M[bb, h] = P
+    if T == 0:
+        return np.zeros((B, H, N, N)), M
+    _, E = forward(r, w, k, v, a, b, None)
+    return E, M
+
+
+def compose_states(summaries, s0=None):
+    """states [nseg+1,B,H,N,N] from summaries [nseg,2,B,H,N,N] ([E; M] each):
+    states[0] = s0 (or 0), states[k+1] = states[k] M_k + E_k."""
+    summaries = _f64(summaries)
+    nseg, _, B, H, N, _ = summaries.shape
+    states = np.empty((nseg + 1, B, H, N, N))
+    states[0] = 0.0 if s0 is None else _f64(s0)
+    for kk in range(nseg):
+        states[kk + 1] = states[kk] @ summaries[kk, 1] + summaries[kk, 0]
+    return states

@@ -89,3 +89,41 @@ def test_step_and_backward_reject_invalid_arguments(lib):
     assert lib.wkv7_backward(1, 32, 1, 64, 0, 0, *ptrs, P, 16, None) == wkv7.ERR_INVALID_ARG
     ptrs[15] = None                                  # ds0 is required
     assert lib.wkv7_backward(1, 32, 1, 64, 0, 0, *ptrs, P, 1 << 40, None) == wkv7.ERR_INVALID_ARG
+
+
+def test_summary_and_compose_reject_invalid_arguments(lib):
+    summ = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ptrs=None, ws=None: lib.wkv7_forward_summary(
+        B, T, H, N, dt, *(ptrs or [P] * 7), ws, 0, None)
+    assert summ(N=32) == wkv7.ERR_UNSUPPORTED
+    assert summ(dt=wkv7.F32) == wkv7.ERR_UNSUPPORTED     # computed by the chunked form
+    assert summ(dt=5) == wkv7.ERR_INVALID_ARG
+    assert summ(T=-1) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 7
+    bad[6] = None                                        # summary output missing
+    assert summ(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 7
+    bad[3] = ctypes.c_void_p(24)                         # v misaligned
+    assert summ(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert summ(ws=ctypes.c_void_p(40)) == wkv7.ERR_INVALID_ARG  # workspace misaligned
+    assert summ(B=0) == wkv7.OK
+    cont = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ydt=wkv7.BF16, ptrs=None: lib.wkv7_forward_continue(
+        B, T, H, N, dt, ydt, *(ptrs or [P] * 9), None, 0, None)
+    assert cont(N=128) == wkv7.ERR_UNSUPPORTED
+    assert cont(dt=wkv7.F32) == wkv7.ERR_UNSUPPORTED
+    assert cont(ydt=3) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 9
+    bad[7] = None                                        # y missing
+    assert cont(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 9
+    bad[6] = ctypes.c_void_p(36)                         # s_in misaligned
+    assert cont(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert cont(H=0) == wkv7.OK
+    assert lib.wkv7_forward_summary_workspace_size(1, 64, 1, 32) == 0
+    comp = lambda nseg=2, B=1, H=1, N=64, s0=None, sums=P, out=P: lib.wkv7_compose_states(
+        nseg, B, H, N, s0, sums, out, None)
+    assert comp(N=16) == wkv7.ERR_UNSUPPORTED
+    assert comp(nseg=-1) == wkv7.ERR_INVALID_ARG
+    assert comp(sums=None) == wkv7.ERR_INVALID_ARG       # nseg > 0 needs summaries
+    assert comp(out=None) == wkv7.ERR_INVALID_ARG
+    assert comp(s0=ctypes.c_void_p(20)) == wkv7.ERR_INVALID_ARG
+    assert comp(H=0) == wkv7.OK

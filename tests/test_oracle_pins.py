@@ -247,6 +247,90 @@ def test_state_passing_split():
     np.testing.assert_array_equal(s2, sT)
 
 
+def test_summary_is_the_affine_map_of_the_state():
+    """The final state from any entry state is S_in M + E: checked against the
+    C forward run from a random S_in (a reversed product order, a transposed
+    M or a dropped a b^T term breaks it); T = 0 is the identity map."""
+    B, T, H, N = 2, 23, 2, 8
+    (r, w, k, v, a, b), _ = recipe(B, T, H, N, seed=43)
+    S_in = np.random.default_rng(47).standard_normal((B, H, N, N))
+    E, M = oracle.forward_summary(r, w, k, v, a, b)
+    _, sT = oracle.forward(r, w, k, v, a, b, s0=S_in)
+    assert rel_err(S_in @ M + E, sT) < 1e-12
+    E0, M0 = oracle.forward_summary(*(x[:, :0] for x in (r, w, k, v, a, b)))
+    np.testing.assert_array_equal(E0, 0.0)
+    np.testing.assert_array_equal(M0, np.broadcast_to(np.eye(N), M0.shape))
+
+
+def test_summary_closed_forms():
+    """a = b = 0: M is the diagonal of the decay products.  w = 1 with
+    a = -k_hat, b = 2 k_hat: every transition is a Householder reflection, so M
+    is orthogonal (M M^T = I) with determinant (-1)^T."""
+    B, T, H, N = 1, 9, 2, 8
+    (r, w, k, v, a, b), _ = recipe(B, T, H, N, seed=53)
+    zero = np.zeros_like(a)
+    _, M = oracle.forward_summary(r, w, k, v, zero, zero)
+    for h in range(H):
+        np.testing.assert_allclose(M[0, h], np.diag(np.prod(w[0, :, h], axis=0)), rtol=1e-14, atol=0)
+    kh = unit_rows(np.random.default_rng(59).standard_normal((B, T, H, N)))
+    _, M = oracle.forward_summary(r, np.ones_like(w), k, v, -kh, 2.0 * kh)
+    for h in range(H):
+        np.testing.assert_allclose(M[0, h] @ M[0, h].T, np.eye(N), atol=1e-13)
+        assert abs(np.linalg.det(M[0, h]) - (-1.0) ** T) < 1e-12
+
+
+def test_compose_states_match_prefix_forwards():
+    """Composing the summaries of consecutive stretches (ragged lengths, one
+    empty) gives the state after every prefix, and the final state."""
+    B, T, H, N = 2, 41, 2, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=61)
+    cuts = [0, 13, 13, 30, 41]
+    sums = []
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        E, M = oracle.forward_summary(*(x[:, c0:c1] for x in (r, w, k, v, a, b)))
+        sums.append(np.stack([E, M]))
+    states = oracle.compose_states(np.stack(sums), s0)
+    assert states.shape == (len(cuts), B, H, N, N)
+    np.testing.assert_array_equal(states[0], s0)
+    for i, c in enumerate(cuts[1:], start=1):
+        _, s_pref = oracle.forward(*(x[:, :c] for x in (r, w, k, v, a, b)), s0=s0)
+        assert rel_err(states[i], s_pref) < 1e-12, i
+    np.testing.assert_array_equal(oracle.compose_states(np.zeros((0, 2, B, H, N, N)))[0], 0.0)
+
+
+SUMMARY_MUTANTS = {
+    "reversed_product": ("P = P @ (np.diag(", "P = (np.diag("),
+    "compose_left_multiply": ("states[kk] @ summaries[kk, 1]", "summaries[kk, 1] @ states[kk]"),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(SUMMARY_MUTANTS))
+def test_summary_mutants_are_caught(mutant):
+    import inspect
+    fn = "forward_summary" if mutant == "reversed_product" else "compose_states"
+    src = inspect.getsource(getattr(oracle, fn))
+    old, new = SUMMARY_MUTANTS[mutant]
+    assert src.count(old) == 1, "mutation anchor not found"
+    if mutant == "reversed_product":
+        new_src = src.replace(old, new).replace("b[bb, t, h]))", "b[bb, t, h])) @ P")
+    else:
+        new_src = src.replace(old, new)
+    ns = dict(np=np, _f64=oracle._f64, forward=oracle.forward)
+    exec(new_src, ns)
+    B, T, H, N = 1, 7, 1, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=67)
+    S_in = np.random.default_rng(71).standard_normal((B, H, N, N))
+    if mutant == "reversed_product":
+        E, M = ns["forward_summary"](r, w, k, v, a, b)
+        _, sT = oracle.forward(r, w, k, v, a, b, s0=S_in)
+        assert rel_err(S_in @ M + E, sT) > 1e-6
+    else:
+        E, M = oracle.forward_summary(r, w, k, v, a, b)
+        states = ns["compose_states"](np.stack([E, M])[None], S_in)
+        _, sT = oracle.forward(r, w, k, v, a, b, s0=S_in)
+        assert rel_err(states[1], sT) > 1e-6
+
+
 def test_step_equals_forward_t1():
     B, H, N = 3, 2, 8
     (r, w, k, v, a, b), s0 = recipe(B, 1, H, N, seed=29)
