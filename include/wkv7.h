@@ -18,9 +18,10 @@
  * key; k, v the write key and value; r the receptance.
  *
  * Conventions shared by every entry point
- *  - Pointers are DEVICE pointers owned by the caller.  The library
- *    allocates no memory; scratch comes from the caller through the
- *    *_workspace_size queries.  Every pointer must be 16-byte aligned.
+ *  - Pointers are DEVICE pointers owned by the caller (wkv7_forward_host
+ *    takes host tensors).  The library allocates no memory; scratch comes
+ *    from the caller through the *_workspace_size queries.  Every pointer
+ *    must be 16-byte aligned.
  *  - Tensors are contiguous, row-major.  Per-token tensors (r, w, k, v, a, b,
  *    y, dy and their gradients) are [B, T, H, N]; a decode step's tensors are
  *    [B, H, N]; states (s0, sT, dsT, ds0, state) are [B, H, N, N] fp32 with
@@ -180,6 +181,32 @@ WKV7_API wkv7_status wkv7_forward_continue(int B, int T, int H, int N, wkv7_dtyp
  */
 WKV7_API wkv7_status wkv7_compose_states(int nseg, int B, int H, int N, const float *s0,
                                          const float *summaries, float *states, cudaStream_t stream);
+
+/*
+ * wkv7_forward with r..b, s0, y and sT in HOST memory (page-locked memory
+ * lets the copies overlap the computation; pageable memory works, slower).
+ * The sequence is cut into up to 8 time slices of whole 32-token chunks; the
+ * upload of slice k+1 and the download of slice k-1's y run on two internal
+ * streams while slice k computes on `stream`, and the state is carried from
+ * slice to slice on the device.  The algorithm is resolved once for the whole
+ * T.  Results equal wkv7_forward's up to the chunked form's segment choice,
+ * which is made per slice.
+ *   host tensors : same shapes and dtypes as wkv7_forward; s0 / sT may be NULL
+ *   workspace    : DEVICE scratch of wkv7_forward_host_workspace_size() bytes
+ *                  (two slots of slice inputs and y, the state, the forward's
+ *                  own workspace); required, also for T = 0.
+ * Asynchronous on `stream` like every call: the host buffers must stay valid
+ * and unmodified (y, sT unread) until `stream` reaches this point.  Each call
+ * creates two streams and a few events and releases them before returning
+ * (the driver frees them when their work completes), so it is not meant for
+ * stream capture.
+ */
+WKV7_API size_t wkv7_forward_host_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                                 wkv7_dtype y_dtype, wkv7_algo algo, int chunk_len);
+WKV7_API wkv7_status wkv7_forward_host(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
+                                       const void *r, const void *w, const void *k, const void *v, const void *a,
+                                       const void *b, const float *s0, void *y, float *sT, wkv7_algo algo,
+                                       int chunk_len, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * The algorithm wkv7_forward runs for these arguments (WKV7_ALGO_SEQ or

@@ -7,3 +7,4 @@
 #include "bwd_chunk.cu"
 #include "fwd_chunk.cu"
 #include "bwd_noalloc.cu"
+#include "fwd_host.cu"

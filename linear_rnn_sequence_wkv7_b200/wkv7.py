@@ -26,7 +26,7 @@ EXPORTED_SYMBOLS = (
     "wkv7_step", "wkv7_backward_workspace_size", "wkv7_backward", "wkv7_get_device_status",
     "wkv7_forward_resolve_algo", "wkv7_backward_noalloc", "wkv7_set_wait_limit",
     "wkv7_forward_summary", "wkv7_compose_states", "wkv7_forward_summary_workspace_size",
-    "wkv7_forward_continue",
+    "wkv7_forward_continue", "wkv7_forward_host_workspace_size", "wkv7_forward_host",
 )
 
 _lib = None
@@ -70,6 +70,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_forward_continue.restype = i
     lib.wkv7_compose_states.argtypes = [i, i, i, i, vp, vp, vp, vp]
     lib.wkv7_compose_states.restype = i
+    lib.wkv7_forward_host_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+    lib.wkv7_forward_host_workspace_size.restype = z
+    lib.wkv7_forward_host.argtypes = [i, i, i, i, i, i] + [vp] * 9 + [i, i, vp, z, vp]
+    lib.wkv7_forward_host.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_set_wait_limit.argtypes = [ctypes.c_longlong]
@@ -205,6 +209,46 @@ def compose_states(summaries, s0=None, *, out=None, stream=None):
     st = lib.wkv7_compose_states(nseg, B, H, N, _ptr(s0), _ptr(summaries), _ptr(out), _stream(stream))
     _check("wkv7_compose_states", st)
     return out
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host tensors must be contiguous CPU tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward_host_workspace_size(B, T, H, N, in_dtype=torch.bfloat16, y_dtype=None, algo="auto", chunk_len=0) -> int:
+    ic = F32 if in_dtype == torch.float32 else BF16
+    yc = ic if y_dtype is None else (F32 if y_dtype == torch.float32 else BF16)
+    return load_library().wkv7_forward_host_workspace_size(B, T, H, N, ic, yc, ALGOS[algo], chunk_len)
+
+
+def forward_host(r, w, k, v, a, b, s0=None, *, y, sT=None, algo="auto", chunk_len=0, workspace=None,
+                 device=None, stream=None):
+    """wkv7_forward_host: inputs and outputs are CPU tensors (pinned for
+    overlap), ``y`` [B,T,H,N] and optional ``sT`` written in place once the
+    stream reaches the call; ``workspace`` is a CUDA uint8 tensor (allocated
+    on ``device`` when None)."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    ycode = _dt(y)
+    if tuple(y.shape) != (B, T, H, N):
+        raise ValueError("y must be [B, T, H, N]")
+    if s0 is not None:
+        _same((s0,), (B, H, N, N), torch.float32)
+    if sT is not None:
+        _same((sT,), (B, H, N, N), torch.float32)
+    ws_bytes = lib.wkv7_forward_host_workspace_size(B, T, H, N, _dt(r), ycode, ALGOS[algo], chunk_len)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8,
+                                device=device if device is not None else torch.cuda.current_device())
+    st = lib.wkv7_forward_host(B, T, H, N, _dt(r), ycode, *map(_host_ptr, (r, w, k, v, a, b, s0, y, sT)),
+                               ALGOS[algo], chunk_len, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("wkv7_forward_host", st)
+    return y, sT
 
 
 def resolve_algo(T, in_dtype=torch.bfloat16, algo="auto") -> str:

@@ -127,3 +127,24 @@ def test_summary_and_compose_reject_invalid_arguments(lib):
     assert comp(out=None) == wkv7.ERR_INVALID_ARG
     assert comp(s0=ctypes.c_void_p(20)) == wkv7.ERR_INVALID_ARG
     assert comp(H=0) == wkv7.OK
+
+
+def test_forward_host_rejects_invalid_arguments(lib):
+    fh = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ydt=wkv7.BF16, ptrs=None, algo=0, chunk=0, ws=P, nb=1 << 40: (
+        lib.wkv7_forward_host(B, T, H, N, dt, ydt, *(ptrs or [P] * 9), algo, chunk, ws, nb, None))
+    assert fh(N=32) == wkv7.ERR_UNSUPPORTED
+    assert fh(dt=4) == wkv7.ERR_INVALID_ARG
+    assert fh(algo=5) == wkv7.ERR_INVALID_ARG
+    assert fh(chunk=16) == wkv7.ERR_UNSUPPORTED
+    assert fh(dt=wkv7.F32, algo=wkv7.ALGO_CHUNK) == wkv7.ERR_UNSUPPORTED
+    assert fh(ws=None) == wkv7.ERR_INVALID_ARG                     # device workspace is required
+    assert fh(nb=16) == wkv7.ERR_INVALID_ARG                       # ... and must be large enough
+    bad = [P] * 9
+    bad[7] = None                                                  # y missing
+    assert fh(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert fh(B=0) == wkv7.OK
+    # two slots of 8 slices' inputs and y, the state, no forward scratch for 256 heads
+    B, T, H = 8, 4096, 32
+    need = lib.wkv7_forward_host_workspace_size(B, T, H, 64, wkv7.BF16, wkv7.BF16, wkv7.ALGO_CHUNK, 0)
+    assert need >= 2 * 7 * B * (T // 8) * H * 64 * 2 + B * H * 64 * 64 * 4
+    assert lib.wkv7_forward_host_workspace_size(B, T, H, 16, wkv7.BF16, wkv7.BF16, 0, 0) == 0
