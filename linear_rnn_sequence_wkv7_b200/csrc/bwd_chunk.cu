@@ -201,13 +201,37 @@ __device__ __forceinline__ void load_a(float (&av)[Acc<M>::RM], const float *A, 
     }
 }
 
-// K is a multiple of 4; the operands of step k + 1 are loaded while step k
-// is multiplied
+// K is a multiple of 4.  A row-major (A[m * lda + k]): four k steps per pass,
+// each thread's A rows read as float4 along k (one load per row and pass
+// instead of one per row and k).  A column-major (A[k * lda + m]): the
+// operands of step k + 1 are loaded while step k is multiplied.
 template <int M, bool A_COL>
 __device__ __forceinline__ void mm(Acc<M> &acc, const float *A, int lda, const float *B, int ldb, int K) {
     constexpr int RM = Acc<M>::RM;
     const int tid = threadIdx.x;
     const int m0 = RM * (tid >> 4), n0 = 4 * (tid & 15);
+    if constexpr (!A_COL) {
+#pragma unroll 2
+        for (int k4 = 0; k4 < K; k4 += 4) {
+            float4 a4[RM], b4[4];
+#pragma unroll
+            for (int i = 0; i < RM; ++i) a4[i] = *reinterpret_cast<const float4 *>(A + (size_t)(m0 + i) * lda + k4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) b4[kk] = *reinterpret_cast<const float4 *>(B + (size_t)(k4 + kk) * ldb + n0);
+#pragma unroll
+            for (int i = 0; i < RM; ++i) {
+                const float av[4] = {a4[i].x, a4[i].y, a4[i].z, a4[i].w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    acc.c[i][0] = fmaf(av[kk], b4[kk].x, acc.c[i][0]);
+                    acc.c[i][1] = fmaf(av[kk], b4[kk].y, acc.c[i][1]);
+                    acc.c[i][2] = fmaf(av[kk], b4[kk].z, acc.c[i][2]);
+                    acc.c[i][3] = fmaf(av[kk], b4[kk].w, acc.c[i][3]);
+                }
+            }
+        }
+        return;
+    }
     float4 bn = *reinterpret_cast<const float4 *>(B + n0);
     float an[RM];
     load_a<M, A_COL>(an, A, lda, 0, m0);
@@ -584,10 +608,16 @@ size_t bwd_chunk_ckpt_bytes(int B, int T, int H) {
     return (size_t)B * H * nck * kN * kN * sizeof(float);
 }
 
+cudaError_t bwd_chunk_tc(int B, int T, int H, wkv7_dtype g_dt, const void *r, const void *w, const void *k,
+                         const void *v, const void *a, const void *b, const void *dy, const float *ckpt,
+                         const float *sfin, const float *dS_out, void *dr, void *dw, void *dk, void *dv, void *da,
+                         void *db, long long wait_limit, cudaStream_t st);
+
 cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
-                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st) {
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
+                        cudaStream_t st) {
     using namespace bwdc;
     const int heads = B * H, nck = (T + L - 1) / L;
     {   // dS at every chunk end, and ds0; split rows over two CTAs when the
@@ -613,6 +643,10 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    // chunk gradients: tensor cores for bf16 inputs, fp32 CUDA-core products for fp32 inputs
+    if (in_dt == WKV7_BF16)
+        return bwd_chunk_tc(B, T, H, g_dt, r, w, k, v, a, b, dy, ckpt, sfin, dS_out, dr, dw, dk, dv, da, db,
+                            wait_limit, st);
     const dim3 grid((unsigned)((size_t)heads * nck));
 #define WKV7_CHUNK_BWD(I, G)                                                                                 \
     do {                                                                                                     \

@@ -5,6 +5,7 @@
 #include "fwd_seq.cu"
 #include "step.cu"
 #include "bwd_chunk.cu"
+#include "bwd_chunk_tc.cu"
 #include "fwd_chunk.cu"
 #include "bwd_noalloc.cu"
 #include "fwd_host.cu"

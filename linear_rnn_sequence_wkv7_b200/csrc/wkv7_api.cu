@@ -23,7 +23,8 @@ cudaError_t step(int B, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
 cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
-                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, cudaStream_t st);
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
+                        cudaStream_t st);
 size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
@@ -277,7 +278,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
                         : fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
-                                 dv, da, db, ds0, stream));
+                                 dv, da, db, ds0, lim > 0 ? lim : kDefaultWaitCycles, stream));
 }
 
 void wkv7_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }

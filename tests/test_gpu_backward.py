@@ -50,9 +50,12 @@ def test_fp32_small(cuda_device, T):
         assert_close(got, ref, TAU_F32, name)
 
 
-@pytest.mark.parametrize("T", [16, 77])
-def test_bf16_inputs(cuda_device, T):
-    d = _case(2, T, 3, 400 + T, "bf16", dsT=False)
+@pytest.mark.parametrize("T,with_dsT", [(1, True), (16, False), (32, True), (33, False), (77, False),
+                                         (200, True)])
+def test_bf16_inputs(cuda_device, T, with_dsT):
+    """bf16 inputs (chunk gradients on the tensor cores): one token, a full
+    chunk, ragged tails, several chunks, with and without dsT."""
+    d = _case(2, T, 3, 400 + T, "bf16", dsT=with_dsT)
     ref = _ref(d)
     for name, got, r in zip(GRAD_NAMES, _gpu(d), ref):
         assert_close(got, r, TAU_BF16, name)
@@ -111,4 +114,23 @@ def test_training_workload_sampled_heads(cuda_device):
     got = _gpu(d, heads=heads)
     ref = _ref(d, heads)
     for name, g, r in zip(GRAD_NAMES, got, ref):
+        assert_close(g, r, TAU_BF16, name)
+
+
+def test_bf16_wait_timeout_reports_and_recovers(cuda_device):
+    """Device-side waits forced to run out (limit 1 cycle): the backward's
+    tensor-core kernels report WKV7_ERR_TIMEOUT without a fault, and the next
+    call at the default limit is correct."""
+    d = _case(1, 70, 2, 450, "bf16")
+    assert wkv7.device_status() == wkv7.OK
+    wkv7.set_wait_limit(1)
+    try:
+        _gpu(d)
+        status = wkv7.device_status()
+    finally:
+        wkv7.set_wait_limit(0)
+    assert status == wkv7.ERR_TIMEOUT
+    got = _gpu(d)
+    assert wkv7.device_status() == wkv7.OK
+    for name, g, r in zip(GRAD_NAMES, got, _ref(d)):
         assert_close(g, r, TAU_BF16, name)
