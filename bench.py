@@ -336,8 +336,10 @@ def bench_backward(args, dist, peaks, device, d):
             "ms_per_step": per * 1e3,
             "steps": steps, "launches": 3 * steps,
             "roofline": {"bound": "alu", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                         "per_unit": "28*N^2 flop per head-token",
-                         "kernels": "checkpoints (chunked forward), dS chain, per-chunk gradients (fp32)",
+                         "per_unit": "28*N^2 flop per head-token (the fp32 algebra of the chunked adjoint)",
+                         "kernels": "checkpoints (chunked forward), dS chain, per-chunk gradients "
+                                    "(tcgen05, bf16 hi/lo operands, fp32 accumulation)",
+                         "tensor_frac": ach / peaks["bf16_tflops"],
                          "hbm_frac": bwd_bytes(B, T, H) / per / 1e9 / peaks["hbm_gbs"]},
             "config": {"workload": "train_bwd_b8_t4096_h32", "B": B, "T": T, "H": H, "N": N,
                        "grad_dtype": "bf16", "dsT": "zero"}}

@@ -236,7 +236,9 @@ WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
  * input and the initial state.  Three launches: state checkpoints every 32
  * tokens, a reverse sweep of the state gradient that records dL/dS at every
  * chunk end (and ds0), then the input gradients of every chunk independently
- * (the adjoint of the chunked form of the recurrence, in fp32).
+ * (the adjoint of the chunked form of the recurrence): on the tensor cores
+ * for bf16 inputs (bf16 hi/lo operands, fp32 accumulation), in fp32 on the
+ * CUDA cores for fp32 inputs.
  *   r..b, s0         : the forward's inputs (s0 NULL = zeros)
  *   dy               : [B, T, H, N] of in_dtype
  *   dsT              : [B, H, N, N] fp32, or NULL for zeros
@@ -278,8 +280,8 @@ WKV7_API wkv7_status wkv7_backward_noalloc(int B, int T, int H, int N, wkv7_dtyp
 
 /*
  * Bound, in SM clock cycles, on every device-side wait of kernels launched
- * afterwards from this process (the chunked forward's tensor-core round
- * handshakes).  A wait that runs out sets WKV7_ERR_TIMEOUT in the device status
+ * afterwards from this process (the tensor-core round handshakes of the
+ * chunked forward and of the backward's chunk gradients).  A wait that runs out sets WKV7_ERR_TIMEOUT in the device status
  * word, lets already-committed tensor-core work finish, frees its tensor
  * memory and returns; the context stays usable.  0 restores the default
  * (about one second).  Meant for testing that path.
