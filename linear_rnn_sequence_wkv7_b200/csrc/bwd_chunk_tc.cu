@@ -79,6 +79,8 @@ constexpr int LDQ = 68;
 constexpr uint32_t CQ = VYZ_HI;                       // fp32 [4][32][68]: q terms of dr, da, db, dk
 constexpr uint32_t CPART = CQ + 4 * 32 * LDQ * 4;     // fp32 [8][64]: per-warp sums of S_out dS
 constexpr uint32_t DWTOT = CPART + 8 * 64 * 4;        // fp32 [4][64]: token-block sums of q
+constexpr uint32_t GSTG = DWTOT + 4 * 64 * 4;         // the four gradient tiles, rows padded by 16 B (<= 34816 B)
+static_assert(GSTG + 4 * 32 * (64 * 4 + 16) <= RAW, "gradient staging ends before the token tiles");
 constexpr uint32_t BAR = ZSM + 1024;                  // 5 mbarriers (rounds A..E)
 constexpr uint32_t TMEM_SLOT = BAR + 40;
 constexpr uint32_t FLAG = BAR + 44;
@@ -621,8 +623,10 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     for (int e = 0; e < 32; ++e) x[e] = x[e] * pv[e];
                     dst = q4 == 2 ? db : dk;
                 }
-                if (rrow < Lc) {
-                    GradT *o = dst + base + (size_t)rrow * tok_stride + j0;
+                (void)dst;
+                {   // into the staging tile of this gradient (row rrow, columns j0 ..); written out coalesced below
+                    constexpr int PITCH = kN * (int)sizeof(GradT) + 16;
+                    GradT *o = reinterpret_cast<GradT *>(sm + GSTG + (q4 * L + rrow) * PITCH) + j0;
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
                         store4(o + 4 * u, make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
@@ -659,6 +663,17 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 }
             }
             csync();
+            {   // the four gradient tiles to global memory, 16 bytes per thread and step, a row per 8 or 16 threads
+                constexpr int PITCH = kN * (int)sizeof(GradT) + 16;
+                constexpr int CPR = kN * (int)sizeof(GradT) / 16;                // 16-byte chunks per row
+                for (int x = tid; x < 4 * L * CPR; x += NC) {
+                    const int ch = x % CPR, row = (x / CPR) % L, tile = x / (CPR * L);
+                    GradT *g = tile == 0 ? dr : tile == 1 ? da : tile == 2 ? db : dk;
+                    if (row < Lc)
+                        *reinterpret_cast<uint4 *>(g + base + (size_t)row * tok_stride + ch * 16 / (int)sizeof(GradT)) =
+                            *reinterpret_cast<const uint4 *>(sm + GSTG + (tile * L + row) * PITCH + 16 * ch);
+                }
+            }
             {   // dw_m = sum_{t >= m} q_t / w_m: thread -> column j, block of 8 tokens
                 const float *cq = reinterpret_cast<const float *>(sm + CQ);
                 const float *cp = reinterpret_cast<const float *>(sm + CPART);
