@@ -58,7 +58,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--algo", default="auto", choices=["auto", "seq", "chunk"])
-    p.add_argument("--parts", default="fwd,bwd,decode,long")
+    p.add_argument("--parts", default="fwd,bwd,train,decode,long")
     p.add_argument("--decode-steps", type=int, default=DEC["steps"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -345,6 +345,47 @@ def bench_backward(args, dist, peaks, device, d):
                        "grad_dtype": "bf16", "dsT": "zero"}}
 
 
+def bench_train(args, dist, peaks, device, d):
+    """One training step of the recurrence on the training workload: the
+    forward that keeps the chunk states, then the backward from them, against
+    the forward followed by the self-contained backward."""
+    import torch
+    from linear_rnn_sequence_wkv7_b200 import wkv7
+    cfg = BWD
+    B, T, H = cfg["B"], cfg["T"], cfg["H"]
+    dev = [to_dev(d[n], device) for n in inputs.INPUT_NAMES]
+    s0 = to_dev(d["s0"], device)
+    dy = to_dev(inputs.gen_dy(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16"), device)
+    y = torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device)
+    sT = torch.empty(B, H, N, N, dtype=torch.float32, device=device)
+    states = torch.empty(B, H, (T + 31) // 32, N, N, dtype=torch.float32, device=device)
+    grads = [torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device) for _ in range(6)]
+    grads.append(torch.empty(B, H, N, N, dtype=torch.float32, device=device))
+    ws_b = torch.empty(wkv7.backward_from_states_workspace_size(B, T, H, N), dtype=torch.uint8, device=device)
+    ws_full = torch.empty(wkv7.backward_workspace_size(B, T, H, N), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        wkv7.forward_train(*dev, s0, y=y, sT=sT, states=states, stream=stream)
+        wkv7.backward_from_states(*dev, states, sT, dy, None, grad_dtype=torch.bfloat16, workspace=ws_b,
+                                  out=grads, stream=stream)
+
+    def step_separate():
+        wkv7.forward(*dev, s0=s0, y=y, sT=sT, stream=stream)
+        wkv7.backward(*dev, s0, dy, None, grad_dtype=torch.bfloat16, workspace=ws_full, out=grads, stream=stream)
+
+    steps = max(3, min(args.steps // 20, 10))
+    per = timed(step, steps, 2, dist, stream) / steps
+    per_sep = timed(step_separate, steps, 2, dist, stream) / steps
+    return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
+            "ms_per_step": per * 1e3, "steps": steps, "launches": 4 * steps,
+            "separate_ms_per_step": per_sep * 1e3,
+            "note": "wkv7_forward_train + wkv7_backward_from_states; separate = wkv7_forward + wkv7_backward "
+                    "(which recomputes the chunk states)",
+            "config": {"workload": "train_bwd_b8_t4096_h32", "B": B, "T": T, "H": H, "N": N,
+                       "y_dtype": "bf16", "grad_dtype": "bf16", "dsT": "zero"}}
+
+
 def bench_decode(args, dist, peaks, device, steps_in):
     import torch
     from linear_rnn_sequence_wkv7_b200 import wkv7
@@ -466,6 +507,8 @@ def run_ours(args):
     launches = fwd["launches"]
     if "bwd" in parts:
         out_parts["backward"] = bench_backward(args, dist, peaks, device, fwd["sample"])
+    if "train" in parts:
+        out_parts["train_step"] = bench_train(args, dist, peaks, device, fwd["sample"])
     if gen_thread is not None:
         gen_thread.join()
         out_parts["decode"] = bench_decode(args, dist, peaks, device, steps_in)

@@ -255,6 +255,46 @@ WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dty
                           cudaStream_t stream);
 
 /*
+ * Training pair: a forward that also keeps what the backward needs, and a
+ * backward that starts from it instead of recomputing the states (saves the
+ * checkpoint pass, about a sixth of wkv7_backward on the training workload).
+ *
+ * Bytes of the saved states: the state before every 32-token chunk,
+ * [B, H, ceil(T / 32), N, N] fp32 (512 B per head-token at N = 64).
+ */
+WKV7_API size_t wkv7_saved_states_size(int B, int T, int H, int N);
+
+/*
+ * wkv7_forward that also writes `states` (wkv7_saved_states_size() bytes,
+ * device, overwritten; states[b][h][c] = the state before token 32 c).  sT is
+ * required here (the backward reads it as the state after the last chunk).
+ * Same arguments, algorithms, results and errors as wkv7_forward otherwise.
+ */
+WKV7_API wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
+                                        const void *r, const void *w, const void *k, const void *v,
+                                        const void *a, const void *b, const float *s0, void *y, float *sT,
+                                        float *states, wkv7_algo algo, int chunk_len, void *workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of scratch wkv7_backward_from_states needs: dL/dS at the end of every
+ * 32-token chunk, fp32. */
+WKV7_API size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, int N);
+
+/*
+ * wkv7_backward given the states and sT that wkv7_forward_train wrote for the
+ * same inputs (s0 is not needed: states[.][.][0] is it).  Two launches: the
+ * state-gradient sweep and the chunk gradients.  Same gradients, dtypes and
+ * errors as wkv7_backward.
+ */
+WKV7_API wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                               wkv7_dtype grad_dtype, const void *r, const void *w,
+                                               const void *k, const void *v, const void *a, const void *b,
+                                               const float *states, const float *sT, const void *dy,
+                                               const float *dsT, void *dr, void *dw, void *dk, void *dv,
+                                               void *da, void *db, float *ds0, void *workspace,
+                                               size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * wkv7_backward without workspace: the same computation, arguments and
  * outputs, with its scratch taken from a fixed 32 MiB array in device memory
  * that belongs to the library.  The pages have no counterpart of this call; it

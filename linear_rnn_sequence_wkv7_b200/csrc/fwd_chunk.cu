@@ -143,9 +143,10 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     float *sTp = (sT && (st_only_z < 0 || st_only_z == z)) ? sT + (st_only_z < 0 ? (size_t)z * sT_zstride : 0) + st_base
                                                             : nullptr;
     const int nchunks = (T + L - 1) / L;
-    // optional state checkpoints (one-segment runs): the state before every
-    // chunk, [B][H][nchunks][64][64]
-    float *ckp = ckpt ? ckpt + ((size_t)bb * H + h) * nchunks * kN * kN : nullptr;
+    // optional state checkpoints: the state before every chunk of the whole
+    // sequence, [B][H][ceil(T_total / L)][64][64]; a segment writes the slots
+    // of its own chunks (t_seg is a multiple of L)
+    float *ckp = ckpt ? ckpt + (((size_t)bb * H + h) * ((T_total + L - 1) / L) + t_begin / L) * kN * kN : nullptr;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
     int last_k = -1;                                 // issuer: last committed round and its parity
     uint32_t last_par = 0;
@@ -831,13 +832,13 @@ cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      int nseg, void *workspace, long long wait_limit, cudaStream_t st) {
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt) {
     if (nseg <= 1)
-        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt);
     int t_seg;
     seg_split(T, nseg, t_seg, nseg);
     if (nseg <= 1)
-        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt);
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
     float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg][B][H][64][64]
@@ -850,7 +851,7 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
     if (e != cudaSuccess) return e;
     // pass 3: every segment from its true entry state; the last one writes sT
     return launch_chunk(B, T, H, t_seg, nseg, nseg, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 1,
-                        wait_limit, st);
+                        wait_limit, st, ckpt);
 }
 
 }  // namespace wkv7

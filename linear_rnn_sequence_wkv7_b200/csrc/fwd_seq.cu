@@ -16,13 +16,13 @@
 // CTA; every lane reads them as broadcast float4s (the interleaved column
 // assignment keeps the 4 lanes of a row group on distinct banks).
 //
-// CKPT mode (used by the backward) writes the state before every CK-th token
-// to a checkpoint buffer instead of producing y.
+// CKPT mode writes the state before every CK-th token to a checkpoint buffer
+// (the backward's first pass, without y; the training forward, with y).
 #include "common.cuh"
 
 namespace wkv7 {
 
-template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT>
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT>
 __global__ void __launch_bounds__((RB / RPT) * 4)
 fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
                const InT *__restrict__ k, const InT *__restrict__ v, const InT *__restrict__ a,
@@ -165,10 +165,10 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
                         float s = S[rr][4 * m + e];
                         s = fmaf(s, wj[e], fmaf(p[rr], bj[e], vi[rr] * kj[e]));
                         S[rr][4 * m + e] = s;
-                        if constexpr (!CKPT) yacc[rr] = fmaf(s, rj[e], yacc[rr]);
+                        if constexpr (YOUT) yacc[rr] = fmaf(s, rj[e], yacc[rr]);
                     }
             }
-            if constexpr (!CKPT) {
+            if constexpr (YOUT) {
 #pragma unroll
                 for (int rr = 0; rr < RPT; ++rr) {
                     yacc[rr] += __shfl_xor_sync(0xffffffffu, yacc[rr], 1);
@@ -194,14 +194,14 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
     }
 }
 
-template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT>
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT = !CKPT>
 static cudaError_t launch_fwd_seq(int B, int T, int H, const void *r, const void *w, const void *k,
                                   const void *v, const void *a, const void *b, const float *s0, void *y,
                                   float *sT, float *ckpt, int CK, cudaStream_t st) {
     constexpr int NT = (RB / RPT) * 4;
     size_t smem = 2 * 6 * TT * kN * sizeof(InT);
     if (!std::is_same<InT, float>::value) smem += 6 * TT * kN * sizeof(float);
-    auto kern = fwd_seq_kernel<InT, OutT, RPT, RB, TT, CKPT>;
+    auto kern = fwd_seq_kernel<InT, OutT, RPT, RB, TT, CKPT, YOUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(H * (kN / RB), B);
@@ -234,6 +234,24 @@ cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r
     if (in_dt == WKV7_F32)
         return launch_fwd_seq<float, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
     return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
+}
+
+// The forward with y and the state checkpoints every CK tokens (the training
+// forward: the backward then skips its own checkpoint pass).
+cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
+                          const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
+                          float *sT, float *ckpt, int CK, cudaStream_t st) {
+    constexpr int RPT = 2, RB = 32, TT = 16;
+    if (in_dt == WKV7_F32 && y_dt == WKV7_F32)
+        return launch_fwd_seq<float, float, RPT, RB, TT, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
+    if (in_dt == WKV7_F32 && y_dt == WKV7_BF16)
+        return launch_fwd_seq<float, __nv_bfloat16, RPT, RB, TT, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK,
+                                                                             st);
+    if (in_dt == WKV7_BF16 && y_dt == WKV7_F32)
+        return launch_fwd_seq<__nv_bfloat16, float, RPT, RB, TT, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK,
+                                                                             st);
+    return launch_fwd_seq<__nv_bfloat16, __nv_bfloat16, RPT, RB, TT, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT,
+                                                                                 ckpt, CK, st);
 }
 
 }  // namespace wkv7

@@ -28,7 +28,10 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
 size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      int nseg, void *workspace, long long wait_limit, cudaStream_t st);
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt);
+cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
+                          const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
+                          float *sT, float *ckpt, int CK, cudaStream_t st);
 int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last);
 cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
                                   const void *a, const void *b, const float *s0, float *ckpt, float *sT,
@@ -137,10 +140,17 @@ size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dty
     return chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms, false));
 }
 
-wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+}  // extern "C"
+
+namespace wkv7 {
+namespace {
+
+// wkv7_forward, and with ckpt non-null the training forward that also keeps
+// the state before every 32-token chunk
+wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
                          const void *w, const void *k, const void *v, const void *a, const void *b,
-                         const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len,
-                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+                         const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream, float *ckpt) {
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
@@ -165,9 +175,67 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
                 nseg = want;
         }
         return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
-                                   lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt));
     }
+    if (ckpt) return from_cuda(fwd_seq_train(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, ckpt, kBwdChunk, stream));
     return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+}
+
+}  // namespace
+}  // namespace wkv7
+
+extern "C" {
+
+wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                         const void *w, const void *k, const void *v, const void *a, const void *b,
+                         const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
+                        workspace_bytes, stream, nullptr);
+}
+
+size_t wkv7_saved_states_size(int B, int T, int H, int N) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
+    return bwd_ckpt_bytes(B, T, H);
+}
+
+wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
+                               const void *w, const void *k, const void *v, const void *a, const void *b,
+                               const float *s0, void *y, float *sT, float *states, wkv7_algo algo, int chunk_len,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if ((size_t)B * H > 0 && (!ptr_ok(sT) || (T > 0 && !ptr_ok(states)))) return WKV7_ERR_INVALID_ARG;
+    return forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
+                        workspace_bytes, stream, states);
+}
+
+size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, int N) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
+    return round_up(bwd_ckpt_bytes(B, T, H));
+}
+
+wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt,
+                                      const void *r, const void *w, const void *k, const void *v, const void *a,
+                                      const void *b, const float *states, const float *sT, const void *dy,
+                                      const float *dsT, void *dr, void *dw, void *dk, void *dv, void *da,
+                                      void *db, float *ds0, void *workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(g_dt)) return WKV7_ERR_INVALID_ARG;
+    if (!opt_ptr_ok(dsT) || !ptr_ok(ds0)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (T == 0) return copy_or_zero_state(ds0, dsT, B, H, stream);
+    for (const void *p : {r, w, k, v, a, b, dy, (const void *)states, (const void *)sT, (const void *)dr,
+                          (const void *)dw, (const void *)dk, (const void *)dv, (const void *)da, (const void *)db})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    if (workspace_bytes < wkv7_backward_from_states_workspace_size(B, T, H, N) || !ptr_ok(workspace))
+        return WKV7_ERR_INVALID_ARG;
+    const long long lim = g_wait_limit.load();
+    return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, states, sT,
+                                 static_cast<float *>(workspace), dr, dw, dk, dv, da, db, ds0,
+                                 lim > 0 ? lim : kDefaultWaitCycles, stream));
 }
 
 size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N) {

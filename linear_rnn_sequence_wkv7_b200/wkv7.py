@@ -27,6 +27,8 @@ EXPORTED_SYMBOLS = (
     "wkv7_forward_resolve_algo", "wkv7_backward_noalloc", "wkv7_set_wait_limit",
     "wkv7_forward_summary", "wkv7_compose_states", "wkv7_forward_summary_workspace_size",
     "wkv7_forward_continue", "wkv7_forward_host_workspace_size", "wkv7_forward_host",
+    "wkv7_saved_states_size", "wkv7_forward_train", "wkv7_backward_from_states_workspace_size",
+    "wkv7_backward_from_states",
 )
 
 _lib = None
@@ -74,6 +76,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_forward_host_workspace_size.restype = z
     lib.wkv7_forward_host.argtypes = [i, i, i, i, i, i] + [vp] * 9 + [i, i, vp, z, vp]
     lib.wkv7_forward_host.restype = i
+    lib.wkv7_saved_states_size.argtypes = [i, i, i, i]
+    lib.wkv7_saved_states_size.restype = z
+    lib.wkv7_forward_train.argtypes = [i, i, i, i, i, i] + [vp] * 10 + [i, i, vp, z, vp]
+    lib.wkv7_forward_train.restype = i
+    lib.wkv7_backward_from_states_workspace_size.argtypes = [i, i, i, i]
+    lib.wkv7_backward_from_states_workspace_size.restype = z
+    lib.wkv7_backward_from_states.argtypes = [i, i, i, i, i, i] + [vp] * 17 + [vp, z, vp]
+    lib.wkv7_backward_from_states.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_set_wait_limit.argtypes = [ctypes.c_longlong]
@@ -294,6 +304,61 @@ def backward(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.float32, wo
                            *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)),
                            _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     _check("wkv7_backward", st)
+    return tuple(out)
+
+
+def saved_states_size(B, T, H, N) -> int:
+    return load_library().wkv7_saved_states_size(B, T, H, N)
+
+
+def backward_from_states_workspace_size(B, T, H, N) -> int:
+    return load_library().wkv7_backward_from_states_workspace_size(B, T, H, N)
+
+
+def forward_train(r, w, k, v, a, b, s0=None, *, y=None, sT=None, states=None, y_dtype=None, algo="auto",
+                  chunk_len=0, workspace=None, stream=None):
+    """(y, sT, states): the forward plus the state before every 32-token chunk,
+    [B, H, ceil(T/32), N, N] fp32, for ``backward_from_states``."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    ycode = _dt(r) if y_dtype is None else (F32 if y_dtype == torch.float32 else BF16)
+    if y is None:
+        y = torch.empty((B, T, H, N), dtype=_tdt(ycode), device=r.device)
+    if sT is None:
+        sT = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    if states is None:
+        states = torch.empty((B, H, (T + 31) // 32, N, N), dtype=torch.float32, device=r.device)
+    if s0 is not None:
+        _same((s0,), (B, H, N, N), torch.float32)
+    ws_bytes = lib.wkv7_forward_workspace_size(B, T, H, N, _dt(r), ALGOS[algo], chunk_len)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=r.device)
+    st = lib.wkv7_forward_train(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s0, y, sT, states)),
+                                ALGOS[algo], chunk_len, _ptr(workspace),
+                                0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("wkv7_forward_train", st)
+    return y, sT, states
+
+
+def backward_from_states(r, w, k, v, a, b, states, sT, dy, dsT=None, *, grad_dtype=torch.float32,
+                         workspace=None, out=None, stream=None):
+    """(dr, dw, dk, dv, da, db, ds0) from the states and sT of ``forward_train``."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b, dy), r.shape, r.dtype)
+    gcode = F32 if grad_dtype == torch.float32 else BF16
+    if out is None:
+        out = [torch.empty((B, T, H, N), dtype=grad_dtype, device=r.device) for _ in range(6)]
+        out.append(torch.empty((B, H, N, N), dtype=torch.float32, device=r.device))
+    ws_bytes = lib.wkv7_backward_from_states_workspace_size(B, T, H, N)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=r.device)
+    st = lib.wkv7_backward_from_states(B, T, H, N, _dt(r), gcode,
+                                       *map(_ptr, (r, w, k, v, a, b, states, sT, dy, dsT, *out)),
+                                       _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                       _stream(stream))
+    _check("wkv7_backward_from_states", st)
     return tuple(out)
 
 

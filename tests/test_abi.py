@@ -148,3 +148,27 @@ def test_forward_host_rejects_invalid_arguments(lib):
     need = lib.wkv7_forward_host_workspace_size(B, T, H, 64, wkv7.BF16, wkv7.BF16, wkv7.ALGO_CHUNK, 0)
     assert need >= 2 * 7 * B * (T // 8) * H * 64 * 2 + B * H * 64 * 64 * 4
     assert lib.wkv7_forward_host_workspace_size(B, T, H, 16, wkv7.BF16, wkv7.BF16, 0, 0) == 0
+
+
+def test_training_pair_rejects_invalid_arguments(lib):
+    ft = lambda B=1, T=64, H=1, N=64, ptrs=None: lib.wkv7_forward_train(
+        B, T, H, N, wkv7.BF16, wkv7.BF16, *(ptrs or [P] * 10), 0, 0, None, 0, None)
+    assert ft(N=32) == wkv7.ERR_UNSUPPORTED
+    bad = [P] * 10
+    bad[8] = None                                        # sT is required
+    assert ft(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 10
+    bad[9] = None                                        # states are required
+    assert ft(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert ft(B=0) == wkv7.OK
+    bs = lambda T=64, ptrs=None, nb=1 << 40: lib.wkv7_backward_from_states(
+        1, T, 1, 64, wkv7.BF16, wkv7.F32, *(ptrs or [P] * 17), P, nb, None)
+    assert bs(nb=16) == wkv7.ERR_INVALID_ARG             # workspace too small
+    bad = [P] * 17
+    bad[6] = None                                        # states missing
+    assert bs(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 17
+    bad[16] = None                                       # ds0 is required
+    assert bs(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert lib.wkv7_saved_states_size(2, 100, 3, 64) == 2 * 3 * 4 * 64 * 64 * 4
+    assert lib.wkv7_backward_from_states_workspace_size(2, 100, 3, 64) >= 2 * 3 * 4 * 64 * 64 * 4
