@@ -178,3 +178,32 @@ def test_orchestration_without_process_group(cuda_device):
     assert torch.equal(s_in, s0)
     assert_close(to_f64(y), to_f64(y1), TAU_BF16, "y", bf16_out=True)
     assert_close(to_f64(s_fin), to_f64(s1), TAU_BF16, "sT")
+
+
+def test_orchestration_over_a_one_rank_nccl_group(cuda_device):
+    """forward_context_parallel inside an NCCL process group of one rank: the
+    all-gather, composition and continue run on the GPU through NCCL and the
+    library; the result equals the plain forward."""
+    import os
+    import socket
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        B, T, H, N = 1, 1000, 4, 64
+        d = inputs.gen_sequence(B, T, H, N, seed=811, dtype="bf16", s0_std=0.1)
+        args = _dev_args(d)
+        s0 = to_dev(d["s0"])
+        y, s_in, s_fin = forward_context_parallel(*args, s0)
+        y1, s1 = wkv7.forward(*args, s0=s0)
+        torch.cuda.synchronize()
+        assert torch.equal(s_in, s0)
+        assert_close(to_f64(y), to_f64(y1), TAU_BF16, "y", bf16_out=True)
+        assert_close(to_f64(s_fin), to_f64(s1), TAU_BF16, "sT")
+    finally:
+        dist.destroy_process_group()
