@@ -144,8 +144,9 @@ WKV7_API size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N);
  *   workspace        : wkv7_forward_summary_workspace_size() bytes, or NULL.
  *                      With it the stretch runs as segments whose summaries
  *                      are chained into E and M and stay in the workspace for
- *                      wkv7_forward_continue; without it, one launch of the
- *                      two runs (from S = 0, and from S = I with v read as 0).
+ *                      wkv7_forward_continue; without it, one launch that
+ *                      carries both states through the stretch (from S = 0,
+ *                      and from S = I with v read as 0).
  * Shares the chunked form's numeric domain (see wkv7_forward).
  */
 WKV7_API wkv7_status wkv7_forward_summary(int B, int T, int H, int N, wkv7_dtype in_dtype,

@@ -7,8 +7,9 @@ v_t k_t^T is affine in the state, because the transition does not depend on S
 state to its final state as S_out = S_in M + E.  So each rank
 
   1. computes the summary [E; M] of its own stretch (wkv7_forward_summary: the
-     stretch's segments run side by side from S = 0 and from S = I with v read
-     as 0, and their summaries are chained into E and M);
+     stretch's segments run side by side, each carrying one state from S = 0
+     and one from S = I with v read as 0, and their summaries are chained
+     into E and M);
   2. all-gathers the summaries (2 B H N^2 fp32 per rank: 1 MiB for B = 1,
      H = 32, N = 64);
   3. composes the entry state of every stretch (wkv7_compose_states), which

@@ -70,6 +70,7 @@ constexpr int NC = 256;            // compute threads (warps 0-7)
 constexpr int NT = NC + 32;        // + the MMA warp
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_X = 0, COL_Z = 64, COL_MQ = 192;
+constexpr uint32_t TMEM_COLS_DUAL = 512, COL_S2 = 256;   // dual runs: the second state's [S_out^T; .]
 
 // shared memory map (bytes)
 constexpr uint32_t IN_W = 0, IN_R = 4096, IN_K = 8192, IN_A = 12288, IN_B = 16384;   // [32][128 B], rotated
@@ -86,6 +87,8 @@ constexpr uint32_t LABT = R + 8192;                 //   P1: fp32 L_ab^T [32][36
 constexpr uint32_t LAK = R + 12800;                 //   P1: fp32 L_ak [32][33] (padded)
 constexpr uint32_t WU_HI = R, WU_LO = R + 8192;     //   P2..R3: [128][32] = W'^T rows, U~^T rows
 constexpr uint32_t SMEM_BYTES = R + 17024;
+constexpr uint32_t S2_HI = SMEM_BYTES, S2_LO = S2_HI + 8192;   // dual runs: S^T of the second state
+constexpr uint32_t SMEM_BYTES_DUAL = S2_LO + 8192;
 // in the free halves of RZ (bytes [1024, 2048) of each 2 KB group)
 constexpr uint32_t TSM = RZ_HI + 1024;              // fp32 T, row t at TSM + (t/8)*2048 + (t%8)*128
 constexpr uint32_t ZSM = RZ_LO + 1024;              // fp32 [16][16]
@@ -116,13 +119,19 @@ constexpr uint32_t BAR_READY = 2, BAR_DONE = 6;
 
 }  // namespace chunk
 
-template <typename OutT>
-__global__ void __launch_bounds__(chunk::NT, 2)
+// DUAL: a summary run that carries two states through the same chunk algebra,
+// S from S_in (here 0, giving the segment's E) and S2 from I (giving M): the
+// chunk's operands, T, W', M and Q do not depend on the state, so only the
+// state round R4 and its read-out are done twice.  No y.  It needs a second S
+// operand and 64 more TMEM columns, so these CTAs run one per SM.
+template <typename OutT, bool DUAL>
+__global__ void __launch_bounds__(chunk::NT, DUAL ? 1 : 2)
 fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *__restrict__ r,
                  const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
-                 float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt) {
+                 float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt,
+                 float *m_out, long long m_zstride) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -133,7 +142,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     // "transition" run of segment z - nseg (state starts at I, v taken as 0),
     // whose final state is the segment's linear map S -> S M_seg.
     const int seg = z % nseg;
-    const bool transition = z >= nseg;
+    const bool transition = !DUAL && z >= nseg;
     const int t_begin = seg * t_seg;
     const int T = min(t_seg, T_total - t_begin);     // tokens of this segment
     const size_t tok_stride = (size_t)H * kN;
@@ -186,7 +195,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         }
         *abort_flag = 0;
     }
-    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
+    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
     if (tid < NC) {
         {   // v columns of AV: lo always zero (v is exact), hi zero in transition runs
             const int t = tid >> 3, ch = tid & 7;
@@ -205,6 +214,12 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         }
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part, 64), x);
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part + 8, 64), x + 8);
+        if constexpr (DUAL) {                         // the second state starts at I
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = (16 * part + e == j) ? 1.f : 0.f;
+            store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part, 64), x);
+            store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part + 8, 64), x + 8);
+        }
         if (ckp) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) ckp[(size_t)(16 * part + e) * kN + j] = x[e];
@@ -233,6 +248,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             const OpD wu = opd_k(sbase + WU_HI, sbase + WU_LO, L);            // [W' | U~], K = tokens
             const OpD vv = opd_mn(sbase + AV_HI + 1024, 0, 128);              // V, exact
             const OpD ss = opd_mn(sbase + S_HI, sbase + S_LO, 64);            // S^T, K = key j
+            const OpD ss2 = opd_mn(sbase + S2_HI, sbase + S2_LO, 64);         // dual runs: S2^T
             // One tensor-core round: wait until the compute warps hand it over
             // (bar.arrive on its ready barrier), issue and commit it, wait for
             // the commit, and release the compute warps (bar.sync on its done
@@ -264,6 +280,8 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 });
                 round(3, par, [&] {                         // [S_out^T; Y] += [M^T; Q] S^T
                     gemm_split_ts(tmem + COL_Z + 64, tmem + COL_MQ, tmem + COL_MQ + 32, ss, id_r4, 4, true);
+                    if constexpr (DUAL)                      // [S2_out^T; .] = [M^T; Q] S2^T (no E: v plays no part)
+                        gemm_split_ts(tmem + COL_S2, tmem + COL_MQ, tmem + COL_MQ + 32, ss2, id_r4, 4, false);
                 });
             }
         }
@@ -565,6 +583,24 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dst[(size_t)(32 * hc + e) * kN] = x[e];
                 }
+                if constexpr (DUAL) {             // the same for the second state
+                    tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc, r0);
+                    tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc + 16, r1);
+                    tmem_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        x[e] = __uint_as_float(r0[e]);
+                        x[16 + e] = __uint_as_float(r1[e]);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        store8_split(sm + S2_HI, sm + S2_LO, cm_off(rho, 32 * hc + 8 * u, 64), x + 8 * u);
+                    if (c == nchunks - 1 && m_out != nullptr) {
+                        float *mp = m_out + (size_t)z * m_zstride + st_base;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) mp[(size_t)(32 * hc + e) * kN + rho] = x[e];
+                    }
+                }
             } else if (y) {                       // y row t, channels 32 hc .. 32 hc + 31
                 const int t = rho - 64;
                 if (t < Lv) {
@@ -621,7 +657,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         __syncthreads();
     }
     fence_after_sync();
-    if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 8) tmem_dealloc(tmem, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
 }
 
 // One launch of the chunked kernel over nz = gridDim.z segment runs.
@@ -633,17 +669,36 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
     const size_t smem = chunk::SMEM_BYTES;
 #define WKV7_CHUNK_LAUNCH(O)                                                                                  \
     do {                                                                                                      \
-        auto kern = fwd_chunk_kernel<O>;                                                                      \
+        auto kern = fwd_chunk_kernel<O, false>;                                                               \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
         if (e != cudaSuccess) return e;                                                                       \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
-                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt);             \
+                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0); \
     } while (0)
     if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
     else WKV7_CHUNK_LAUNCH(__nv_bfloat16);
 #undef WKV7_CHUNK_LAUNCH
+    return cudaGetLastError();
+}
+
+// One launch of dual summary runs over nz segments of t_seg tokens: E of
+// segment z (its final state from 0) to e_out + z e_zstride, M (from I, v read
+// as 0) to m_out + z m_zstride.
+static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const void *r, const void *w, const void *k,
+                               const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
+                               float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st) {
+    static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
+    dim3 grid(H, B, nz);
+    const size_t smem = chunk::SMEM_BYTES_DUAL;
+    auto kern = fwd_chunk_kernel<float, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    using bf = __nv_bfloat16;
+    kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k, (const bf *)v,
+                                        (const bf *)a, (const bf *)b, nullptr, 0, (float *)nullptr, e_out, e_zstride,
+                                        -1, wait_limit, nullptr, m_out, m_zstride);
     return cudaGetLastError();
 }
 
@@ -712,15 +767,23 @@ static double launch_rounds(long long n, int sms) {
     return t;
 }
 
+// Relative time of one launch of n dual summary runs (one CTA per SM, each
+// about kDualCost times a plain run alone on its SM; measured on the
+// long-context shape).
+constexpr double kDualCost = 1.15;
+static double dual_rounds(long long n, int sms) {
+    return n > 0 ? kDualCost * (double)((n + sms - 1) / sms) : 0.0;
+}
+
 // Number of sequence segments for a chunked forward over B*H heads.  The
-// segmented form runs 2 (nseg - 1) summary runs and nseg output runs of T/nseg
-// tokens each, i.e. about 3x the work of one pass, so it only pays when B*H
-// CTAs leave most of the GPU idle.  Picks the nseg (segments of at least 4
+// segmented form runs nseg - 1 dual summary runs and nseg output runs of
+// T/nseg tokens each, about 2.3x the work of one pass, so it only pays when
+// B*H CTAs leave most of the GPU idle.  Picks the nseg (segments of at least 4
 // chunks) with the lowest estimated time, if that is below 95% of one pass;
 // among near-ties (within 3%) the fewest segments, which need the least scratch.
 // With summarize_last (the summary / continue pair) the last segment's summary
 // runs too and one segment means two launches (summary, then output), so the
-// cost model counts 2 nseg summary runs and n = 1 competes on equal terms.
+// cost model counts nseg summary runs and n = 1 competes on equal terms.
 int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last) {
     static_assert(2 * (chunk::SMEM_BYTES + 1024) <= 228 * 1024, "two chunk CTAs per SM");
     const long long heads = (long long)B * H;
@@ -729,7 +792,7 @@ int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last) {
     const long long max_n = std::min<long long>(64, chunks / 4);
     const long long extra = summarize_last ? 0 : 1;
     auto cost = [&](long long n) {
-        return (launch_rounds(2 * (n - extra) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
+        return (dual_rounds((n - extra) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
     };
     double best = summarize_last ? cost(1) : 0.95 * launch_rounds(heads, sm_count);
     for (long long n = 2; n <= max_n; ++n) best = std::min(best, cost(n));
@@ -767,11 +830,11 @@ __global__ void summary_empty_kernel(long long zst, float *summary) {
 }
 
 // Affine summary of a whole sequence, S_out = S_in M + E, E to summary[0] and
-// M to summary[1] ([B][H][64][64] each).  One segment: one launch of two runs,
-// E from S_in = 0 and M from S_in = I with v read as 0.  nseg segments: the
-// same two runs for every segment in one launch (their summaries stay in the
-// workspace for fwd_chunk_continue), then E and M of the whole sequence by
-// chaining them: E from 0 through every (E_k, M_k), M from I through the M_k.
+// M to summary[1] ([B][H][64][64] each).  One segment: one dual run (E from
+// S_in = 0 and M from S_in = I with v read as 0).  nseg segments: a dual run
+// for every segment in one launch (their summaries stay in the workspace for
+// fwd_chunk_continue), then E and M of the whole sequence by chaining them:
+// E from 0 through every (E_k, M_k), M from I through the M_k.
 cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
                               const void *a, const void *b, float *summary, int nseg, void *workspace,
                               long long wait_limit, cudaStream_t st) {
@@ -780,14 +843,11 @@ cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w,
         summary_empty_kernel<<<(unsigned)((2 * zst + 255) / 256), 256, 0, st>>>(zst, summary);
         return cudaGetLastError();
     }
-    if (nseg <= 1)
-        return launch_chunk(B, T, H, T, 1, 2, WKV7_BF16, r, w, k, v, a, b, nullptr, 0, nullptr, summary, zst, -1,
-                            wait_limit, st);
+    if (nseg <= 1) return launch_dual(B, T, H, T, 1, r, w, k, v, a, b, summary, zst, summary + zst, zst, wait_limit, st);
     int t_seg, n;
     seg_split(T, nseg, t_seg, n);
     float *em = static_cast<float *>(workspace);                // E_0..E_{n-1}, M_0..M_{n-1}
-    cudaError_t e = launch_chunk(B, T, H, t_seg, n, 2 * n, WKV7_BF16, r, w, k, v, a, b, nullptr, 0, nullptr, em,
-                                 zst, -1, wait_limit, st);
+    cudaError_t e = launch_dual(B, T, H, t_seg, n, r, w, k, v, a, b, em, zst, em + n * zst, zst, wait_limit, st);
     if (e != cudaSuccess) return e;
     e = launch_combine(B, H, n, nullptr, false, em, zst, em + n * zst, zst, summary, 0, st);
     if (e != cudaSuccess) return e;
@@ -842,9 +902,9 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
     float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg][B][H][64][64]
-    // pass 1: E_k (s0 = 0) and M_k (s0 = I, v = 0) for segments 0..nseg-2, no y
-    cudaError_t e = launch_chunk(B, T, H, t_seg, nseg - 1, 2 * (nseg - 1), y_dt, r, w, k, v, a, b, nullptr, 0,
-                                 nullptr, em, zst, -1, wait_limit, st);
+    // pass 1: E_k (from 0) and M_k (from I, v = 0) for segments 0..nseg-2, one dual run each, no y
+    cudaError_t e = launch_dual(B, T, H, t_seg, nseg - 1, r, w, k, v, a, b, em, zst, em + (size_t)(nseg - 1) * zst,
+                                zst, wait_limit, st);
     if (e != cudaSuccess) return e;
     // pass 2: entry state of every segment
     e = launch_combine(B, H, nseg - 1, s0, false, em, zst, em + (size_t)(nseg - 1) * zst, zst, sin, zst, st);
