@@ -131,7 +131,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
                  float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt,
-                 float *m_out, long long m_zstride) {
+                 float *m_out, long long m_zstride, int seg0, int first_out) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -141,21 +141,27 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     // blockIdx.z selects a segment of the sequence; z >= nseg marks a
     // "transition" run of segment z - nseg (state starts at I, v taken as 0),
     // whose final state is the segment's linear map S -> S M_seg.
-    const int seg = z % nseg;
+    const int seg = seg0 + z % nseg;              // seg0: the first segment of this launch
     const bool transition = !DUAL && z >= nseg;
     const int t_begin = seg * t_seg;
     const int T = min(t_seg, T_total - t_begin);     // tokens of this segment
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = (((size_t)bb * T_total + t_begin) * H + h) * kN;
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
-    const float *s0p = s0 ? s0 + (size_t)z * s0_zstride + st_base : nullptr;
+    // A dual launch with first_out makes its first run an output run: from
+    // s0, with y and checkpoints (its E is then the next segment's entry
+    // state).  Every other dual run starts from 0 and writes no y.
+    const bool out_run = !DUAL || (first_out && z == 0);
+    const float *s0p = (s0 && out_run) ? s0 + (size_t)z * s0_zstride + st_base : nullptr;
+    OutT *yo = out_run ? y : nullptr;
     float *sTp = (sT && (st_only_z < 0 || st_only_z == z)) ? sT + (st_only_z < 0 ? (size_t)z * sT_zstride : 0) + st_base
                                                             : nullptr;
     const int nchunks = (T + L - 1) / L;
     // optional state checkpoints: the state before every chunk of the whole
     // sequence, [B][H][ceil(T_total / L)][64][64]; a segment writes the slots
     // of its own chunks (t_seg is a multiple of L)
-    float *ckp = ckpt ? ckpt + (((size_t)bb * H + h) * ((T_total + L - 1) / L) + t_begin / L) * kN * kN : nullptr;
+    float *ckp = (ckpt && out_run) ? ckpt + (((size_t)bb * H + h) * ((T_total + L - 1) / L) + t_begin / L) * kN * kN
+                                   : nullptr;
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + FLAG);
     int last_k = -1;                                 // issuer: last committed round and its parity
     uint32_t last_par = 0;
@@ -214,15 +220,15 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         }
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part, 64), x);
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part + 8, 64), x + 8);
+        if (ckp) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ckp[(size_t)(16 * part + e) * kN + j] = x[e];
+        }
         if constexpr (DUAL) {                         // the second state starts at I
 #pragma unroll
             for (int e = 0; e < 16; ++e) x[e] = (16 * part + e == j) ? 1.f : 0.f;
             store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part, 64), x);
             store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part + 8, 64), x + 8);
-        }
-        if (ckp) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ckp[(size_t)(16 * part + e) * kN + j] = x[e];
         }
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -601,10 +607,10 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                         for (int e = 0; e < 32; ++e) mp[(size_t)(32 * hc + e) * kN + rho] = x[e];
                     }
                 }
-            } else if (y) {                       // y row t, channels 32 hc .. 32 hc + 31
+            } else if (yo) {                      // y row t, channels 32 hc .. 32 hc + 31
                 const int t = rho - 64;
                 if (t < Lv) {
-                    OutT *dst = y + base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+                    OutT *dst = yo + base + (size_t)(c * L + t) * tok_stride + 32 * hc;
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
                         store4(dst + 4 * u, make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
@@ -664,7 +670,8 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz, wkv7_dtype y_dt, const void *r,
                                 const void *w, const void *k, const void *v, const void *a, const void *b,
                                 const float *s0, long long s0_zstride, void *y, float *sT, long long sT_zstride,
-                                int st_only_z, long long wait_limit, cudaStream_t st, float *ckpt = nullptr) {
+                                int st_only_z, long long wait_limit, cudaStream_t st, float *ckpt = nullptr,
+                                int seg0 = 0) {
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES;
 #define WKV7_CHUNK_LAUNCH(O)                                                                                  \
@@ -675,7 +682,8 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
-                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0); \
+                                            (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0,  \
+                                            seg0, 0);                                                         \
     } while (0)
     if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
     else WKV7_CHUNK_LAUNCH(__nv_bfloat16);
@@ -685,20 +693,30 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
 
 // One launch of dual summary runs over nz segments of t_seg tokens: E of
 // segment z (its final state from 0) to e_out + z e_zstride, M (from I, v read
-// as 0) to m_out + z m_zstride.
+// as 0) to m_out + z m_zstride.  With y given, the first segment instead runs
+// from s0 and writes y (and ckpt, if given): its "E" is its true final state.
 static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const void *r, const void *w, const void *k,
                                const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
-                               float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st) {
+                               float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st,
+                               void *y = nullptr, wkv7_dtype y_dt = WKV7_F32, const float *s0 = nullptr,
+                               float *ckpt = nullptr) {
     static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES_DUAL;
-    auto kern = fwd_chunk_kernel<float, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    const int first_out = y != nullptr ? 1 : 0;
     using bf = __nv_bfloat16;
-    kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k, (const bf *)v,
-                                        (const bf *)a, (const bf *)b, nullptr, 0, (float *)nullptr, e_out, e_zstride,
-                                        -1, wait_limit, nullptr, m_out, m_zstride);
+#define WKV7_DUAL_LAUNCH(O)                                                                                    \
+    do {                                                                                                       \
+        auto kern = fwd_chunk_kernel<O, true>;                                                                 \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+        if (e != cudaSuccess) return e;                                                                        \
+        kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k,      \
+                                            (const bf *)v, (const bf *)a, (const bf *)b, s0, 0, (O *)y, e_out, \
+                                            e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out);  \
+    } while (0)
+    if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf);
+    else WKV7_DUAL_LAUNCH(float);
+#undef WKV7_DUAL_LAUNCH
     return cudaGetLastError();
 }
 
@@ -776,9 +794,10 @@ static double dual_rounds(long long n, int sms) {
 }
 
 // Number of sequence segments for a chunked forward over B*H heads.  The
-// segmented form runs nseg - 1 dual summary runs and nseg output runs of
-// T/nseg tokens each, about 2.3x the work of one pass, so it only pays when
-// B*H CTAs leave most of the GPU idle.  Picks the nseg (segments of at least 4
+// segmented form runs nseg - 1 dual summary runs (the first of them also the
+// output run of segment 0) and nseg - 1 output runs of T/nseg tokens each,
+// about twice the work of one pass, so it only pays when B*H CTAs leave most
+// of the GPU idle.  Picks the nseg (segments of at least 4
 // chunks) with the lowest estimated time, if that is below 95% of one pass;
 // among near-ties (within 3%) the fewest segments, which need the least scratch.
 // With summarize_last (the summary / continue pair) the last segment's summary
@@ -790,9 +809,11 @@ int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last) {
     const long long chunks = (T + chunk::L - 1) / chunk::L;
     if (sm_count <= 0 || heads <= 0) return 1;
     const long long max_n = std::min<long long>(64, chunks / 4);
+    // plain forward: dual runs for segments 0..n-2 (the first also writes its
+    // y), output runs for segments 1..n-1; summary / continue: both for all n
     const long long extra = summarize_last ? 0 : 1;
     auto cost = [&](long long n) {
-        return (dual_rounds((n - extra) * heads, sm_count) + launch_rounds(n * heads, sm_count)) / n;
+        return (dual_rounds((n - extra) * heads, sm_count) + launch_rounds((n - extra) * heads, sm_count)) / n;
     };
     double best = summarize_last ? cost(1) : 0.95 * launch_rounds(heads, sm_count);
     for (long long n = 2; n <= max_n; ++n) best = std::min(best, cost(n));
@@ -901,17 +922,19 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
         return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt);
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
-    float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg][B][H][64][64]
-    // pass 1: E_k (from 0) and M_k (from I, v = 0) for segments 0..nseg-2, one dual run each, no y
+    float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg - 1][B][H][64][64]
+    // pass 1: one dual launch over segments 0..nseg-2.  Segment 0 starts
+    // from s0 and writes its y (and checkpoints): its E is the entry state of
+    // segment 1.  Segments k >= 1 give E_k (from 0) and M_k (from I, v = 0).
     cudaError_t e = launch_dual(B, T, H, t_seg, nseg - 1, r, w, k, v, a, b, em, zst, em + (size_t)(nseg - 1) * zst,
-                                zst, wait_limit, st);
+                                zst, wait_limit, st, y, y_dt, s0, ckpt);
     if (e != cudaSuccess) return e;
-    // pass 2: entry state of every segment
-    e = launch_combine(B, H, nseg - 1, s0, false, em, zst, em + (size_t)(nseg - 1) * zst, zst, sin, zst, st);
+    // pass 2: entry states of segments 1..nseg-1, from segment 1's
+    e = launch_combine(B, H, nseg - 2, em, false, em + zst, zst, em + (size_t)nseg * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
-    // pass 3: every segment from its true entry state; the last one writes sT
-    return launch_chunk(B, T, H, t_seg, nseg, nseg, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 1,
-                        wait_limit, st, ckpt);
+    // pass 3: segments 1..nseg-1 from their true entry states; the last one writes sT
+    return launch_chunk(B, T, H, t_seg, nseg - 1, nseg - 1, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 2,
+                        wait_limit, st, ckpt, 1);
 }
 
 }  // namespace wkv7
