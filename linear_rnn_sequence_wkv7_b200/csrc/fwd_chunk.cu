@@ -138,11 +138,9 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x, bb = blockIdx.y, z = blockIdx.z;
-    // blockIdx.z selects a segment of the sequence; z >= nseg marks a
-    // "transition" run of segment z - nseg (state starts at I, v taken as 0),
-    // whose final state is the segment's linear map S -> S M_seg.
-    const int seg = seg0 + z % nseg;              // seg0: the first segment of this launch
-    const bool transition = !DUAL && z >= nseg;
+    // blockIdx.z selects a segment of the sequence (seg0 + z, nseg of them
+    // in this launch).
+    const int seg = seg0 + z % nseg;
     const int t_begin = seg * t_seg;
     const int T = min(t_seg, T_total - t_begin);     // tokens of this segment
     const size_t tok_stride = (size_t)H * kN;
@@ -185,7 +183,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     // v of chunk c straight into its operand (AV columns 64-127); rows past the
     // end keep the zeros P0 writes.  Transition runs keep v = 0.
     auto issue_v = [&](int c) {
-        if (c < nchunks && !transition) {
+        if (c < nchunks) {
             const int t0 = c * L;
             const int t = tid >> 3, ch = tid & 7;
             if (t0 + t < T)
@@ -203,9 +201,8 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
     if (tid < NC) {
-        {   // v columns of AV: lo always zero (v is exact), hi zero in transition runs
+        {   // v columns of AV: lo always zero (v is exact)
             const int t = tid >> 3, ch = tid & 7;
-            if (transition) *reinterpret_cast<uint4 *>(sm + AV_HI + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(sm + AV_LO + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
         }
         issue_in(0);
@@ -216,7 +213,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int i = 16 * part + e;
-            x[e] = transition ? (i == j ? 1.f : 0.f) : (s0p ? s0p[(size_t)i * kN + j] : 0.f);
+            x[e] = s0p ? s0p[(size_t)i * kN + j] : 0.f;
         }
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part, 64), x);
         store8_split(sm + S_HI, sm + S_LO, cm_off(j, 16 * part + 8, 64), x + 8);
