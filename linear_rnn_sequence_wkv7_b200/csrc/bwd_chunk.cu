@@ -8,15 +8,18 @@
 //
 // Three launches:
 //  1. state checkpoints S_in(c) before every chunk of L = 32 tokens and the
-//     final state (the sequential forward in checkpoint mode, fwd_seq.cu);
+//     final state (the chunked forward's epilogue for bf16 inputs,
+//     fwd_chunk.cu; the sequential forward in checkpoint mode for fp32
+//     inputs, fwd_seq.cu);
 //  2. bwd_dstate_kernel: dS_out(c) = dL/dS at the end of every chunk, through
 //     the chunk's own outputs excluded, by a reverse sweep of the state
 //     gradient alone (per row i: g += dy_t[i] r_t; g = g w_t + (g . b_t) a_t);
 //     it needs no state and no column sums (rows are independent, two CTAs
 //     per head), and ends with ds0;
-//  3. bwd_chunk_kernel: one CTA per chunk, all chunks independent given
-//     S_in(c) and dS_out(c): the chunk's six input gradients by fp32 matrix
-//     products in shared memory.
+//  3. the chunks' input gradients, all chunks independent given S_in(c) and
+//     dS_out(c): on the tensor cores for bf16 inputs (bwd_chunk_tc.cu), else
+//     bwd_chunk_kernel below, one CTA per chunk with fp32 matrix products in
+//     shared memory.
 //
 // Per chunk (local t, s in [0, L), suffix decay products p_t = prod_{m>=t} w_m,
 // p_L = 1, G = p_0; all decay ratios that appear are <= 1):

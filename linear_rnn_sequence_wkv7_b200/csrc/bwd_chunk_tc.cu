@@ -32,9 +32,12 @@
 // the operands, invert the 32 x 32 unit lower triangular I - L_ab by 16 x 16
 // blocks, move results between rounds and finish the gradients.
 //
-// One CTA per chunk: warps 0-7 compute, warp 8 issues the tensor-core rounds;
-// hand-offs through named barriers (ready: compute -> issuer, done: issuer ->
-// compute), every wait of the issuer bounded.
+// A persistent grid, one CTA per SM walking the chunks: warps 0-7 compute,
+// warp 8 issues the tensor-core rounds; hand-offs through named barriers
+// (ready: compute -> issuer, done: issuer -> compute), every wait of the issuer
+// bounded.  The next chunk's token tiles arrive by cp.async into the raw tile
+// buffer as soon as the current chunk has read it (first phase), and its
+// states are pulled into L2 one chunk ahead.
 #include "umma.cuh"
 
 namespace wkv7 {
