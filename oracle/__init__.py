@@ -34,6 +34,13 @@ section "Summary").
   S_in M + E with M the ordered product of its transitions and E its final
   state from S = 0.  Both are written as those definitions: the product taken
   token by token, E from ``forward``.
+* ``state_gradient`` / ``compose_adjoints``: the same affinity backwards.
+  dL/dS before a stretch is (dL/dS after it) M^T + F, F being the stretch's
+  own contribution (its outputs' gradient with nothing after it).
+  ``state_gradient`` is the reverse sweep of the state gradient alone, token
+  by token (the adjoint of S_t = S_{t-1} A_t + v_t k_t^T, y_t = S_t r_t, taken
+  for S only): G <- G + dy_t r_t^T, then G <- G A_t^T.  ``compose_adjoints``
+  chains those maps over stretches, last stretch first.
 """
 from __future__ import annotations
 
@@ -309,3 +316,37 @@ def compose_states(summaries, s0=None):
     for kk in range(nseg):
         states[kk + 1] = states[kk] @ summaries[kk, 1] + summaries[kk, 0]
     return states
+
+
+def state_gradient(r, w, a, b, dy, dsT=None):
+    """dL/dS_0 [B,H,N,N] fp64 of L = sum(dy * y) + sum(dsT * S_T) for a stretch
+    shaped [B,T,H,N]: the reverse sweep G_T = dsT (or 0), then for t = T-1..0
+    G <- G + dy_t r_t^T and G <- G (diag(w_t) + a_t b_t^T)^T (the adjoint of
+    S_t = S_{t-1} A_t + ..., y_t = S_t r_t, for the state alone).  k, v and the
+    initial state play no part."""
+    r, w, a, b, dy = (_f64(x) for x in (r, w, a, b, dy))
+    B, T, H, N = r.shape
+    out = np.empty((B, H, N, N))
+    for bb in range(B):
+        for h in range(H):
+            G = np.zeros((N, N)) if dsT is None else _f64(dsT)[bb, h].copy()
+            for t in range(T - 1, -1, -1):
+                G = G + np.outer(dy[bb, t, h], r[bb, t, h])
+                A = np.diag(w[bb, t, h]) + np.outer(a[bb, t, h], b[bb, t, h])
+                G = G @ A.T
+            out[bb, h] = G
+    return out
+
+
+def compose_adjoints(summaries, F, dsT=None):
+    """adj [nseg+1,B,H,N,N] for consecutive stretches with summaries
+    [nseg,2,B,H,N,N] ([E; M] each) and own state gradients F [nseg,B,H,N,N]:
+    adj[nseg] = dsT (or 0), adj[k] = adj[k+1] M_k^T + F_k (adj[k] = dL/dS
+    before stretch k)."""
+    summaries, F = _f64(summaries), _f64(F)
+    nseg, _, B, H, N, _ = summaries.shape
+    adj = np.empty((nseg + 1, B, H, N, N))
+    adj[nseg] = 0.0 if dsT is None else _f64(dsT)
+    for kk in range(nseg - 1, -1, -1):
+        adj[kk] = adj[kk + 1] @ np.swapaxes(summaries[kk, 1], -1, -2) + F[kk]
+    return adj

@@ -298,6 +298,76 @@ def test_compose_states_match_prefix_forwards():
     np.testing.assert_array_equal(oracle.compose_states(np.zeros((0, 2, B, H, N, N)))[0], 0.0)
 
 
+def test_state_gradient_is_the_backward_ds0():
+    """The state-gradient sweep equals ds0 of the C backward (an independent
+    implementation pinned by central differences), for any k, v, s0."""
+    B, T, H, N = 2, 29, 2, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=73)
+    rng = np.random.default_rng(79)
+    dy = rng.standard_normal((B, T, H, N))
+    dsT = rng.standard_normal((B, H, N, N))
+    g = oracle.state_gradient(r, w, a, b, dy, dsT)
+    assert rel_err(g, oracle.backward(r, w, k, v, a, b, s0, dy, dsT)[6]) < 1e-12
+    k2, v2 = rng.standard_normal(k.shape), rng.standard_normal(v.shape)
+    assert rel_err(g, oracle.backward(r, w, k2, v2, a, b, None, dy, dsT)[6]) < 1e-12
+    np.testing.assert_array_equal(oracle.state_gradient(*(x[:, :0] for x in (r, w, a, b, dy)), dsT), dsT)
+
+
+def test_compose_adjoints_match_suffix_backwards():
+    """Chaining (M_k, F_k) of consecutive stretches, last first, gives dL/dS
+    before every stretch: ds0 of the C backward over the suffix from there."""
+    B, T, H, N = 1, 37, 2, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=83)
+    rng = np.random.default_rng(89)
+    dy = rng.standard_normal((B, T, H, N))
+    dsT = rng.standard_normal((B, H, N, N))
+    cuts = [0, 11, 11, 25, 37]
+    sums, F = [], []
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        sl = lambda x: x[:, c0:c1]
+        E, M = oracle.forward_summary(*map(sl, (r, w, k, v, a, b)))
+        sums.append(np.stack([E, M]))
+        F.append(oracle.state_gradient(*map(sl, (r, w, a, b, dy))))
+    adj = oracle.compose_adjoints(np.stack(sums), np.stack(F), dsT)
+    np.testing.assert_array_equal(adj[-1], dsT)
+    for i, c in enumerate(cuts[:-1]):
+        sl = lambda x: x[:, c:]
+        ref = oracle.backward(*map(sl, (r, w, k, v, a, b)), s0, sl(dy), dsT)[6]
+        assert rel_err(adj[i], ref) < 1e-12, i
+
+
+ADJOINT_MUTANTS = {
+    "untransposed_transition": ("state_gradient", "G = G @ A.T", "G = G @ A"),
+    "readout_after_transition": ("state_gradient",
+                                 "G = G + np.outer(dy[bb, t, h], r[bb, t, h])\n                A = np.diag(w[bb, t, h]) + np.outer(a[bb, t, h], b[bb, t, h])\n                G = G @ A.T",
+                                 "A = np.diag(w[bb, t, h]) + np.outer(a[bb, t, h], b[bb, t, h])\n                G = G @ A.T\n                G = G + np.outer(dy[bb, t, h], r[bb, t, h])"),
+    "untransposed_summary": ("compose_adjoints", "np.swapaxes(summaries[kk, 1], -1, -2)", "summaries[kk, 1]"),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(ADJOINT_MUTANTS))
+def test_adjoint_mutants_are_caught(mutant):
+    import inspect
+    fn, old, new = ADJOINT_MUTANTS[mutant]
+    src = inspect.getsource(getattr(oracle, fn))
+    assert src.count(old) == 1, "mutation anchor not found"
+    ns = dict(np=np, _f64=oracle._f64)
+    exec(src.replace(old, new), ns)
+    B, T, H, N = 1, 9, 1, 8
+    (r, w, k, v, a, b), s0 = recipe(B, T, H, N, seed=97)
+    rng = np.random.default_rng(101)
+    dy = rng.standard_normal((B, T, H, N))
+    dsT = rng.standard_normal((B, H, N, N))
+    ref = oracle.backward(r, w, k, v, a, b, s0, dy, dsT)[6]
+    if fn == "state_gradient":
+        got = ns["state_gradient"](r, w, a, b, dy, dsT)
+    else:
+        E, M = oracle.forward_summary(r, w, k, v, a, b)
+        F = oracle.state_gradient(r, w, a, b, dy)
+        got = ns["compose_adjoints"](np.stack([E, M])[None], F[None], dsT)[0]
+    assert rel_err(got, ref) > 1e-6, f"mutant {mutant} slipped through"
+
+
 SUMMARY_MUTANTS = {
     "reversed_product": ("P = P @ (np.diag(", "P = (np.diag("),
     "compose_left_multiply": ("states[kk] @ summaries[kk, 1]", "summaries[kk, 1] @ states[kk]"),
