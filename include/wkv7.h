@@ -184,6 +184,45 @@ WKV7_API wkv7_status wkv7_compose_states(int nseg, int B, int H, int N, const fl
                                          const float *summaries, float *states, cudaStream_t stream);
 
 /*
+ * Sequence-parallel backward, the forward's steps in reverse.  The state
+ * gradient is affine too: for a stretch with summary M (see above),
+ *     dL/dS_in = dL/dS_out M^T + F,
+ * F being the stretch's own contribution (dL/dS_in with dL/dS_out = 0).  On
+ * device i with stretch i, after the sequence-parallel forward:
+ *   wkv7_state_gradient (dsT = NULL) -> F_i
+ *   (exchange the P F's: an all-gather)
+ *   wkv7_compose_adjoints            -> dL/dS before and after every stretch
+ *   wkv7_backward (s0 = the stretch's entry state, dsT = dL/dS after it)
+ * which gives the gradients of one wkv7_backward over the whole sequence.
+ */
+
+/*
+ * dL/dS_0 of L = sum(dy * y) + sum(dsT * S_T) over a stretch: the reverse
+ * sweep of the state gradient alone (G += dy_t r_t^T, then G <- G A_t^T), one
+ * launch.  Needs neither k, v nor the states.
+ *   r, w, a, b, dy : [B, T, H, N] of in_dtype
+ *   dsT            : [B, H, N, N] fp32, or NULL for zeros
+ *   ds0            : [B, H, N, N] fp32, written
+ */
+WKV7_API wkv7_status wkv7_state_gradient(int B, int T, int H, int N, wkv7_dtype in_dtype, const void *r,
+                                         const void *w, const void *a, const void *b, const void *dy,
+                                         const float *dsT, float *ds0, cudaStream_t stream);
+
+/*
+ * dL/dS before every one of nseg consecutive stretches, last stretch first:
+ *     adj[nseg] = dsT (or zeros when dsT is NULL)
+ *     adj[k] = adj[k + 1] M_k^T + F_k,  k = nseg - 1 .. 0
+ *   summaries : [nseg, 2, B, H, N, N] fp32 as for wkv7_compose_states (M_k in
+ *               summaries[k][1]; may be NULL if nseg = 0)
+ *   F         : [nseg, B, H, N, N] fp32, the stretches' own state gradients
+ *   adj       : [nseg + 1, B, H, N, N] fp32, written; stretch k's backward
+ *               takes dsT = adj[k + 1], and adj[0] is the whole sequence's ds0.
+ *               adj must not overlap the inputs.
+ */
+WKV7_API wkv7_status wkv7_compose_adjoints(int nseg, int B, int H, int N, const float *dsT, const float *summaries,
+                                           const float *F, float *adj, cudaStream_t stream);
+
+/*
  * wkv7_forward with r..b, s0, y and sT in HOST memory (page-locked memory
  * lets the copies overlap the computation; pageable memory works, slower).
  * The sequence is cut into up to 8 time slices of whole 32-token chunks; the

@@ -108,7 +108,7 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         cp_async_wait<0>();
         __syncthreads();
         if (c > 0) issue(c - 1, stage ^ 1);
-        {   // dL/dS after the chunk's last token, before its own output is added
+        if (dS_out) {   // dL/dS after the chunk's last token, before its own output is added
             float *dst = dS_out + ((size_t)head * nck + c) * kN * kN + (size_t)row0 * kN + 4 * q;
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr)
@@ -616,14 +616,13 @@ cudaError_t bwd_chunk_tc(int B, int T, int H, wkv7_dtype g_dt, const void *r, co
                          const float *sfin, const float *dS_out, void *dr, void *dw, void *dk, void *dv, void *da,
                          void *db, long long wait_limit, cudaStream_t st);
 
-cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
-                        const void *k, const void *v, const void *a, const void *b, const void *dy,
-                        const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
-                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
-                        cudaStream_t st) {
+// dL/dS at every chunk end (into dS_out, skipped when it is null) and ds0, by
+// the reverse sweep of the state gradient; reads r, w, a, b, dy only
+cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
+                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, cudaStream_t st) {
     using namespace bwdc;
-    const int heads = B * H, nck = (T + L - 1) / L;
-    {   // dS at every chunk end, and ds0; split rows over two CTAs when the
+    const int heads = B * H;
+    {   // split rows over two CTAs when the
         // heads alone leave SMs idle (measured: 1.45 vs 1.67 ms at 256 heads)
         const size_t smem = 2 * 5 * L * kN * (in_dt == WKV7_F32 ? 4 : 2);
         const bool split = heads <= 148;
@@ -643,10 +642,19 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
             else WKV7_DSTATE(__nv_bfloat16, 2);
         }
 #undef WKV7_DSTATE
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
     }
-    // chunk gradients: tensor cores for bf16 inputs, fp32 CUDA-core products for fp32 inputs
+    return cudaGetLastError();
+}
+
+// The input gradients of every chunk from its checkpoint, the next one (or
+// the final state) and dS at its end: tensor cores for bf16 inputs, fp32
+// CUDA-core products for fp32 inputs.
+cudaError_t bwd_chunk_grads(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
+                            const void *k, const void *v, const void *a, const void *b, const void *dy,
+                            const float *ckpt, const float *sfin, const float *dS_out, void *dr, void *dw, void *dk,
+                            void *dv, void *da, void *db, long long wait_limit, cudaStream_t st) {
+    using namespace bwdc;
+    const int heads = B * H, nck = (T + L - 1) / L;
     if (in_dt == WKV7_BF16)
         return bwd_chunk_tc(B, T, H, g_dt, r, w, k, v, a, b, dy, ckpt, sfin, dS_out, dr, dw, dk, dv, da, db,
                             wait_limit, st);
@@ -666,6 +674,17 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
     else WKV7_CHUNK_BWD(__nv_bfloat16, __nv_bfloat16);
 #undef WKV7_CHUNK_BWD
     return cudaGetLastError();
+}
+
+cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
+                        const void *k, const void *v, const void *a, const void *b, const void *dy,
+                        const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
+                        cudaStream_t st) {
+    cudaError_t e = bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, dS_out, ds0, st);
+    if (e != cudaSuccess) return e;
+    return bwd_chunk_grads(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, ckpt, sfin, dS_out, dr, dw, dk, dv, da, db,
+                           wait_limit, st);
 }
 
 }  // namespace wkv7

@@ -718,9 +718,10 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
 }
 
 // Chain of affine state maps, per head: X_0 = s0 (I when s0_eye, zeros when
-// s0 is null), X_{k+1} = X_k M_k + E_k for k < nsteps, with M_k at
-// m_base + k m_stride and E_k at e_base + k e_stride ([B*H][64][64] each; E
-// read as zeros when e_base is null).  With out_stride != 0 writes every X_k,
+// s0 is null), X_{k+1} = X_k M_k + E_k for k < nsteps (X_k M_k^T + E_k with
+// transpose_m), with M_k at m_base + k m_stride and E_k at e_base + k e_stride
+// ([B*H][64][64] each; strides may be negative; E read as zeros when e_base
+// is null).  With out_stride != 0 writes every X_k,
 // k <= nsteps, at out + k out_stride; else only X_nsteps at out.  The rows of
 // X are independent: CTA (head, rb) owns rows 8 rb .. 8 rb + 7, thread ->
 // (row, two columns); M_k is staged in shared memory.  fp32 on CUDA cores.
@@ -729,7 +730,7 @@ constexpr int kCombineRows = 8;
 __global__ void __launch_bounds__(256)
 seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const float *__restrict__ e_base,
                    long long e_stride, const float *__restrict__ m_base, long long m_stride,
-                   float *__restrict__ out, long long out_stride) {
+                   float *__restrict__ out, long long out_stride, int transpose_m) {
     __shared__ __align__(16) float Msm[kN * kN];
     __shared__ float Ssm[kCombineRows][kN];
     const int head = blockIdx.x, tid = threadIdx.x;
@@ -744,8 +745,12 @@ seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const f
         const float *M = m_base + kk * m_stride + hoff;
         Ssm[rr][c2] = cur.x;
         Ssm[rr][c2 + 1] = cur.y;
-        for (int x = tid; x < kN * kN / 4; x += 256)
-            reinterpret_cast<float4 *>(Msm)[x] = reinterpret_cast<const float4 *>(M)[x];
+        if (transpose_m) {                            // Msm[m][c] = M[c][m]
+            for (int x = tid; x < kN * kN; x += 256) Msm[(x & 63) * kN + (x >> 6)] = M[x];
+        } else {
+            for (int x = tid; x < kN * kN / 4; x += 256)
+                reinterpret_cast<float4 *>(Msm)[x] = reinterpret_cast<const float4 *>(M)[x];
+        }
         __syncthreads();
         float2 acc = e_base ? *reinterpret_cast<const float2 *>(e_base + kk * e_stride + eoff) : make_float2(0.f, 0.f);
 #pragma unroll 16
@@ -762,9 +767,10 @@ seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const f
 
 static cudaError_t launch_combine(int B, int H, int nsteps, const float *s0, bool s0_eye, const float *e_base,
                                   long long e_stride, const float *m_base, long long m_stride, float *out,
-                                  long long out_stride, cudaStream_t st) {
+                                  long long out_stride, cudaStream_t st, bool transpose_m = false) {
     seg_combine_kernel<<<dim3(B * H, kN / kCombineRows), 256, 0, st>>>(nsteps, s0, s0_eye ? 1 : 0, e_base, e_stride,
-                                                                       m_base, m_stride, out, out_stride);
+                                                                       m_base, m_stride, out, out_stride,
+                                                                       transpose_m ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -888,6 +894,17 @@ cudaError_t fwd_chunk_continue(int B, int T, int H, wkv7_dtype y_dt, const void 
     cudaError_t e = launch_combine(B, H, n - 1, s_in, false, em, zst, em + n * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
     return launch_chunk(B, T, H, t_seg, n, n, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, n - 1, wait_limit, st);
+}
+
+// dL/dS before each of nseg consecutive segments, last segment first:
+// adj[nseg] = dsT (or 0), adj[k] = adj[k+1] M_k^T + F_k, with M_k in
+// summary[k] = [E_k; M_k] and F_k the segment's own state gradient.
+cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const float *summary, const float *F,
+                             float *adj, cudaStream_t st) {
+    const long long zst = (long long)B * H * kN * kN;
+    if (nseg == 0) return launch_combine(B, H, 0, dsT, false, nullptr, 0, nullptr, 0, adj, 0, st);
+    return launch_combine(B, H, nseg, dsT, false, F + (nseg - 1) * zst, -zst, summary + (2LL * (nseg - 1) + 1) * zst,
+                          -2 * zst, adj + nseg * zst, -zst, st, true);
 }
 
 // Entry states of nseg consecutive segments and the state after the last:

@@ -26,6 +26,10 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
                         void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
                         cudaStream_t st);
 size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
+cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
+                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, cudaStream_t st);
+cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const float *summary, const float *F,
+                             float *adj, cudaStream_t st);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt);
@@ -347,6 +351,30 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
                                  dv, da, db, ds0, lim > 0 ? lim : kDefaultWaitCycles, stream));
+}
+
+wkv7_status wkv7_state_gradient(int B, int T, int H, int N, wkv7_dtype in_dt, const void *r, const void *w,
+                                const void *a, const void *b, const void *dy, const float *dsT, float *ds0,
+                                cudaStream_t stream) {
+    wkv7_status s = check_dims(B, T, H, N);
+    if (s != WKV7_OK) return s;
+    if (!dtype_ok(in_dt)) return WKV7_ERR_INVALID_ARG;
+    if (!opt_ptr_ok(dsT) || !ptr_ok(ds0)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (T == 0) return copy_or_zero_state(ds0, dsT, B, H, stream);
+    for (const void *p : {r, w, a, b, dy})
+        if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
+    return from_cuda(bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, nullptr, ds0, stream));
+}
+
+wkv7_status wkv7_compose_adjoints(int nseg, int B, int H, int N, const float *dsT, const float *summaries,
+                                  const float *F, float *adj, cudaStream_t stream) {
+    wkv7_status s = check_dims(B, 0, H, N);
+    if (s != WKV7_OK) return s;
+    if (nseg < 0 || !opt_ptr_ok(dsT)) return WKV7_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0) return WKV7_OK;
+    if (!ptr_ok(adj) || (nseg > 0 && (!ptr_ok(summaries) || !ptr_ok(F)))) return WKV7_ERR_INVALID_ARG;
+    return from_cuda(compose_adjoints(B, H, nseg, dsT, summaries, F, adj, stream));
 }
 
 void wkv7_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }

@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = (
     "wkv7_forward_summary", "wkv7_compose_states", "wkv7_forward_summary_workspace_size",
     "wkv7_forward_continue", "wkv7_forward_host_workspace_size", "wkv7_forward_host",
     "wkv7_saved_states_size", "wkv7_forward_train", "wkv7_backward_from_states_workspace_size",
-    "wkv7_backward_from_states",
+    "wkv7_backward_from_states", "wkv7_state_gradient", "wkv7_compose_adjoints",
 )
 
 _lib = None
@@ -84,6 +84,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward_from_states_workspace_size.restype = z
     lib.wkv7_backward_from_states.argtypes = [i, i, i, i, i, i] + [vp] * 17 + [vp, z, vp]
     lib.wkv7_backward_from_states.restype = i
+    lib.wkv7_state_gradient.argtypes = [i, i, i, i, i] + [vp] * 7 + [vp]
+    lib.wkv7_state_gradient.restype = i
+    lib.wkv7_compose_adjoints.argtypes = [i, i, i, i, vp, vp, vp, vp, vp]
+    lib.wkv7_compose_adjoints.restype = i
     lib.wkv7_forward_resolve_algo.argtypes = [i, i, i]
     lib.wkv7_forward_resolve_algo.restype = i
     lib.wkv7_set_wait_limit.argtypes = [ctypes.c_longlong]
@@ -259,6 +263,36 @@ def forward_host(r, w, k, v, a, b, s0=None, *, y, sT=None, algo="auto", chunk_le
                                ALGOS[algo], chunk_len, _ptr(workspace), workspace.numel(), _stream(stream))
     _check("wkv7_forward_host", st)
     return y, sT
+
+
+def state_gradient(r, w, a, b, dy, dsT=None, *, out=None, stream=None):
+    """dL/dS_0 [B,H,N,N] fp32 of a stretch [B,T,H,N] given dL/dS_T (dsT, None = 0)."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, a, b, dy), r.shape, r.dtype)
+    if dsT is not None:
+        _same((dsT,), (B, H, N, N), torch.float32)
+    if out is None:
+        out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    st = lib.wkv7_state_gradient(B, T, H, N, _dt(r), *map(_ptr, (r, w, a, b, dy, dsT, out)), _stream(stream))
+    _check("wkv7_state_gradient", st)
+    return out
+
+
+def compose_adjoints(summaries, F, dsT=None, *, out=None, stream=None):
+    """adj [nseg+1,B,H,N,N]: adj[nseg] = dsT (or 0), adj[k] = adj[k+1] @ M_k^T + F_k."""
+    lib = load_library()
+    nseg, two, B, H, N, _ = summaries.shape
+    if two != 2:
+        raise ValueError("summaries must be [nseg, 2, B, H, N, N]")
+    _same((F,), (nseg, B, H, N, N), torch.float32)
+    if dsT is not None:
+        _same((dsT,), (B, H, N, N), torch.float32)
+    if out is None:
+        out = torch.empty((nseg + 1, B, H, N, N), dtype=torch.float32, device=summaries.device)
+    st = lib.wkv7_compose_adjoints(nseg, B, H, N, _ptr(dsT), _ptr(summaries), _ptr(F), _ptr(out), _stream(stream))
+    _check("wkv7_compose_adjoints", st)
+    return out
 
 
 def resolve_algo(T, in_dtype=torch.bfloat16, algo="auto") -> str:

@@ -172,3 +172,30 @@ def test_training_pair_rejects_invalid_arguments(lib):
     assert bs(ptrs=bad) == wkv7.ERR_INVALID_ARG
     assert lib.wkv7_saved_states_size(2, 100, 3, 64) == 2 * 3 * 4 * 64 * 64 * 4
     assert lib.wkv7_backward_from_states_workspace_size(2, 100, 3, 64) >= 2 * 3 * 4 * 64 * 64 * 4
+
+
+def test_state_gradient_and_adjoints_reject_invalid_arguments(lib):
+    sg = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ptrs=None: lib.wkv7_state_gradient(
+        B, T, H, N, dt, *(ptrs or [P] * 7), None)
+    assert sg(N=32) == wkv7.ERR_UNSUPPORTED
+    assert sg(dt=7) == wkv7.ERR_INVALID_ARG
+    assert sg(T=-2) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 7
+    bad[6] = None                                        # ds0 is required
+    assert sg(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 7
+    bad[4] = None                                        # dy missing
+    assert sg(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    bad = [P] * 7
+    bad[5] = ctypes.c_void_p(12)                         # dsT misaligned
+    assert sg(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert sg(H=0) == wkv7.OK
+    ca = lambda nseg=2, B=1, H=1, N=64, dsT=None, sums=P, F=P, adj=P: lib.wkv7_compose_adjoints(
+        nseg, B, H, N, dsT, sums, F, adj, None)
+    assert ca(N=128) == wkv7.ERR_UNSUPPORTED
+    assert ca(nseg=-1) == wkv7.ERR_INVALID_ARG
+    assert ca(sums=None) == wkv7.ERR_INVALID_ARG         # nseg > 0 needs summaries ...
+    assert ca(F=None) == wkv7.ERR_INVALID_ARG            # ... and the stretches' F
+    assert ca(adj=None) == wkv7.ERR_INVALID_ARG
+    assert ca(dsT=ctypes.c_void_p(8)) == wkv7.ERR_INVALID_ARG
+    assert ca(B=0) == wkv7.OK

@@ -1,9 +1,11 @@
-"""The sequence-parallel forward's host logic on CPU: gloo ranks (one process
-each) hold consecutive stretches of one sequence, exchange their summaries by
-all-gather and compose their entry states.  The per-rank compute is the fp64
-oracle, injected through ``StretchOps``, so the test checks the orchestration
-(rank order = time order, the gather, which composed state each rank takes)
-against the oracle's forward over the whole sequence."""
+"""The sequence-parallel forward's and backward's host logic on CPU: gloo ranks
+(one process each) hold consecutive stretches of one sequence, exchange their
+summaries (and, backward, their own state gradients) by all-gather and compose
+their entry states (and the state gradients after their stretches).  The
+per-rank compute is the fp64 oracle, injected through ``StretchOps``, so the
+test checks the orchestration (rank order = time order, the gathers, which
+composed state each rank takes) against the oracle's forward and backward
+over the whole sequence."""
 import os
 import socket
 
@@ -14,7 +16,8 @@ import torch.multiprocessing as mp
 
 import oracle
 from linear_rnn_sequence_wkv7_b200 import inputs
-from linear_rnn_sequence_wkv7_b200.context_parallel import StretchOps, forward_context_parallel, split_lengths
+from linear_rnn_sequence_wkv7_b200.context_parallel import (StretchOps, backward_context_parallel,
+                                                            forward_context_parallel, split_lengths)
 from linear_rnn_sequence_wkv7_b200.dist import Dist
 
 
@@ -40,7 +43,17 @@ def oracle_ops():
         y, _ = oracle.forward(*map(_np, (r, w, k, v, a, b)), s0=_np(s_in))
         return torch.from_numpy(y)
 
-    return StretchOps(summary=summary, compose=compose, forward=forward)
+    def state_gradient(r, w, a, b, dy):
+        return torch.from_numpy(oracle.state_gradient(*map(_np, (r, w, a, b, dy))))
+
+    def compose_adjoints(sums, F, dsT):
+        return torch.from_numpy(oracle.compose_adjoints(_np(sums), _np(F), _np(dsT)))
+
+    def backward(r, w, k, v, a, b, s_in, dy, ds_out):
+        return tuple(map(torch.from_numpy, oracle.backward(*map(_np, (r, w, k, v, a, b, s_in, dy, ds_out)))))
+
+    return StretchOps(summary=summary, compose=compose, forward=forward, state_gradient=state_gradient,
+                      compose_adjoints=compose_adjoints, backward=backward)
 
 
 def _sequence(T, seed):
@@ -87,6 +100,56 @@ def test_gloo_ranks_match_whole_sequence(world, T):
         np.testing.assert_allclose(s_fin, sT_ref, rtol=0, atol=1e-12)
         ys.append(y)
     np.testing.assert_allclose(np.concatenate(ys, axis=1), y_ref, rtol=0, atol=1e-12)
+
+
+def _dy(T, seed):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((1, T, 2, 16)), 0.1 * rng.standard_normal((1, 2, 16, 16))
+
+
+def _rank_main_bwd(rank, world, port, T, seed, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    d = Dist("gloo").init(timeout_s=60)
+    try:
+        args, s0 = _sequence(T, seed)
+        dy, dsT = _dy(T, seed + 1)
+        lens = split_lengths(T, world, chunk=8)
+        c0 = sum(lens[:rank])
+        cut = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, c0:c0 + lens[rank]]))
+        mine = [cut(x) for x in args]
+        ops = oracle_ops()
+        _, s_in, _, sums = forward_context_parallel(*mine, torch.from_numpy(s0), ops=ops, return_summaries=True)
+        grads = backward_context_parallel(*mine, s_in, sums, cut(dy), torch.from_numpy(dsT), ops=ops)
+        out.put((rank, [g.numpy() for g in grads]))
+    finally:
+        d.close()
+
+
+@pytest.mark.parametrize("world,T", [(2, 70), (3, 17), (4, 45)])
+def test_gloo_ranks_backward_match_whole_sequence(world, T):
+    """Each rank's gradients from its stretch, the exchanged own state
+    gradients F and the composed adjoints equal the oracle's single backward
+    over the whole sequence (with a dL/dS_T term); dL/dS_0 agrees on every
+    rank.  T = 17 over 3 ranks leaves the last stretch empty."""
+    seed, port = 120 + world, _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main_bwd, args=(r, world, port, T, seed, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted((out.get(timeout=120) for _ in range(world)), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    args, s0 = _sequence(T, seed)
+    dy, dsT = _dy(T, seed + 1)
+    ref = oracle.backward(*args, s0, dy, dsT)
+    for i in range(6):
+        got = np.concatenate([g[i] for _, g in results], axis=1)
+        np.testing.assert_allclose(got, ref[i], rtol=0, atol=1e-10 * max(1.0, np.abs(ref[i]).max()))
+    for _, g in results:
+        np.testing.assert_allclose(g[6], ref[6], rtol=0, atol=1e-10 * max(1.0, np.abs(ref[6]).max()))
 
 
 def test_single_process_is_plain_forward():
