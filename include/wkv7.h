@@ -198,15 +198,21 @@ WKV7_API wkv7_status wkv7_compose_states(int nseg, int B, int H, int N, const fl
 
 /*
  * dL/dS_0 of L = sum(dy * y) + sum(dsT * S_T) over a stretch: the reverse
- * sweep of the state gradient alone (G += dy_t r_t^T, then G <- G A_t^T), one
- * launch.  Needs neither k, v nor the states.
+ * sweep of the state gradient alone (G += dy_t r_t^T, then G <- G A_t^T).
+ * Needs neither k, v nor the states.  With a workspace of at least
+ * wkv7_state_gradient_workspace_size bytes, a sweep over few heads runs as
+ * segments side by side (each carrying G from 0 and a second G from I, the
+ * two chained afterwards), else as one pass per head.
  *   r, w, a, b, dy : [B, T, H, N] of in_dtype
  *   dsT            : [B, H, N, N] fp32, or NULL for zeros
  *   ds0            : [B, H, N, N] fp32, written
+ *   workspace      : device scratch, 16-byte aligned, or NULL
  */
+WKV7_API size_t wkv7_state_gradient_workspace_size(int B, int T, int H, int N);
 WKV7_API wkv7_status wkv7_state_gradient(int B, int T, int H, int N, wkv7_dtype in_dtype, const void *r,
                                          const void *w, const void *a, const void *b, const void *dy,
-                                         const float *dsT, float *ds0, cudaStream_t stream);
+                                         const float *dsT, float *ds0, void *workspace, size_t workspace_bytes,
+                                         cudaStream_t stream);
 
 /*
  * dL/dS before every one of nseg consecutive stretches, last stretch first:
@@ -268,17 +274,22 @@ WKV7_API wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dtype, wkv7_dt
 
 /* Bytes of scratch wkv7_backward needs: per (b, h), the state before every
  * 32-token chunk, dL/dS at the end of every chunk, and the final state
- * (fp32, 16 KiB each). */
+ * (fp32, 16 KiB each); for few heads over many tokens also 3 states per
+ * segment of the state-gradient sweep (see below).  Depends on the current
+ * device's SM count. */
 WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
 
 /*
  * Backward: gradients of L = sum(dy * y) + sum(dsT * sT) with respect to every
- * input and the initial state.  Three launches: state checkpoints every 32
+ * input and the initial state.  Three steps: state checkpoints every 32
  * tokens, a reverse sweep of the state gradient that records dL/dS at every
  * chunk end (and ds0), then the input gradients of every chunk independently
  * (the adjoint of the chunked form of the recurrence): on the tensor cores
  * for bf16 inputs (bf16 hi/lo operands, fp32 accumulation), in fp32 on the
- * CUDA cores for fp32 inputs.
+ * CUDA cores for fp32 inputs.  When the heads leave most SMs idle the sweep
+ * runs as segments side by side: a dual pass per segment (dL/dS from 0 with
+ * dy, and the segment's transposed transition product from I), a chain of
+ * those for every segment's exit adjoint, and a second pass that records dS.
  *   r..b, s0         : the forward's inputs (s0 NULL = zeros)
  *   dy               : [B, T, H, N] of in_dtype
  *   dsT              : [B, H, N, N] fp32, or NULL for zeros
@@ -317,7 +328,7 @@ WKV7_API wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype i
                                         size_t workspace_bytes, cudaStream_t stream);
 
 /* Bytes of scratch wkv7_backward_from_states needs: dL/dS at the end of every
- * 32-token chunk, fp32. */
+ * 32-token chunk, fp32, and the segmented sweep's scratch. */
 WKV7_API size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, int N);
 
 /*

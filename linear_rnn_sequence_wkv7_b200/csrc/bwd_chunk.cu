@@ -61,23 +61,44 @@ constexpr float kMinDecay = 1e-30f;
 // one CTA; RPT = 1 splits it over two CTAs (rows 32 q .. 32 q + 31), for
 // problems with too few heads to fill the GPU.  Token tiles of r w a b dy are
 // prefetched by cp.async, 32 tokens ahead.
+//
+// A launch runs nz segments of t_seg tokens (segment seg0 + z, whole chunks;
+// only the last one of the sequence is ragged), each for all heads.  The
+// sweep is affine in G: over a segment, G_in = G_out M^T + F with M the
+// segment's transition product and F its own part (G_out = 0).  So a long
+// sweep with few heads splits into segments: a dual run carries G from 0
+// with dy (-> F) and a second G from I without dy (-> M^T) through one pass;
+// the entry adjoints are chained from those, and an output run per segment
+// sweeps again from its true G_out, storing dS_out.  In a DUAL launch only
+// the last segment (z = nz - 1) is an output run.
+//   g_in   : G at the segment's end per z (stride g_in_zstride), NULL = 0
+//   g_out  : G at the segment's start, for runs z < g_out_nz
+//   m_out  : the dual runs' M^T
 // ---------------------------------------------------------------------------
-template <typename InT, int RPT>
+template <typename InT, int RPT, bool DUAL>
 __global__ void __launch_bounds__(128)
-bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
-                  const InT *__restrict__ a, const InT *__restrict__ b, const InT *__restrict__ dy,
-                  const float *__restrict__ dsT, float *__restrict__ dS_out, float *__restrict__ ds0) {
+bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r, const InT *__restrict__ w,
+                  const InT *__restrict__ a, const InT *__restrict__ b, const InT *__restrict__ dy, int H,
+                  const float *__restrict__ g_in, long long g_in_zstride, float *__restrict__ dS_out,
+                  float *__restrict__ g_out, long long g_out_zstride, int g_out_nz, float *__restrict__ m_out,
+                  long long m_zstride) {
     constexpr int L = bwdc::L, NTEN = 5, VEC = 16 / sizeof(InT), CPV = kN / VEC;
+    constexpr int NR = DUAL ? 2 * RPT : RPT;   // rows RPT.. carry the dual run's second G
     extern __shared__ __align__(16) unsigned char dsmem[];
     auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
     constexpr int SPLIT = 2 / RPT;     // CTAs per head
     const int tid = threadIdx.x, q = tid & 3;
-    const int head = blockIdx.x / SPLIT;
+    const int per_z = gridDim.x / nz;
+    const int z = blockIdx.x / per_z, head = (blockIdx.x % per_z) / SPLIT;
     const int row0 = 32 * (blockIdx.x % SPLIT) * (SPLIT - 1) + RPT * (tid >> 2);
     const int bb = head / H, h = head % H;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
-    const int nck = (T + L - 1) / L;
+    const int nck_total = (T + L - 1) / L;
+    const int t_begin = (seg0 + z) * t_seg, t_end = min(T, t_begin + t_seg);
+    const int c_begin = t_begin / L, c_last = (t_end + L - 1) / L - 1;
+    const bool out_run = !DUAL || z == nz - 1;
+    const size_t hoff = (size_t)head * kN * kN;
     const InT *src[NTEN] = {r, w, a, b, dy};
 
     auto issue = [&](int c, int stage) {
@@ -92,24 +113,32 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         cp_async_commit();
     };
 
-    float g[RPT][16];
+    float g[NR][16];
 #pragma unroll
-    for (int rr = 0; rr < RPT; ++rr)
+    for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (dsT) d4 = load4(dsT + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q);
+            const int row = row0 + rr % RPT, col = 16 * m + 4 * q;
+            if (rr >= RPT) {             // identity start of the product run
+                d4.x = row == col ? 1.f : 0.f;
+                d4.y = row == col + 1 ? 1.f : 0.f;
+                d4.z = row == col + 2 ? 1.f : 0.f;
+                d4.w = row == col + 3 ? 1.f : 0.f;
+            } else if (out_run && g_in) {
+                d4 = load4(g_in + z * g_in_zstride + hoff + (size_t)row * kN + col);
+            }
             g[rr][4 * m] = d4.x; g[rr][4 * m + 1] = d4.y; g[rr][4 * m + 2] = d4.z; g[rr][4 * m + 3] = d4.w;
         }
-    issue(nck - 1, 0);
-    for (int c = nck - 1; c >= 0; --c) {
-        const int stage = (nck - 1 - c) & 1;
+    if (t_begin < t_end) issue(c_last, 0);   // an empty segment passes G through
+    for (int c = c_last; c >= c_begin; --c) {
+        const int stage = (c_last - c) & 1;
         const int t0 = c * L, Lc = min(L, T - t0);
         cp_async_wait<0>();
         __syncthreads();
-        if (c > 0) issue(c - 1, stage ^ 1);
-        if (dS_out) {   // dL/dS after the chunk's last token, before its own output is added
-            float *dst = dS_out + ((size_t)head * nck + c) * kN * kN + (size_t)row0 * kN + 4 * q;
+        if (c > c_begin) issue(c - 1, stage ^ 1);
+        if (out_run && dS_out) {   // dL/dS after the chunk's last token, before its own output is added
+            float *dst = dS_out + ((size_t)head * nck_total + c) * kN * kN + (size_t)row0 * kN + 4 * q;
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
@@ -120,29 +149,29 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
         for (int tt = Lc - 1; tt >= 0; --tt) {
             const InT *rv = tile[stage][0][tt], *wv = tile[stage][1][tt], *av = tile[stage][2][tt];
             const InT *bv = tile[stage][3][tt];
-            float dyi[RPT], dp4[RPT][4];   // four partial sums per row: a shorter dependency chain
+            float dyi[RPT], dp4[NR][4];   // four partial sums per row: a shorter dependency chain
 #pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) {
-                dyi[rr] = to_f32(tile[stage][4][tt][row0 + rr]);
+            for (int rr = 0; rr < RPT; ++rr) dyi[rr] = to_f32(tile[stage][4][tt][row0 + rr]);
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dp4[rr][e] = 0.f;
-            }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 r4 = load4(rv + 16 * m + 4 * q), b4 = load4(bv + 16 * m + 4 * q);
                 const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                for (int rr = 0; rr < RPT; ++rr)
+                for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float gg = fmaf(dyi[rr], rj[e], g[rr][4 * m + e]);
+                        const float gg = rr < RPT ? fmaf(dyi[rr], rj[e], g[rr][4 * m + e]) : g[rr][4 * m + e];
                         g[rr][4 * m + e] = gg;
                         dp4[rr][e] = fmaf(gg, bj[e], dp4[rr][e]);
                     }
             }
-            float dp[RPT];
+            float dp[NR];
 #pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) {
+            for (int rr = 0; rr < NR; ++rr) {
                 dp[rr] = (dp4[rr][0] + dp4[rr][1]) + (dp4[rr][2] + dp4[rr][3]);
                 dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 1);
                 dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 2);
@@ -152,18 +181,23 @@ bwd_dstate_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict
                 const float4 w4 = load4(wv + 16 * m + 4 * q), a4 = load4(av + 16 * m + 4 * q);
                 const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                for (int rr = 0; rr < RPT; ++rr)
+                for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) g[rr][4 * m + e] = fmaf(g[rr][4 * m + e], wj[e], dp[rr] * aj[e]);
             }
         }
     }
+    auto store_rows = [&](float *dst, int r_first) {
 #pragma unroll
-    for (int rr = 0; rr < RPT; ++rr)
+        for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-            store4(ds0 + (size_t)head * kN * kN + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
-                   make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
+            for (int m = 0; m < 4; ++m)
+                store4(dst + hoff + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+                       make_float4(g[r_first + rr][4 * m], g[r_first + rr][4 * m + 1], g[r_first + rr][4 * m + 2],
+                                   g[r_first + rr][4 * m + 3]));
+    };
+    if (z < g_out_nz) store_rows(g_out + z * g_out_zstride, 0);
+    if (DUAL && !out_run) store_rows(m_out + z * m_zstride, DUAL ? RPT : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -616,34 +650,182 @@ cudaError_t bwd_chunk_tc(int B, int T, int H, wkv7_dtype g_dt, const void *r, co
                          const float *sfin, const float *dS_out, void *dr, void *dw, void *dk, void *dv, void *da,
                          void *db, long long wait_limit, cudaStream_t st);
 
-// dL/dS at every chunk end (into dS_out, skipped when it is null) and ds0, by
-// the reverse sweep of the state gradient; reads r, w, a, b, dy only
-cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
-                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, cudaStream_t st) {
-    using namespace bwdc;
-    const int heads = B * H;
-    {   // split rows over two CTAs when the
-        // heads alone leave SMs idle (measured: 1.45 vs 1.67 ms at 256 heads)
-        const size_t smem = 2 * 5 * L * kN * (in_dt == WKV7_F32 ? 4 : 2);
-        const bool split = heads <= 148;
-#define WKV7_DSTATE(I, R)                                                                                 \
-    do {                                                                                                  \
-        auto kern = bwd_dstate_kernel<I, R>;                                                              \
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        if (e != cudaSuccess) return e;                                                                   \
-        kern<<<(2 / R) * heads, 128, smem, st>>>(T, H, (const I *)r, (const I *)w, (const I *)a,          \
-                                                 (const I *)b, (const I *)dy, dsT, dS_out, ds0);          \
+static cudaError_t launch_combine(int B, int H, int nsteps, const float *s0, bool s0_eye, const float *e_base,
+                                  long long e_stride, const float *m_base, long long m_stride, float *out,
+                                  long long out_stride, cudaStream_t st, bool transpose_m);   // fwd_chunk.cu
+
+size_t dstate_scratch_bytes(int B, int H, int nseg) {
+    return nseg > 1 ? 3ULL * nseg * B * H * kN * kN * sizeof(float) : 0;
+}
+
+namespace {
+
+// One launch of the sweep kernel: nz segments from seg0, all heads.
+template <typename I>
+cudaError_t launch_dstate(int rpt, bool dual, int heads, int T, int H, int t_seg, int seg0, int nz, const void *r,
+                          const void *w, const void *a, const void *b, const void *dy, const float *g_in,
+                          long long g_in_zs, float *dS_out, float *g_out, long long g_out_zs, int g_out_nz,
+                          float *m_out, long long m_zs, cudaStream_t st) {
+    const size_t smem = 2 * 5 * bwdc::L * kN * sizeof(I);
+    const unsigned grid = (unsigned)((size_t)nz * heads * (2 / rpt));
+#define WKV7_DSTATE(R, D)                                                                                    \
+    do {                                                                                                     \
+        auto kern = bwd_dstate_kernel<I, R, D>;                                                              \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+        if (e != cudaSuccess) return e;                                                                      \
+        kern<<<grid, 128, smem, st>>>(T, t_seg, seg0, nz, (const I *)r, (const I *)w, (const I *)a,         \
+                                      (const I *)b, (const I *)dy, H, g_in, g_in_zs, dS_out, g_out, g_out_zs, \
+                                      g_out_nz, m_out, m_zs);                                                \
     } while (0)
-        if (in_dt == WKV7_F32) {
-            if (split) WKV7_DSTATE(float, 1);
-            else WKV7_DSTATE(float, 2);
-        } else {
-            if (split) WKV7_DSTATE(__nv_bfloat16, 1);
-            else WKV7_DSTATE(__nv_bfloat16, 2);
-        }
-#undef WKV7_DSTATE
+    if (rpt == 1) {
+        if (dual) WKV7_DSTATE(1, true);
+        else WKV7_DSTATE(1, false);
+    } else {
+        if (dual) WKV7_DSTATE(2, true);
+        else WKV7_DSTATE(2, false);
     }
+#undef WKV7_DSTATE
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// The sweep's plan: segments (whole chunks, all non-empty) and rows per
+// thread, for B*H heads of T tokens.
+struct DstatePlan {
+    int nseg = 1, t_seg = 0, rpt = 2;
+};
+
+DstatePlan dstate_split(int T, int nseg_want, int rpt) {
+    DstatePlan p;
+    const int chunks = (T + bwdc::L - 1) / bwdc::L;
+    const int want = std::max(1, std::min(nseg_want, chunks));
+    const int per = (chunks + want - 1) / want;
+    p.t_seg = per * bwdc::L;
+    p.nseg = (chunks + per - 1) / per;
+    p.rpt = rpt;
+    return p;
+}
+
+// Estimated time (ns) of one sweep launch of n CTAs over `steps` tokens.  A
+// step of a CTA alone on its SM is latency-bound; each further co-resident
+// CTA adds its issue time; CTAs beyond the resident ones run in later waves.
+// Fitted on B200 (bf16 inputs; B = 1 and 8, H = 32, T = 4096 .. 65536).
+static double dstate_launch_ns(long long n, long long steps, int rpt, bool dual, bool f32, int sms) {
+    const double lat = rpt == 1 ? (dual ? 198.0 : 156.0) : (dual ? 252.0 : 221.0);
+    const double add = rpt == 1 ? (dual ? 115.0 : 156.0) : (dual ? 191.0 : 109.0);
+    const int res = f32 ? 2 : (rpt == 2 && dual ? 4 : 5);    // shared memory, registers
+    const long long per_sm = (n + sms - 1) / sms;
+    const long long waves = (per_sm + res - 1) / res;
+    const long long k = std::min<long long>(per_sm, res);
+    return (double)waves * (double)steps * (lat + add * (double)(k - 1));
+}
+
+// The plan with the lowest estimated time whose scratch fits scratch_cap
+// bytes: rpt 1 or 2, nseg = 1 or a split into segments of at least two chunks.
+// need_dS: dS at every chunk end is wanted (the backward), else ds0 alone.
+DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, size_t scratch_cap) {
+    const long long heads = (long long)B * H;
+    const int chunks = (T + bwdc::L - 1) / bwdc::L;
+    if (sms <= 0) sms = 148;
+    constexpr double kCombineStepNs = 3000.0, kLaunchNs = 4000.0;
+    DstatePlan best;
+    double best_ns = 0.0;
+    for (int rpt = 1; rpt <= 2; ++rpt) {
+        const long long per_head = 2 / rpt;
+        for (int want = 1; want <= std::min(64, std::max(1, chunks / 2)); ++want) {
+            const DstatePlan p = dstate_split(T, want, rpt);
+            if (p.nseg != want) continue;
+            if (p.nseg > 1 && dstate_scratch_bytes(B, H, p.nseg) > scratch_cap) break;
+            const int n = p.nseg;
+            double ns;
+            if (n == 1) {
+                ns = dstate_launch_ns(heads * per_head, T, rpt, false, f32, sms);
+            } else if (need_dS) {
+                const long long ctas = (n - 1) * heads * per_head;
+                ns = dstate_launch_ns(ctas, p.t_seg, rpt, n > 2, f32, sms) +
+                     dstate_launch_ns(ctas, p.t_seg, rpt, false, f32, sms) + kCombineStepNs * (n - 2) +
+                     kLaunchNs * (n > 2 ? 2 : 1);
+            } else {
+                ns = dstate_launch_ns(n * heads * per_head, p.t_seg, rpt, true, f32, sms) +
+                     kCombineStepNs * (n - 1) + kLaunchNs;
+            }
+            if (best_ns == 0.0 || ns < 0.97 * best_ns) {
+                best = p;
+                best_ns = ns;
+            }
+        }
+    }
+    return best;
+}
+
+// Scratch of the plan dstate_plan picks with room to spare, for either input
+// dtype (workspace sizes do not depend on it).
+size_t dstate_scratch_for(int B, int T, int H, int sms, bool need_dS) {
+    size_t need = 0;
+    for (bool f32 : {false, true}) {
+        const DstatePlan p = dstate_plan(B, T, H, sms, f32, need_dS, (size_t)-1);
+        need = std::max(need, dstate_scratch_bytes(B, H, p.nseg));
+    }
+    return need;
+}
+
+// dL/dS at every chunk end (into dS_out, skipped when it is null) and ds0, by
+// the reverse sweep of the state gradient; reads r, w, a, b, dy only.  With
+// nseg > 1 segments (scratch: dstate_scratch_bytes), the segments' dual runs,
+// a chain of their summaries for the entry adjoints, and (for dS_out) output
+// runs of all segments but the last.
+template <typename I>
+cudaError_t bwd_dstate_run(int B, int T, int H, const DstatePlan &p, const void *r, const void *w, const void *a,
+                           const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0,
+                           float *scratch, cudaStream_t st) {
+    const int heads = B * H, n = p.nseg;
+    if (n <= 1)
+        return launch_dstate<I>(p.rpt, false, heads, T, H, std::max(p.t_seg, T), 0, 1, r, w, a, b, dy, dsT, 0,
+                                dS_out, ds0, 0, 1, nullptr, 0, st);
+    const long long zs = (long long)heads * kN * kN;
+    float *FA = scratch, *MT = scratch + n * zs, *ADJ = scratch + 2 * n * zs;
+    cudaError_t e;
+    if (!dS_out) {
+        // every segment summarised (the last one from dsT), then one chain to ds0
+        e = launch_dstate<I>(p.rpt, true, heads, T, H, p.t_seg, 0, n, r, w, a, b, dy, dsT, 0, nullptr, FA, zs, n,
+                             MT, zs, st);
+        if (e != cudaSuccess) return e;
+        return launch_combine(B, H, n - 1, FA + (n - 1) * zs, false, FA + (n - 2) * zs, -zs, MT + (n - 2) * zs, -zs,
+                              ds0, 0, st, false);
+    }
+    // pass 1: segments 1..n-1, the last as an output run from dsT
+    e = launch_dstate<I>(p.rpt, n > 2, heads, T, H, p.t_seg, 1, n - 1, r, w, a, b, dy, dsT, 0, dS_out, FA + zs, zs,
+                         n - 1, MT + zs, zs, st);
+    if (e != cudaSuccess) return e;
+    // pass 2: dL/dS at the end of segments 0..n-2: adj[k] = adj[k+1] M_k^T + F_k
+    const float *entry = FA + zs;
+    if (n > 2) {
+        e = launch_combine(B, H, n - 2, FA + (n - 1) * zs, false, FA + (n - 2) * zs, -zs, MT + (n - 2) * zs, -zs,
+                           ADJ + (n - 1) * zs, -zs, st, false);
+        if (e != cudaSuccess) return e;
+        entry = ADJ + zs;
+    }
+    // pass 3: output runs of segments 0..n-2; segment 0 ends with ds0
+    return launch_dstate<I>(p.rpt, false, heads, T, H, p.t_seg, 0, n - 1, r, w, a, b, dy, entry, zs, dS_out, ds0, 0,
+                            1, nullptr, 0, st);
+}
+
+cudaError_t bwd_dstate_plan(int B, int T, int H, wkv7_dtype in_dt, const DstatePlan &p, const void *r,
+                            const void *w, const void *a, const void *b, const void *dy, const float *dsT,
+                            float *dS_out, float *ds0, float *scratch, cudaStream_t st) {
+    return in_dt == WKV7_F32
+               ? bwd_dstate_run<float>(B, T, H, p, r, w, a, b, dy, dsT, dS_out, ds0, scratch, st)
+               : bwd_dstate_run<__nv_bfloat16>(B, T, H, p, r, w, a, b, dy, dsT, dS_out, ds0, scratch, st);
+}
+
+// The sweep under the cost model's plan, within scratch_bytes of scratch.
+cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
+                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, float *scratch,
+                       size_t scratch_bytes, int sms, cudaStream_t st) {
+    const DstatePlan p =
+        dstate_plan(B, T, H, sms, in_dt == WKV7_F32, dS_out != nullptr, scratch ? scratch_bytes : 0);
+    return bwd_dstate_plan(B, T, H, in_dt, p, r, w, a, b, dy, dsT, dS_out, ds0, scratch, st);
 }
 
 // The input gradients of every chunk from its checkpoint, the next one (or
@@ -679,9 +861,9 @@ cudaError_t bwd_chunk_grads(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_
 cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
-                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
-                        cudaStream_t st) {
-    cudaError_t e = bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, dS_out, ds0, st);
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, float *scratch,
+                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st) {
+    cudaError_t e = bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, dS_out, ds0, scratch, scratch_bytes, sms, st);
     if (e != cudaSuccess) return e;
     return bwd_chunk_grads(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, ckpt, sfin, dS_out, dr, dw, dk, dv, da, db,
                            wait_limit, st);

@@ -23,11 +23,13 @@ cudaError_t step(int B, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
 cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
-                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, long long wait_limit,
-                        cudaStream_t st);
+                        void *dw, void *dk, void *dv, void *da, void *db, float *ds0, float *scratch,
+                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st);
 size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
 cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
-                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, cudaStream_t st);
+                       const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, float *scratch,
+                       size_t scratch_bytes, int sms, cudaStream_t st);
+size_t dstate_scratch_for(int B, int T, int H, int sms, bool need_dS);
 cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const float *summary, const float *F,
                              float *adj, cudaStream_t st);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
@@ -216,7 +218,8 @@ wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dt, wkv
 
 size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
-    return round_up(bwd_ckpt_bytes(B, T, H));
+    // dL/dS at every chunk end, the segmented sweep's scratch
+    return round_up(bwd_ckpt_bytes(B, T, H)) + round_up(dstate_scratch_for(B, T, H, current_sm_count(), true));
 }
 
 wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt,
@@ -237,9 +240,12 @@ wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_
     if (workspace_bytes < wkv7_backward_from_states_workspace_size(B, T, H, N) || !ptr_ok(workspace))
         return WKV7_ERR_INVALID_ARG;
     const long long lim = g_wait_limit.load();
+    const size_t ds_bytes = round_up(bwd_ckpt_bytes(B, T, H));
+    char *ws = static_cast<char *>(workspace);
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, states, sT,
-                                 static_cast<float *>(workspace), dr, dw, dk, dv, da, db, ds0,
-                                 lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                 reinterpret_cast<float *>(ws), dr, dw, dk, dv, da, db, ds0,
+                                 reinterpret_cast<float *>(ws + ds_bytes), workspace_bytes - ds_bytes,
+                                 current_sm_count(), lim > 0 ? lim : kDefaultWaitCycles, stream));
 }
 
 size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N) {
@@ -317,8 +323,10 @@ wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, co
 
 size_t wkv7_backward_workspace_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
-    // state before every chunk, the final state, dL/dS at every chunk end
-    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
+    // state before every chunk, dL/dS at every chunk end, the final state, the
+    // segmented sweep's scratch
+    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H)) +
+           round_up(dstate_scratch_for(B, T, H, current_sm_count(), true));
 }
 
 wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
@@ -349,22 +357,30 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
                                                 lim > 0 ? lim : kDefaultWaitCycles, stream)
                         : fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
+    const size_t used = 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
-                                 dv, da, db, ds0, lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                 dv, da, db, ds0, reinterpret_cast<float *>(ws + used), workspace_bytes - used,
+                                 current_sm_count(), lim > 0 ? lim : kDefaultWaitCycles, stream));
+}
+
+size_t wkv7_state_gradient_workspace_size(int B, int T, int H, int N) {
+    if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
+    return dstate_scratch_for(B, T, H, current_sm_count(), false);
 }
 
 wkv7_status wkv7_state_gradient(int B, int T, int H, int N, wkv7_dtype in_dt, const void *r, const void *w,
                                 const void *a, const void *b, const void *dy, const float *dsT, float *ds0,
-                                cudaStream_t stream) {
+                                void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt)) return WKV7_ERR_INVALID_ARG;
-    if (!opt_ptr_ok(dsT) || !ptr_ok(ds0)) return WKV7_ERR_INVALID_ARG;
+    if (!opt_ptr_ok(dsT) || !ptr_ok(ds0) || !opt_ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
     if ((size_t)B * H == 0) return WKV7_OK;
     if (T == 0) return copy_or_zero_state(ds0, dsT, B, H, stream);
     for (const void *p : {r, w, a, b, dy})
         if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
-    return from_cuda(bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, nullptr, ds0, stream));
+    return from_cuda(bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, nullptr, ds0, static_cast<float *>(workspace),
+                                workspace ? workspace_bytes : 0, current_sm_count(), stream));
 }
 
 wkv7_status wkv7_compose_adjoints(int nseg, int B, int H, int N, const float *dsT, const float *summaries,

@@ -28,7 +28,8 @@ EXPORTED_SYMBOLS = (
     "wkv7_forward_summary", "wkv7_compose_states", "wkv7_forward_summary_workspace_size",
     "wkv7_forward_continue", "wkv7_forward_host_workspace_size", "wkv7_forward_host",
     "wkv7_saved_states_size", "wkv7_forward_train", "wkv7_backward_from_states_workspace_size",
-    "wkv7_backward_from_states", "wkv7_state_gradient", "wkv7_compose_adjoints",
+    "wkv7_backward_from_states", "wkv7_state_gradient", "wkv7_state_gradient_workspace_size",
+    "wkv7_compose_adjoints",
 )
 
 _lib = None
@@ -84,7 +85,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_backward_from_states_workspace_size.restype = z
     lib.wkv7_backward_from_states.argtypes = [i, i, i, i, i, i] + [vp] * 17 + [vp, z, vp]
     lib.wkv7_backward_from_states.restype = i
-    lib.wkv7_state_gradient.argtypes = [i, i, i, i, i] + [vp] * 7 + [vp]
+    lib.wkv7_state_gradient.argtypes = [i, i, i, i, i] + [vp] * 8 + [z, vp]
+    lib.wkv7_state_gradient_workspace_size.argtypes = [i, i, i, i]
+    lib.wkv7_state_gradient_workspace_size.restype = z
     lib.wkv7_state_gradient.restype = i
     lib.wkv7_compose_adjoints.argtypes = [i, i, i, i, vp, vp, vp, vp, vp]
     lib.wkv7_compose_adjoints.restype = i
@@ -265,8 +268,13 @@ def forward_host(r, w, k, v, a, b, s0=None, *, y, sT=None, algo="auto", chunk_le
     return y, sT
 
 
-def state_gradient(r, w, a, b, dy, dsT=None, *, out=None, stream=None):
-    """dL/dS_0 [B,H,N,N] fp32 of a stretch [B,T,H,N] given dL/dS_T (dsT, None = 0)."""
+def state_gradient_workspace_size(B, T, H, N) -> int:
+    return load_library().wkv7_state_gradient_workspace_size(B, T, H, N)
+
+
+def state_gradient(r, w, a, b, dy, dsT=None, *, out=None, workspace=None, stream=None):
+    """dL/dS_0 [B,H,N,N] fp32 of a stretch [B,T,H,N] given dL/dS_T (dsT, None = 0).
+    ``workspace=False`` runs the sweep unsegmented."""
     lib = load_library()
     B, T, H, N = r.shape
     _same((w, a, b, dy), r.shape, r.dtype)
@@ -274,7 +282,13 @@ def state_gradient(r, w, a, b, dy, dsT=None, *, out=None, stream=None):
         _same((dsT,), (B, H, N, N), torch.float32)
     if out is None:
         out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
-    st = lib.wkv7_state_gradient(B, T, H, N, _dt(r), *map(_ptr, (r, w, a, b, dy, dsT, out)), _stream(stream))
+    if workspace is None:
+        nbytes = lib.wkv7_state_gradient_workspace_size(B, T, H, N)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=r.device) if nbytes else None
+    elif workspace is False:
+        workspace = None
+    st = lib.wkv7_state_gradient(B, T, H, N, _dt(r), *map(_ptr, (r, w, a, b, dy, dsT, out, workspace)),
+                                 0 if workspace is None else workspace.numel(), _stream(stream))
     _check("wkv7_state_gradient", st)
     return out
 

@@ -175,8 +175,8 @@ def test_training_pair_rejects_invalid_arguments(lib):
 
 
 def test_state_gradient_and_adjoints_reject_invalid_arguments(lib):
-    sg = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ptrs=None: lib.wkv7_state_gradient(
-        B, T, H, N, dt, *(ptrs or [P] * 7), None)
+    sg = lambda B=1, T=64, H=1, N=64, dt=wkv7.BF16, ptrs=None, ws=None: lib.wkv7_state_gradient(
+        B, T, H, N, dt, *(ptrs or [P] * 7), ws, 0, None)
     assert sg(N=32) == wkv7.ERR_UNSUPPORTED
     assert sg(dt=7) == wkv7.ERR_INVALID_ARG
     assert sg(T=-2) == wkv7.ERR_INVALID_ARG
@@ -189,7 +189,13 @@ def test_state_gradient_and_adjoints_reject_invalid_arguments(lib):
     bad = [P] * 7
     bad[5] = ctypes.c_void_p(12)                         # dsT misaligned
     assert sg(ptrs=bad) == wkv7.ERR_INVALID_ARG
+    assert sg(ws=ctypes.c_void_p(40)) == wkv7.ERR_INVALID_ARG     # workspace misaligned
     assert sg(H=0) == wkv7.OK
+    # the segmented sweep's scratch: 3 states per segment, none for many heads
+    assert lib.wkv7_state_gradient_workspace_size(1, 65536, 32, 64) % (3 * 32 * 64 * 64 * 4) == 0
+    assert lib.wkv7_state_gradient_workspace_size(1, 65536, 32, 64) > 0
+    assert lib.wkv7_state_gradient_workspace_size(16, 4096, 32, 64) == 0
+    assert lib.wkv7_state_gradient_workspace_size(1, 64, 1, 16) == 0
     ca = lambda nseg=2, B=1, H=1, N=64, dsT=None, sums=P, F=P, adj=P: lib.wkv7_compose_adjoints(
         nseg, B, H, N, dsT, sums, F, adj, None)
     assert ca(N=128) == wkv7.ERR_UNSUPPORTED

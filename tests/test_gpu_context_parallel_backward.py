@@ -55,6 +55,25 @@ def test_state_gradient_matches_oracle(cuda_device, dtype, tau, T, with_dsT):
     assert_close(to_f64(ds0), ref, tau, "ds0")
 
 
+@pytest.mark.parametrize("T", [700, 2001, 8192])
+def test_segmented_sweep_matches_oracle(cuda_device, T):
+    """Few heads over many tokens: with its workspace the sweep runs as
+    segments (dual passes, then the chained adjoints); ds0 vs the oracle and
+    vs the one-pass sweep, w near 1 so every segment's product matters."""
+    B, H = 1, 2
+    assert wkv7.state_gradient_workspace_size(B, T, H, 64) > 0
+    d = _case(B, T, H, 930 + T, "bf16", x_mean=-4.0)
+    r, w, k, v, a, b = _dev_args(d)
+    dy, dsT = to_dev(d["dy"]), to_dev(d["dsT"])
+    seg = wkv7.state_gradient(r, w, a, b, dy, dsT)
+    one = wkv7.state_gradient(r, w, a, b, dy, dsT, workspace=False)
+    assert wkv7.device_status() == wkv7.OK
+    rf, wf, kf, vf, af, bf = _f64(d)
+    ref = oracle.state_gradient(rf, wf, af, bf, inputs.to_f64(d["dy"]), d["dsT"].astype(np.float64))
+    assert_close(to_f64(seg), ref, TAU_BF16, "segmented ds0")
+    assert_close(to_f64(seg), to_f64(one), TAU_BF16, "segmented vs one pass")
+
+
 def test_state_gradient_equals_backward_ds0(cuda_device):
     """The sweep's ds0 is the same quantity the full backward returns."""
     d = _case(1, 300, 4, 950, "bf16")
