@@ -690,8 +690,8 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
 
 // One launch of dual summary runs over nz segments of t_seg tokens: E of
 // segment z (its final state from 0) to e_out + z e_zstride, M (from I, v read
-// as 0) to m_out + z m_zstride.  With y given, the first segment instead runs
-// from s0 and writes y (and ckpt, if given): its "E" is its true final state.
+// as 0) to m_out + z m_zstride.  With y or ckpt given, the first segment
+// instead runs from s0 and writes them: its "E" is its true final state.
 static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const void *r, const void *w, const void *k,
                                const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
                                float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st,
@@ -700,7 +700,7 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
     static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES_DUAL;
-    const int first_out = y != nullptr ? 1 : 0;
+    const int first_out = (y != nullptr || ckpt != nullptr) ? 1 : 0;
     using bf = __nv_bfloat16;
 #define WKV7_DUAL_LAUNCH(O)                                                                                    \
     do {                                                                                                       \
@@ -914,15 +914,6 @@ cudaError_t compose_states(int B, int H, int nseg, const float *s0, const float 
     const long long zst = (long long)B * H * kN * kN;
     const float *m0 = summary ? summary + zst : nullptr;     // nseg = 0 reads no summary
     return launch_combine(B, H, nseg, s0, false, summary, 2 * zst, m0, 2 * zst, out, zst, st);
-}
-
-// State checkpoints before every 32-token chunk (and the final state) for the
-// backward: one pass of the chunked kernel without y.
-cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
-                                  const void *a, const void *b, const float *s0, float *ckpt, float *sT,
-                                  long long wait_limit, cudaStream_t st) {
-    return launch_chunk(B, T, H, T, 1, 1, WKV7_BF16, r, w, k, v, a, b, s0, 0, nullptr, sT, 0, -1, wait_limit, st,
-                        ckpt);
 }
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,

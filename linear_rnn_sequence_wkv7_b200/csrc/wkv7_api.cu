@@ -39,9 +39,6 @@ cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt
                           const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
                           float *sT, float *ckpt, int CK, cudaStream_t st);
 int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last);
-cudaError_t fwd_chunk_checkpoints(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
-                                  const void *a, const void *b, const float *s0, float *ckpt, float *sT,
-                                  long long wait_limit, cudaStream_t st);
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
 cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
                               const void *a, const void *b, float *summary, int nseg, void *workspace,
@@ -112,6 +109,15 @@ int summary_segments(int B, int T, int H, const void *workspace, size_t workspac
 }
 
 size_t bwd_ckpt_bytes(int B, int T, int H) { return bwd_chunk_ckpt_bytes(B, T, H); }
+
+// Scratch shared by the backward's checkpoint pass (the segmented chunked
+// forward, bf16 inputs) and then its state-gradient sweep (segments too).
+int bwd_ckpt_segments(int B, int T, int H, int sms) { return sms > 0 ? chunk_segments(B, T, H, sms, false) : 1; }
+size_t bwd_scratch_bytes(int B, int T, int H) {
+    const int sms = current_sm_count();
+    return std::max(round_up(chunk_workspace_bytes(B, T, H, bwd_ckpt_segments(B, T, H, sms))),
+                    round_up(dstate_scratch_for(B, T, H, sms, true)));
+}
 size_t state_bytes(int B, int H) { return (size_t)B * H * kN * kN * sizeof(float); }
 
 }  // namespace
@@ -324,9 +330,8 @@ wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, co
 size_t wkv7_backward_workspace_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
     // state before every chunk, dL/dS at every chunk end, the final state, the
-    // segmented sweep's scratch
-    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H)) +
-           round_up(dstate_scratch_for(B, T, H, current_sm_count(), true));
+    // segmented passes' scratch
+    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H)) + bwd_scratch_bytes(B, T, H);
 }
 
 wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
@@ -349,18 +354,27 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     float *ckpt = reinterpret_cast<float *>(ws);
     float *dSo = reinterpret_cast<float *>(ws + round_up(bwd_ckpt_bytes(B, T, H)));
     float *sfin = reinterpret_cast<float *>(ws + 2 * round_up(bwd_ckpt_bytes(B, T, H)));
-    // checkpoints: the chunked tensor-core forward for bf16 inputs (its chunk
-    // is the backward's), the sequential scan for fp32 inputs
-    const long long lim = g_wait_limit.load();
-    cudaError_t e = in_dt == WKV7_BF16
-                        ? fwd_chunk_checkpoints(B, T, H, r, w, k, v, a, b, s0, ckpt, sfin,
-                                                lim > 0 ? lim : kDefaultWaitCycles, stream)
-                        : fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
-    if (e != cudaSuccess) return WKV7_ERR_CUDA;
     const size_t used = 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
+    char *scratch = ws + used;
+    const size_t scratch_bytes = workspace_bytes - used;
+    const int sms = current_sm_count();
+    // checkpoints: the chunked tensor-core forward without y for bf16 inputs
+    // (its chunk is the backward's; sequence segments side by side when the
+    // heads are few), the sequential scan for fp32 inputs
+    const long long lim = g_wait_limit.load();
+    cudaError_t e;
+    if (in_dt == WKV7_BF16) {
+        const int want = bwd_ckpt_segments(B, T, H, sms);
+        const int nseg = (want > 1 && scratch_bytes >= chunk_workspace_bytes(B, T, H, want)) ? want : 1;
+        e = fwd_chunk(B, T, H, WKV7_BF16, r, w, k, v, a, b, s0, nullptr, sfin, nseg, scratch,
+                      lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt);
+    } else {
+        e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
+    }
+    if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
-                                 dv, da, db, ds0, reinterpret_cast<float *>(ws + used), workspace_bytes - used,
-                                 current_sm_count(), lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                 dv, da, db, ds0, reinterpret_cast<float *>(scratch), scratch_bytes, sms,
+                                 lim > 0 ? lim : kDefaultWaitCycles, stream));
 }
 
 size_t wkv7_state_gradient_workspace_size(int B, int T, int H, int N) {
