@@ -50,6 +50,17 @@ def test_fp32_small(cuda_device, T):
         assert_close(got, ref, TAU_F32, name)
 
 
+@pytest.mark.parametrize("dtype,T", [("f32", 1000), ("bf16", 3000)])
+def test_few_heads_long_sequence(cuda_device, dtype, T):
+    """One head: the state-gradient sweep runs as segments (and, for bf16,
+    the checkpoint pass as the segmented forward); the fp32 path keeps 1e-5."""
+    d = _case(1, T, 1, 350 + T, dtype)
+    assert wkv7.backward_workspace_size(1, T, 1, 64) > 2 * ((T + 31) // 32 + 1) * 64 * 64 * 4
+    tau = TAU_F32 if dtype == "f32" else TAU_BF16
+    for name, got, ref in zip(GRAD_NAMES, _gpu(d), _ref(d)):
+        assert_close(got, ref, tau, name)
+
+
 @pytest.mark.parametrize("T,with_dsT", [(1, True), (16, False), (32, True), (33, False), (77, False),
                                          (200, True)])
 def test_bf16_inputs(cuda_device, T, with_dsT):

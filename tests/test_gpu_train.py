@@ -58,8 +58,11 @@ def test_forward_train_matches_forward_and_oracle(cuda_device, dtype, B, T, H, a
         assert_close(to_f64(states[:, :, c]), ref[:, :, c], tau, f"state before chunk {c}")
 
 
-@pytest.mark.parametrize("dtype,B,T,H", [("bf16", 2, 200, 3), ("f32", 2, 100, 2), ("bf16", 1, 33, 1)])
+@pytest.mark.parametrize("dtype,B,T,H", [("bf16", 2, 200, 3), ("f32", 2, 100, 2), ("bf16", 1, 33, 1),
+                                         ("bf16", 1, 1500, 2), ("f32", 1, 1100, 1)])
 def test_backward_from_states_matches_oracle(cuda_device, dtype, B, T, H):
+    """(1, 1500, 2) and (1, 1100, 1): few heads, so the forward keeps its
+    states from sequence segments and the sweep runs as segments too."""
     d = _case(B, T, H, 990 + T, dtype)
     x, s0, dy, dsT = _dev(d)
     _, sT, states = wkv7.forward_train(*x, s0)
