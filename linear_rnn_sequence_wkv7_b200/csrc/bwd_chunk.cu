@@ -56,10 +56,11 @@ constexpr float kMinDecay = 1e-30f;
 
 // ---------------------------------------------------------------------------
 // dS_out(c) for every chunk and ds0: reverse sweep of the state gradient.
-// The rows of dS evolve independently.  CTAs of 128 threads, four lanes per
-// row (16 columns each) and RPT rows per thread: RPT = 2 covers a (b, h) with
-// one CTA; RPT = 1 splits it over two CTAs (rows 32 q .. 32 q + 31), for
-// problems with too few heads to fill the GPU.  Token tiles of r w a b dy are
+// The rows of dS evolve independently.  Four lanes per row (16 columns each)
+// and RPT rows per thread: RPT = 4 covers a (b, h) with a CTA of 64 threads,
+// RPT = 2 with 128 threads; RPT = 1 splits it over two CTAs of 128 (rows
+// 32 q .. 32 q + 31), for problems with too few heads to fill the GPU.  More
+// rows per thread share the conversions and loads of r, w, a, b.  Token tiles of r w a b dy are
 // prefetched by cp.async, 32 tokens ahead.
 //
 // A launch runs nz segments of t_seg tokens (segment seg0 + z, whole chunks;
@@ -86,11 +87,12 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
     constexpr int NR = DUAL ? 2 * RPT : RPT;   // rows RPT.. carry the dual run's second G
     extern __shared__ __align__(16) unsigned char dsmem[];
     auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
-    constexpr int SPLIT = 2 / RPT;     // CTAs per head
+    constexpr int SPLIT = RPT == 1 ? 2 : 1;         // CTAs per head
+    constexpr int NTH = 4 * kN / (SPLIT * RPT);     // threads: four lanes per group of RPT rows
     const int tid = threadIdx.x, q = tid & 3;
     const int per_z = gridDim.x / nz;
     const int z = blockIdx.x / per_z, head = (blockIdx.x % per_z) / SPLIT;
-    const int row0 = 32 * (blockIdx.x % SPLIT) * (SPLIT - 1) + RPT * (tid >> 2);
+    const int row0 = (SPLIT == 2 ? 32 * (blockIdx.x % 2) : 0) + RPT * (tid >> 2);
     const int bb = head / H, h = head % H;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
@@ -105,7 +107,7 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
         const int t0 = c * L, Lc = min(L, T - t0);
 #pragma unroll
         for (int ten = 0; ten < NTEN; ++ten)
-            for (int x = tid; x < L * CPV; x += 128) {
+            for (int x = tid; x < L * CPV; x += NTH) {
                 const int tt = x / CPV, ch = x % CPV;
                 if (tt < Lc)
                     cp_async16(&tile[stage][ten][tt][ch * VEC], src[ten] + base + (size_t)(t0 + tt) * tok_stride + ch * VEC);
@@ -667,19 +669,23 @@ cudaError_t launch_dstate(int rpt, bool dual, int heads, int T, int H, int t_seg
                           long long g_in_zs, float *dS_out, float *g_out, long long g_out_zs, int g_out_nz,
                           float *m_out, long long m_zs, cudaStream_t st) {
     const size_t smem = 2 * 5 * bwdc::L * kN * sizeof(I);
-    const unsigned grid = (unsigned)((size_t)nz * heads * (2 / rpt));
+    if (rpt == 4 && dual) rpt = 2;      // eight rows of two states would spill
+    const unsigned grid = (unsigned)((size_t)nz * heads * (rpt == 1 ? 2 : 1));
+    const int threads = rpt == 4 ? 64 : 128;
 #define WKV7_DSTATE(R, D)                                                                                    \
     do {                                                                                                     \
         auto kern = bwd_dstate_kernel<I, R, D>;                                                              \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
         if (e != cudaSuccess) return e;                                                                      \
-        kern<<<grid, 128, smem, st>>>(T, t_seg, seg0, nz, (const I *)r, (const I *)w, (const I *)a,         \
+        kern<<<grid, threads, smem, st>>>(T, t_seg, seg0, nz, (const I *)r, (const I *)w, (const I *)a,     \
                                       (const I *)b, (const I *)dy, H, g_in, g_in_zs, dS_out, g_out, g_out_zs, \
                                       g_out_nz, m_out, m_zs);                                                \
     } while (0)
     if (rpt == 1) {
         if (dual) WKV7_DSTATE(1, true);
         else WKV7_DSTATE(1, false);
+    } else if (rpt == 4 && !dual) {
+        WKV7_DSTATE(4, false);
     } else {
         if (dual) WKV7_DSTATE(2, true);
         else WKV7_DSTATE(2, false);
@@ -709,20 +715,33 @@ DstatePlan dstate_split(int T, int nseg_want, int rpt) {
 
 // Estimated time (ns) of one sweep launch of n CTAs over `steps` tokens.  A
 // step of a CTA alone on its SM is latency-bound; each further co-resident
-// CTA adds its issue time; CTAs beyond the resident ones run in later waves.
-// Fitted on B200 (bf16 inputs; B = 1 and 8, H = 32, T = 4096 .. 65536).
+// CTA adds its issue time (for the two-warp CTAs of rpt 4, from the third on);
+// CTAs beyond the resident ones run in later waves.  Fitted on B200 (bf16
+// inputs; B = 1 .. 16, H = 32, T = 4096 .. 65536).
 static double dstate_launch_ns(long long n, long long steps, int rpt, bool dual, bool f32, int sms) {
-    const double lat = rpt == 1 ? (dual ? 198.0 : 156.0) : (dual ? 252.0 : 221.0);
-    const double add = rpt == 1 ? (dual ? 115.0 : 156.0) : (dual ? 191.0 : 109.0);
+    double lat, add;
+    long long free_k = 1;
+    if (rpt == 1) {
+        lat = dual ? 198.0 : 156.0;
+        add = dual ? 115.0 : 156.0;
+    } else if (rpt == 2) {
+        lat = dual ? 252.0 : 221.0;
+        add = dual ? 191.0 : 109.0;
+    } else {
+        lat = 306.0;
+        add = 110.0;
+        free_k = 2;
+    }
     const int res = f32 ? 2 : (rpt == 2 && dual ? 4 : 5);    // shared memory, registers
     const long long per_sm = (n + sms - 1) / sms;
     const long long waves = (per_sm + res - 1) / res;
     const long long k = std::min<long long>(per_sm, res);
-    return (double)waves * (double)steps * (lat + add * (double)(k - 1));
+    return (double)waves * (double)steps * (lat + add * (double)std::max<long long>(0, k - free_k));
 }
 
 // The plan with the lowest estimated time whose scratch fits scratch_cap
-// bytes: rpt 1 or 2, nseg = 1 or a split into segments of at least two chunks.
+// bytes: rpt 1, 2 or 4 (one pass only), nseg = 1 or a split into segments of
+// at least two chunks.
 // need_dS: dS at every chunk end is wanted (the backward), else ds0 alone.
 DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, size_t scratch_cap) {
     const long long heads = (long long)B * H;
@@ -731,9 +750,9 @@ DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, siz
     constexpr double kCombineStepNs = 3000.0, kLaunchNs = 4000.0;
     DstatePlan best;
     double best_ns = 0.0;
-    for (int rpt = 1; rpt <= 2; ++rpt) {
-        const long long per_head = 2 / rpt;
-        for (int want = 1; want <= std::min(64, std::max(1, chunks / 2)); ++want) {
+    for (int rpt : {1, 2, 4}) {
+        const long long per_head = rpt == 1 ? 2 : 1;
+        for (int want = 1; want <= (rpt == 4 ? 1 : std::min(64, std::max(1, chunks / 2))); ++want) {
             const DstatePlan p = dstate_split(T, want, rpt);
             if (p.nseg != want) continue;
             if (p.nseg > 1 && dstate_scratch_bytes(B, H, p.nseg) > scratch_cap) break;
