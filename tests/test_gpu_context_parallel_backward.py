@@ -164,3 +164,31 @@ def test_backward_orchestration_without_process_group(cuda_device):
     torch.cuda.synchronize()
     for j, name in enumerate(GRADS + ("ds0",)):
         assert_close(to_f64(got[j]), to_f64(ref[j]), TAU_BF16, name)
+
+
+def test_backward_orchestration_over_a_one_rank_nccl_group(cuda_device):
+    """forward_context_parallel + backward_context_parallel inside an NCCL
+    process group of one rank: both all-gathers go through NCCL on the GPU;
+    the gradients equal the plain backward's."""
+    import os
+    import socket
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        d = _case(1, 1000, 4, 995, "bf16")
+        args = _dev_args(d)
+        s0, dy, dsT = to_dev(d["s0"]), to_dev(d["dy"]), to_dev(d["dsT"])
+        _, s_in, _, sums = forward_context_parallel(*args, s0, return_summaries=True)
+        got = backward_context_parallel(*args, s_in, sums, dy, dsT)
+        ref = wkv7.backward(*args, s0, dy, dsT)
+        torch.cuda.synchronize()
+        for j, name in enumerate(GRADS + ("ds0",)):
+            assert_close(to_f64(got[j]), to_f64(ref[j]), TAU_BF16, name)
+    finally:
+        dist.destroy_process_group()
