@@ -56,11 +56,13 @@ constexpr float kMinDecay = 1e-30f;
 
 // ---------------------------------------------------------------------------
 // dS_out(c) for every chunk and ds0: reverse sweep of the state gradient.
-// The rows of dS evolve independently.  Four lanes per row (16 columns each)
-// and RPT rows per thread: RPT = 4 covers a (b, h) with a CTA of 64 threads,
-// RPT = 2 with 128 threads; RPT = 1 splits it over two CTAs of 128 (rows
-// 32 q .. 32 q + 31), for problems with too few heads to fill the GPU.  More
-// rows per thread share the conversions and loads of r, w, a, b.  Token tiles of r w a b dy are
+// The rows of dS evolve independently.  LPR lanes per row (64 / LPR columns
+// each, in groups of 4 at a stride of 4 LPR) and RPT rows per thread: with
+// four lanes, RPT = 4 covers a (b, h) with a CTA of 64 threads, RPT = 2 with
+// 128 threads, and RPT = 1 splits it over two CTAs of 128 (rows 32 q ..
+// 32 q + 31) for problems with too few heads to fill the GPU; eight lanes and
+// RPT = 4 make 128-thread CTAs, more warps per head at the same instructions
+// per row.  More rows per thread share the conversions and loads of r, w, a, b.  Token tiles of r w a b dy are
 // prefetched by cp.async, 32 tokens ahead.
 //
 // A launch runs nz segments of t_seg tokens (segment seg0 + z, whole chunks;
@@ -76,7 +78,7 @@ constexpr float kMinDecay = 1e-30f;
 //   g_out  : G at the segment's start, for runs z < g_out_nz
 //   m_out  : the dual runs' M^T
 // ---------------------------------------------------------------------------
-template <typename InT, int RPT, bool DUAL>
+template <typename InT, int RPT, int LPR, bool DUAL>
 __global__ void __launch_bounds__(128)
 bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r, const InT *__restrict__ w,
                   const InT *__restrict__ a, const InT *__restrict__ b, const InT *__restrict__ dy, int H,
@@ -85,14 +87,16 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
                   long long m_zstride) {
     constexpr int L = bwdc::L, NTEN = 5, VEC = 16 / sizeof(InT), CPV = kN / VEC;
     constexpr int NR = DUAL ? 2 * RPT : RPT;   // rows RPT.. carry the dual run's second G
+    constexpr int CPL = kN / LPR, NG = CPL / 4;   // columns per lane, in groups of 4 (stride 4 LPR)
     extern __shared__ __align__(16) unsigned char dsmem[];
     auto tile = reinterpret_cast<InT(*)[NTEN][L][kN]>(dsmem);   // [2 stages]
     constexpr int SPLIT = RPT == 1 ? 2 : 1;         // CTAs per head
-    constexpr int NTH = 4 * kN / (SPLIT * RPT);     // threads: four lanes per group of RPT rows
-    const int tid = threadIdx.x, q = tid & 3;
+    constexpr int NTH = LPR * kN / (SPLIT * RPT);   // threads: LPR lanes per group of RPT rows
+    static_assert(NTH <= 128 && (LPR == 4 || LPR == 8), "sweep CTA shape");
+    const int tid = threadIdx.x, q = tid % LPR;
     const int per_z = gridDim.x / nz;
     const int z = blockIdx.x / per_z, head = (blockIdx.x % per_z) / SPLIT;
-    const int row0 = (SPLIT == 2 ? 32 * (blockIdx.x % 2) : 0) + RPT * (tid >> 2);
+    const int row0 = (SPLIT == 2 ? 32 * (blockIdx.x % 2) : 0) + RPT * (tid / LPR);
     const int bb = head / H, h = head % H;
     const size_t tok_stride = (size_t)H * kN;
     const size_t base = ((size_t)bb * T * H + h) * kN;
@@ -102,6 +106,7 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
     const bool out_run = !DUAL || z == nz - 1;
     const size_t hoff = (size_t)head * kN * kN;
     const InT *src[NTEN] = {r, w, a, b, dy};
+    auto col = [&](int m) { return 4 * LPR * m + 4 * q; };   // first of this lane's 4 columns in group m
 
     auto issue = [&](int c, int stage) {
         const int t0 = c * L, Lc = min(L, T - t0);
@@ -115,20 +120,20 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
         cp_async_commit();
     };
 
-    float g[NR][16];
+    float g[NR][CPL];
 #pragma unroll
     for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < NG; ++m) {
             float4 d4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int row = row0 + rr % RPT, col = 16 * m + 4 * q;
+            const int row = row0 + rr % RPT, c0 = col(m);
             if (rr >= RPT) {             // identity start of the product run
-                d4.x = row == col ? 1.f : 0.f;
-                d4.y = row == col + 1 ? 1.f : 0.f;
-                d4.z = row == col + 2 ? 1.f : 0.f;
-                d4.w = row == col + 3 ? 1.f : 0.f;
+                d4.x = row == c0 ? 1.f : 0.f;
+                d4.y = row == c0 + 1 ? 1.f : 0.f;
+                d4.z = row == c0 + 2 ? 1.f : 0.f;
+                d4.w = row == c0 + 3 ? 1.f : 0.f;
             } else if (out_run && g_in) {
-                d4 = load4(g_in + z * g_in_zstride + hoff + (size_t)row * kN + col);
+                d4 = load4(g_in + z * g_in_zstride + hoff + (size_t)row * kN + c0);
             }
             g[rr][4 * m] = d4.x; g[rr][4 * m + 1] = d4.y; g[rr][4 * m + 2] = d4.z; g[rr][4 * m + 3] = d4.w;
         }
@@ -140,12 +145,12 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
         __syncthreads();
         if (c > c_begin) issue(c - 1, stage ^ 1);
         if (out_run && dS_out) {   // dL/dS after the chunk's last token, before its own output is added
-            float *dst = dS_out + ((size_t)head * nck_total + c) * kN * kN + (size_t)row0 * kN + 4 * q;
+            float *dst = dS_out + ((size_t)head * nck_total + c) * kN * kN + (size_t)row0 * kN;
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    store4(dst + (size_t)rr * kN + 16 * m,
+                for (int m = 0; m < NG; ++m)
+                    store4(dst + (size_t)rr * kN + col(m),
                            make_float4(g[rr][4 * m], g[rr][4 * m + 1], g[rr][4 * m + 2], g[rr][4 * m + 3]));
         }
         for (int tt = Lc - 1; tt >= 0; --tt) {
@@ -159,8 +164,8 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dp4[rr][e] = 0.f;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 r4 = load4(rv + 16 * m + 4 * q), b4 = load4(bv + 16 * m + 4 * q);
+            for (int m = 0; m < NG; ++m) {
+                const float4 r4 = load4(rv + col(m)), b4 = load4(bv + col(m));
                 const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
                 for (int rr = 0; rr < NR; ++rr)
@@ -175,12 +180,12 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
 #pragma unroll
             for (int rr = 0; rr < NR; ++rr) {
                 dp[rr] = (dp4[rr][0] + dp4[rr][1]) + (dp4[rr][2] + dp4[rr][3]);
-                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 1);
-                dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], 2);
+#pragma unroll
+                for (int o = 1; o < LPR; o <<= 1) dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], o);
             }
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 w4 = load4(wv + 16 * m + 4 * q), a4 = load4(av + 16 * m + 4 * q);
+            for (int m = 0; m < NG; ++m) {
+                const float4 w4 = load4(wv + col(m)), a4 = load4(av + col(m));
                 const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                 for (int rr = 0; rr < NR; ++rr)
@@ -193,8 +198,8 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr)
 #pragma unroll
-            for (int m = 0; m < 4; ++m)
-                store4(dst + hoff + (size_t)(row0 + rr) * kN + 16 * m + 4 * q,
+            for (int m = 0; m < NG; ++m)
+                store4(dst + hoff + (size_t)(row0 + rr) * kN + col(m),
                        make_float4(g[r_first + rr][4 * m], g[r_first + rr][4 * m + 1], g[r_first + rr][4 * m + 2],
                                    g[r_first + rr][4 * m + 3]));
     };
@@ -662,33 +667,40 @@ size_t dstate_scratch_bytes(int B, int H, int nseg) {
 
 namespace {
 
-// One launch of the sweep kernel: nz segments from seg0, all heads.
+// One launch of the sweep kernel: nz segments from seg0, all heads; rpt rows
+// per thread and lpr lanes per row (rpt 1 splits a head over two CTAs).
 template <typename I>
-cudaError_t launch_dstate(int rpt, bool dual, int heads, int T, int H, int t_seg, int seg0, int nz, const void *r,
-                          const void *w, const void *a, const void *b, const void *dy, const float *g_in,
-                          long long g_in_zs, float *dS_out, float *g_out, long long g_out_zs, int g_out_nz,
-                          float *m_out, long long m_zs, cudaStream_t st) {
+cudaError_t launch_dstate(int rpt, int lpr, bool dual, int heads, int T, int H, int t_seg, int seg0, int nz,
+                          const void *r, const void *w, const void *a, const void *b, const void *dy,
+                          const float *g_in, long long g_in_zs, float *dS_out, float *g_out, long long g_out_zs,
+                          int g_out_nz, float *m_out, long long m_zs, cudaStream_t st) {
     const size_t smem = 2 * 5 * bwdc::L * kN * sizeof(I);
-    if (rpt == 4 && dual) rpt = 2;      // eight rows of two states would spill
-    const unsigned grid = (unsigned)((size_t)nz * heads * (rpt == 1 ? 2 : 1));
-    const int threads = rpt == 4 ? 64 : 128;
-#define WKV7_DSTATE(R, D)                                                                                    \
+    if (lpr != 8) lpr = 4;
+    if (lpr == 8) rpt = 4;
+    if (rpt == 4 && lpr == 4 && dual) rpt = 2;     // eight rows of two states in 16 columns would spill
+    const int split = rpt == 1 ? 2 : 1;
+    const unsigned grid = (unsigned)((size_t)nz * heads * split);
+    const int threads = lpr * kN / (split * rpt);
+#define WKV7_DSTATE(R, P, D)                                                                                 \
     do {                                                                                                     \
-        auto kern = bwd_dstate_kernel<I, R, D>;                                                              \
+        auto kern = bwd_dstate_kernel<I, R, P, D>;                                                           \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
         if (e != cudaSuccess) return e;                                                                      \
         kern<<<grid, threads, smem, st>>>(T, t_seg, seg0, nz, (const I *)r, (const I *)w, (const I *)a,     \
-                                      (const I *)b, (const I *)dy, H, g_in, g_in_zs, dS_out, g_out, g_out_zs, \
-                                      g_out_nz, m_out, m_zs);                                                \
+                                          (const I *)b, (const I *)dy, H, g_in, g_in_zs, dS_out, g_out,     \
+                                          g_out_zs, g_out_nz, m_out, m_zs);                                  \
     } while (0)
-    if (rpt == 1) {
-        if (dual) WKV7_DSTATE(1, true);
-        else WKV7_DSTATE(1, false);
-    } else if (rpt == 4 && !dual) {
-        WKV7_DSTATE(4, false);
+    if (lpr == 8) {
+        if (dual) WKV7_DSTATE(4, 8, true);
+        else WKV7_DSTATE(4, 8, false);
+    } else if (rpt == 1) {
+        if (dual) WKV7_DSTATE(1, 4, true);
+        else WKV7_DSTATE(1, 4, false);
+    } else if (rpt == 4) {
+        WKV7_DSTATE(4, 4, false);
     } else {
-        if (dual) WKV7_DSTATE(2, true);
-        else WKV7_DSTATE(2, false);
+        if (dual) WKV7_DSTATE(2, 4, true);
+        else WKV7_DSTATE(2, 4, false);
     }
 #undef WKV7_DSTATE
     return cudaGetLastError();
@@ -699,10 +711,10 @@ cudaError_t launch_dstate(int rpt, bool dual, int heads, int T, int H, int t_seg
 // The sweep's plan: segments (whole chunks, all non-empty) and rows per
 // thread, for B*H heads of T tokens.
 struct DstatePlan {
-    int nseg = 1, t_seg = 0, rpt = 2;
+    int nseg = 1, t_seg = 0, rpt = 2, lpr = 4;
 };
 
-DstatePlan dstate_split(int T, int nseg_want, int rpt) {
+DstatePlan dstate_split(int T, int nseg_want, int rpt, int lpr = 4) {
     DstatePlan p;
     const int chunks = (T + bwdc::L - 1) / bwdc::L;
     const int want = std::max(1, std::min(nseg_want, chunks));
@@ -710,6 +722,7 @@ DstatePlan dstate_split(int T, int nseg_want, int rpt) {
     p.t_seg = per * bwdc::L;
     p.nseg = (chunks + per - 1) / per;
     p.rpt = rpt;
+    p.lpr = lpr;
     return p;
 }
 
@@ -718,10 +731,13 @@ DstatePlan dstate_split(int T, int nseg_want, int rpt) {
 // CTA adds its issue time (for the two-warp CTAs of rpt 4, from the third on);
 // CTAs beyond the resident ones run in later waves.  Fitted on B200 (bf16
 // inputs; B = 1 .. 16, H = 32, T = 4096 .. 65536).
-static double dstate_launch_ns(long long n, long long steps, int rpt, bool dual, bool f32, int sms) {
+static double dstate_launch_ns(long long n, long long steps, int rpt, int lpr, bool dual, bool f32, int sms) {
     double lat, add;
     long long free_k = 1;
-    if (rpt == 1) {
+    if (lpr == 8) {
+        lat = 197.0;
+        add = 120.0;
+    } else if (rpt == 1) {
         lat = dual ? 198.0 : 156.0;
         add = dual ? 115.0 : 156.0;
     } else if (rpt == 2) {
@@ -740,8 +756,9 @@ static double dstate_launch_ns(long long n, long long steps, int rpt, bool dual,
 }
 
 // The plan with the lowest estimated time whose scratch fits scratch_cap
-// bytes: rpt 1, 2 or 4 (one pass only), nseg = 1 or a split into segments of
-// at least two chunks.
+// bytes: rpt 1, 2 or 4 rows per thread with four lanes per row, or 4 rows
+// with eight lanes (those two one-pass only), nseg = 1 or a split into
+// segments of at least two chunks.
 // need_dS: dS at every chunk end is wanted (the backward), else ds0 alone.
 DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, size_t scratch_cap) {
     const long long heads = (long long)B * H;
@@ -750,23 +767,24 @@ DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, siz
     constexpr double kCombineStepNs = 3000.0, kLaunchNs = 4000.0;
     DstatePlan best;
     double best_ns = 0.0;
-    for (int rpt : {1, 2, 4}) {
+    for (int variant = 0; variant < 4; ++variant) {
+        const int rpt = variant == 0 ? 1 : variant == 1 ? 2 : 4, lpr = variant == 3 ? 8 : 4;
         const long long per_head = rpt == 1 ? 2 : 1;
         for (int want = 1; want <= (rpt == 4 ? 1 : std::min(64, std::max(1, chunks / 2))); ++want) {
-            const DstatePlan p = dstate_split(T, want, rpt);
+            const DstatePlan p = dstate_split(T, want, rpt, lpr);
             if (p.nseg != want) continue;
             if (p.nseg > 1 && dstate_scratch_bytes(B, H, p.nseg) > scratch_cap) break;
             const int n = p.nseg;
             double ns;
             if (n == 1) {
-                ns = dstate_launch_ns(heads * per_head, T, rpt, false, f32, sms);
+                ns = dstate_launch_ns(heads * per_head, T, rpt, lpr, false, f32, sms);
             } else if (need_dS) {
                 const long long ctas = (n - 1) * heads * per_head;
-                ns = dstate_launch_ns(ctas, p.t_seg, rpt, n > 2, f32, sms) +
-                     dstate_launch_ns(ctas, p.t_seg, rpt, false, f32, sms) + kCombineStepNs * (n - 2) +
+                ns = dstate_launch_ns(ctas, p.t_seg, rpt, lpr, n > 2, f32, sms) +
+                     dstate_launch_ns(ctas, p.t_seg, rpt, lpr, false, f32, sms) + kCombineStepNs * (n - 2) +
                      kLaunchNs * (n > 2 ? 2 : 1);
             } else {
-                ns = dstate_launch_ns(n * heads * per_head, p.t_seg, rpt, true, f32, sms) +
+                ns = dstate_launch_ns(n * heads * per_head, p.t_seg, rpt, lpr, true, f32, sms) +
                      kCombineStepNs * (n - 1) + kLaunchNs;
             }
             if (best_ns == 0.0 || ns < 0.97 * best_ns) {
@@ -800,21 +818,21 @@ cudaError_t bwd_dstate_run(int B, int T, int H, const DstatePlan &p, const void 
                            float *scratch, cudaStream_t st) {
     const int heads = B * H, n = p.nseg;
     if (n <= 1)
-        return launch_dstate<I>(p.rpt, false, heads, T, H, std::max(p.t_seg, T), 0, 1, r, w, a, b, dy, dsT, 0,
+        return launch_dstate<I>(p.rpt, p.lpr, false, heads, T, H, std::max(p.t_seg, T), 0, 1, r, w, a, b, dy, dsT, 0,
                                 dS_out, ds0, 0, 1, nullptr, 0, st);
     const long long zs = (long long)heads * kN * kN;
     float *FA = scratch, *MT = scratch + n * zs, *ADJ = scratch + 2 * n * zs;
     cudaError_t e;
     if (!dS_out) {
         // every segment summarised (the last one from dsT), then one chain to ds0
-        e = launch_dstate<I>(p.rpt, true, heads, T, H, p.t_seg, 0, n, r, w, a, b, dy, dsT, 0, nullptr, FA, zs, n,
+        e = launch_dstate<I>(p.rpt, p.lpr, true, heads, T, H, p.t_seg, 0, n, r, w, a, b, dy, dsT, 0, nullptr, FA, zs, n,
                              MT, zs, st);
         if (e != cudaSuccess) return e;
         return launch_combine(B, H, n - 1, FA + (n - 1) * zs, false, FA + (n - 2) * zs, -zs, MT + (n - 2) * zs, -zs,
                               ds0, 0, st, false);
     }
     // pass 1: segments 1..n-1, the last as an output run from dsT
-    e = launch_dstate<I>(p.rpt, n > 2, heads, T, H, p.t_seg, 1, n - 1, r, w, a, b, dy, dsT, 0, dS_out, FA + zs, zs,
+    e = launch_dstate<I>(p.rpt, p.lpr, n > 2, heads, T, H, p.t_seg, 1, n - 1, r, w, a, b, dy, dsT, 0, dS_out, FA + zs, zs,
                          n - 1, MT + zs, zs, st);
     if (e != cudaSuccess) return e;
     // pass 2: dL/dS at the end of segments 0..n-2: adj[k] = adj[k+1] M_k^T + F_k
@@ -826,7 +844,7 @@ cudaError_t bwd_dstate_run(int B, int T, int H, const DstatePlan &p, const void 
         entry = ADJ + zs;
     }
     // pass 3: output runs of segments 0..n-2; segment 0 ends with ds0
-    return launch_dstate<I>(p.rpt, false, heads, T, H, p.t_seg, 0, n - 1, r, w, a, b, dy, entry, zs, dS_out, ds0, 0,
+    return launch_dstate<I>(p.rpt, p.lpr, false, heads, T, H, p.t_seg, 0, n - 1, r, w, a, b, dy, entry, zs, dS_out, ds0, 0,
                             1, nullptr, 0, st);
 }
 

@@ -114,6 +114,18 @@ def test_central_differences_slice(cuda_device):
         assert np.max(np.abs(sel - fd)) <= 1e-5 * scale + 1e-7, name
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_mid_head_count_sampled_heads(cuda_device, dtype):
+    """B=4, T=1024, H=32 (128 heads): the state-gradient sweep takes four
+    rows per thread with eight lanes per row; sampled heads vs the oracle,
+    with a dL/dS_T term."""
+    d = _case(4, 1024, 32, 360, dtype)
+    heads = [5, 30]
+    tau = TAU_F32 if dtype == "f32" else TAU_BF16
+    for name, got, ref in zip(GRAD_NAMES, _gpu(d, heads=heads), _ref(d, heads=heads)):
+        assert_close(got, ref, tau, name)
+
+
 def test_training_workload_sampled_heads(cuda_device):
     """B=8, T=4096, H=32 bf16 with dy ~ N(0,1) bf16 and dsT = 0: sampled heads."""
     cfg = inputs.WORKLOADS["train_bwd_b8_t4096_h32"]
