@@ -26,7 +26,9 @@
 //      and dL^T (lanes 64-127, cols 0-63);  dV^T += [dY; dZ]^T [L_rk; L_ak]
 //   E  ZYUV [SG | dS] + [dL; dL^T] [[b-; k-] | [r'; a']] -> [dr'; da'] (lanes
 //      0-63, cols 0-63) and [db'; dk'] (lanes 64-127, cols 64-127); the B
-//      operands are side-by-side copies made after round D
+//      operands are side-by-side copies ([SG | dS] made in P3 by the warps
+//      that idle there, so the first half is issued after round D and runs
+//      under P4)
 // Operands are bf16 hi/lo splits (three passes, two when one side is an exact
 // bf16 input: v, dy), accumulation in fp32 in TMEM.  The CUDA cores prepare
 // the operands, invert the 32 x 32 unit lower triangular I - L_ab by 16 x 16
@@ -36,8 +38,9 @@
 // warp 8 issues the tensor-core rounds; hand-offs through named barriers
 // (ready: compute -> issuer, done: issuer -> compute), every wait of the issuer
 // bounded.  The next chunk's token tiles arrive by cp.async into the raw tile
-// buffer as soon as the current chunk has read it (first phase), and its
-// states are pulled into L2 one chunk ahead.
+// buffer as soon as the current chunk has read it (first phase), its S_in and
+// dS into the [SG; dS] tiles' space once round E is done; its states are
+// pulled into L2 one chunk ahead.
 #include "umma.cuh"
 
 namespace wkv7 {
@@ -74,20 +77,28 @@ constexpr uint32_t LABT = PSM + 33 * LDP * 4;         // fp32 [32][36]: L_ab^T (
 constexpr int LDTS = 33;
 constexpr uint32_t TSM = LABT + 32 * LDT * 4;         // fp32 [32][33]: T
 constexpr uint32_t ZSM = TSM + 32 * LDTS * 4;         // fp32 [16][16]
-// after round D (VYZ, ZDU, LB2, TT are no longer read): round E's side-by-side B operands
-constexpr uint32_t SGDC_HI = VYZ_HI, SGDC_LO = VYZ_LO;  // [64][128]: rows i: [SG | dS]
-constexpr uint32_t X1C_HI = ZDU_HI, X1C_LO = ZDU_HI + 16384;   // [64][128]: rows: [[b-; k-] | [r'; a']]
+// round E's side-by-side B operands: [SG | dS] after round C (ZDU, LB2, TT are
+// no longer read), so that round E's first half can run under P4;
+// [[b-; k-] | [r'; a']] after round D (VYZ is no longer read)
+constexpr uint32_t SGDC_HI = ZDU_HI, SGDC_LO = ZDU_HI + 16384;   // [64][128]: rows i: [SG | dS]
+constexpr uint32_t X1C_HI = VYZ_HI, X1C_LO = VYZ_LO;             // [64][128]: rows: [[b-; k-] | [r'; a']]
 // after round E: fp32 scratch of the q and dw sums
 constexpr int LDQ = 68;
 constexpr uint32_t CQ = VYZ_HI;                       // fp32 [4][32][68]: q terms of dr, da, db, dk
-constexpr uint32_t CPART = CQ + 4 * 32 * LDQ * 4;     // fp32 [8][64]: per-warp sums of S_out dS
-constexpr uint32_t DWTOT = CPART + 8 * 64 * 4;        // fp32 [4][64]: token-block sums of q
+constexpr uint32_t DWTOT = CQ + 4 * 32 * LDQ * 4;     // fp32 [4][64]: token-block sums of q
 constexpr uint32_t GSTG = DWTOT + 4 * 64 * 4;         // the four gradient tiles, rows padded by 16 B (<= 34816 B)
 static_assert(GSTG + 4 * 32 * (64 * 4 + 16) <= RAW, "gradient staging ends before the token tiles");
-constexpr uint32_t BAR = ZSM + 1024;                  // 5 mbarriers (rounds A..E)
-constexpr uint32_t TMEM_SLOT = BAR + 40;
-constexpr uint32_t FLAG = BAR + 44;
-constexpr uint32_t SMEM_BYTES = BAR + 64;
+constexpr uint32_t BAR = ZSM + 1024;                  // 6 mbarriers: rounds A..E, round E's first half
+constexpr uint32_t TMEM_SLOT = BAR + 48;
+constexpr uint32_t FLAG = BAR + 52;
+constexpr uint32_t CPART = BAR + 64;                  // fp32 [8][64]: per-warp sums of S_out dS (P0b -> P5)
+constexpr uint32_t SMEM_BYTES = CPART + 8 * 64 * 4;
+// staged states (fp32, row-major) arriving by cp.async: the chunk's S_in and
+// dS into the [SG; dS] tiles' space during the previous chunk's last phase
+// (round E no longer reads it); S_out, rows 0-31 and 32-63, at the top of the
+// chunk into the halves of VYZ that nothing reads before P3
+constexpr uint32_t ST_SIN = SGD_HI, ST_DS = SGD_LO;
+constexpr uint32_t ST_SOUT0 = VYZ_HI + 8192, ST_SOUT1 = VYZ_LO + 8192;
 
 constexpr uint32_t BAR_READY = 2, BAR_DONE = 7;      // named barriers 2-6, 7-11
 constexpr long long kDrainCycles = 200000000LL;
@@ -181,9 +192,27 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         cp_async_commit();
     };
     // The states a chunk reads (S_in, dS, S_out: 16 KB each) are pulled into
-    // L2 one chunk ahead; the register loads at the top of the chunk then hit L2.
+    // L2 one chunk ahead, then staged in shared memory by cp.async.
     auto s_out_of = [&](int id) {
         return (id % nck) + 1 < nck ? ckpt + (size_t)(id + 1) * kN * kN : sfin + (size_t)(id / nck) * kN * kN;
+    };
+    // S_out of a chunk into ST_SOUT0 / ST_SOUT1 (compute threads, 4 x 16 B each)
+    auto issue_sout = [&](int id) {
+        const float *src = s_out_of(id);
+        for (int x = tid; x < 1024; x += NC)
+            cp_async16(sm + (x < 512 ? ST_SOUT0 : ST_SOUT1) + 16 * (x & 511), src + 4 * x);
+        cp_async_commit();
+    };
+    // S_in and dS of a chunk into ST_SIN / ST_DS (compute threads, 8 x 16 B each)
+    auto issue_states = [&](int id) {
+        if (id < total) {
+            for (int x = tid; x < 2048; x += NC) {
+                const int which = x >> 10, o4 = 4 * (x & 1023);
+                const float *src = (which ? dS_out : ckpt) + (size_t)id * kN * kN + o4;
+                cp_async16(sm + (which ? ST_DS : ST_SIN) + 4 * o4, src);
+            }
+        }
+        cp_async_commit();
     };
     auto prefetch_states = [&](int id) {
         if (id >= total || tid >= 3) return;
@@ -193,12 +222,13 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
 
     // ---- set-up (once per CTA) ------------------------------------------------------------
     if (tid == 0) {
-        for (int rd = 0; rd < 5; ++rd) mbar_init(done_bar(rd), 1);
+        for (int rd = 0; rd < 6; ++rd) mbar_init(done_bar(rd), 1);
         *abort_flag = 0;
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if (tid < NC) {
         issue_tiles(blockIdx.x);
+        issue_states(blockIdx.x);
         prefetch_states(blockIdx.x);
         for (int x = tid; x < 256; x += NC) {          // ZYUV lo rows 0-31 (dY) and 96-127 (V): exact, 4 KB each
             *reinterpret_cast<uint4 *>(sm + ZY_LO + 16 * x) = make_uint4(0, 0, 0, 0);
@@ -232,10 +262,15 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         const OpD sgdc = opd_mn(sbase + SGDC_HI, sbase + SGDC_LO, 128);             // [SG | dS], K = i
         const OpD x1c = opd_mn(sbase + X1C_HI, sbase + X1C_LO, 128);                // [[b-; k-] | [r'; a']], K = s', t'
         // one round: wait for the hand-over, issue, commit, wait for the
-        // commit, release the compute warps; every barrier is passed once
-        // whatever happens, nothing is issued after a wait gave up
+        // commit, release the compute warps, then issue any work that runs on
+        // under the next compute phase (with its own commit, so that a drain
+        // after an abort covers it); every barrier is passed once whatever
+        // happens, nothing is issued after a wait gave up.  Issuing blocks
+        // while the tensor pipe is busy, so the extra work goes in only after
+        // the round's completion has been handed over.
         uint32_t par = 0;                            // phase parity of this chunk's round barriers
-        auto round = [&](int rd, auto &&issue) {
+        auto nothing = [] { return false; };
+        auto round = [&](int rd, auto &&issue, auto &&more) {
             named_sync(BAR_READY + rd, NT);
             fence_after_sync();
             if (lane == 0 && *abort_flag == 0u) {
@@ -248,23 +283,28 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             __syncwarp();
             fence_before_sync();
             named_arrive(BAR_DONE + rd, NT);
+            if (lane == 0 && *abort_flag == 0u && more()) {
+                commit(done_bar(5));
+                last_rd = 5;
+            }
+            __syncwarp();
         };
         for (int id = blockIdx.x, it = 0; id < total; id += gridDim.x, ++it) {
             par = (uint32_t)it & 1u;
-            round(0, [&] { gemm_split_d(tmem + CA, x1, x1, id_a, 4, false); });
+            round(0, [&] { gemm_split_d(tmem + CA, x1, x1, id_a, 4, false); }, nothing);
             round(1, [&] {
                 gemm_split_d(tmem + CB, sgd, x1_abk, id_b1, 4, false);
                 gemm_split_d(tmem + CB, vy, lb2, id_b2, 2, true);
-            });
-            round(2, [&] { gemm_split_d(tmem + CC, tt, zdu, id_c, 2, false); });
+            }, nothing);
+            round(2, [&] { gemm_split_d(tmem + CC, tt, zdu, id_c, 2, false); }, nothing);
             round(3, [&] {
                 gemm_split_d(tmem + CA, zy, zy, id_a, 4, false);
                 gemm_split_d(tmem + CB + 64, vyz, lrk, id_d2, 4, true);
-            });
-            round(4, [&] {
+            }, [&] {                                 // round E's first half, ZYUV [SG | dS], under P4
                 gemm_split_d(tmem + CE, zy, sgdc, id_e, 4, false);
-                gemm_split_ts(tmem + CE, tmem + ADL_HI, tmem + ADL_LO, x1c, id_e, 4, true);
+                return true;
             });
+            round(4, [&] { gemm_split_ts(tmem + CE, tmem + ADL_HI, tmem + ADL_LO, x1c, id_e, 4, true); }, nothing);
         }
         __syncwarp();
     } else {
@@ -296,30 +336,16 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         for (int id = blockIdx.x; id < total; id += gridDim.x) {
             const int Lc = chunk_len(id);
             const size_t base = chunk_base(id);
-            const float *S_out = s_out_of(id);
             csync();                                 // the previous chunk's last reads are done
-            // clear VYZ: rows 32-63 (columns 0-63 are never written, 64-127
-            // take dZ) and the lo copy of rows 0-31 (V, dY are exact)
+            issue_sout(id);
+            // zero the lo copy of dY in VYZ (rows 0-31, columns 64-127; dY is
+            // exact), which round D reads; columns 0-63 of VYZ feed only
+            // accumulator lanes that are never read, and rows 32-63 take dZ
             {
-                for (int x = tid; x < 512; x += NC) {
-                    *reinterpret_cast<uint4 *>(sm + VYZ_HI + 8192 + 16 * x) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(sm + VYZ_LO + 8192 + 16 * x) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(sm + VYZ_LO + 16 * x) = make_uint4(0, 0, 0, 0);
-                }
+                const int t = tid >> 3, ch = tid & 7;
+                *reinterpret_cast<uint4 *>(sm + VYZ_LO + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
             }
-            // S_in and dS rows (from L2): thread -> row tid / 4, columns 16 (tid % 4) ..
-            float4 s_in[4], ds_o[4];
-            {
-                const float *S_in = ckpt + (size_t)id * kN * kN, *dSo = dS_out + (size_t)id * kN * kN;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const size_t x = (size_t)(tid >> 2) * kN + 16 * (tid & 3) + 4 * u;
-                    s_in[u] = __ldcg(reinterpret_cast<const float4 *>(S_in + x));
-                    ds_o[u] = __ldcg(reinterpret_cast<const float4 *>(dSo + x));
-                }
-            }
-            prefetch_states(id + gridDim.x);         // the next chunk's states into L2
-            cp_async_wait<0>();                      // this chunk's token tiles (issued one chunk ago)
+            cp_async_wait<1>();                      // this chunk's token tiles, S_in and dS (not yet S_out)
             csync();
             // ---- P0a: suffix decay products and the decayed operands (warp -> 8
             //      channels, lane -> token) ----
@@ -383,18 +409,44 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             {
                 const int i = tid >> 2, c0 = 16 * (tid & 3);
                 float sg[16], dsv[16];
+                const float *sin_s = reinterpret_cast<const float *>(sm + ST_SIN) + i * kN + c0;
+                const float *ds_s = reinterpret_cast<const float *>(sm + ST_DS) + i * kN + c0;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 s4 = s_in[u], d4 = ds_o[u];
+                    const float4 s4 = *reinterpret_cast<const float4 *>(sin_s + 4 * u);
+                    const float4 d4 = *reinterpret_cast<const float4 *>(ds_s + 4 * u);
                     const int j = c0 + 4 * u;
                     sg[4 * u] = s4.x * psm[j]; sg[4 * u + 1] = s4.y * psm[j + 1];
                     sg[4 * u + 2] = s4.z * psm[j + 2]; sg[4 * u + 3] = s4.w * psm[j + 3];
                     dsv[4 * u] = d4.x; dsv[4 * u + 1] = d4.y; dsv[4 * u + 2] = d4.z; dsv[4 * u + 3] = d4.w;
                 }
+                cp_async_wait<1>();                      // S_out (the next chunk's tiles may still be in flight)
+                csync();                                 // the staged states are read before SGD replaces them
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0, 64), sg);
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0 + 8, 64), sg + 8);
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(64 + i, c0, 64), dsv);
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(64 + i, c0 + 8, 64), dsv + 8);
+                // the chunk's last token also scales S_out: q_{Lc-1} += sum_i S_out dS
+                // (the 8 rows of a warp summed by shuffles, then per-warp partial sums)
+                float cs[16];
+                const float *so = reinterpret_cast<const float *>(sm + (i < 32 ? ST_SOUT0 : ST_SOUT1)) + (i & 31) * kN + c0;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 s4 = *reinterpret_cast<const float4 *>(so + 4 * u);
+                    cs[4 * u] = s4.x * dsv[4 * u]; cs[4 * u + 1] = s4.y * dsv[4 * u + 1];
+                    cs[4 * u + 2] = s4.z * dsv[4 * u + 2]; cs[4 * u + 3] = s4.w * dsv[4 * u + 3];
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 4);
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 8);
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 16);
+                }
+                if (lane < 4) {
+                    float *cp = reinterpret_cast<float *>(sm + CPART) + warp * kN + c0;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) cp[e] = cs[e];
+                }
             }
 
             // ---- P1: Gram rows -> L tiles (lane = row of X X^T) ----
@@ -508,6 +560,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 store8_split(sm + ZDU_HI, sm + ZDU_LO, cm_off(row, 16 * hc + 8, 32), x + 8);
             }
             ready_arrive(2);                             // round C: [T; T^T], [Z^T; dU^T]
+            prefetch_states(id + gridDim.x);             // the next chunk's states into L2, under round C
             // ---- P3: U rows (lanes 0-31), dZ rows (lanes 32-63) -> ZYUV, VYZ ----
             done_wait(2);
             if (q4 < 2) {
@@ -525,21 +578,28 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                         store8_split(sm + VYZ_HI, sm + VYZ_LO, cm_off(32 + t, 64 + 32 * hc + 8 * u, 128), x + 8 * u);
                     }
                 }
+            } else {                                     // the other four warps: [SG | dS] side by side
+                const int u = (2 * hc + q4 - 2) * 32 + lane;   // 0 .. 127; SG rows to columns 0-63, dS to 64-127
+                for (int x = u; x < 2048; x += 128) {
+                    const int blk = x >> 6, hl = (blk >> 4) & 1, G = blk & 15;
+                    const uint32_t src = (hl ? SGD_LO : SGD_HI) + G * 1024;
+                    const uint32_t dst = (hl ? SGDC_LO : SGDC_HI) + ((G & 7) * 16 + (G < 8 ? 0 : 8)) * 128;
+                    *reinterpret_cast<uint4 *>(sm + dst + 16 * (x & 63)) =
+                        *reinterpret_cast<const uint4 *>(sm + src + 16 * (x & 63));
+                }
             }
             ready_arrive(3);                             // round D: ZYUV, VYZ, [L_rk; L_ak]
 
             // ---- P4: dV out; the masked dL block as round E's A operand in TMEM ----
             done_wait(3);
-            // side-by-side copies for round E: [SG | dS] from the SGD rows,
-            // [[b-; k-] | [r'; a']] from the X1 rows.  A group of 8 rows is 1 KB
-            // in both layouts (8 column chunks of 8 rows), so each moves as one
-            // contiguous block; consecutive lanes move consecutive 16 bytes.
-            for (int x = tid; x < 4096; x += NC) {
-                const int blk = x >> 6, tile = blk >> 5, hl = (blk >> 4) & 1, G = blk & 15;
-                const int dbase = (tile == 0) == (G < 8) ? 0 : 8;
-                const uint32_t src = (tile == 0 ? (hl ? SGD_LO : SGD_HI) : (hl ? X1_LO : X1_HI)) + G * 1024;
-                const uint32_t dst = (tile == 0 ? (hl ? SGDC_LO : SGDC_HI) : (hl ? X1C_LO : X1C_HI)) +
-                                     ((G & 7) * 16 + dbase) * 128;
+            // side-by-side copy for round E's second half: [[b-; k-] | [r'; a']]
+            // from the X1 rows.  A group of 8 rows is 1 KB in both layouts (8
+            // column chunks of 8 rows), so each moves as one contiguous block;
+            // consecutive lanes move consecutive 16 bytes.
+            for (int x = tid; x < 2048; x += NC) {
+                const int blk = x >> 6, hl = (blk >> 4) & 1, G = blk & 15;
+                const uint32_t src = (hl ? X1_LO : X1_HI) + G * 1024;
+                const uint32_t dst = (hl ? X1C_LO : X1C_HI) + ((G & 7) * 16 + (G < 8 ? 8 : 0)) * 128;
                 *reinterpret_cast<uint4 *>(sm + dst + 16 * (x & 63)) =
                     *reinterpret_cast<const uint4 *>(sm + src + 16 * (x & 63));
             }
@@ -578,6 +638,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             ready_arrive(4);                             // round E
             // ---- P5: the four gradients, q, dw ----
             done_wait(4);
+            issue_states(id + gridDim.x);                // SGD is no longer read in this chunk
             {
                 const int rrow = lane;                   // token t (q4 0, 1) or s (q4 2, 3)
                 float x[32];
@@ -633,36 +694,6 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
                         store4(o + 4 * u, make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
-                }
-            }
-            {   // the chunk's last token also scales S_out: q_{Lc-1} += sum_i S_out dS
-                // (thread -> row tid / 4, columns 16 (tid % 4) ..; the 8 rows of a
-                // warp summed by shuffles, then per-warp partial sums)
-                const int i = tid >> 2, c0 = 16 * (tid & 3);
-                float cs[16];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 so = __ldcg(reinterpret_cast<const float4 *>(S_out + (size_t)i * kN + c0 + 4 * u));
-                    float dsv[4];                        // dS row i from SGD (hi + lo)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t off = cm_off(64 + i, c0 + 4 * u + e, 64);
-                        dsv[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + SGD_HI + off)) +
-                                 __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + SGD_LO + off));
-                    }
-                    cs[4 * u] = so.x * dsv[0]; cs[4 * u + 1] = so.y * dsv[1];
-                    cs[4 * u + 2] = so.z * dsv[2]; cs[4 * u + 3] = so.w * dsv[3];
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 4);
-                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 8);
-                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 16);
-                }
-                if (lane < 4) {
-                    float *cp = reinterpret_cast<float *>(sm + CPART) + warp * kN + c0;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) cp[e] = cs[e];
                 }
             }
             csync();
