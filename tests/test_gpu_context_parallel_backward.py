@@ -192,3 +192,32 @@ def test_backward_orchestration_over_a_one_rank_nccl_group(cuda_device):
             assert_close(to_f64(got[j]), to_f64(ref[j]), TAU_BF16, name)
     finally:
         dist.destroy_process_group()
+
+
+def test_long_context_backward_over_eight_stretches(cuda_device):
+    """B=1, T=65536, H=32, w near 1 (the long-context workload's inputs), split
+    over 8 stretches of 8192 tokens (one per GPU of a node), with dy ~ N(0,1)
+    and a dL/dS_T term: sampled heads vs the oracle's backward over the whole
+    sequence, every head vs one wkv7.backward (which itself runs the
+    segmented checkpoint pass and sweep)."""
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    B, T, H, N = cfg["B"], cfg["T"], cfg["H"], cfg["N"]
+    d = inputs.gen_sequence(B, T, H, N, seed=cfg["seed"], dtype="bf16", x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
+    d["dy"] = inputs.gen_dy(B, T, H, N, seed=cfg["seed"], dtype="bf16")
+    d["dsT"] = (inputs.gen_normal(B * H * N, N, seed=cfg["seed"], stream=inputs.STREAM_DST, std=0.1)
+                .reshape(B, H, N, N))
+    grads, adj, _ = _stretches_backward_on_one_gpu(d, 8)
+    assert wkv7.device_status() == wkv7.OK
+    heads = [7, 26]
+    raw = [d[n][:, :, heads] for n in inputs.INPUT_NAMES]
+    ref = oracle.backward(*map(inputs.to_f64, raw), d["s0"][:, heads].astype(np.float64),
+                          inputs.to_f64(d["dy"][:, :, heads]), d["dsT"][:, heads].astype(np.float64))
+    for j, name in enumerate(GRADS):
+        assert_close(to_f64(grads[j][:, :, heads]), ref[j], TAU_BF16, f"{name} vs oracle")
+    assert_close(to_f64(adj[0][:, heads]), ref[6], TAU_BF16, "ds0 vs oracle")
+    whole = wkv7.backward(*_dev_args(d), to_dev(d["s0"]), to_dev(d["dy"]), to_dev(d["dsT"]))
+    torch.cuda.synchronize()
+    for j, name in enumerate(GRADS):
+        for h in range(H):
+            assert_close(to_f64(grads[j][:, :, h]), to_f64(whole[j][:, :, h]), TAU_BF16, f"{name} head {h} vs whole")
+    assert_close(to_f64(adj[0]), to_f64(whole[6]), TAU_BF16, "ds0 vs whole")
