@@ -111,12 +111,13 @@ def test_compose_adjoints_matches_oracle(cuda_device, nseg, with_dsT):
         assert_close(to_f64(adj[kk]), ref[kk], TAU_F32, f"adj[{kk}]")
 
 
-def _stretches_backward_on_one_gpu(d, world):
-    """Every rank's forward and backward steps in turn on this GPU."""
+def _stretches_backward_on_one_gpu(d, world, lens=None):
+    """Every rank's forward and backward steps in turn on this GPU (stretch
+    lengths from split_lengths, or as given)."""
     args = _dev_args(d)
     dy, dsT = to_dev(d["dy"]), to_dev(d["dsT"])
     T = args[0].shape[1]
-    bounds = np.cumsum([0] + split_lengths(T, world))
+    bounds = np.cumsum([0] + (lens if lens is not None else split_lengths(T, world)))
     cut = lambda x, i: x[:, bounds[i]:bounds[i + 1]].contiguous()
     parts = [[cut(x, i) for x in args] for i in range(world)]
     sums = torch.stack([wkv7.forward_summary(*p) for p in parts])
@@ -149,6 +150,24 @@ def test_stretch_backwards_match_whole_sequence(cuda_device, T, world):
     for j, name in enumerate(GRADS):
         assert_close(to_f64(grads[j]), to_f64(whole[j]), TAU_BF16, f"{name} vs whole")
     for i in range(world):
+        assert_close(to_f64(ds_ins[i]), to_f64(adj[i]), TAU_BF16, f"stretch {i} ds_in vs adj")
+
+
+def test_stretches_of_any_length(cuda_device):
+    """Stretch boundaries off the 32-token chunk grid, a one-token stretch and
+    an empty one: the composed forward and backward still equal the oracle's
+    over the whole sequence."""
+    lens = [333, 1, 0, 500, 77]
+    T = sum(lens)
+    d = _case(1, T, 2, 985, "bf16")
+    grads, adj, ds_ins = _stretches_backward_on_one_gpu(d, len(lens), lens)
+    assert wkv7.device_status() == wkv7.OK
+    ref = oracle.backward(*_f64(d), d["s0"].astype(np.float64), inputs.to_f64(d["dy"]),
+                          d["dsT"].astype(np.float64))
+    for j, name in enumerate(GRADS):
+        assert_close(to_f64(grads[j]), ref[j], TAU_BF16, name)
+    assert_close(to_f64(adj[0]), ref[6], TAU_BF16, "ds0")
+    for i in range(len(lens)):
         assert_close(to_f64(ds_ins[i]), to_f64(adj[i]), TAU_BF16, f"stretch {i} ds_in vs adj")
 
 
