@@ -38,9 +38,10 @@
 // warp 8 issues the tensor-core rounds; hand-offs through named barriers
 // (ready: compute -> issuer, done: issuer -> compute), every wait of the issuer
 // bounded.  The next chunk's token tiles arrive by cp.async into the raw tile
-// buffer as soon as the current chunk has read it (first phase), its S_in and
-// dS into the [SG; dS] tiles' space once round E is done; its states are
-// pulled into L2 one chunk ahead.
+// buffer (read only in the first phase), issued while the compute warps wait
+// for round C; its S_in and dS into the [SG; dS] tiles' space (last read in
+// P3), issued while they wait for round D; its states are pulled into L2 one
+// chunk ahead.
 #include "umma.cuh"
 
 namespace wkv7 {
@@ -94,8 +95,8 @@ constexpr uint32_t FLAG = BAR + 52;
 constexpr uint32_t CPART = BAR + 64;                  // fp32 [8][64]: per-warp sums of S_out dS (P0b -> P5)
 constexpr uint32_t SMEM_BYTES = CPART + 8 * 64 * 4;
 // staged states (fp32, row-major) arriving by cp.async: the chunk's S_in and
-// dS into the [SG; dS] tiles' space during the previous chunk's last phase
-// (round E no longer reads it); S_out, rows 0-31 and 32-63, at the top of the
+// dS into the [SG; dS] tiles' space, issued under the previous chunk's round
+// D (P3 was its last reader); S_out, rows 0-31 and 32-63, at the top of the
 // chunk into the halves of VYZ that nothing reads before P3
 constexpr uint32_t ST_SIN = SGD_HI, ST_DS = SGD_LO;
 constexpr uint32_t ST_SOUT0 = VYZ_HI + 8192, ST_SOUT1 = VYZ_LO + 8192;
@@ -163,8 +164,8 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
     };
 
     // The token tiles of a chunk (r w k v a b dy) go to RAW by cp.async one
-    // chunk ahead, as soon as the current chunk's tiles have been read (RAW
-    // is read only at the start of a chunk); thread -> (token tid / 8,
+    // chunk ahead, once the current chunk's tiles have been read (RAW is read
+    // only at the start of a chunk); thread -> (token tid / 8,
     // channels 8 (tid % 8) ..).  Rows past the end are no-op tokens (w = 1,
     // the rest 0), written directly.
     auto issue_tiles = [&](int id) {
@@ -403,7 +404,6 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             }
             ready_arrive(0);                                     // round A: X1
             csync();                                             // p_t visible; RAW no longer read
-            issue_tiles(id + gridDim.x);                         // the next chunk's token tiles
             // ---- P0b: SG = S_in diag(G) (rows 0-63) and dS (rows 64-127); thread ->
             //      row tid / 4, columns 16 (tid % 4) .. ----
             {
@@ -420,7 +420,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     sg[4 * u + 2] = s4.z * psm[j + 2]; sg[4 * u + 3] = s4.w * psm[j + 3];
                     dsv[4 * u] = d4.x; dsv[4 * u + 1] = d4.y; dsv[4 * u + 2] = d4.z; dsv[4 * u + 3] = d4.w;
                 }
-                cp_async_wait<1>();                      // S_out (the next chunk's tiles may still be in flight)
+                cp_async_wait<0>();                      // S_out
                 csync();                                 // the staged states are read before SGD replaces them
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0, 64), sg);
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0 + 8, 64), sg + 8);
@@ -560,6 +560,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 store8_split(sm + ZDU_HI, sm + ZDU_LO, cm_off(row, 16 * hc + 8, 32), x + 8);
             }
             ready_arrive(2);                             // round C: [T; T^T], [Z^T; dU^T]
+            issue_tiles(id + gridDim.x);                 // the next chunk's token tiles, while round C runs
             prefetch_states(id + gridDim.x);             // the next chunk's states into L2, under round C
             // ---- P3: U rows (lanes 0-31), dZ rows (lanes 32-63) -> ZYUV, VYZ ----
             done_wait(2);
@@ -589,6 +590,8 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 }
             }
             ready_arrive(3);                             // round D: ZYUV, VYZ, [L_rk; L_ak]
+            csync();                                     // every warp's P3 reads of SGD are done
+            issue_states(id + gridDim.x);                // S_in, dS of the next chunk, under round D
 
             // ---- P4: dV out; the masked dL block as round E's A operand in TMEM ----
             done_wait(3);
@@ -638,7 +641,6 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             ready_arrive(4);                             // round E
             // ---- P5: the four gradients, q, dw ----
             done_wait(4);
-            issue_states(id + gridDim.x);                // SGD is no longer read in this chunk
             {
                 const int rrow = lane;                   // token t (q4 0, 1) or s (q4 2, 3)
                 float x[32];
