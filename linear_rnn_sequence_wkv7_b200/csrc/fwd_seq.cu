@@ -11,35 +11,59 @@
 // j = 16 m + 4 q + e (m, e in 0..3) of each of its rows in registers, so the
 // two dot products per token are 16-term in-thread sums plus two xor-shuffle
 // steps, and the update is 3 FP32 instructions per element.  The token
-// vectors are streamed through shared memory in tiles of TT tokens with
-// double-buffered cp.async (16-byte, L2-only) and converted to fp32 once per
-// CTA; every lane reads them as broadcast float4s (the interleaved column
-// assignment keeps the 4 lanes of a row group on distinct banks).
+// vectors are streamed through shared memory in double-buffered tiles of TT
+// tokens: with TMA, one thread issues a tile load per tensor ([TT tokens] x
+// [64 channels] of the (b, h) slice, rows past T filled with zeros), each
+// stage completing on its own mbarrier; otherwise every thread issues 16-byte
+// cp.async copies.  bf16 tiles are converted to fp32 once per CTA, and every
+// lane reads them as broadcast float4s (the interleaved column assignment
+// keeps the 4 lanes of a row group on distinct banks).
 //
 // CKPT mode writes the state before every CK-th token to a checkpoint buffer
 // (the backward's first pass, without y; the training forward, with y).
-#include "common.cuh"
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "umma.cuh"
 
 namespace wkv7 {
 
-template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT>
+// TMA descriptors of the six token tensors r w k v a b, each seen as a 3D
+// array {x: H * 64 channels, y: T tokens, z: B}
+struct SeqMaps {
+    CUtensorMap m[6];
+};
+
+__device__ __forceinline__ void seq_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// one box of a 3D tensor map into shared memory (no multicast), completing
+// on the mbarrier at `bar`
+__device__ __forceinline__ void seq_tma_load(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT, bool TMA>
 __global__ void __launch_bounds__((RB / RPT) * 4)
-fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ w,
-               const InT *__restrict__ k, const InT *__restrict__ v, const InT *__restrict__ a,
-               const InT *__restrict__ b, const float *s0, OutT *__restrict__ y, float *sT,
-               float *__restrict__ ckpt, int CK) {
+fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__restrict__ r,
+               const InT *__restrict__ w, const InT *__restrict__ k, const InT *__restrict__ v,
+               const InT *__restrict__ a, const InT *__restrict__ b, const float *s0, OutT *__restrict__ y,
+               float *sT, float *__restrict__ ckpt, int CK, long long wait_limit) {
     constexpr int NT = (RB / RPT) * 4;
     constexpr int NTEN = 6;                          // r w k v a b
-    constexpr int VEC = 16 / sizeof(InT);            // elements per 16-byte chunk
-    constexpr int CHUNKS_PER_VEC = kN / VEC;         // 16-byte chunks per N-vector
-    constexpr int CHUNKS_PER_TILE = TT * NTEN * CHUNKS_PER_VEC;
+    constexpr uint32_t TILE_BYTES = TT * kN * sizeof(InT);        // one tensor's tile
     constexpr bool kConvert = !std::is_same<InT, float>::value;
 
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     InT *raw = reinterpret_cast<InT *>(smem_raw);                 // [2][NTEN][TT][kN]
-    float *f32buf = kConvert ? reinterpret_cast<float *>(smem_raw + 2 * NTEN * TT * kN * sizeof(InT))
+    float *f32buf = kConvert ? reinterpret_cast<float *>(smem_raw + 2 * NTEN * TILE_BYTES)
                              : nullptr;                           // [NTEN][TT][kN]
-
+    const uint32_t bar0 = smem_u32(smem_raw + 2 * NTEN * TILE_BYTES +
+                                   (kConvert ? NTEN * TT * kN * sizeof(float) : 0));   // 2 mbarriers
     const int tid = threadIdx.x;
     const int q = tid & 3;
     const int rg = tid >> 2;
@@ -51,7 +75,12 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
     const size_t base = ((size_t)bb * T * H + h) * kN;            // (bb, t=0, h, 0)
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
 
-    const InT *src[NTEN] = {r, w, k, v, a, b};
+    if (tid == 0) {
+        umma::mbar_init(bar0, 1);
+        umma::mbar_init(bar0 + 8, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
 
     float S[RPT][16];
 #pragma unroll
@@ -67,26 +96,47 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
         }
 
     const int ntiles = (T + TT - 1) / TT;
+    // tile `tile` into stage `stage` (thread 0): the six tensors' boxes at
+    // x = 64 h (128-byte aligned), y = first token, z = b
+    const InT *src[NTEN] = {r, w, k, v, a, b};
     auto issue_tile = [&](int tile, int stage) {
-        const int t0 = tile * TT;
-        for (int c = tid; c < CHUNKS_PER_TILE; c += NT) {
-            const int ten = c / (TT * CHUNKS_PER_VEC);
-            const int rem = c % (TT * CHUNKS_PER_VEC);
-            const int tt = rem / CHUNKS_PER_VEC;
-            const int ch = rem % CHUNKS_PER_VEC;
-            if (t0 + tt < T) {
-                InT *dst = raw + (((size_t)stage * NTEN + ten) * TT + tt) * kN + ch * VEC;
-                cp_async16(dst, src[ten] + base + (size_t)(t0 + tt) * tok_stride + ch * VEC);
+        if constexpr (TMA) {
+            if (tid != 0) return;
+            const uint32_t bar = bar0 + 8u * (uint32_t)stage;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the stage's last generic reads
+            seq_expect_tx(bar, NTEN * TILE_BYTES);
+#pragma unroll
+            for (int ten = 0; ten < NTEN; ++ten)
+                seq_tma_load(smem_u32(raw + ((size_t)stage * NTEN + ten) * TT * kN), &maps.m[ten], h * kN, tile * TT,
+                             bb, bar);
+        } else {
+            constexpr int VEC = 16 / sizeof(InT), CPV = kN / VEC;       // 16-byte chunks per N-vector
+            const int t0 = tile * TT;
+            for (int c = tid; c < TT * NTEN * CPV; c += NT) {
+                const int ten = c / (TT * CPV), rem = c % (TT * CPV), tt = rem / CPV, ch = rem % CPV;
+                if (t0 + tt < T)
+                    cp_async16(raw + (((size_t)stage * NTEN + ten) * TT + tt) * kN + ch * VEC,
+                               src[ten] + base + (size_t)(t0 + tt) * tok_stride + ch * VEC);
             }
+            cp_async_commit();
         }
-        cp_async_commit();
     };
 
+    bool timed_out = false;
     if (ntiles > 0) issue_tile(0, 0);
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it & 1;
         const int t0 = it * TT;
-        cp_async_wait<0>();
+        // the tile's bytes have landed: with TMA phase it / 2 of its stage's
+        // mbarrier (bounded; polled with test_wait), else this thread's copies
+        if constexpr (TMA) {
+            if (!umma::mbar_spin(bar0 + 8u * (uint32_t)stage, (uint32_t)(it >> 1) & 1u, wait_limit)) {
+                if (!timed_out) raise_status(WKV7_ERR_TIMEOUT);
+                timed_out = true;
+            }
+        } else {
+            cp_async_wait<0>();
+        }
         __syncthreads();
         const float *buf;
         if constexpr (kConvert) {
@@ -182,6 +232,10 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
         }
     }
 
+    if (timed_out && tid == 0 && ntiles > 0) {   // let a late tile land before the CTA exits
+        umma::mbar_wait(bar0 + 8u * (uint32_t)((ntiles - 1) & 1), (uint32_t)((ntiles - 1) >> 1) & 1u, 200000000LL);
+        if (ntiles > 1) umma::mbar_wait(bar0 + 8u * (uint32_t)(ntiles & 1), (uint32_t)((ntiles - 2) >> 1) & 1u, 200000000LL);
+    }
     if (sT) {
         // Every CTA read its own rows of s0 before its first tile, so writing
         // sT here is safe even when sT aliases s0.
@@ -194,47 +248,93 @@ fwd_seq_kernel(int T, int H, const InT *__restrict__ r, const InT *__restrict__ 
     }
 }
 
-template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT = !CKPT>
+// cuTensorMapEncodeTiled, looked up in the driver once (no link-time
+// dependency on the driver library)
+static PFN_cuTensorMapEncodeTiled_v12000 seq_encode_fn() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// The six token tensors [B, T, H, 64] as 3D maps {H * 64, T, B} with boxes of
+// {64, TT, 1}: a (b, h) slice of TT tokens, rows past T read as zeros.  Base
+// addresses are 16-byte aligned (the API checks every pointer) and the row
+// strides are multiples of 128 bytes.
+template <typename InT, int TT>
+static cudaError_t seq_maps(int B, int T, int H, const void *const src[6], SeqMaps &maps) {
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = seq_encode_fn();
+    if (!encode) return cudaErrorNotSupported;
+    const CUtensorMapDataType dt =
+        std::is_same<InT, float>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[3] = {(cuuint64_t)H * kN, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)H * kN * sizeof(InT), (cuuint64_t)T * H * kN * sizeof(InT)};
+    const cuuint32_t box[3] = {(cuuint32_t)kN, (cuuint32_t)TT, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    for (int x = 0; x < 6; ++x) {
+        const CUresult res = encode(&maps.m[x], dt, 3, const_cast<void *>(src[x]), dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (res != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
+template <typename InT, typename OutT, int RPT, int RB, int TT, bool CKPT, bool YOUT, bool TMA>
 static cudaError_t launch_fwd_seq(int B, int T, int H, const void *r, const void *w, const void *k,
                                   const void *v, const void *a, const void *b, const float *s0, void *y,
-                                  float *sT, float *ckpt, int CK, cudaStream_t st) {
+                                  float *sT, float *ckpt, int CK, long long wait_limit, cudaStream_t st) {
     constexpr int NT = (RB / RPT) * 4;
     size_t smem = 2 * 6 * TT * kN * sizeof(InT);
     if (!std::is_same<InT, float>::value) smem += 6 * TT * kN * sizeof(float);
-    auto kern = fwd_seq_kernel<InT, OutT, RPT, RB, TT, CKPT, YOUT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    smem += 16;                                      // two mbarriers
+    SeqMaps maps{};
+    const void *src[6] = {r, w, k, v, a, b};
+    cudaError_t e = TMA ? seq_maps<InT, TT>(B, T, H, src, maps) : cudaSuccess;
+    if (e != cudaSuccess) return e;
+    auto kern = fwd_seq_kernel<InT, OutT, RPT, RB, TT, CKPT, YOUT, TMA>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(H * (kN / RB), B);
-    kern<<<grid, NT, smem, st>>>(T, H, (const InT *)r, (const InT *)w, (const InT *)k, (const InT *)v,
-                                 (const InT *)a, (const InT *)b, s0, (OutT *)y, sT, ckpt, CK);
+    kern<<<grid, NT, smem, st>>>(T, H, maps, (const InT *)r, (const InT *)w, (const InT *)k, (const InT *)v,
+                                 (const InT *)a, (const InT *)b, s0, (OutT *)y, sT, ckpt, CK, wait_limit);
     return cudaGetLastError();
 }
 
 // Layout of the scan: with more heads than SMs, one CTA per head with four
-// rows per thread and 32-token tiles (fewer loads and conversions of the token
-// vectors per row: 1.89 vs 2.29 ms at B=8, T=4096, H=32, bf16); otherwise two
-// CTAs per head with two rows per thread, which keeps more SMs busy (1.69 vs
-// 1.85 ms at B=2).
+// rows per thread and 32-token tiles loaded by TMA (fewer loads and
+// conversions of the token vectors per row: 1.87 vs 2.29 ms at B=8, T=4096,
+// H=32, bf16, of which TMA instead of cp.async 0.013 ms); otherwise two CTAs
+// per head with two rows per thread and 16-token tiles by cp.async, which
+// keeps more SMs busy (1.69 vs 1.85 ms at B=2; TMA tiles measured 1.89 ms
+// there).
 template <typename InT, typename OutT, bool CKPT, bool YOUT = !CKPT>
 static cudaError_t dispatch_fwd_seq(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
                                     const void *a, const void *b, const float *s0, void *y, float *sT, float *ckpt,
-                                    int CK, cudaStream_t st) {
+                                    int CK, long long lim, cudaStream_t st) {
     if ((long long)B * H > 148 && (!CKPT || CK % 32 == 0))   // checkpoints fall on tile starts
-        return launch_fwd_seq<InT, OutT, 4, 64, 32, CKPT, YOUT>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
-    return launch_fwd_seq<InT, OutT, 2, 32, 16, CKPT, YOUT>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
+        return launch_fwd_seq<InT, OutT, 4, 64, 32, CKPT, YOUT, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK,
+                                                                      lim, st);
+    return launch_fwd_seq<InT, OutT, 2, 32, 16, CKPT, YOUT, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, lim,
+                                                                   st);
 }
 
 // Host entry used by the API layer.
 cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
                     const void *w, const void *k, const void *v, const void *a, const void *b,
-                    const float *s0, void *y, float *sT, cudaStream_t st) {
+                    const float *s0, void *y, float *sT, long long lim, cudaStream_t st) {
     if (in_dt == WKV7_F32 && y_dt == WKV7_F32)
-        return dispatch_fwd_seq<float, float, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+        return dispatch_fwd_seq<float, float, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, lim, st);
     if (in_dt == WKV7_F32 && y_dt == WKV7_BF16)
-        return dispatch_fwd_seq<float, __nv_bfloat16, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+        return dispatch_fwd_seq<float, __nv_bfloat16, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, lim, st);
     if (in_dt == WKV7_BF16 && y_dt == WKV7_F32)
-        return dispatch_fwd_seq<__nv_bfloat16, float, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
-    return dispatch_fwd_seq<__nv_bfloat16, __nv_bfloat16, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, st);
+        return dispatch_fwd_seq<__nv_bfloat16, float, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, lim, st);
+    return dispatch_fwd_seq<__nv_bfloat16, __nv_bfloat16, false>(B, T, H, r, w, k, v, a, b, s0, y, sT, nullptr, 0, lim, st);
 }
 
 // State checkpoints every CK tokens (CK a multiple of 16; they are written at
@@ -243,25 +343,25 @@ cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, cons
 // the state before token c * CK.  Used by the backward's first pass.
 cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
                             const void *k, const void *v, const void *a, const void *b, const float *s0,
-                            float *ckpt, int CK, float *sT, cudaStream_t st) {
+                            float *ckpt, int CK, float *sT, long long lim, cudaStream_t st) {
     if (in_dt == WKV7_F32)
-        return dispatch_fwd_seq<float, float, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
-    return dispatch_fwd_seq<__nv_bfloat16, float, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, st);
+        return dispatch_fwd_seq<float, float, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, lim, st);
+    return dispatch_fwd_seq<__nv_bfloat16, float, true>(B, T, H, r, w, k, v, a, b, s0, nullptr, sT, ckpt, CK, lim, st);
 }
 
 // The forward with y and the state checkpoints every CK tokens (the training
 // forward: the backward then skips its own checkpoint pass).
 cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                           const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
-                          float *sT, float *ckpt, int CK, cudaStream_t st) {
+                          float *sT, float *ckpt, int CK, long long lim, cudaStream_t st) {
     if (in_dt == WKV7_F32 && y_dt == WKV7_F32)
-        return dispatch_fwd_seq<float, float, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
+        return dispatch_fwd_seq<float, float, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, lim, st);
     if (in_dt == WKV7_F32 && y_dt == WKV7_BF16)
-        return dispatch_fwd_seq<float, __nv_bfloat16, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
+        return dispatch_fwd_seq<float, __nv_bfloat16, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, lim, st);
     if (in_dt == WKV7_BF16 && y_dt == WKV7_F32)
-        return dispatch_fwd_seq<__nv_bfloat16, float, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, st);
+        return dispatch_fwd_seq<__nv_bfloat16, float, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK, lim, st);
     return dispatch_fwd_seq<__nv_bfloat16, __nv_bfloat16, true, true>(B, T, H, r, w, k, v, a, b, s0, y, sT, ckpt, CK,
-                                                                       st);
+                                                                       lim, st);
 }
 
 }  // namespace wkv7

@@ -13,10 +13,10 @@ namespace wkv7 {
 
 cudaError_t fwd_seq(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
                     const void *w, const void *k, const void *v, const void *a, const void *b,
-                    const float *s0, void *y, float *sT, cudaStream_t st);
+                    const float *s0, void *y, float *sT, long long wait_limit, cudaStream_t st);
 cudaError_t fwd_checkpoints(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w,
                             const void *k, const void *v, const void *a, const void *b, const float *s0,
-                            float *ckpt, int CK, float *sT, cudaStream_t st);
+                            float *ckpt, int CK, float *sT, long long wait_limit, cudaStream_t st);
 cudaError_t step(int B, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                  const void *k, const void *v, const void *a, const void *b, float *state, void *y,
                  cudaStream_t st);
@@ -37,7 +37,7 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt);
 cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                           const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
-                          float *sT, float *ckpt, int CK, cudaStream_t st);
+                          float *sT, float *ckpt, int CK, long long wait_limit, cudaStream_t st);
 int chunk_segments(int B, int T, int H, int sm_count, bool summarize_last);
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg);
 cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w, const void *k, const void *v,
@@ -189,8 +189,10 @@ wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
         return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
                                    lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt));
     }
-    if (ckpt) return from_cuda(fwd_seq_train(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, ckpt, kBwdChunk, stream));
-    return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, stream));
+    const long long lim = g_wait_limit.load() > 0 ? g_wait_limit.load() : kDefaultWaitCycles;
+    if (ckpt)
+        return from_cuda(fwd_seq_train(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, ckpt, kBwdChunk, lim, stream));
+    return from_cuda(fwd_seq(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, lim, stream));
 }
 
 }  // namespace
@@ -369,7 +371,8 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
         e = fwd_chunk(B, T, H, WKV7_BF16, r, w, k, v, a, b, s0, nullptr, sfin, nseg, scratch,
                       lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt);
     } else {
-        e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin, stream);
+        e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin,
+                            lim > 0 ? lim : kDefaultWaitCycles, stream);
     }
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
