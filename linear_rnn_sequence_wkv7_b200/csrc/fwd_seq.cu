@@ -75,12 +75,14 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
     const size_t base = ((size_t)bb * T * H + h) * kN;            // (bb, t=0, h, 0)
     const size_t st_base = ((size_t)bb * H + h) * kN * kN;
 
-    if (tid == 0) {
-        umma::mbar_init(bar0, 1);
-        umma::mbar_init(bar0 + 8, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if constexpr (TMA) {                                          // one mbarrier per tile stage
+        if (tid == 0) {
+            umma::mbar_init(bar0, 1);
+            umma::mbar_init(bar0 + 8, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncthreads();
     }
-    __syncthreads();
 
     float S[RPT][16];
 #pragma unroll
@@ -96,8 +98,9 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
         }
 
     const int ntiles = (T + TT - 1) / TT;
-    // tile `tile` into stage `stage` (thread 0): the six tensors' boxes at
-    // x = 64 h (128-byte aligned), y = first token, z = b
+    // tile `tile` into stage `stage`: with TMA, thread 0 loads the six
+    // tensors' boxes at x = 64 h (128-byte aligned), y = first token, z = b;
+    // else all threads copy the tile's rows that lie before T
     const InT *src[NTEN] = {r, w, k, v, a, b};
     auto issue_tile = [&](int tile, int stage) {
         if constexpr (TMA) {
