@@ -295,7 +295,7 @@ def bench_forward(args, dist, peaks, device):
                 "peak_source": peaks["source"], "per_unit": "896 B per head-token + 32 KiB state per head",
                 "units_per_launch": head_tokens,
                 "tensor_tflops": fwd_chunk_flops(B, T, H) / per_launch / 1e12}
-    src = {"fwd_seq": ("fwd_seq.cu", "common.cuh"), "fwd_chunk": ("fwd_chunk.cu", "umma.cuh", "common.cuh")}[kernel]
+    src = {"fwd_seq": ("fwd_seq.cu", "umma.cuh", "common.cuh"), "fwd_chunk": ("fwd_chunk.cu", "umma.cuh", "common.cuh")}[kernel]
     roof["traffic"] = recorded_traffic(kernel, source_hash(*src))
     roof["kernel"] = kernel
     roof["hbm_frac"] = nbytes / per_launch / 1e9 / peaks["hbm_gbs"]
