@@ -125,22 +125,27 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
         }
     };
 
-    bool timed_out = false;
     if (ntiles > 0) issue_tile(0, 0);
     for (int it = 0; it < ntiles; ++it) {
         const int stage = it & 1;
         const int t0 = it * TT;
         // the tile's bytes have landed: with TMA phase it / 2 of its stage's
         // mbarrier (bounded; polled with test_wait), else this thread's copies
-        if constexpr (TMA) {
-            if (!umma::mbar_spin(bar0 + 8u * (uint32_t)stage, (uint32_t)(it >> 1) & 1u, wait_limit)) {
-                if (!timed_out) raise_status(WKV7_ERR_TIMEOUT);
-                timed_out = true;
-            }
-        } else {
+        bool late = false;
+        if constexpr (TMA)
+            late = !umma::mbar_spin(bar0 + 8u * (uint32_t)stage, (uint32_t)(it >> 1) & 1u, wait_limit);
+        else
             cp_async_wait<0>();
+        if (__syncthreads_or(late)) {
+            // a tile did not arrive within the limit: report it, give the one
+            // copy in flight (this tile's; the next is not issued yet) a
+            // bounded time to land, and stop without writing y or sT
+            if (tid == 0) {
+                raise_status(WKV7_ERR_TIMEOUT);
+                umma::mbar_wait(bar0 + 8u * (uint32_t)stage, (uint32_t)(it >> 1) & 1u, 200000000LL);
+            }
+            return;
         }
-        __syncthreads();
         const float *buf;
         if constexpr (kConvert) {
             const InT *rs = raw + (size_t)stage * NTEN * TT * kN;
@@ -235,10 +240,6 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
         }
     }
 
-    if (timed_out && tid == 0 && ntiles > 0) {   // let a late tile land before the CTA exits
-        umma::mbar_wait(bar0 + 8u * (uint32_t)((ntiles - 1) & 1), (uint32_t)((ntiles - 1) >> 1) & 1u, 200000000LL);
-        if (ntiles > 1) umma::mbar_wait(bar0 + 8u * (uint32_t)(ntiles & 1), (uint32_t)((ntiles - 2) >> 1) & 1u, 200000000LL);
-    }
     if (sT) {
         // Every CTA read its own rows of s0 before its first tile, so writing
         // sT here is safe even when sT aliases s0.

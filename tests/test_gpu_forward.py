@@ -226,6 +226,31 @@ def test_chunked_wait_timeout_reports_and_recovers(cuda_device):
     assert_close(to_f64(sT), sr, TAU_BF16, "sT after recovery")
 
 
+def test_scan_tile_wait_timeout_reports_and_recovers(cuda_device):
+    """The sequential scan's wait for its TMA tile (the one-CTA-per-head
+    layout: more heads than SMs) with the limit forced to 1 cycle: every CTA
+    gives up on its first tile, lets that copy land and stops; the status word
+    reads WKV7_ERR_TIMEOUT, nothing faults, and the next launch with the
+    default limit is correct (sampled heads vs the oracle)."""
+    B, T, H, N = 5, 40, 32, 64                   # 160 heads
+    d = inputs.gen_sequence(B, T, H, N, seed=78, dtype="bf16", s0_std=0.1)
+    assert wkv7.device_status() == wkv7.OK
+    wkv7.set_wait_limit(1)
+    try:
+        run_forward(d, y_dtype=torch.float32, algo="seq")
+        status = wkv7.device_status()
+    finally:
+        wkv7.set_wait_limit(0)
+    assert status == wkv7.ERR_TIMEOUT
+    y, sT = run_forward(d, y_dtype=torch.float32, algo="seq")
+    assert wkv7.device_status() == wkv7.OK
+    heads = [0, 31]
+    raw = [d[n][:, :, heads] for n in inputs.INPUT_NAMES]
+    yr, sr = oracle.forward(*map(inputs.to_f64, raw), s0=d["s0"][:, heads].astype(np.float64))
+    assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y after recovery")
+    assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT after recovery")
+
+
 # --- chunked form over sequence segments (few heads, long sequences) -----------------
 
 @pytest.mark.parametrize("T", [512, 700, 2000, 4097])
