@@ -175,3 +175,20 @@ def test_split_lengths(T, world):
         assert nonempty == list(range(len(nonempty)))
         full = [n // 32 for n in lens[:-1]] + [-(-lens[-1] // 32)]
         assert max(full) - min(full) <= 1 or T < 32 * world
+
+
+def test_single_process_backward_is_plain_backward():
+    """Without a process group the backward orchestration is one stretch: its
+    gradients and ds0 are the oracle backward's; summaries for another world
+    size are rejected."""
+    args, s0 = _sequence(21, 6)
+    dy, dsT = _dy(21, 7)
+    ops = oracle_ops()
+    t = [torch.from_numpy(x) for x in args]
+    _, s_in, _, sums = forward_context_parallel(*t, torch.from_numpy(s0), ops=ops, return_summaries=True)
+    got = backward_context_parallel(*t, s_in, sums, torch.from_numpy(dy), torch.from_numpy(dsT), ops=ops)
+    ref = oracle.backward(*args, s0, dy, dsT)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g.numpy(), r, rtol=0, atol=1e-10 * max(1.0, np.abs(r).max()))
+    with pytest.raises(ValueError):
+        backward_context_parallel(*t, s_in, torch.cat([sums, sums]), torch.from_numpy(dy), ops=ops)
