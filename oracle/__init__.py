@@ -41,6 +41,10 @@ section "Summary").
   by token (the adjoint of S_t = S_{t-1} A_t + v_t k_t^T, y_t = S_t r_t, taken
   for S only): G <- G + dy_t r_t^T, then G <- G A_t^T.  ``compose_adjoints``
   chains those maps over stretches, last stretch first.
+* ``timemix_out`` / ``forward_timemix``: the output epilogue of the time-mix
+  block (the current-token term, the per-head normalisation and the gate; Paper
+  Review, section "The approach").  The pages describe it in words only, so it
+  is our plainest reading of them, written out token by token.
 """
 from __future__ import annotations
 
@@ -350,3 +354,44 @@ def compose_adjoints(summaries, F, dsT=None):
     for kk in range(nseg - 1, -1, -1):
         adj[kk] = adj[kk + 1] @ np.swapaxes(summaries[kk, 1], -1, -2) + F[kk]
     return adj
+
+
+def timemix_out(y, r, k, v, rho, gamma=None, beta=None, g=None, eps=1e-5):
+    """Output epilogue of the time-mix block, fp64, for per-token tensors
+    [B,T,H,N] and per-head parameters [H,N].  Paper Review: RWKV-7 "Goose"
+    with Expressive Dynamic State Evolution, section "The approach": after the
+    state update the receptance reads the state (y_t = S_t r_t, from
+    ``forward``); the block also attends to the current token directly,
+    without that token being stored in the state; the result is normalised,
+    the heads are combined, gated, and a linear layer follows.  The pages give
+    no formula; this is the plainest reading of those words:
+
+        o_t   = y_t + (sum_j r_t[j] rho[j] k_t[j]) v_t     (current-token term)
+        mu_t  = mean_i o_t[i],  var_t = mean_i (o_t[i] - mu_t)^2   (per head)
+        z_t   = g_t * (gamma * (o_t - mu_t) / sqrt(var_t + eps) + beta)
+
+    The heads are combined by concatenation (the [B,T,H,N] layout already is
+    it); the gate g arrives as values (its projection, like the final linear
+    layer, needs trained weights).  gamma / beta / g default to 1 / 0 / 1."""
+    y, r, k, v = (_f64(x) for x in (y, r, k, v))
+    B, T, H, N = y.shape
+    rho = _f64(rho)
+    gamma = np.ones((H, N)) if gamma is None else _f64(gamma)
+    beta = np.zeros((H, N)) if beta is None else _f64(beta)
+    g = np.ones((B, T, H, N)) if g is None else _f64(g)
+    z = np.empty((B, T, H, N))
+    for bb in range(B):
+        for t in range(T):
+            for h in range(H):
+                bonus = float(np.sum(r[bb, t, h] * rho[h] * k[bb, t, h]))
+                o = y[bb, t, h] + bonus * v[bb, t, h]
+                mu = float(np.sum(o)) / N
+                var = float(np.sum((o - mu) ** 2)) / N
+                z[bb, t, h] = g[bb, t, h] * (gamma[h] * (o - mu) / np.sqrt(var + eps) + beta[h])
+    return z
+
+
+def forward_timemix(r, w, k, v, a, b, s0, rho, gamma=None, beta=None, g=None, eps=1e-5):
+    """(z, sT): ``forward`` followed by ``timemix_out`` on its y."""
+    y, sT = forward(r, w, k, v, a, b, s0=s0)
+    return timemix_out(y, r, k, v, rho, gamma, beta, g, eps), sT
