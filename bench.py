@@ -45,8 +45,10 @@ N = 64
 FWD = inputs.WORKLOADS["prefill_b8_t4096_h32_bf16"]
 BWD = inputs.WORKLOADS["train_bwd_b8_t4096_h32"]
 DEC = inputs.WORKLOADS["decode_b256_h40_x1000"]
-LONG = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+LONG = inputs.WORKLOADS["long_b1_t65536_h32_chunk32"]
 SM_COUNT = 148
+TC_OPERANDS = ("bf16 hi/lo split (3 passes; 2 where one side is an exact bf16 input), fp32 accumulate "
+               "in TMEM; state fp32")
 FP32_LANES_PER_SM = 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
 
@@ -215,12 +217,23 @@ def to_pinned(x):
     return t.pin_memory()
 
 
-def timed(fn, steps, warmup, dist, stream):
+def require_ok_status(what, stream):
+    """The library's device status word must read OK after a timed part: a
+    bounded wait that ran out or a chunk outside the chunked form's range
+    leaves outputs unspecified, so such a run is no measurement."""
+    from linear_rnn_sequence_wkv7_b200 import wkv7
+    st = wkv7.last_status(stream)
+    if st != wkv7.OK:
+        raise RuntimeError(f"{what}: device status {wkv7.status_string(st)} ({st}) after the timed run")
+
+
+def timed(fn, steps, warmup, dist, stream, what="timed run"):
     """Device time of `steps` calls of fn (CUDA events on `stream`), max over ranks."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
+    require_ok_status(what + " (warm-up)", stream)
     dist.barrier()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -230,7 +243,9 @@ def timed(fn, steps, warmup, dist, stream):
     end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
-    return dist.max(start.elapsed_time(end) / 1e3)
+    elapsed = start.elapsed_time(end) / 1e3
+    require_ok_status(what, stream)
+    return dist.max(elapsed)
 
 
 def bench_forward(args, dist, peaks, device):
@@ -254,7 +269,7 @@ def bench_forward(args, dist, peaks, device):
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     with sampler:
-        secs = timed(step, args.steps, args.warmup, dist, stream)
+        secs = timed(step, args.steps, args.warmup, dist, stream, "prefill forward")
     clocks = sampler.summary()
 
     # end to end through the host-buffer entry point: pinned host inputs in,
@@ -274,7 +289,7 @@ def bench_forward(args, dist, peaks, device):
                           stream=stream)
 
     e2e_steps = max(3, min(args.steps, 20))
-    e2e_secs = timed(e2e_step, e2e_steps, 2, dist, stream)
+    e2e_secs = timed(e2e_step, e2e_steps, 2, dist, stream, "prefill forward from host buffers")
     h2d = sum(t.numel() * t.element_size() for t in host_in) + host_s0.numel() * 4
     d2h = host_y.numel() * 2 + host_sT.numel() * 4
 
@@ -328,19 +343,24 @@ def bench_backward(args, dist, peaks, device, d):
         wkv7.backward(*dev, s0, dy, None, grad_dtype=torch.bfloat16, workspace=ws, out=out, stream=stream)
 
     steps = max(3, min(args.steps // 20, 10))
-    secs = timed(step, steps, 2, dist, stream)
+    secs = timed(step, steps, 2, dist, stream, "training backward")
     per = secs / steps
     pk = fp32_peak_tflops(peaks["sm_max_mhz"])
-    ach = bwd_flops(B, T, H) / per / 1e12
+    ach_flops = bwd_flops(B, T, H) / per / 1e12
+    nbytes = bwd_bytes(B, T, H)
+    ach = nbytes / per / 1e9
     return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
             "ms_per_step": per * 1e3,
             "steps": steps, "launches": 3 * steps,
-            "roofline": {"bound": "alu", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                         "per_unit": "28*N^2 flop per head-token (the fp32 algebra of the chunked adjoint)",
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                         "per_unit": "1664 B per head-token (6 inputs + dy read, 6 bf16 gradients written) "
+                                     "+ 32 KiB state per head", "bytes_per_launch": nbytes,
                          "kernels": "checkpoints (chunked forward), dS chain, per-chunk gradients "
                                     "(tcgen05, bf16 hi/lo operands, fp32 accumulation)",
-                         "tensor_frac": ach / peaks["bf16_tflops"],
-                         "hbm_frac": bwd_bytes(B, T, H) / per / 1e9 / peaks["hbm_gbs"]},
+                         "fp32_alu": {"achieved": ach_flops, "peak": pk, "unit": "TFLOP/s", "frac": ach_flops / pk,
+                                      "per_unit": "28*N^2 flop per head-token (the sequential scan's algebra)"},
+                         "tensor_frac": ach_flops / peaks["bf16_tflops"]},
             "config": {"workload": "train_bwd_b8_t4096_h32", "B": B, "T": T, "H": H, "N": N,
                        "grad_dtype": "bf16", "dsT": "zero"}}
 
@@ -375,8 +395,8 @@ def bench_train(args, dist, peaks, device, d):
         wkv7.backward(*dev, s0, dy, None, grad_dtype=torch.bfloat16, workspace=ws_full, out=grads, stream=stream)
 
     steps = max(3, min(args.steps // 20, 10))
-    per = timed(step, steps, 2, dist, stream) / steps
-    per_sep = timed(step_separate, steps, 2, dist, stream) / steps
+    per = timed(step, steps, 2, dist, stream, "training step") / steps
+    per_sep = timed(step_separate, steps, 2, dist, stream, "forward + backward") / steps
     return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
             "ms_per_step": per * 1e3, "steps": steps, "launches": 4 * steps,
             "separate_ms_per_step": per_sep * 1e3,
@@ -398,7 +418,7 @@ def bench_decode(args, dist, peaks, device, steps_in):
     g = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap):
+    with torch.cuda.stream(cap), wkv7.status_checks(False):     # no synchronizing check inside a capture
         for s in range(2):   # warm the launch path outside the capture
             wkv7.step(*(dev[nm][s] for nm in inputs.INPUT_NAMES), state, y=y[s], stream=cap)
         torch.cuda.synchronize()
@@ -407,7 +427,7 @@ def bench_decode(args, dist, peaks, device, steps_in):
                 wkv7.step(*(dev[nm][s] for nm in inputs.INPUT_NAMES), state, y=y[s], stream=cap)
     torch.cuda.synchronize()
     reps = 3
-    secs = timed(g.replay, reps, 1, dist, torch.cuda.current_stream())
+    secs = timed(g.replay, reps, 1, dist, torch.cuda.current_stream(), "decode steps")
     per_step = secs / (reps * n)
     nbytes = step_bytes(B, H)
     ach = nbytes / per_step / 1e9
@@ -443,7 +463,7 @@ def bench_long(args, dist, peaks, device):
         wkv7.forward(*dev, s0=s0, y=y, sT=sT, algo="chunk", workspace=ws, stream=stream)
 
     steps = max(3, min(args.steps // 20, 10))
-    secs = timed(step, steps, 2, dist, stream)
+    secs = timed(step, steps, 2, dist, stream, "long-context forward")
     per = secs / steps
     nbytes = fwd_bytes(B, T, H)
     ach = nbytes / per / 1e9
@@ -455,7 +475,9 @@ def bench_long(args, dist, peaks, device):
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "per_unit": "896 B per head-token + 32 KiB state per head",
                          "units_per_launch": B * T * H},
-            "config": {"workload": "long_b1_t65536_h32", "B": B, "T": T, "H": H, "N": N, "algo": "chunk",
+            "config": {"workload": "long_b1_t65536_h32_chunk32", "B": B, "T": T, "H": H, "N": N, "algo": "chunk",
+                       "chunk_len": cfg["chunk_len"],
+                       "tc_operands": TC_OPERANDS,
                        "w": "exp(-0.6065 sigmoid(x)), x ~ N(-2, 1)",
                        "l2": "no flush: each step reads 1.6 GB of inputs (> 126 MB L2)"}}
 
@@ -533,6 +555,7 @@ def run_ours(args):
         "config": {"workload": "prefill_b8_t4096_h32_bf16", "B": FWD["B"], "T": FWD["T"], "H": FWD["H"],
                    "N": N, "io_dtype": "bf16", "state_dtype": "f32", "algo": args.algo,
                    "kernel": fwd["roofline"]["kernel"],
+                   "tc_operands": TC_OPERANDS if fwd["roofline"]["kernel"] == "fwd_chunk" else None,
                    "l2": "no flush: each step reads 805 MB of inputs (> 126 MB L2)",
                    "parallelism": f"dp{dist.world} (independent batches per GPU)"},
         "roofline": fwd["roofline"],

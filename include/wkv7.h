@@ -27,7 +27,7 @@
  *    [B, H, N]; states (s0, sT, dsT, ds0, state) are [B, H, N, N] fp32 with
  *    element S[b][h][i][j] (i = value row, j = key column).
  *  - Calls are asynchronous on `stream`; they never synchronize (except
- *    wkv7_get_device_status).  Launch errors are reported as WKV7_ERR_CUDA.
+ *    wkv7_get_last_status).  Launch errors are reported as WKV7_ERR_CUDA.
  *  - Arguments are validated on the host before any launch; an invalid
  *    argument returns WKV7_ERR_INVALID_ARG (N other than 64 returns
  *    WKV7_ERR_UNSUPPORTED) and launches nothing.
@@ -81,7 +81,11 @@ WKV7_API const char *wkv7_status_string(wkv7_status status);
 
 /*
  * Bytes of scratch wkv7_forward can use for these arguments on the current
- * device (0 when the chosen algorithm needs none).  The chunked form uses it to
+ * device (0 when the chosen algorithm needs none).  The split it pays for
+ * rests on the state update being affine in S: the transition is a diagonal
+ * plus a rank-one term built from the token's own inputs (Paper Review:
+ * RWKV-7 "Goose", section "Architecture"), so a stretch of tokens maps its
+ * entry state S to S M + E.  The chunked form uses it to
  * split long sequences into segments that run in parallel when B*H heads are
  * too few to fill the GPU (a per-segment summary S -> S M + E, a scan of the
  * entry states, then every segment from its entry state).  Without it (NULL
@@ -99,13 +103,17 @@ WKV7_API size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dty
  *   sT               : [B, H, N, N] fp32 final state, or NULL to skip.
  *                      sT may alias s0 (in-place continuation); no other
  *                      output may alias an input.
- *   algo, chunk_len  : algorithm choice; chunk_len 0 means 32 (the only
- *                      length the chunked form implements).
+ *   algo, chunk_len  : algorithm choice; chunk_len 0 means 32, the only
+ *                      length the chunked form implements (any other value
+ *                      returns WKV7_ERR_UNSUPPORTED; the result of the
+ *                      recurrence does not depend on the chunk length).
  *   workspace        : wkv7_forward_workspace_size() bytes, or NULL if 0.
  * The chunked form needs the per-chunk decay product of every channel to stay
  * in fp32's normal range (prod of 32 consecutive w >= 1e-30); a chunk outside
- * it raises WKV7_ERR_RANGE in the device status word (wkv7_get_device_status)
- * and its outputs are unspecified.  The SEQ form has no such limit.
+ * it raises WKV7_ERR_RANGE in the device status word (read it with
+ * wkv7_get_last_status) and its outputs are unspecified.  The SEQ form has no
+ * such limit: callers whose decays can be that strong poll the status word
+ * or choose WKV7_ALGO_SEQ.
  */
 WKV7_API wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
                          const void *r, const void *w, const void *k, const void *v,
@@ -262,6 +270,41 @@ WKV7_API wkv7_status wkv7_forward_host(int B, int T, int H, int N, wkv7_dtype in
 WKV7_API int wkv7_forward_resolve_algo(int T, wkv7_dtype in_dtype, wkv7_algo algo);
 
 /*
+ * Forward with the time-mix block's output epilogue.  The pages describe it in
+ * words (Paper Review: RWKV-7 "Goose" with Expressive Dynamic State Evolution,
+ * section "The approach"): after the state update the receptance reads the
+ * state; the block also attends to the current token directly, without that
+ * token being stored in the state; the result is normalised per head, the
+ * heads are combined, and a gate is applied (the linear layer that follows
+ * needs trained weights and is not part of this call).  Our reading of those
+ * words, per (b, t, h):
+ *     o_t = S_t r_t + (sum_j r_t[j] rho[h][j] k_t[j]) v_t
+ *     z_t[i] = g_t[i] * (gamma[h][i] (o_t[i] - mean(o_t)) / sqrt(var(o_t) + eps) + beta[h][i])
+ * with the mean and the population variance over the head's N channels.
+ *   r..b, s0, sT, algo, chunk_len : as wkv7_forward (sT is the plain
+ *                      recurrence's final state: the current-token term never
+ *                      enters the state)
+ *   rho              : [H, N] fp32 current-token weight (required; zeros give
+ *                      the normalised readout)
+ *   gamma, beta      : [H, N] fp32, or NULL for 1 and 0
+ *   g                : [B, T, H, N] of in_dtype gate values, or NULL for 1
+ *   eps              : >= 0, added to the variance
+ *   z                : [B, T, H, N] of out_dtype, written
+ *   workspace        : wkv7_forward_timemix_workspace_size() bytes.  The
+ *                      chunked form applies the epilogue inside its kernel
+ *                      (same scratch as wkv7_forward); the sequential scan
+ *                      writes an fp32 y there and maps it to z in a second pass.
+ */
+WKV7_API size_t wkv7_forward_timemix_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dtype,
+                                                    wkv7_algo algo, int chunk_len);
+WKV7_API wkv7_status wkv7_forward_timemix(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype out_dtype,
+                                          const void *r, const void *w, const void *k, const void *v,
+                                          const void *a, const void *b, const float *s0, const float *rho,
+                                          const float *gamma, const float *beta, const void *g, float eps,
+                                          void *z, float *sT, wkv7_algo algo, int chunk_len, void *workspace,
+                                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * One decode token (T = 1) for every (b, h), updating the state IN PLACE
  * (constant memory and time per token: RWKV-7 "Goose" abstract).
  *   r, w, k, v, a, b : [B, H, N] of in_dtype
@@ -276,12 +319,19 @@ WKV7_API wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dtype, wkv7_dt
  * 32-token chunk, dL/dS at the end of every chunk, and the final state
  * (fp32, 16 KiB each); for few heads over many tokens also 3 states per
  * segment of the state-gradient sweep (see below).  Depends on the current
- * device's SM count. */
+ * device's SM count.  The checkpoints are what lets the backward run its
+ * chunks in parallel instead of token by token: the method is presented as
+ * keeping training parallelisable (RWKV-7 "Goose" with Expressive Dynamic
+ * State Evolution, abstract). */
 WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
 
 /*
  * Backward: gradients of L = sum(dy * y) + sum(dsT * sT) with respect to every
- * input and the initial state.  Three steps: state checkpoints every 32
+ * input and the initial state, i.e. the training pass of the recurrence above.
+ * The pages give no gradient formula; they say the formulation keeps training
+ * parallelisable (RWKV-7 "Goose" with Expressive Dynamic State Evolution,
+ * abstract), and this call is the reverse-mode derivative of the recurrence
+ * taken chunk by chunk.  Three steps: state checkpoints every 32
  * tokens, a reverse sweep of the state gradient that records dL/dS at every
  * chunk end (and ds0), then the input gradients of every chunk independently
  * (the adjoint of the chunked form of the recurrence): on the tensor cores
@@ -382,8 +432,17 @@ WKV7_API void wkv7_set_wait_limit(long long cycles);
 /*
  * Synchronizes `stream`, then returns and clears the sticky device-side status
  * word of the current device (WKV7_OK, WKV7_ERR_TIMEOUT or WKV7_ERR_RANGE), or
- * WKV7_ERR_CUDA if the synchronization itself failed.
+ * WKV7_ERR_CUDA if the synchronization itself failed.  Kernels cannot return
+ * a status to the host, so conditions found on the device (a bounded wait
+ * that ran out; a chunk whose decay product leaves the chunked form's range,
+ * which matters because the recurrence is sensitive to numerical precision:
+ * Elamur Research summary of RWKV-7 "Goose", section "Limitations") are
+ * recorded in this word until read.  A caller of the chunked form that wants
+ * to know its outputs are valid calls this after the work it cares about.
  */
+WKV7_API wkv7_status wkv7_get_last_status(cudaStream_t stream);
+
+/* The same call as wkv7_get_last_status, under its earlier name. */
 WKV7_API wkv7_status wkv7_get_device_status(cudaStream_t stream);
 
 #ifdef __cplusplus

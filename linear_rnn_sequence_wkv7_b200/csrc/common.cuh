@@ -19,6 +19,25 @@ __device__ int g_device_status = 0;
 
 __device__ __forceinline__ void raise_status(int code) { atomicMax(&g_device_status, code); }
 
+// Optional output epilogue of the time-mix block (Paper Review: RWKV-7
+// "Goose", section "The approach": the receptance reads the state, the block
+// also attends to the current token without storing it, and the output is
+// normalised per head and gated).  With rho set, y_t is replaced by
+//     o_t = S_t r_t + (sum_j r_t[j] rho[j] k_t[j]) v_t
+//     z_t = g_t * (gamma * (o_t - mean(o_t)) / sqrt(var(o_t) + eps) + beta)
+// (mean and population variance over the head's N channels; gamma, beta, g
+// default to 1, 0, 1).  The chunked kernel applies it in place of its y
+// store and adds the current-token term to the diagonal of the chunk's L_rk
+// (token t's own write already reaches y_t through r_t . k_t, so the term only
+// reweights it): it never enters the state.  The sequential path runs it as a
+// separate pass over an fp32 y.
+struct EpiArgs {
+    const float *rho;             // [H][64] or null: no epilogue, plain y
+    const float *gamma, *beta;    // [H][64] or null
+    const void *g;                // [B][T][H][64] of the input dtype, or null
+    float eps;
+};
+
 // ---- element load / store ---------------------------------------------------
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -96,6 +96,12 @@ constexpr uint32_t GAML = RZ_LO + 3072;             // fp32 [64]: G per channel
 constexpr uint32_t BAR = GAML + 256;                // 4 mbarriers: tcgen05.commit of R1..R4
 constexpr uint32_t TMEM_SLOT = BAR + 64;
 constexpr uint32_t FLAG = BAR + 68;                 // set by whichever role gives up first
+// time-mix epilogue (EpiArgs): per-warp parts of the current-token weight
+// u_t = sum_j r_t[j] rho[j] k_t[j], fp32 [32 t][8 warps]; and the two rounds of
+// the per-head mean / variance exchange between the two halves of a y row
+constexpr uint32_t UPART = RZ_LO + 5120;
+constexpr uint32_t EXCH = RZ_LO + 7168;             // fp32 [2 rounds][2 halves][32 rows]
+constexpr uint32_t BAR_EPI = 10;                    // named barrier of warps 2 and 6 (the y rows)
 
 constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
 constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (prod of 32 w)
@@ -119,19 +125,21 @@ constexpr uint32_t BAR_READY = 2, BAR_DONE = 6;
 
 }  // namespace chunk
 
+
 // DUAL: a summary run that carries two states through the same chunk algebra,
 // S from S_in (here 0, giving the segment's E) and S2 from I (giving M): the
 // chunk's operands, T, W', M and Q do not depend on the state, so only the
 // state round R4 and its read-out are done twice.  No y.  It needs a second S
 // operand and 64 more TMEM columns, so these CTAs run one per SM.
-template <typename OutT, bool DUAL>
+// EPI: the time-mix output epilogue (EpiArgs) replaces the y store.
+template <typename OutT, bool DUAL, bool EPI>
 __global__ void __launch_bounds__(chunk::NT, DUAL ? 1 : 2)
 fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *__restrict__ r,
                  const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
                  float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt,
-                 float *m_out, long long m_zstride, int seg0, int first_out) {
+                 float *m_out, long long m_zstride, int seg0, int first_out, EpiArgs epi) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -355,6 +363,15 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 xb[e] = bv[e] * nxt;
                 xk[e] = kv[e] * nxt;
             }
+            if constexpr (EPI) {                  // part of u_t over this warp's 8 channels
+                const float4 *rp = reinterpret_cast<const float4 *>(epi.rho + (size_t)h * kN + 8 * g);
+                const float4 q0 = rp[0], q1 = rp[1];
+                const float rr[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                float part = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) part = fmaf(rv[e] * rr[e], kv[e], part);
+                reinterpret_cast<float *>(sm + UPART)[t * 8 + g] = part;
+            }
             store8_split(sm + AV_HI, sm + AV_LO, cm_off(t, 8 * g, 128), xa);
             store8_split(sm + AV_HI, sm + AV_LO, cm_off(L + t, 8 * g, 128), xr);     // RZ rows
             store8_split(sm + BB_HI, sm + BB_LO, cm_off(t, 8 * g, 96), xb);
@@ -392,11 +409,18 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
                         for (int t = 0; t < L; ++t) dst[t * 33] = t > s ? g[t] : 0.f;
                     } else {                          // column s of L_rb / L_rk -> columns 64.. of row s / 32+s
+                        float u = 0.f;            // epilogue: u_s on the diagonal of L_rk
+                        if (EPI && row >= L) {
+                            const float4 *up = reinterpret_cast<const float4 *>(sm + UPART) + 2 * s;
+                            const float4 u0 = up[0], u1 = up[1];
+                            u = ((u0.x + u0.y) + (u0.z + u0.w)) + ((u1.x + u1.y) + (u1.z + u1.w));
+                        }
 #pragma unroll
                         for (int qq = 0; qq < 4; ++qq) {
                             float x[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] = (8 * qq + e >= s) ? g[8 * qq + e] : 0.f;
+                            for (int e = 0; e < 8; ++e)
+                                x[e] = (8 * qq + e >= s) ? g[8 * qq + e] + (8 * qq + e == s ? u : 0.f) : 0.f;
                             store8_split(sm + BB_HI, sm + BB_LO, cm_off(row, 64 + 8 * qq, 96), x);
                         }
                     }
@@ -604,6 +628,44 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                         for (int e = 0; e < 32; ++e) mp[(size_t)(32 * hc + e) * kN + rho] = x[e];
                     }
                 }
+            } else if (EPI && yo) {               // epilogue: z row t from o row t (halves in warps 2, 6)
+                const int t = rho - 64;
+                float *ex = reinterpret_cast<float *>(sm + EXCH);
+                float s1 = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s1 += x[e];
+                ex[32 * hc + lane] = s1;
+                named_sync(BAR_EPI, 64);
+                const float mu = (s1 + ex[32 * (1 - hc) + lane]) * (1.f / kN);
+                float s2 = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s2 = fmaf(x[e] - mu, x[e] - mu, s2);
+                ex[64 + 32 * hc + lane] = s2;
+                named_sync(BAR_EPI, 64);
+                const float inv = rsqrtf((s2 + ex[64 + 32 * (1 - hc) + lane]) * (1.f / kN) + epi.eps);
+                if (t < Lv) {
+                    const size_t off = base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+                    OutT *dst = yo + off;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {  // 8 channels at a time
+                        float gv[8], gm[8], bt[8];
+                        if (epi.g)
+                            bf8_to_f32(*reinterpret_cast<const uint4 *>(
+                                           static_cast<const __nv_bfloat16 *>(epi.g) + off + 8 * u), gv);
+                        else for (int e = 0; e < 8; ++e) gv[e] = 1.f;
+                        const size_t po = (size_t)h * kN + 32 * hc + 8 * u;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            gm[e] = epi.gamma ? epi.gamma[po + e] : 1.f;
+                            bt[e] = epi.beta ? epi.beta[po + e] : 0.f;
+                        }
+                        float zz[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) zz[e] = fmaf((x[8 * u + e] - mu) * inv, gm[e], bt[e]) * gv[e];
+                        store4(dst + 8 * u, make_float4(zz[0], zz[1], zz[2], zz[3]));
+                        store4(dst + 8 * u + 4, make_float4(zz[4], zz[5], zz[6], zz[7]));
+                    }
+                }
             } else if (yo) {                      // y row t, channels 32 hc .. 32 hc + 31
                 const int t = rho - 64;
                 if (t < Lv) {
@@ -668,22 +730,27 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
                                 const void *w, const void *k, const void *v, const void *a, const void *b,
                                 const float *s0, long long s0_zstride, void *y, float *sT, long long sT_zstride,
                                 int st_only_z, long long wait_limit, cudaStream_t st, float *ckpt = nullptr,
-                                int seg0 = 0) {
+                                int seg0 = 0, EpiArgs epi = EpiArgs{}) {
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES;
-#define WKV7_CHUNK_LAUNCH(O)                                                                                  \
+#define WKV7_CHUNK_LAUNCH(O, E)                                                                               \
     do {                                                                                                      \
-        auto kern = fwd_chunk_kernel<O, false>;                                                               \
+        auto kern = fwd_chunk_kernel<O, false, E>;                                                            \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
         if (e != cudaSuccess) return e;                                                                       \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
                                             (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0,  \
-                                            seg0, 0);                                                         \
+                                            seg0, 0, epi);                                                    \
     } while (0)
-    if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float);
-    else WKV7_CHUNK_LAUNCH(__nv_bfloat16);
+    if (epi.rho) {
+        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, true);
+        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, true);
+    } else {
+        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, false);
+        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, false);
+    }
 #undef WKV7_CHUNK_LAUNCH
     return cudaGetLastError();
 }
@@ -696,23 +763,29 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
                                const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
                                float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st,
                                void *y = nullptr, wkv7_dtype y_dt = WKV7_F32, const float *s0 = nullptr,
-                               float *ckpt = nullptr) {
+                               float *ckpt = nullptr, EpiArgs epi = EpiArgs{}) {
     static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES_DUAL;
     const int first_out = (y != nullptr || ckpt != nullptr) ? 1 : 0;
     using bf = __nv_bfloat16;
-#define WKV7_DUAL_LAUNCH(O)                                                                                    \
+#define WKV7_DUAL_LAUNCH(O, E)                                                                                 \
     do {                                                                                                       \
-        auto kern = fwd_chunk_kernel<O, true>;                                                                 \
+        auto kern = fwd_chunk_kernel<O, true, E>;                                                              \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
         if (e != cudaSuccess) return e;                                                                        \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k,      \
                                             (const bf *)v, (const bf *)a, (const bf *)b, s0, 0, (O *)y, e_out, \
-                                            e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out);  \
+                                            e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out,   \
+                                            epi);                                                              \
     } while (0)
-    if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf);
-    else WKV7_DUAL_LAUNCH(float);
+    if (epi.rho && first_out) {
+        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, true);
+        else WKV7_DUAL_LAUNCH(float, true);
+    } else {
+        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, false);
+        else WKV7_DUAL_LAUNCH(float, false);
+    }
 #undef WKV7_DUAL_LAUNCH
     return cudaGetLastError();
 }
@@ -918,13 +991,16 @@ cudaError_t compose_states(int B, int H, int nseg, const float *s0, const float 
 
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt) {
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
+                      const EpiArgs &epi) {
     if (nseg <= 1)
-        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt);
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt, 0,
+                            epi);
     int t_seg;
     seg_split(T, nseg, t_seg, nseg);
     if (nseg <= 1)
-        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt);
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt, 0,
+                            epi);
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
     float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg - 1][B][H][64][64]
@@ -932,14 +1008,14 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
     // from s0 and writes its y (and checkpoints): its E is the entry state of
     // segment 1.  Segments k >= 1 give E_k (from 0) and M_k (from I, v = 0).
     cudaError_t e = launch_dual(B, T, H, t_seg, nseg - 1, r, w, k, v, a, b, em, zst, em + (size_t)(nseg - 1) * zst,
-                                zst, wait_limit, st, y, y_dt, s0, ckpt);
+                                zst, wait_limit, st, y, y_dt, s0, ckpt, epi);
     if (e != cudaSuccess) return e;
     // pass 2: entry states of segments 1..nseg-1, from segment 1's
     e = launch_combine(B, H, nseg - 2, em, false, em + zst, zst, em + (size_t)nseg * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
     // pass 3: segments 1..nseg-1 from their true entry states; the last one writes sT
     return launch_chunk(B, T, H, t_seg, nseg - 1, nseg - 1, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 2,
-                        wait_limit, st, ckpt, 1);
+                        wait_limit, st, ckpt, 1, epi);
 }
 
 }  // namespace wkv7

@@ -9,3 +9,4 @@
 #include "fwd_chunk.cu"
 #include "bwd_noalloc.cu"
 #include "fwd_host.cu"
+#include "timemix.cu"

@@ -1,7 +1,7 @@
 // extern "C" entry points of libwkv7.so: argument validation, workspace
 // layout and kernel dispatch.  Every check happens on the host before any
 // launch; nothing here allocates device memory or synchronizes (except
-// wkv7_get_device_status).
+// wkv7_get_last_status / wkv7_get_device_status).
 #include <stdint.h>
 
 #include <algorithm>
@@ -34,7 +34,8 @@ cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const flo
                              float *adj, cudaStream_t st);
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
-                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt);
+                      int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
+                      const EpiArgs &epi = EpiArgs{});
 cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                           const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
                           float *sT, float *ckpt, int CK, long long wait_limit, cudaStream_t st);
@@ -158,11 +159,13 @@ namespace wkv7 {
 namespace {
 
 // wkv7_forward, and with ckpt non-null the training forward that also keeps
-// the state before every 32-token chunk
+// the state before every 32-token chunk; with epi.rho set (the chunked form
+// only) the time-mix output epilogue replaces y
 wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
                          const void *w, const void *k, const void *v, const void *a, const void *b,
                          const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len, void *workspace,
-                         size_t workspace_bytes, cudaStream_t stream, float *ckpt) {
+                         size_t workspace_bytes, cudaStream_t stream, float *ckpt,
+                         const EpiArgs &epi = EpiArgs{}) {
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
@@ -187,8 +190,9 @@ wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
                 nseg = want;
         }
         return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
-                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt));
+                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, epi));
     }
+    if (epi.rho) return WKV7_ERR_UNSUPPORTED;      // the scan's epilogue is a separate pass (timemix.cu)
     const long long lim = g_wait_limit.load() > 0 ? g_wait_limit.load() : kDefaultWaitCycles;
     if (ckpt)
         return from_cuda(fwd_seq_train(B, T, H, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, ckpt, kBwdChunk, lim, stream));
@@ -412,12 +416,14 @@ wkv7_status wkv7_compose_adjoints(int nseg, int B, int H, int N, const float *ds
 
 void wkv7_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }
 
-wkv7_status wkv7_get_device_status(cudaStream_t stream) {
+wkv7_status wkv7_get_last_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV7_ERR_CUDA;
     int h = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
     if (h != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
     return static_cast<wkv7_status>(h);
 }
+
+wkv7_status wkv7_get_device_status(cudaStream_t stream) { return wkv7_get_last_status(stream); }
 
 }  // extern "C"

@@ -37,6 +37,7 @@ BLOCK_VECS = 16384
 
 STREAM_R, STREAM_W, STREAM_K, STREAM_V, STREAM_KHAT, STREAM_LR = 1, 2, 3, 4, 5, 6
 STREAM_S0, STREAM_DY, STREAM_DST = 7, 8, 9
+STREAM_GATE, STREAM_PARAMS = 10, 11
 
 INPUT_NAMES = ("r", "w", "k", "v", "a", "b")
 
@@ -99,27 +100,41 @@ def gen_vectors(nvec: int, N: int, *, seed: int, dtype: str = "bf16",
 
     Returns a dict of arrays shaped [nvec, N] (uint16 bf16 bits or float32).
     """
+    return gen_vectors_range(0, nvec, N, seed=seed, dtype=dtype, x_mean=x_mean, threads=threads)
+
+
+def gen_vectors_range(first: int, stop: int, N: int, *, seed: int, dtype: str = "bf16",
+                      x_mean: float = 0.0, threads: int | None = None) -> dict:
+    """Vectors ``first`` .. ``stop - 1`` of the flat stream that ``gen_vectors``
+    draws (the same values, regenerating only the blocks that hold them)."""
+    nvec = stop - first
     out = {name: _empty(nvec, N, dtype) for name in INPUT_NAMES}
+    c0 = first // BLOCK_VECS
+    c1 = (stop + BLOCK_VECS - 1) // BLOCK_VECS
+    blocks = [(c, max(first, c * BLOCK_VECS), min(stop, (c + 1) * BLOCK_VECS)) for c in range(c0, c1)]
 
     def block(blk):
-        c, lo, hi = blk
-        n = hi - lo
+        c, lo_abs, hi_abs = blk
+        off = lo_abs - c * BLOCK_VECS      # the block's leading vectors are drawn and dropped
+        n = hi_abs - c * BLOCK_VECS        # draws up to the last vector needed
+        lo, hi = lo_abs - first, hi_abs - first
         buf = np.empty((n, N), dtype=np.float32)
         for name, stream in (("r", STREAM_R), ("k", STREAM_K), ("v", STREAM_V)):
             _rng(seed, stream, c).standard_normal(out=buf, dtype=np.float32)
-            out[name][lo:hi] = _store(buf, dtype)
+            out[name][lo:hi] = _store(buf[off:], dtype)
         _rng(seed, STREAM_W, c).standard_normal(out=buf, dtype=np.float32)
         buf += np.float32(x_mean)
-        out["w"][lo:hi] = _store(np.exp(np.float32(-0.6065) / (np.float32(1.0) + np.exp(-buf))), dtype)
+        out["w"][lo:hi] = _store(np.exp(np.float32(-0.6065) / (np.float32(1.0) + np.exp(-buf[off:]))), dtype)
         _rng(seed, STREAM_KHAT, c).standard_normal(out=buf, dtype=np.float32)
-        khat = buf / np.sqrt(np.einsum("ij,ij->i", buf, buf))[:, None]
+        kb = buf[off:]
+        khat = kb / np.sqrt(np.einsum("ij,ij->i", kb, kb))[:, None]
         lr = np.empty((n, N), dtype=np.float32)
         _rng(seed, STREAM_LR, c).standard_normal(out=lr, dtype=np.float32)
-        lr = np.float32(1.0) / (np.float32(1.0) + np.exp(-lr))
+        lr = np.float32(1.0) / (np.float32(1.0) + np.exp(-lr[off:]))
         out["a"][lo:hi] = _store(-khat, dtype)
         out["b"][lo:hi] = _store(khat * lr, dtype)
 
-    _run(block, _blocks(nvec), threads)
+    _run(block, blocks, threads)
     return out
 
 
@@ -159,10 +174,32 @@ def gen_steps(steps: int, B: int, H: int, N: int, *, seed: int, dtype: str = "bf
     return {name: arr.reshape(steps, B, H, N) for name, arr in vecs.items()}
 
 
+def gen_steps_range(first: int, stop: int, B: int, H: int, N: int, *, seed: int, dtype: str = "bf16",
+                    threads: int | None = None) -> dict:
+    """Steps ``first`` .. ``stop - 1`` of ``gen_steps`` (same values), [stop - first, B, H, N]."""
+    vecs = gen_vectors_range(first * B * H, stop * B * H, N, seed=seed, dtype=dtype, threads=threads)
+    return {name: arr.reshape(stop - first, B, H, N) for name, arr in vecs.items()}
+
+
 def gen_dy(B: int, T: int, H: int, N: int, *, seed: int, dtype: str = "bf16",
            threads: int | None = None) -> np.ndarray:
     return gen_normal(B * T * H, N, seed=seed, stream=STREAM_DY, dtype=dtype,
                       threads=threads).reshape(B, T, H, N)
+
+
+def gen_gate(B: int, T: int, H: int, N: int, *, seed: int, dtype: str = "bf16",
+             threads: int | None = None) -> np.ndarray:
+    """Gate values of the time-mix output, sigmoid(N(0, 1)) per channel, [B, T, H, N]."""
+    x = gen_normal(B * T * H, N, seed=seed, stream=STREAM_GATE, dtype="f32", threads=threads)
+    return _store(np.float32(1.0) / (np.float32(1.0) + np.exp(-x)), dtype).reshape(B, T, H, N)
+
+
+def gen_timemix_params(H: int, N: int, *, seed: int):
+    """Per-head parameters of the time-mix output, float32 [H, N] each: the
+    current-token weight rho ~ U(-1, 1), the norm's gamma ~ U(0.5, 1.5) and
+    beta ~ U(-0.5, 0.5)."""
+    u = _rng(seed, STREAM_PARAMS, 0).random((3, H, N), dtype=np.float32)
+    return (u[0] * np.float32(2.0) - np.float32(1.0), u[1] + np.float32(0.5), u[2] - np.float32(0.5))
 
 
 # Named workloads: (kind, shape, recipe).  Sizes follow the workload list of
@@ -174,8 +211,10 @@ WORKLOADS = {
                                       x_mean=0.0, s0_std=0.1, seed=1),
     "decode_b256_h40_x1000": dict(kind="step", B=256, H=40, N=64, dtype="bf16",
                                   steps=1000, s0_std=0.1, seed=2),
-    "long_b1_t65536_h32_chunk64": dict(kind="forward", B=1, T=65536, H=32, N=64, dtype="bf16",
-                                       x_mean=-2.0, s0_std=0.1, seed=3, chunk_len=64),
+    # served by the chunked form's 32-token chunks (the result does not depend
+    # on the chunk length; a 64-token chunk is not implemented)
+    "long_b1_t65536_h32_chunk32": dict(kind="forward", B=1, T=65536, H=32, N=64, dtype="bf16",
+                                       x_mean=-2.0, s0_std=0.1, seed=3, chunk_len=32),
     "train_bwd_b8_t4096_h32": dict(kind="backward", B=8, T=4096, H=32, N=64, dtype="bf16",
                                    x_mean=0.0, s0_std=0.1, seed=4),
 }

@@ -8,6 +8,7 @@ is missing or fails to load, the first call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -29,7 +30,8 @@ EXPORTED_SYMBOLS = (
     "wkv7_forward_continue", "wkv7_forward_host_workspace_size", "wkv7_forward_host",
     "wkv7_saved_states_size", "wkv7_forward_train", "wkv7_backward_from_states_workspace_size",
     "wkv7_backward_from_states", "wkv7_state_gradient", "wkv7_state_gradient_workspace_size",
-    "wkv7_compose_adjoints",
+    "wkv7_compose_adjoints", "wkv7_get_last_status", "wkv7_forward_timemix",
+    "wkv7_forward_timemix_workspace_size",
 )
 
 _lib = None
@@ -97,6 +99,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wkv7_set_wait_limit.restype = None
     lib.wkv7_get_device_status.argtypes = [vp]
     lib.wkv7_get_device_status.restype = i
+    lib.wkv7_get_last_status.argtypes = [vp]
+    lib.wkv7_get_last_status.restype = i
+    lib.wkv7_forward_timemix_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    lib.wkv7_forward_timemix_workspace_size.restype = z
+    lib.wkv7_forward_timemix.argtypes = ([i, i, i, i, i, i] + [vp] * 11 + [ctypes.c_float] + [vp, vp] +
+                                         [i, i, vp, z, vp])
+    lib.wkv7_forward_timemix.restype = i
     _lib = lib
     return lib
 
@@ -105,9 +114,37 @@ def status_string(status: int) -> str:
     return load_library().wkv7_status_string(int(status)).decode()
 
 
-def _check(fn, status):
+# Status checks after every call: off by default (a check synchronizes the
+# stream).  WKV7_CHECK_STATUS=1 in the environment, set_status_checks(True) or
+# the status_checks() context turn them on; then each call also reads the
+# device status word (wkv7_get_last_status) and raises on a device-side
+# condition such as a chunk outside the chunked form's range.
+_status_checks = os.environ.get("WKV7_CHECK_STATUS", "") not in ("", "0")
+
+
+def set_status_checks(on: bool) -> bool:
+    """Turn the per-call device status check on or off; returns the old setting."""
+    global _status_checks
+    old, _status_checks = _status_checks, bool(on)
+    return old
+
+
+@contextlib.contextmanager
+def status_checks(on: bool):
+    old = set_status_checks(on)
+    try:
+        yield
+    finally:
+        set_status_checks(old)
+
+
+def _check(fn, status, stream=None):
     if status != OK:
         raise WKV7Error(fn, status)
+    if _status_checks:
+        dev = load_library().wkv7_get_last_status(_stream(stream))
+        if dev != OK:
+            raise WKV7Error(fn, dev)
 
 
 def _dt(t: torch.Tensor) -> int:
@@ -165,8 +202,44 @@ def forward(r, w, k, v, a, b, s0=None, *, y=None, sT=None, y_dtype=None, algo="a
     st = lib.wkv7_forward(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s0, y, sT)),
                           ALGOS[algo], chunk_len, _ptr(workspace),
                           0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("wkv7_forward", st)
+    _check("wkv7_forward", st, stream)
     return (y, sT) if return_state else y
+
+
+def forward_timemix_workspace_size(B, T, H, N, in_dtype=torch.bfloat16, algo="auto", chunk_len=0) -> int:
+    code = F32 if in_dtype == torch.float32 else BF16
+    return load_library().wkv7_forward_timemix_workspace_size(B, T, H, N, code, ALGOS[algo], chunk_len)
+
+
+def forward_timemix(r, w, k, v, a, b, s0=None, *, rho, gamma=None, beta=None, g=None, eps=1e-5, z=None, sT=None,
+                    out_dtype=None, algo="auto", chunk_len=0, workspace=None, return_state=True, stream=None):
+    """wkv7_forward_timemix: z [B,T,H,N] (and sT) of the forward followed by the
+    time-mix output epilogue (current-token term with weight ``rho`` [H,N],
+    per-head normalisation with ``gamma``/``beta`` [H,N], gate ``g`` [B,T,H,N])."""
+    lib = load_library()
+    B, T, H, N = r.shape
+    _same((w, k, v, a, b), r.shape, r.dtype)
+    _same((rho,), (H, N), torch.float32)
+    for p in (gamma, beta):
+        if p is not None:
+            _same((p,), (H, N), torch.float32)
+    if g is not None:
+        _same((g,), r.shape, r.dtype)
+    ocode = _dt(r) if out_dtype is None else (F32 if out_dtype == torch.float32 else BF16)
+    if z is None:
+        z = torch.empty((B, T, H, N), dtype=_tdt(ocode), device=r.device)
+    if return_state and sT is None:
+        sT = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    if s0 is not None:
+        _same((s0,), (B, H, N, N), torch.float32)
+    ws_bytes = lib.wkv7_forward_timemix_workspace_size(B, T, H, N, _dt(r), ALGOS[algo], chunk_len)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=r.device)
+    st = lib.wkv7_forward_timemix(B, T, H, N, _dt(r), ocode, *map(_ptr, (r, w, k, v, a, b, s0, rho, gamma, beta, g)),
+                                  float(eps), _ptr(z), _ptr(sT), ALGOS[algo], chunk_len, _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("wkv7_forward_timemix", st, stream)
+    return (z, sT) if return_state else z
 
 
 def forward_summary_workspace_size(B, T, H, N) -> int:
@@ -185,7 +258,7 @@ def forward_summary(r, w, k, v, a, b, *, out=None, workspace=None, stream=None):
     _same((out,), (2, B, H, N, N), torch.float32)
     st = lib.wkv7_forward_summary(B, T, H, N, _dt(r), *map(_ptr, (r, w, k, v, a, b, out)), _ptr(workspace),
                                   0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("wkv7_forward_summary", st)
+    _check("wkv7_forward_summary", st, stream)
     return out
 
 
@@ -206,7 +279,7 @@ def forward_continue(r, w, k, v, a, b, s_in=None, *, workspace=None, y=None, sT=
     st = lib.wkv7_forward_continue(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s_in, y, sT)),
                                    _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                    _stream(stream))
-    _check("wkv7_forward_continue", st)
+    _check("wkv7_forward_continue", st, stream)
     return (y, sT) if return_state else y
 
 
@@ -224,7 +297,7 @@ def compose_states(summaries, s0=None, *, out=None, stream=None):
         out = torch.empty((nseg + 1, B, H, N, N), dtype=torch.float32, device=summaries.device)
     _same((out,), (nseg + 1, B, H, N, N), torch.float32)
     st = lib.wkv7_compose_states(nseg, B, H, N, _ptr(s0), _ptr(summaries), _ptr(out), _stream(stream))
-    _check("wkv7_compose_states", st)
+    _check("wkv7_compose_states", st, stream)
     return out
 
 
@@ -264,7 +337,7 @@ def forward_host(r, w, k, v, a, b, s0=None, *, y, sT=None, algo="auto", chunk_le
                                 device=device if device is not None else torch.cuda.current_device())
     st = lib.wkv7_forward_host(B, T, H, N, _dt(r), ycode, *map(_host_ptr, (r, w, k, v, a, b, s0, y, sT)),
                                ALGOS[algo], chunk_len, _ptr(workspace), workspace.numel(), _stream(stream))
-    _check("wkv7_forward_host", st)
+    _check("wkv7_forward_host", st, stream)
     return y, sT
 
 
@@ -289,7 +362,7 @@ def state_gradient(r, w, a, b, dy, dsT=None, *, out=None, workspace=None, stream
         workspace = None
     st = lib.wkv7_state_gradient(B, T, H, N, _dt(r), *map(_ptr, (r, w, a, b, dy, dsT, out, workspace)),
                                  0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("wkv7_state_gradient", st)
+    _check("wkv7_state_gradient", st, stream)
     return out
 
 
@@ -305,7 +378,7 @@ def compose_adjoints(summaries, F, dsT=None, *, out=None, stream=None):
     if out is None:
         out = torch.empty((nseg + 1, B, H, N, N), dtype=torch.float32, device=summaries.device)
     st = lib.wkv7_compose_adjoints(nseg, B, H, N, _ptr(dsT), _ptr(summaries), _ptr(F), _ptr(out), _stream(stream))
-    _check("wkv7_compose_adjoints", st)
+    _check("wkv7_compose_adjoints", st, stream)
     return out
 
 
@@ -327,7 +400,7 @@ def step(r, w, k, v, a, b, state, *, y=None, y_dtype=None, stream=None):
     if y is None:
         y = torch.empty((B, H, N), dtype=_tdt(ycode), device=r.device)
     st = lib.wkv7_step(B, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, state, y)), _stream(stream))
-    _check("wkv7_step", st)
+    _check("wkv7_step", st, stream)
     return y
 
 
@@ -351,7 +424,7 @@ def backward(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.float32, wo
     st = lib.wkv7_backward(B, T, H, N, _dt(r), gcode,
                            *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)),
                            _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("wkv7_backward", st)
+    _check("wkv7_backward", st, stream)
     return tuple(out)
 
 
@@ -385,7 +458,7 @@ def forward_train(r, w, k, v, a, b, s0=None, *, y=None, sT=None, states=None, y_
     st = lib.wkv7_forward_train(B, T, H, N, _dt(r), ycode, *map(_ptr, (r, w, k, v, a, b, s0, y, sT, states)),
                                 ALGOS[algo], chunk_len, _ptr(workspace),
                                 0 if workspace is None else workspace.numel(), _stream(stream))
-    _check("wkv7_forward_train", st)
+    _check("wkv7_forward_train", st, stream)
     return y, sT, states
 
 
@@ -406,7 +479,7 @@ def backward_from_states(r, w, k, v, a, b, states, sT, dy, dsT=None, *, grad_dty
                                        *map(_ptr, (r, w, k, v, a, b, states, sT, dy, dsT, *out)),
                                        _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                        _stream(stream))
-    _check("wkv7_backward_from_states", st)
+    _check("wkv7_backward_from_states", st, stream)
     return tuple(out)
 
 
@@ -424,7 +497,7 @@ def backward_noalloc(r, w, k, v, a, b, s0, dy, dsT=None, *, grad_dtype=torch.flo
         out.append(torch.empty((B, H, N, N), dtype=torch.float32, device=r.device))
     st = lib.wkv7_backward_noalloc(B, T, H, N, _dt(r), gcode,
                                    *map(_ptr, (r, w, k, v, a, b, s0, dy, dsT, *out)), _stream(stream))
-    _check("wkv7_backward_noalloc", st)
+    _check("wkv7_backward_noalloc", st, stream)
     return tuple(out)
 
 
@@ -433,6 +506,9 @@ def set_wait_limit(cycles: int = 0) -> None:
     load_library().wkv7_set_wait_limit(int(cycles))
 
 
-def device_status(stream=None) -> int:
+def last_status(stream=None) -> int:
     """Synchronize and read/clear the library's sticky device status word."""
-    return load_library().wkv7_get_device_status(_stream(stream))
+    return load_library().wkv7_get_last_status(_stream(stream))
+
+
+device_status = last_status

@@ -205,3 +205,36 @@ def test_state_gradient_and_adjoints_reject_invalid_arguments(lib):
     assert ca(adj=None) == wkv7.ERR_INVALID_ARG
     assert ca(dsT=ctypes.c_void_p(8)) == wkv7.ERR_INVALID_ARG
     assert ca(B=0) == wkv7.OK
+
+
+def test_last_status_without_a_device(lib):
+    """wkv7_get_last_status (and its earlier name wkv7_get_device_status)
+    synchronize the stream first; without a usable device that fails and the
+    call says so instead of reporting a status word it could not read."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present (the GPU tests read the status word)")
+    lib.wkv7_get_last_status.argtypes = [ctypes.c_void_p]
+    lib.wkv7_get_device_status.argtypes = [ctypes.c_void_p]
+    assert lib.wkv7_get_last_status(None) == wkv7.ERR_CUDA
+    assert lib.wkv7_get_device_status(None) == wkv7.ERR_CUDA
+
+
+def test_timemix_rejects_invalid_arguments(lib):
+    """wkv7_forward_timemix validates on the host before any CUDA call."""
+    lib.wkv7_forward_timemix.argtypes = ([ctypes.c_int] * 6 + [ctypes.c_void_p] * 11 + [ctypes.c_float] +
+                                         [ctypes.c_void_p] * 2 + [ctypes.c_int] * 2 +
+                                         [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p])
+
+    def call(N=64, rho=P, eps=1e-5, algo=2, ws=None, wsb=0, g=None, T=64):
+        return lib.wkv7_forward_timemix(1, T, 1, N, wkv7.BF16, wkv7.BF16, P, P, P, P, P, P, None, rho, None, None,
+                                        g, eps, P, None, algo, 0, ws, wsb, None)
+
+    assert call(rho=None) == wkv7.ERR_INVALID_ARG                  # rho is required
+    assert call(eps=-1.0) == wkv7.ERR_INVALID_ARG
+    assert call(eps=float("nan")) == wkv7.ERR_INVALID_ARG
+    assert call(N=32) == wkv7.ERR_UNSUPPORTED
+    assert call(g=ctypes.c_void_p(18)) == wkv7.ERR_INVALID_ARG      # misaligned gate
+    assert call(algo=1) == wkv7.ERR_INVALID_ARG                    # the scan path needs its fp32 y workspace
+    assert call(algo=7) == wkv7.ERR_INVALID_ARG
+    assert lib.wkv7_forward_timemix_workspace_size(2, 100, 3, 64, wkv7.BF16, wkv7.ALGO_SEQ, 0) == 2 * 100 * 3 * 64 * 4

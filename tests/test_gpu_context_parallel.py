@@ -148,7 +148,7 @@ def test_long_context_over_eight_stretches(cuda_device):
     """B=1, T=65536, H=32, w near 1, split over 8 stretches of 8192 tokens (one
     per GPU of a node): sampled heads vs the oracle, every head vs the whole
     sequence's chunked forward."""
-    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk32"]
     d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
                             x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
     y, states, _ = _stretches_on_one_gpu(d, 8)

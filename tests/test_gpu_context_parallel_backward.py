@@ -219,7 +219,7 @@ def test_long_context_backward_over_eight_stretches(cuda_device):
     and a dL/dS_T term: sampled heads vs the oracle's backward over the whole
     sequence, every head vs one wkv7.backward (which itself runs the
     segmented checkpoint pass and sweep)."""
-    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk32"]
     B, T, H, N = cfg["B"], cfg["T"], cfg["H"], cfg["N"]
     d = inputs.gen_sequence(B, T, H, N, seed=cfg["seed"], dtype="bf16", x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
     d["dy"] = inputs.gen_dy(B, T, H, N, seed=cfg["seed"], dtype="bf16")

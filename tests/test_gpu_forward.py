@@ -111,7 +111,7 @@ def test_prefill_workload_sampled_heads(cuda_device):
     assert wkv7.resolve_algo(cfg["T"], torch.bfloat16, "auto") == "chunk"
     y, sT = run_forward(d, algo="auto")
     assert wkv7.device_status() == wkv7.OK
-    heads = _sample_heads(cfg["H"], 3, 0)
+    heads = _sample_heads(cfg["H"], cfg["H"] // 8, 0)      # an eighth of the heads of every batch row
     yr, sr = oracle_forward(d, heads)
     assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y", bf16_out=True)
     assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT")
@@ -119,11 +119,11 @@ def test_prefill_workload_sampled_heads(cuda_device):
 
 def test_long_context_workload_sampled_heads(cuda_device):
     """B=1, T=65536, H=32 with w near 1 (long memory): sequential scan on sampled heads."""
-    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk32"]
     d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
                             x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
     y, sT = run_forward(d, y_dtype=torch.float32, algo="seq")
-    heads = _sample_heads(cfg["H"], 2, 1)
+    heads = _sample_heads(cfg["H"], cfg["H"] // 8, 1)
     yr, sr = oracle_forward(d, heads)
     assert_close(to_f64(y[:, :, heads]), yr, TAU_BF16, "y")
     assert_close(to_f64(sT[:, heads]), sr, TAU_BF16, "sT")
@@ -180,8 +180,16 @@ def test_chunked_flags_out_of_domain_decay(cuda_device):
     d["w"] = inputs.f32_to_bf16_bits(np.full((B, T, H, N), 0.05, np.float32))
     assert wkv7.device_status() == wkv7.OK
     run_forward(d, y_dtype=torch.float32, algo="chunk")
-    assert wkv7.device_status() == wkv7.ERR_RANGE
-    assert wkv7.device_status() == wkv7.OK          # cleared by the read
+    assert wkv7.last_status() == wkv7.ERR_RANGE
+    assert wkv7.last_status() == wkv7.OK            # cleared by the read
+    lib = wkv7.load_library()
+    run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert lib.wkv7_get_device_status(None) == wkv7.ERR_RANGE     # the earlier name of the same call
+    with wkv7.status_checks(True):                  # the binding's per-call check raises instead
+        with pytest.raises(wkv7.WKV7Error) as ei:
+            run_forward(d, y_dtype=torch.float32, algo="chunk")
+    assert ei.value.status == wkv7.ERR_RANGE
+    assert wkv7.last_status() == wkv7.OK
     y, sT = run_forward(d, y_dtype=torch.float32, algo="seq")
     yr, sr = oracle_forward(d)
     assert_close(to_f64(y), yr, TAU_BF16, "y (seq)")
@@ -190,12 +198,12 @@ def test_chunked_flags_out_of_domain_decay(cuda_device):
 def test_long_context_chunked_matches_oracle_and_sequential(cuda_device):
     """B=1, T=65536, H=32, w near 1, chunked form: sampled heads vs the oracle,
     and every head vs the sequential scan."""
-    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk64"]
+    cfg = inputs.WORKLOADS["long_b1_t65536_h32_chunk32"]
     d = inputs.gen_sequence(cfg["B"], cfg["T"], cfg["H"], cfg["N"], seed=cfg["seed"], dtype="bf16",
                             x_mean=cfg["x_mean"], s0_std=cfg["s0_std"])
     yc, sc = run_forward(d, y_dtype=torch.float32, algo="chunk")
     assert wkv7.device_status() == wkv7.OK
-    heads = _sample_heads(cfg["H"], 2, 2)
+    heads = _sample_heads(cfg["H"], cfg["H"] // 8, 2)
     yr, sr = oracle_forward(d, heads)
     assert_close(to_f64(yc[:, :, heads]), yr, TAU_BF16, "y vs oracle")
     assert_close(to_f64(sc[:, heads]), sr, TAU_BF16, "sT vs oracle")

@@ -75,3 +75,43 @@ def test_decode_workload_full_state(cuda_device):
     yr, Sr = _oracle_steps(st, s0, n)
     assert_close(y, yr, TAU_BF16, "y", bf16_out=True)
     assert_close(S, Sr, TAU_BF16, "state")
+
+
+def test_decode_workload_1000_steps_sampled_heads(cuda_device):
+    """The decode workload as specified: B=256, H=40, all 1000 consecutive
+    steps from the workload's seeds, through the step kernel in the benchmark's
+    launch.  A random eighth of the (b, h) heads is checked: y of every step
+    and the final state vs the oracle.  The steps of one head are one sequence
+    of the recurrence (a decode step is one token of it), so the oracle runs
+    them as a forward over the steps of each block, carrying its state."""
+    cfg = inputs.WORKLOADS["decode_b256_h40_x1000"]
+    B, H, N, n = cfg["B"], cfg["H"], cfg["N"], cfg["steps"]
+    rng = np.random.default_rng(1000)
+    flat = np.sort(rng.choice(B * H, size=B * H // 8, replace=False))
+    sb, sh = flat // H, flat % H
+    sel_b, sel_h = torch.as_tensor(sb, device="cuda"), torch.as_tensor(sh, device="cuda")
+    s0 = inputs.gen_normal(B * H * N, N, seed=cfg["seed"], stream=inputs.STREAM_S0,
+                           std=cfg["s0_std"]).reshape(B, H, N, N)
+    state = to_dev(s0)
+    S_ref = s0[sb, sh][:, None].astype(np.float64)          # [nsel, 1, N, N]
+    y_got = np.empty((n, len(flat), N), np.float32)
+    y_ref = np.empty((n, len(flat), N), np.float32)
+    block = 100
+    for s_lo in range(0, n, block):
+        s_hi = min(n, s_lo + block)
+        st = inputs.gen_steps_range(s_lo, s_hi, B, H, N, seed=cfg["seed"], dtype="bf16")
+        dev = {nm: to_dev(st[nm]) for nm in inputs.INPUT_NAMES}
+        y = torch.empty((s_hi - s_lo, B, H, N), dtype=torch.bfloat16, device="cuda")
+        for s in range(s_hi - s_lo):
+            wkv7.step(*(dev[nm][s] for nm in inputs.INPUT_NAMES), state, y=y[s])
+        y_got[s_lo:s_hi] = y[:, sel_b, sel_h].float().cpu().numpy()
+        # oracle: each sampled head is a batch row of a one-head sequence over these steps
+        seq = [inputs.to_f64(np.ascontiguousarray(st[nm][:, sb, sh].transpose(1, 0, 2)))[:, :, None]
+               for nm in inputs.INPUT_NAMES]
+        yr, S_ref = oracle.forward(*seq, s0=S_ref)
+        y_ref[s_lo:s_hi] = yr[:, :, 0].transpose(1, 0, 2)
+        del dev, y
+    torch.cuda.synchronize()
+    assert wkv7.last_status() == wkv7.OK
+    assert_close(y_got, y_ref, TAU_BF16, "y (every step, bf16 out)", bf16_out=True)
+    assert_close(to_f64(state[sel_b, sel_h]), S_ref[:, 0], TAU_BF16, "state after 1000 steps")

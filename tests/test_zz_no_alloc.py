@@ -7,9 +7,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from linear_rnn_sequence_wkv7_b200 import inputs, wkv7
 from tests._dev import to_dev, to_f64
-from tests._tol import TAU_F32, assert_close
+from tests._tol import TAU_BF16, TAU_F32, assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -35,6 +36,27 @@ def test_noalloc_backward_matches_workspace_backward(cuda_device):
         torch.cuda.synchronize()
         for name, g, r in zip(NAMES, got, ref):
             assert_close(to_f64(g), to_f64(r), TAU_F32, name)
+
+
+def test_noalloc_backward_bf16_segmented_then_small(cuda_device):
+    """bf16 inputs (checkpoints by the chunked forward, chunk gradients on the
+    tensor cores).  First a few-head long sequence (B=1, T=1024, H=2) whose
+    checkpoint pass and state-gradient sweep run as segments, so their
+    per-segment scratch lives in the fixed array too; then a smaller problem
+    on the same array.  Each call vs the backward with a workspace, and vs
+    the oracle."""
+    for seed, (B, T, H) in ((920, (1, 1024, 2)), (921, (2, 77, 3))):
+        assert wkv7.backward_workspace_size(B, T, H, 64) <= (32 << 20)
+        x, s0, dy, dsT = _case(seed, B=B, T=T, H=H, dtype="bf16")
+        ref = wkv7.backward(*x, s0, dy, dsT)
+        got = wkv7.backward_noalloc(*x, s0, dy, dsT)
+        torch.cuda.synchronize()
+        assert wkv7.last_status() == wkv7.OK
+        args = [to_f64(t) for t in x]
+        want = oracle.backward(*args, to_f64(s0), to_f64(dy), to_f64(dsT))
+        for name, g, r, o in zip(NAMES, got, ref, want):
+            assert_close(to_f64(g), to_f64(r), TAU_BF16, name + " vs workspace backward")
+            assert_close(to_f64(g), o, TAU_BF16, name + " vs oracle")
 
 
 def test_noalloc_backward_rejects_oversized_problems(cuda_device):
