@@ -60,7 +60,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--algo", default="auto", choices=["auto", "seq", "chunk"])
-    p.add_argument("--parts", default="fwd,bwd,train,decode,long")
+    p.add_argument("--parts", default="fwd,bwd,train,decode,long,timemix")
     p.add_argument("--decode-steps", type=int, default=DEC["steps"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -406,6 +406,43 @@ def bench_train(args, dist, peaks, device, d):
                        "y_dtype": "bf16", "grad_dtype": "bf16", "dsT": "zero"}}
 
 
+def bench_timemix(args, dist, peaks, device, d, plain_ms):
+    """The prefill forward with the time-mix output epilogue (current-token
+    term, per-head norm, gate) fused into the chunked kernel, bf16 z: its cost
+    over the plain forward on the same inputs."""
+    import torch
+    from linear_rnn_sequence_wkv7_b200 import wkv7
+    cfg = FWD
+    B, T, H = cfg["B"], cfg["T"], cfg["H"]
+    dev = [to_dev(d[n], device) for n in inputs.INPUT_NAMES]
+    s0 = to_dev(d["s0"], device)
+    rho, gamma, beta = (torch.from_numpy(x).to(device) for x in inputs.gen_timemix_params(H, N, seed=cfg["seed"]))
+    g = to_dev(inputs.gen_gate(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16"), device)
+    z = torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device)
+    sT = torch.empty(B, H, N, N, dtype=torch.float32, device=device)
+    ws_n = wkv7.forward_timemix_workspace_size(B, T, H, N, torch.bfloat16, args.algo)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=device) if ws_n else None
+    stream = torch.cuda.current_stream()
+
+    def step():
+        wkv7.forward_timemix(*dev, s0, rho=rho, gamma=gamma, beta=beta, g=g, z=z, sT=sT, algo=args.algo,
+                             workspace=ws, stream=stream)
+
+    steps = max(3, min(args.steps // 4, 50))
+    per = timed(step, steps, 3, dist, stream, "time-mix forward") / steps
+    nbytes = fwd_bytes(B, T, H) + B * T * H * N * 2          # + the gate read
+    ach = nbytes / per / 1e9
+    return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
+            "ms_per_step": per * 1e3, "steps": steps, "launches": steps,
+            "plain_forward_ms": plain_ms, "overhead_frac": per * 1e3 / plain_ms - 1.0,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"],
+                         "per_unit": "1024 B per head-token (six inputs, gate, z) + 32 KiB state per head"},
+            "config": {"workload": "prefill_b8_t4096_h32_bf16 + time-mix epilogue", "B": B, "T": T, "H": H,
+                       "N": N, "z_dtype": "bf16", "eps": 1e-5,
+                       "params": "rho ~ U(-1,1), gamma ~ U(0.5,1.5), beta ~ U(-0.5,0.5), g = sigmoid(N(0,1))"}}
+
+
 def bench_decode(args, dist, peaks, device, steps_in):
     import torch
     from linear_rnn_sequence_wkv7_b200 import wkv7
@@ -536,6 +573,8 @@ def run_ours(args):
         out_parts["decode"] = bench_decode(args, dist, peaks, device, steps_in)
     if "long" in parts:
         out_parts["long_context"] = bench_long(args, dist, peaks, device)
+    if "timemix" in parts:
+        out_parts["timemix"] = bench_timemix(args, dist, peaks, device, fwd["sample"], fwd["ms_per_step"])
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(fwd["sample"])
