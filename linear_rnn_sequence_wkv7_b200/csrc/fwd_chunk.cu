@@ -101,6 +101,9 @@ constexpr uint32_t FLAG = BAR + 68;                 // set by whichever role giv
 // the per-head mean / variance exchange between the two halves of a y row
 constexpr uint32_t UPART = RZ_LO + 5120;
 constexpr uint32_t EXCH = RZ_LO + 7168;             // fp32 [2 rounds][2 halves][32 rows]
+constexpr uint32_t GAMBET = RZ_LO + 7680;           // float2 [64]: (gamma, beta) of the head's channels
+// the gate rows of the chunk, bf16 [32][64], arrive by cp.async in TSM's rows
+// (free from the end of P1 to the next P1)
 constexpr uint32_t BAR_EPI = 10;                    // named barrier of warps 2 and 6 (the y rows)
 
 constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
@@ -108,6 +111,7 @@ constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (pr
 
 __device__ __forceinline__ uint32_t in_off(int t, int ch) { return (uint32_t)(t * 128 + (((ch + t) & 7) << 4)); }
 __device__ __forceinline__ uint32_t tsm_row(int t) { return TSM + (uint32_t)((t >> 3) * 2048 + (t & 7) * 128); }
+__device__ __forceinline__ int hc_of(int warp) { return warp >> 2; }
 
 __device__ __forceinline__ void bf8_to_f32(uint4 u, float *o) {
     const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
@@ -208,6 +212,12 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         *abort_flag = 0;
     }
     if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
+    if constexpr (EPI) {
+        if (tid < kN)
+            reinterpret_cast<float2 *>(sm + GAMBET)[tid] =
+                make_float2(epi.gamma ? epi.gamma[(size_t)h * kN + tid] : 1.f,
+                            epi.beta ? epi.beta[(size_t)h * kN + tid] : 0.f);
+    }
     if (tid < NC) {
         {   // v columns of AV: lo always zero (v is exact)
             const int t = tid >> 3, ch = tid & 7;
@@ -644,24 +654,21 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 named_sync(BAR_EPI, 64);
                 const float inv = rsqrtf((s2 + ex[64 + 32 * (1 - hc) + lane]) * (1.f / kN) + epi.eps);
                 if (t < Lv) {
-                    const size_t off = base + (size_t)(c * L + t) * tok_stride + 32 * hc;
-                    OutT *dst = yo + off;
+                    OutT *dst = yo + base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+                    const float4 *gb = reinterpret_cast<const float4 *>(sm + GAMBET) + 16 * hc;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {  // 8 channels at a time
-                        float gv[8], gm[8], bt[8];
-                        if (epi.g)
-                            bf8_to_f32(*reinterpret_cast<const uint4 *>(
-                                           static_cast<const __nv_bfloat16 *>(epi.g) + off + 8 * u), gv);
+                        float gv[8];
+                        if (epi.g) bf8_to_f32(*reinterpret_cast<const uint4 *>(sm + tsm_row(t) + 64 * hc + 16 * u), gv);
                         else for (int e = 0; e < 8; ++e) gv[e] = 1.f;
-                        const size_t po = (size_t)h * kN + 32 * hc + 8 * u;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            gm[e] = epi.gamma ? epi.gamma[po + e] : 1.f;
-                            bt[e] = epi.beta ? epi.beta[po + e] : 0.f;
-                        }
                         float zz[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) zz[e] = fmaf((x[8 * u + e] - mu) * inv, gm[e], bt[e]) * gv[e];
+                        for (int e2 = 0; e2 < 4; ++e2) {   // (gamma, beta) pairs of two channels
+                            const float4 p = gb[4 * u + e2];
+                            const int e = 2 * e2;
+                            zz[e] = fmaf((x[8 * u + e] - mu) * inv, p.x, p.y) * gv[e];
+                            zz[e + 1] = fmaf((x[8 * u + e + 1] - mu) * inv, p.z, p.w) * gv[e + 1];
+                        }
                         store4(dst + 8 * u, make_float4(zz[0], zz[1], zz[2], zz[3]));
                         store4(dst + 8 * u + 4, make_float4(zz[4], zz[5], zz[6], zz[7]));
                     }
@@ -693,6 +700,18 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             cp_async_wait<1>();                            // v(c) is in place
             ready_arrive(1);                               // R2(c)
             done_wait(1, c);
+            if constexpr (EPI) {                           // gate rows of chunk c (P1's T rows are dead)
+                if (yo && epi.g && warp % 4 == 2) {
+                    const int t = lane;
+                    if (c * L + t < T) {
+                        const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(epi.g) + base +
+                                                   (size_t)(c * L + t) * tok_stride + 32 * hc_of(warp);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) cp_async16(sm + tsm_row(t) + 64 * hc_of(warp) + 16 * q, src + 8 * q);
+                    }
+                }
+                cp_async_commit();                         // (empty for the other threads)
+            }
             P2();
             ready_arrive(2);                               // R3(c)
             done_wait(2, c);
@@ -706,6 +725,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 ready_arrive(0);                           // R1(c+1), under P4(c)
             }
             done_wait(3, c);                               // R4(c)
+            if constexpr (EPI) cp_async_wait<1>();         // the gate of chunk c (all but v(c+1))
             P4(c, min(L, T - c * L));
         }
         cp_async_wait<0>();

@@ -3,6 +3,7 @@
     python -m linear_rnn_sequence_wkv7_b200.profile_case --op fwd --algo chunk --B 2 --T 4096 --H 32
     python -m linear_rnn_sequence_wkv7_b200.profile_case --op step --B 256 --H 40 --reps 3
     python -m linear_rnn_sequence_wkv7_b200.profile_case --op bwd --B 1 --T 4096 --H 32
+    python -m linear_rnn_sequence_wkv7_b200.profile_case --op timemix --B 8 --T 4096 --H 32
 
 Inputs follow the prefill workload's distributions (bf16, s0 ~ N(0, 0.1)).
 Runs ``--warmup`` untimed launches, then ``--reps`` launches timed with CUDA
@@ -32,7 +33,7 @@ def to_dev(x):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("--op", choices=["fwd", "step", "bwd"], default="fwd")
+    p.add_argument("--op", choices=["fwd", "step", "bwd", "timemix"], default="fwd")
     p.add_argument("--algo", choices=["auto", "seq", "chunk"], default="auto")
     p.add_argument("--B", type=int, default=2)
     p.add_argument("--T", type=int, default=4096)
@@ -51,6 +52,15 @@ def main():
         nws = wkv7.forward_workspace_size(a.B, T, a.H, N, torch.bfloat16, a.algo)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
         run = lambda: wkv7.forward(*x, s0=s0, y=y, sT=sT, algo=a.algo, workspace=ws)
+    elif a.op == "timemix":
+        z = torch.empty(a.B, T, a.H, N, dtype=torch.bfloat16, device="cuda")
+        sT = torch.empty_like(s0)
+        rho, gamma, beta = (torch.from_numpy(t).cuda() for t in inputs.gen_timemix_params(a.H, N, seed=1))
+        g = to_dev(inputs.gen_gate(a.B, T, a.H, N, seed=1))
+        nws = wkv7.forward_timemix_workspace_size(a.B, T, a.H, N, torch.bfloat16, a.algo)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda")
+        run = lambda: wkv7.forward_timemix(*x, s0, rho=rho, gamma=gamma, beta=beta, g=g, z=z, sT=sT, algo=a.algo,
+                                           workspace=ws)
     elif a.op == "step":
         xs = [t[:, 0].contiguous() for t in x]
         y = torch.empty(a.B, a.H, N, dtype=torch.bfloat16, device="cuda")
