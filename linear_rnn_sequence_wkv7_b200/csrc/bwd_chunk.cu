@@ -156,41 +156,55 @@ bwd_dstate_kernel(int T, int t_seg, int seg0, int nz, const InT *__restrict__ r,
         for (int tt = Lc - 1; tt >= 0; --tt) {
             const InT *rv = tile[stage][0][tt], *wv = tile[stage][1][tt], *av = tile[stage][2][tt];
             const InT *bv = tile[stage][3][tt];
-            float dyi[RPT], dp4[NR][4];   // four partial sums per row: a shorter dependency chain
+            // packed fp32 pairs (fma.rn.f32x2): the same per-element arithmetic as
+            // scalar fmaf, half the FP instructions of an issue-bound loop
+            float2 dyi[RPT], dp4[NR][2];  // four partial sums per row (two pairs)
 #pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) dyi[rr] = to_f32(tile[stage][4][tt][row0 + rr]);
+            for (int rr = 0; rr < RPT; ++rr) {
+                const float d = to_f32(tile[stage][4][tt][row0 + rr]);
+                dyi[rr] = make_float2(d, d);
+            }
 #pragma unroll
-            for (int rr = 0; rr < NR; ++rr)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dp4[rr][e] = 0.f;
+            for (int rr = 0; rr < NR; ++rr) dp4[rr][0] = dp4[rr][1] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < NG; ++m) {
                 const float4 r4 = load4(rv + col(m)), b4 = load4(bv + col(m));
-                const float rj[4] = {r4.x, r4.y, r4.z, r4.w}, bj[4] = {b4.x, b4.y, b4.z, b4.w};
+                const float2 rj[2] = {make_float2(r4.x, r4.y), make_float2(r4.z, r4.w)};
+                const float2 bj[2] = {make_float2(b4.x, b4.y), make_float2(b4.z, b4.w)};
 #pragma unroll
                 for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float gg = rr < RPT ? fmaf(dyi[rr], rj[e], g[rr][4 * m + e]) : g[rr][4 * m + e];
-                        g[rr][4 * m + e] = gg;
-                        dp4[rr][e] = fmaf(gg, bj[e], dp4[rr][e]);
+                    for (int e = 0; e < 2; ++e) {
+                        float2 gg = make_float2(g[rr][4 * m + 2 * e], g[rr][4 * m + 2 * e + 1]);
+                        if (rr < RPT) gg = __ffma2_rn(dyi[rr], rj[e], gg);
+                        g[rr][4 * m + 2 * e] = gg.x;
+                        g[rr][4 * m + 2 * e + 1] = gg.y;
+                        dp4[rr][e] = __ffma2_rn(gg, bj[e], dp4[rr][e]);
                     }
             }
             float dp[NR];
 #pragma unroll
             for (int rr = 0; rr < NR; ++rr) {
-                dp[rr] = (dp4[rr][0] + dp4[rr][1]) + (dp4[rr][2] + dp4[rr][3]);
+                dp[rr] = (dp4[rr][0].x + dp4[rr][0].y) + (dp4[rr][1].x + dp4[rr][1].y);
 #pragma unroll
                 for (int o = 1; o < LPR; o <<= 1) dp[rr] += __shfl_xor_sync(0xffffffffu, dp[rr], o);
             }
 #pragma unroll
             for (int m = 0; m < NG; ++m) {
                 const float4 w4 = load4(wv + col(m)), a4 = load4(av + col(m));
-                const float wj[4] = {w4.x, w4.y, w4.z, w4.w}, aj[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float2 wj[2] = {make_float2(w4.x, w4.y), make_float2(w4.z, w4.w)};
+                const float2 aj[2] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w)};
 #pragma unroll
-                for (int rr = 0; rr < NR; ++rr)
+                for (int rr = 0; rr < NR; ++rr) {
+                    const float2 dpp = make_float2(dp[rr], dp[rr]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) g[rr][4 * m + e] = fmaf(g[rr][4 * m + e], wj[e], dp[rr] * aj[e]);
+                    for (int e = 0; e < 2; ++e) {
+                        const float2 gg = __ffma2_rn(make_float2(g[rr][4 * m + 2 * e], g[rr][4 * m + 2 * e + 1]),
+                                                     wj[e], __fmul2_rn(dpp, aj[e]));
+                        g[rr][4 * m + 2 * e] = gg.x;
+                        g[rr][4 * m + 2 * e + 1] = gg.y;
+                    }
+                }
             }
         }
     }

@@ -575,9 +575,14 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             tmem_wait();
             float xv[32];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                xv[e] = gv[e] * (__uint_as_float(r0[e]) + add[e]);
-                xv[16 + e] = gv[16 + e] * (__uint_as_float(r1[e]) + add[16 + e]);
+            for (int e = 0; e < 16; e += 2) {     // packed pairs: (acc + add) * G
+                const float2 lo = __fmul2_rn(make_float2(gv[e], gv[e + 1]),
+                                             __fadd2_rn(make_float2(__uint_as_float(r0[e]), __uint_as_float(r0[e + 1])),
+                                                        make_float2(add[e], add[e + 1])));
+                const float2 hi = __fmul2_rn(make_float2(gv[16 + e], gv[17 + e]),
+                                             __fadd2_rn(make_float2(__uint_as_float(r1[e]), __uint_as_float(r1[e + 1])),
+                                                        make_float2(add[16 + e], add[17 + e])));
+                xv[e] = lo.x; xv[e + 1] = lo.y; xv[16 + e] = hi.x; xv[17 + e] = hi.y;
             }
             uint32_t ph[16], pl[16];
 #pragma unroll
@@ -585,8 +590,9 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                 const float x0 = xv[2 * e2], x1 = xv[2 * e2 + 1];
                 const __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
                 const uint32_t hu = *reinterpret_cast<const uint32_t *>(&hp);
-                const __nv_bfloat162 lp = __floats2bfloat162_rn(x0 - __uint_as_float(hu << 16),
-                                                                x1 - __uint_as_float(hu & 0xffff0000u));
+                const float2 rr = __ffma2_rn(make_float2(__uint_as_float(hu << 16), __uint_as_float(hu & 0xffff0000u)),
+                                             make_float2(-1.f, -1.f), make_float2(x0, x1));
+                const __nv_bfloat162 lp = __floats2bfloat162_rn(rr.x, rr.y);
                 ph[e2] = hu;
                 pl[e2] = *reinterpret_cast<const uint32_t *>(&lp);
             }

@@ -178,20 +178,25 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
             const float *av = buf + (4 * TT + tt) * kN;
             const float *bv = buf + (5 * TT + tt) * kN;
 
-            // p = S_{t-1}[i,:] . a_t
+            // p = S_{t-1}[i,:] . a_t, in packed fp32 pairs (fma.rn.f32x2): two
+            // partial sums per row, half the FP instructions
             float p[RPT];
+            {
+                float2 p2[RPT];
 #pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) p[rr] = 0.f;
+                for (int rr = 0; rr < RPT; ++rr) p2[rr] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(av + 16 * m + 4 * q);
+                for (int m = 0; m < 4; ++m) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(av + 16 * m + 4 * q);
+                    const float2 alo = make_float2(a4.x, a4.y), ahi = make_float2(a4.z, a4.w);
 #pragma unroll
-                for (int rr = 0; rr < RPT; ++rr) {
-                    p[rr] = fmaf(S[rr][4 * m + 0], a4.x, p[rr]);
-                    p[rr] = fmaf(S[rr][4 * m + 1], a4.y, p[rr]);
-                    p[rr] = fmaf(S[rr][4 * m + 2], a4.z, p[rr]);
-                    p[rr] = fmaf(S[rr][4 * m + 3], a4.w, p[rr]);
+                    for (int rr = 0; rr < RPT; ++rr) {
+                        p2[rr] = __ffma2_rn(make_float2(S[rr][4 * m + 0], S[rr][4 * m + 1]), alo, p2[rr]);
+                        p2[rr] = __ffma2_rn(make_float2(S[rr][4 * m + 2], S[rr][4 * m + 3]), ahi, p2[rr]);
+                    }
                 }
+#pragma unroll
+                for (int rr = 0; rr < RPT; ++rr) p[rr] = p2[rr].x + p2[rr].y;
             }
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr) {
@@ -202,30 +207,37 @@ fwd_seq_kernel(int T, int H, const __grid_constant__ SeqMaps maps, const InT *__
 #pragma unroll
             for (int rr = 0; rr < RPT; ++rr) vi[rr] = vv[row0 + rr];
 
-            // S = S * w + p b + v k ;  y = S . r
+            // S = S * w + p b + v k ;  y = S . r   (packed fp32 pairs, the same
+            // per-element rounding for S; y summed as two partial sums)
             float yacc[RPT];
+            float2 y2[RPT];
 #pragma unroll
-            for (int rr = 0; rr < RPT; ++rr) yacc[rr] = 0.f;
+            for (int rr = 0; rr < RPT; ++rr) y2[rr] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const float4 w4 = *reinterpret_cast<const float4 *>(wv + 16 * m + 4 * q);
                 const float4 b4 = *reinterpret_cast<const float4 *>(bv + 16 * m + 4 * q);
                 const float4 k4 = *reinterpret_cast<const float4 *>(kv + 16 * m + 4 * q);
                 const float4 r4 = *reinterpret_cast<const float4 *>(rv + 16 * m + 4 * q);
-                const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
-                const float bj[4] = {b4.x, b4.y, b4.z, b4.w};
-                const float kj[4] = {k4.x, k4.y, k4.z, k4.w};
-                const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+                const float2 wj[2] = {make_float2(w4.x, w4.y), make_float2(w4.z, w4.w)};
+                const float2 bj[2] = {make_float2(b4.x, b4.y), make_float2(b4.z, b4.w)};
+                const float2 kj[2] = {make_float2(k4.x, k4.y), make_float2(k4.z, k4.w)};
+                const float2 rj[2] = {make_float2(r4.x, r4.y), make_float2(r4.z, r4.w)};
 #pragma unroll
-                for (int rr = 0; rr < RPT; ++rr)
+                for (int rr = 0; rr < RPT; ++rr) {
+                    const float2 pp = make_float2(p[rr], p[rr]), vv2 = make_float2(vi[rr], vi[rr]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float s = S[rr][4 * m + e];
-                        s = fmaf(s, wj[e], fmaf(p[rr], bj[e], vi[rr] * kj[e]));
-                        S[rr][4 * m + e] = s;
-                        if constexpr (YOUT) yacc[rr] = fmaf(s, rj[e], yacc[rr]);
+                    for (int e = 0; e < 2; ++e) {
+                        float2 s = make_float2(S[rr][4 * m + 2 * e], S[rr][4 * m + 2 * e + 1]);
+                        s = __ffma2_rn(s, wj[e], __ffma2_rn(pp, bj[e], __fmul2_rn(vv2, kj[e])));
+                        S[rr][4 * m + 2 * e] = s.x;
+                        S[rr][4 * m + 2 * e + 1] = s.y;
+                        if constexpr (YOUT) y2[rr] = __ffma2_rn(s, rj[e], y2[rr]);
                     }
+                }
             }
+#pragma unroll
+            for (int rr = 0; rr < RPT; ++rr) yacc[rr] = y2[rr].x + y2[rr].y;
             if constexpr (YOUT) {
 #pragma unroll
                 for (int rr = 0; rr < RPT; ++rr) {

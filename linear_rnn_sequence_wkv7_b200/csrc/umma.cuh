@@ -270,8 +270,10 @@ __device__ __forceinline__ void store8_split(unsigned char *hi_base, unsigned ch
     for (int q = 0; q < 4; ++q) {
         const __nv_bfloat162 hp = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
         const uint32_t hu = *reinterpret_cast<const uint32_t *>(&hp);
-        const float r0 = x[2 * q] - __uint_as_float(hu << 16);
-        const float r1 = x[2 * q + 1] - __uint_as_float(hu & 0xffff0000u);
+        // x - hi for the pair in one packed fma (exact: -1 * hi is exact)
+        const float2 rr = __ffma2_rn(make_float2(__uint_as_float(hu << 16), __uint_as_float(hu & 0xffff0000u)),
+                                     make_float2(-1.f, -1.f), make_float2(x[2 * q], x[2 * q + 1]));
+        const float r0 = rr.x, r1 = rr.y;
         const __nv_bfloat162 lp = __floats2bfloat162_rn(r0, r1);
         h[q] = hu;
         l[q] = *reinterpret_cast<const uint32_t *>(&lp);
