@@ -437,7 +437,9 @@ def bench_timemix(args, dist, peaks, device, d, plain_ms):
             "plain_forward_ms": plain_ms, "overhead_frac": per * 1e3 / plain_ms - 1.0,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"],
-                         "per_unit": "1024 B per head-token (six inputs, gate, z) + 32 KiB state per head"},
+                         "per_unit": "1024 B per head-token (six inputs, gate, z) + 32 KiB state per head",
+                         "traffic": recorded_traffic("fwd_chunk_timemix",
+                                                     source_hash("fwd_chunk.cu", "umma.cuh", "common.cuh"))},
             "config": {"workload": "prefill_b8_t4096_h32_bf16 + time-mix epilogue", "B": B, "T": T, "H": H,
                        "N": N, "z_dtype": "bf16", "eps": 1e-5,
                        "params": "rho ~ U(-1,1), gamma ~ U(0.5,1.5), beta ~ U(-0.5,0.5), g = sigmoid(N(0,1))"}}
