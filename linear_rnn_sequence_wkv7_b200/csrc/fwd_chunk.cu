@@ -143,7 +143,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
                  float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt,
-                 float *m_out, long long m_zstride, int seg0, int first_out, EpiArgs epi) {
+                 float *m_out, long long m_zstride, int seg0, int first_out, EpiArgs epi, float *y0q) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -644,6 +644,33 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                         for (int e = 0; e < 32; ++e) mp[(size_t)(32 * hc + e) * kN + rho] = x[e];
                     }
                 }
+            } else if (DUAL && !yo && y0q != nullptr) {
+                // a summary run's y rows: y0 (its output from S = 0) and q = M_{<=t} r_t
+                // (the second state's rows, from I), fp32 [2][B][T][H][64] at the
+                // tokens' own positions; y_t = y0_t + S_in q_t once S_in is known
+                const int t = rho - 64;
+                if (t < Lv) {
+                    const size_t off = base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+                    float4 *d0 = reinterpret_cast<float4 *>(y0q + off);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) d0[u] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+                }
+                tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc, r0);
+                tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc + 16, r1);
+                tmem_wait();
+                if (t < Lv) {
+                    const size_t off = base + (size_t)(c * L + t) * tok_stride + 32 * hc;
+                    const size_t plane = (size_t)gridDim.y * T_total * H * kN;
+                    float4 *d1 = reinterpret_cast<float4 *>(y0q + plane + off);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        d1[u] = make_float4(__uint_as_float(r0[4 * u]), __uint_as_float(r0[4 * u + 1]),
+                                            __uint_as_float(r0[4 * u + 2]), __uint_as_float(r0[4 * u + 3]));
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        d1[4 + u] = make_float4(__uint_as_float(r1[4 * u]), __uint_as_float(r1[4 * u + 1]),
+                                                __uint_as_float(r1[4 * u + 2]), __uint_as_float(r1[4 * u + 3]));
+                }
             } else if (EPI && yo) {               // epilogue: z row t from o row t (halves in warps 2, 6)
                 const int t = rho - 64;
                 float *ex = reinterpret_cast<float *>(sm + EXCH);
@@ -768,7 +795,7 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
                                             (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0,  \
-                                            seg0, 0, epi);                                                    \
+                                            seg0, 0, epi, nullptr);                                           \
     } while (0)
     if (epi.rho) {
         if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, true);
@@ -789,7 +816,7 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
                                const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
                                float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st,
                                void *y = nullptr, wkv7_dtype y_dt = WKV7_F32, const float *s0 = nullptr,
-                               float *ckpt = nullptr, EpiArgs epi = EpiArgs{}) {
+                               float *ckpt = nullptr, EpiArgs epi = EpiArgs{}, float *y0q = nullptr) {
     static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES_DUAL;
@@ -803,7 +830,7 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k,      \
                                             (const bf *)v, (const bf *)a, (const bf *)b, s0, 0, (O *)y, e_out, \
                                             e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out,   \
-                                            epi);                                                              \
+                                            epi, y0q);                                                         \
     } while (0)
     if (epi.rho && first_out) {
         if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, true);
@@ -862,6 +889,96 @@ seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const f
         __syncthreads();
         cur = acc;
     }
+}
+
+// The output of segments 1..nseg-1 from their summary runs: a segment's state
+// at token t is S_in M_{<=t} + E_{<=t}, so y_t = y0_t + S_in q_t, with y0_t
+// its output from S = 0 and q_t = M_{<=t} r_t the second state's output
+// (both fp32 in y0q = [2][B][T][H][64]).  One CTA of 128 threads per (head,
+// segment, 256 tokens of it): S_in of the segment staged transposed in shared
+// memory once, then 64-token tiles of q.  Thread -> 4 tokens x 8 value rows
+// (4 rg .. 4 rg + 3 and 32 + 4 rg .. 32 + 4 rg + 3, so a quarter-warp reads 128
+// contiguous bytes of S_in and one broadcast q): 6 shared loads per 16 packed
+// fp32 FMAs.
+constexpr int kFixTokens = 256, kFixTile = 64;
+
+template <typename OutT>
+__global__ void __launch_bounds__(128)
+seg_fixup_kernel(int T, int H, int t_seg, const float *__restrict__ y0q, const float *__restrict__ sin,
+                 long long sin_zstride, OutT *__restrict__ y) {
+    __shared__ __align__(16) float St[kN][kN + 4];    // St[i][i'] = S_in[i'][i]
+    __shared__ __align__(16) float Qs[kFixTile][kN + 4];
+    const int head = blockIdx.x, seg = blockIdx.y + 1, tid = threadIdx.x;
+    const int bb = head / H, h = head % H;
+    const int t_lo = seg * t_seg + kFixTokens * blockIdx.z;
+    const int t_hi = min(T, min((seg + 1) * t_seg, t_lo + kFixTokens));
+    if (t_lo >= t_hi) return;
+    const float *S = sin + (size_t)(seg - 1) * sin_zstride + (size_t)head * kN * kN;
+    for (int x = tid; x < kN * kN; x += 128) St[x & 63][x >> 6] = S[x];
+    const size_t tok_stride = (size_t)H * kN, plane = (size_t)gridDim.x / H * T * tok_stride;
+    const size_t base = ((size_t)bb * T * H + h) * kN;
+    const int tg = tid >> 3, rg = tid & 7;
+    for (int t0 = t_lo; t0 < t_hi; t0 += kFixTile) {
+        const int nt = min(kFixTile, t_hi - t0);
+        __syncthreads();                              // St staged / the previous tile's Qs consumed
+        for (int x = tid; x < kFixTile * kN / 4; x += 128) {
+            const int r = x / (kN / 4), c4 = x % (kN / 4);
+            *reinterpret_cast<float4 *>(&Qs[r][4 * c4]) =
+                r < nt ? *reinterpret_cast<const float4 *>(y0q + plane + base + (size_t)(t0 + r) * tok_stride + 4 * c4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        float2 acc[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = 4 * tg + k;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (r < nt) {
+                const float *src = y0q + base + (size_t)(t0 + r) * tok_stride;
+                a = *reinterpret_cast<const float4 *>(src + 4 * rg);
+                b = *reinterpret_cast<const float4 *>(src + 32 + 4 * rg);
+            }
+            acc[k][0] = make_float2(a.x, a.y); acc[k][1] = make_float2(a.z, a.w);
+            acc[k][2] = make_float2(b.x, b.y); acc[k][3] = make_float2(b.z, b.w);
+        }
+#pragma unroll 8
+        for (int i = 0; i < kN; ++i) {
+            const float4 s0 = *reinterpret_cast<const float4 *>(&St[i][4 * rg]);
+            const float4 s1 = *reinterpret_cast<const float4 *>(&St[i][32 + 4 * rg]);
+            const float2 p0 = make_float2(s0.x, s0.y), p1 = make_float2(s0.z, s0.w);
+            const float2 p2 = make_float2(s1.x, s1.y), p3 = make_float2(s1.z, s1.w);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float qv = Qs[4 * tg + k][i];
+                const float2 q2 = make_float2(qv, qv);
+                acc[k][0] = __ffma2_rn(q2, p0, acc[k][0]);
+                acc[k][1] = __ffma2_rn(q2, p1, acc[k][1]);
+                acc[k][2] = __ffma2_rn(q2, p2, acc[k][2]);
+                acc[k][3] = __ffma2_rn(q2, p3, acc[k][3]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = 4 * tg + k;
+            if (r < nt) {
+                OutT *dst = y + base + (size_t)(t0 + r) * tok_stride;
+                store4(dst + 4 * rg, make_float4(acc[k][0].x, acc[k][0].y, acc[k][1].x, acc[k][1].y));
+                store4(dst + 32 + 4 * rg, make_float4(acc[k][2].x, acc[k][2].y, acc[k][3].x, acc[k][3].y));
+            }
+        }
+    }
+}
+
+static cudaError_t launch_fixup(int B, int T, int H, int t_seg, int nseg, wkv7_dtype y_dt, const float *y0q,
+                                const float *sin, long long sin_zstride, void *y, cudaStream_t st) {
+    if (nseg <= 1) return cudaSuccess;
+    const dim3 grid(B * H, nseg - 1, (t_seg + kFixTokens - 1) / kFixTokens);
+    if (y_dt == WKV7_F32)
+        seg_fixup_kernel<float><<<grid, 128, 0, st>>>(T, H, t_seg, y0q, sin, sin_zstride, static_cast<float *>(y));
+    else
+        seg_fixup_kernel<__nv_bfloat16>
+            <<<grid, 128, 0, st>>>(T, H, t_seg, y0q, sin, sin_zstride, static_cast<__nv_bfloat16 *>(y));
+    return cudaGetLastError();
 }
 
 static cudaError_t launch_combine(int B, int H, int nsteps, const float *s0, bool s0_eye, const float *e_base,
@@ -930,6 +1047,36 @@ static void seg_split(int T, int nseg, int &t_seg, int &n) {
     const int chunks = (T + chunk::L - 1) / chunk::L;
     t_seg = ((chunks + nseg - 1) / nseg) * chunk::L;
     n = (T + t_seg - 1) / t_seg;
+}
+
+// Fix-up form of the segmented forward (no checkpoints, no epilogue): one
+// dual launch over all nseg segments, the first an output run from s0 and the
+// others keeping their y0 and q rows; a chain for the entry states; the
+// fix-up y = y0 + S_in q.  Cost in units of one CTA alone running all of T:
+// nseg dual runs of T/nseg tokens, plus the fix-up pass, which moves 640 B
+// per head-token (measured ~1.6e-10 s per head-token against ~4.9 us per
+// chunk of one CTA alone: 1.0e-3 units per head).
+constexpr double kFixupPerHead = 1.0e-3;
+int chunk_segments_fixup(int B, int T, int H, int sm_count) {
+    const long long heads = (long long)B * H;
+    const long long chunks = (T + chunk::L - 1) / chunk::L;
+    if (sm_count <= 0 || heads <= 0) return 1;
+    const long long max_n = std::min<long long>(64, chunks / 4);
+    auto cost = [&](long long n) {
+        const long long per = (chunks + n - 1) / n;
+        return dual_rounds(n * heads, sm_count) * (double)per / (double)chunks + kFixupPerHead * (double)heads;
+    };
+    double best = 0.95 * launch_rounds(heads, sm_count);
+    for (long long n = 2; n <= max_n; ++n) best = std::min(best, cost(n));
+    for (long long n = 2; n <= max_n; ++n)
+        if (cost(n) <= 1.03 * best) return (int)n;
+    return 1;
+}
+
+size_t chunk_fixup_workspace_bytes(int B, int T, int H, int nseg) {
+    if (nseg <= 1) return 0;
+    // E_k, M_k and S_in(k + 1) for every segment, then y0 and q for every token
+    return (size_t)3 * nseg * B * H * kN * kN * sizeof(float) + (size_t)2 * B * T * H * kN * sizeof(float);
 }
 
 size_t chunk_workspace_bytes(int B, int T, int H, int nseg) {
@@ -1015,10 +1162,39 @@ cudaError_t compose_states(int B, int H, int nseg, const float *s0, const float 
     return launch_combine(B, H, nseg, s0, false, summary, 2 * zst, m0, 2 * zst, out, zst, st);
 }
 
+// The forward in the fix-up form over nseg segments (see chunk_segments_fixup).
+static cudaError_t fwd_chunk_fixup(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w,
+                                   const void *k, const void *v, const void *a, const void *b, const float *s0,
+                                   void *y, float *sT, int nseg, void *workspace, long long wait_limit,
+                                   cudaStream_t st) {
+    int t_seg;
+    seg_split(T, nseg, t_seg, nseg);
+    if (nseg <= 1)
+        return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st);
+    const long long zst = (long long)B * H * kN * kN;
+    float *em = static_cast<float *>(workspace);        // E_k [nseg], then M_k [nseg]
+    float *sin = em + 2 * nseg * zst;                    // S_in(1) .. S_in(nseg) (the last = final state)
+    float *y0q = sin + nseg * zst;                       // [2][B][T][H][64]
+    // pass 1: segment 0 from s0 writes y (its "E" is S_in(1)); segments >= 1
+    // from 0 and from I keep E_k, M_k and their y0, q rows
+    cudaError_t e = launch_dual(B, T, H, t_seg, nseg, r, w, k, v, a, b, em, zst, em + nseg * zst, zst, wait_limit,
+                                st, y, y_dt, s0, nullptr, EpiArgs{}, y0q);
+    if (e != cudaSuccess) return e;
+    // pass 2: S_in(k + 1) = S_in(k) M_k + E_k for k = 1 .. nseg - 1, from S_in(1) = E_0
+    e = launch_combine(B, H, nseg - 1, em, false, em + zst, zst, em + (nseg + 1) * zst, zst, sin, zst, st);
+    if (e != cudaSuccess) return e;
+    // pass 3: y of segments 1 .. nseg - 1, and the final state
+    e = launch_fixup(B, T, H, t_seg, nseg, y_dt, y0q, sin, zst, y, st);
+    if (e != cudaSuccess || sT == nullptr) return e;
+    return cudaMemcpyAsync(sT, sin + (nseg - 1) * zst, zst * sizeof(float), cudaMemcpyDeviceToDevice, st);
+}
+
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
-                      const EpiArgs &epi) {
+                      const EpiArgs &epi, bool fixup) {
+    if (fixup && nseg > 1 && ckpt == nullptr && epi.rho == nullptr && y != nullptr)
+        return fwd_chunk_fixup(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace, wait_limit, st);
     if (nseg <= 1)
         return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt, 0,
                             epi);

@@ -35,7 +35,9 @@ cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const flo
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
-                      const EpiArgs &epi = EpiArgs{});
+                      const EpiArgs &epi = EpiArgs{}, bool fixup = false);
+int chunk_segments_fixup(int B, int T, int H, int sm_count);
+size_t chunk_fixup_workspace_bytes(int B, int T, int H, int nseg);
 cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
                           const void *k, const void *v, const void *a, const void *b, const float *s0, void *y,
                           float *sT, float *ckpt, int CK, long long wait_limit, cudaStream_t st);
@@ -150,7 +152,10 @@ size_t wkv7_forward_workspace_size(int B, int T, int H, int N, wkv7_dtype in_dty
     if (resolve_algo(T, in_dtype, algo) != WKV7_ALGO_CHUNK || in_dtype != WKV7_BF16) return 0;
     const int sms = current_sm_count();
     if (sms <= 0) return 0;
-    return chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms, false));
+    // enough for either segmented form: the fix-up form (plain forward) or
+    // the output-run form (with checkpoints or the time-mix epilogue)
+    return std::max(chunk_workspace_bytes(B, T, H, chunk_segments(B, T, H, sms, false)),
+                    chunk_fixup_workspace_bytes(B, T, H, chunk_segments_fixup(B, T, H, sms)));
 }
 
 }  // extern "C"
@@ -182,15 +187,24 @@ wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
         // sequence segments run in parallel when there are too few heads to
         // fill the GPU and the caller provided the workspace they need
         int nseg = 1;
+        bool fixup = false;
         const int sms = current_sm_count();
-        if (sms > 0) {
-            const int want = chunk_segments(B, T, H, sms, false);
-            if (want > 1 && workspace != nullptr && aligned16(workspace) &&
-                workspace_bytes >= chunk_workspace_bytes(B, T, H, want))
+        const bool ws_ok = workspace != nullptr && aligned16(workspace);
+        if (sms > 0 && ws_ok && ckpt == nullptr && epi.rho == nullptr) {
+            // plain forward: the fix-up form (one dual pass over every segment,
+            // then y = y0 + S_in q) when its scratch is there
+            const int want = chunk_segments_fixup(B, T, H, sms);
+            if (want > 1 && workspace_bytes >= chunk_fixup_workspace_bytes(B, T, H, want)) {
                 nseg = want;
+                fixup = true;
+            }
+        }
+        if (sms > 0 && ws_ok && !fixup) {
+            const int want = chunk_segments(B, T, H, sms, false);
+            if (want > 1 && workspace_bytes >= chunk_workspace_bytes(B, T, H, want)) nseg = want;
         }
         return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
-                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, epi));
+                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, epi, fixup));
     }
     if (epi.rho) return WKV7_ERR_UNSUPPORTED;      // the scan's epilogue is a separate pass (timemix.cu)
     const long long lim = g_wait_limit.load() > 0 ? g_wait_limit.load() : kDefaultWaitCycles;

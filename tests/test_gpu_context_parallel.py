@@ -183,7 +183,9 @@ def test_orchestration_without_process_group(cuda_device):
 def test_orchestration_over_a_one_rank_nccl_group(cuda_device):
     """forward_context_parallel inside an NCCL process group of one rank: the
     all-gather, composition and continue run on the GPU through NCCL and the
-    library; the result equals the plain forward."""
+    library; the result, like the plain forward's, matches the oracle (the two
+    bf16 outputs come from different launch sequences, so each is compared
+    with the exact value rather than with the other)."""
     import os
     import socket
     import torch.distributed as dist
@@ -203,7 +205,10 @@ def test_orchestration_over_a_one_rank_nccl_group(cuda_device):
         y1, s1 = wkv7.forward(*args, s0=s0)
         torch.cuda.synchronize()
         assert torch.equal(s_in, s0)
-        assert_close(to_f64(y), to_f64(y1), TAU_BF16, "y", bf16_out=True)
-        assert_close(to_f64(s_fin), to_f64(s1), TAU_BF16, "sT")
+        yr, sr = oracle.forward(*(inputs.to_f64(d[n]) for n in inputs.INPUT_NAMES), s0=d["s0"].astype(np.float64))
+        assert_close(to_f64(y), yr, TAU_BF16, "y", bf16_out=True)
+        assert_close(to_f64(y1), yr, TAU_BF16, "y (plain forward)", bf16_out=True)
+        assert_close(to_f64(s_fin), sr, TAU_BF16, "sT")
+        assert_close(to_f64(s_fin), to_f64(s1), TAU_BF16, "sT vs the plain forward")
     finally:
         dist.destroy_process_group()

@@ -42,17 +42,25 @@ def _oracle_states(d):
 @pytest.mark.parametrize("dtype,B,T,H,algo", [("bf16", 2, 200, 3, "chunk"), ("bf16", 1, 2000, 2, "chunk"),
                                               ("f32", 2, 100, 2, "seq"), ("bf16", 1, 77, 2, "seq")])
 def test_forward_train_matches_forward_and_oracle(cuda_device, dtype, B, T, H, algo):
-    """y and sT equal wkv7_forward's (same kernels, same segments); the saved
-    states equal the oracle's state at every chunk start.  (1, 2000, 2) runs
-    the chunked form as sequence segments, which write their own slots."""
+    """y and sT equal wkv7_forward's (same kernels) and the saved states equal
+    the oracle's state at every chunk start.  (1, 2000, 2) runs the chunked
+    form as sequence segments, which write their own slots; there the plain
+    forward takes the fix-up form (y = y0 + S_in q after one summary pass)
+    while the training forward keeps the output runs that write the states,
+    so the two agree within the bound rather than bit for bit."""
     d = _case(B, T, H, 970 + T, dtype)
     x, s0, _, _ = _dev(d)
     y, sT, states = wkv7.forward_train(*x, s0, y_dtype=torch.float32, algo=algo)
     y1, s1 = wkv7.forward(*x, s0=s0, y_dtype=torch.float32, algo=algo)
     torch.cuda.synchronize()
     assert wkv7.device_status() == wkv7.OK
-    assert torch.equal(y, y1) and torch.equal(sT, s1)
     tau = TAU_F32 if dtype == "f32" else TAU_BF16
+    segmented = algo == "chunk" and wkv7.forward_workspace_size(B, T, H, 64, torch.bfloat16, algo) > 0
+    if segmented:
+        assert_close(to_f64(y), to_f64(y1), tau, "y vs the plain forward")
+        assert_close(to_f64(sT), to_f64(s1), tau, "sT vs the plain forward")
+    else:
+        assert torch.equal(y, y1) and torch.equal(sT, s1)
     ref = _oracle_states(d)
     for c in range(ref.shape[2]):
         assert_close(to_f64(states[:, :, c]), ref[:, :, c], tau, f"state before chunk {c}")
