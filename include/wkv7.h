@@ -152,7 +152,8 @@ WKV7_API size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N);
  *   workspace        : wkv7_forward_summary_workspace_size() bytes, or NULL.
  *                      With it the stretch runs as segments whose summaries
  *                      are chained into E and M and stay in the workspace for
- *                      wkv7_forward_continue; without it, one launch that
+ *                      wkv7_forward_continue, with every token's two partial
+ *                      outputs (fp32, 512 B per head-token); without it, one launch that
  *                      carries both states through the stretch (from S = 0,
  *                      and from S = I with v read as 0).
  * Shares the chunked form's numeric domain (see wkv7_forward).
@@ -166,8 +167,13 @@ WKV7_API wkv7_status wkv7_forward_summary(int B, int T, int H, int N, wkv7_dtype
  * Forward of one stretch from its entry state s_in (NULL = zeros), after
  * wkv7_forward_summary ran on the SAME inputs with the SAME workspace pointer
  * and size, and nothing wrote the workspace in between (the segment summaries
- * it left there are reused; the results are unspecified otherwise).  With a
- * NULL workspace it is a plain one-pass chunked forward from s_in.
+ * and per-token partial outputs it left there are reused; the results are
+ * unspecified otherwise).  With that workspace it does no chunk work: a
+ * segment's state at token t is S_in M_{<=t} + E_{<=t}, so its output is
+ * y0_t + S_in q_t, where y0 (the output from S = 0) and q_t = M_{<=t} r_t
+ * come from the summary pass; the call chains the segments' entry states
+ * and adds S_in q.  With a NULL workspace it is a plain one-pass chunked
+ * forward from s_in.
  *   y  : [B, T, H, N] of y_dtype, written
  *   sT : [B, H, N, N] fp32 final state of the stretch, or NULL
  */

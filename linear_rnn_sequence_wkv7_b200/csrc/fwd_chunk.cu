@@ -891,7 +891,7 @@ seg_combine_kernel(int nsteps, const float *__restrict__ s0, int s0_eye, const f
     }
 }
 
-// The output of segments 1..nseg-1 from their summary runs: a segment's state
+// The output of segments seg_first..nseg-1 from their summary runs: a segment's state
 // at token t is S_in M_{<=t} + E_{<=t}, so y_t = y0_t + S_in q_t, with y0_t
 // its output from S = 0 and q_t = M_{<=t} r_t the second state's output
 // (both fp32 in y0q = [2][B][T][H][64]).  One CTA of 128 threads per (head,
@@ -904,16 +904,16 @@ constexpr int kFixTokens = 256, kFixTile = 64;
 
 template <typename OutT>
 __global__ void __launch_bounds__(128)
-seg_fixup_kernel(int T, int H, int t_seg, const float *__restrict__ y0q, const float *__restrict__ sin,
-                 long long sin_zstride, OutT *__restrict__ y) {
+seg_fixup_kernel(int T, int H, int t_seg, int seg_first, const float *__restrict__ y0q,
+                 const float *__restrict__ sin, long long sin_zstride, OutT *__restrict__ y) {
     __shared__ __align__(16) float St[kN][kN + 4];    // St[i][i'] = S_in[i'][i]
     __shared__ __align__(16) float Qs[kFixTile][kN + 4];
-    const int head = blockIdx.x, seg = blockIdx.y + 1, tid = threadIdx.x;
+    const int head = blockIdx.x, seg = blockIdx.y + seg_first, tid = threadIdx.x;
     const int bb = head / H, h = head % H;
     const int t_lo = seg * t_seg + kFixTokens * blockIdx.z;
     const int t_hi = min(T, min((seg + 1) * t_seg, t_lo + kFixTokens));
     if (t_lo >= t_hi) return;
-    const float *S = sin + (size_t)(seg - 1) * sin_zstride + (size_t)head * kN * kN;
+    const float *S = sin + (size_t)(seg - seg_first) * sin_zstride + (size_t)head * kN * kN;
     for (int x = tid; x < kN * kN; x += 128) St[x & 63][x >> 6] = S[x];
     const size_t tok_stride = (size_t)H * kN, plane = (size_t)gridDim.x / H * T * tok_stride;
     const size_t base = ((size_t)bb * T * H + h) * kN;
@@ -969,15 +969,18 @@ seg_fixup_kernel(int T, int H, int t_seg, const float *__restrict__ y0q, const f
     }
 }
 
-static cudaError_t launch_fixup(int B, int T, int H, int t_seg, int nseg, wkv7_dtype y_dt, const float *y0q,
-                                const float *sin, long long sin_zstride, void *y, cudaStream_t st) {
-    if (nseg <= 1) return cudaSuccess;
-    const dim3 grid(B * H, nseg - 1, (t_seg + kFixTokens - 1) / kFixTokens);
+// Fix-up of segments seg_first .. nseg - 1, segment k taking its entry state
+// from sin + (k - seg_first) sin_zstride.
+static cudaError_t launch_fixup(int B, int T, int H, int t_seg, int seg_first, int nseg, wkv7_dtype y_dt,
+                                const float *y0q, const float *sin, long long sin_zstride, void *y, cudaStream_t st) {
+    if (nseg <= seg_first) return cudaSuccess;
+    const dim3 grid(B * H, nseg - seg_first, (t_seg + kFixTokens - 1) / kFixTokens);
     if (y_dt == WKV7_F32)
-        seg_fixup_kernel<float><<<grid, 128, 0, st>>>(T, H, t_seg, y0q, sin, sin_zstride, static_cast<float *>(y));
+        seg_fixup_kernel<float>
+            <<<grid, 128, 0, st>>>(T, H, t_seg, seg_first, y0q, sin, sin_zstride, static_cast<float *>(y));
     else
         seg_fixup_kernel<__nv_bfloat16>
-            <<<grid, 128, 0, st>>>(T, H, t_seg, y0q, sin, sin_zstride, static_cast<__nv_bfloat16 *>(y));
+            <<<grid, 128, 0, st>>>(T, H, t_seg, seg_first, y0q, sin, sin_zstride, static_cast<__nv_bfloat16 *>(y));
     return cudaGetLastError();
 }
 
@@ -1087,8 +1090,9 @@ size_t chunk_workspace_bytes(int B, int T, int H, int nseg) {
 
 size_t summary_workspace_bytes(int B, int T, int H, int nseg) {
     if (nseg <= 1) return 0;
-    // E_k, M_k and S_in(k) for every segment
-    return (size_t)3 * nseg * B * H * kN * kN * sizeof(float);
+    // E_k, M_k for every segment, the entry states and the final state, then
+    // y0 and q of every token for the continue's fix-up
+    return (size_t)(3 * nseg + 1) * B * H * kN * kN * sizeof(float) + (size_t)2 * B * T * H * kN * sizeof(float);
 }
 
 // The summary of an empty sequence: E = 0, M = I (one thread per element of both).
@@ -1117,7 +1121,9 @@ cudaError_t fwd_chunk_summary(int B, int T, int H, const void *r, const void *w,
     int t_seg, n;
     seg_split(T, nseg, t_seg, n);
     float *em = static_cast<float *>(workspace);                // E_0..E_{n-1}, M_0..M_{n-1}
-    cudaError_t e = launch_dual(B, T, H, t_seg, n, r, w, k, v, a, b, em, zst, em + n * zst, zst, wait_limit, st);
+    float *y0q = em + (3 * n + 1) * zst;                         // y0, q of every token (for the continue)
+    cudaError_t e = launch_dual(B, T, H, t_seg, n, r, w, k, v, a, b, em, zst, em + n * zst, zst, wait_limit, st,
+                                nullptr, WKV7_F32, nullptr, nullptr, EpiArgs{}, y0q);
     if (e != cudaSuccess) return e;
     e = launch_combine(B, H, n, nullptr, false, em, zst, em + n * zst, zst, summary, 0, st);
     if (e != cudaSuccess) return e;
@@ -1136,10 +1142,15 @@ cudaError_t fwd_chunk_continue(int B, int T, int H, wkv7_dtype y_dt, const void 
     int t_seg, n;
     seg_split(T, nseg, t_seg, n);
     float *em = static_cast<float *>(workspace);
-    float *sin = em + 2 * n * zst;
-    cudaError_t e = launch_combine(B, H, n - 1, s_in, false, em, zst, em + n * zst, zst, sin, zst, st);
+    float *sin = em + 2 * n * zst;                  // entry states of segments 0 .. n - 1, then the final state
+    const float *y0q = em + (3 * n + 1) * zst;      // kept by the summary
+    cudaError_t e = launch_combine(B, H, n, s_in, false, em, zst, em + n * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
-    return launch_chunk(B, T, H, t_seg, n, n, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, n - 1, wait_limit, st);
+    // every segment in fix-up form: y = y0 + S_in q (the summary's dual runs
+    // started every segment from 0 and from I)
+    e = launch_fixup(B, T, H, t_seg, 0, n, y_dt, y0q, sin, zst, y, st);
+    if (e != cudaSuccess || sT == nullptr) return e;
+    return cudaMemcpyAsync(sT, sin + n * zst, zst * sizeof(float), cudaMemcpyDeviceToDevice, st);
 }
 
 // dL/dS before each of nseg consecutive segments, last segment first:
@@ -1184,7 +1195,7 @@ static cudaError_t fwd_chunk_fixup(int B, int T, int H, wkv7_dtype y_dt, const v
     e = launch_combine(B, H, nseg - 1, em, false, em + zst, zst, em + (nseg + 1) * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
     // pass 3: y of segments 1 .. nseg - 1, and the final state
-    e = launch_fixup(B, T, H, t_seg, nseg, y_dt, y0q, sin, zst, y, st);
+    e = launch_fixup(B, T, H, t_seg, 1, nseg, y_dt, y0q, sin, zst, y, st);
     if (e != cudaSuccess || sT == nullptr) return e;
     return cudaMemcpyAsync(sT, sin + (nseg - 1) * zst, zst * sizeof(float), cudaMemcpyDeviceToDevice, st);
 }
