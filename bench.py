@@ -506,7 +506,7 @@ def bench_long(args, dist, peaks, device):
     per = secs / steps
     nbytes = fwd_bytes(B, T, H)
     ach = nbytes / per / 1e9
-    # launches per call: one pass, or summary pass + entry-state scan + output pass
+    # launches per call: one pass, or the dual pass + the entry-state chain + the fix-up
     per_call = 3 if ws_n else 1
     return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
             "ms_per_step": per * 1e3, "steps": steps, "launches": per_call * steps,
