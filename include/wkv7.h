@@ -321,14 +321,17 @@ WKV7_API wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dtype, wkv7_dt
                       const void *r, const void *w, const void *k, const void *v,
                       const void *a, const void *b, float *state, void *y, cudaStream_t stream);
 
-/* Bytes of scratch wkv7_backward needs: per (b, h), the state before every
+/* Bytes of scratch wkv7_backward takes: per (b, h), the state before every
  * 32-token chunk, dL/dS at the end of every chunk, and the final state
  * (fp32, 16 KiB each); for few heads over many tokens also 3 states per
- * segment of the state-gradient sweep (see below).  Depends on the current
- * device's SM count.  The checkpoints are what lets the backward run its
- * chunks in parallel instead of token by token: the method is presented as
- * keeping training parallelisable (RWKV-7 "Goose" with Expressive Dynamic
- * State Evolution, abstract). */
+ * segment of the state-gradient sweep (see below); and every chunk's
+ * transition image (24 KiB per chunk, used for bf16 inputs).  The call also
+ * runs with less, down to this size minus the transition images (dL/dS then
+ * comes from the per-token sweep).  Depends on the current device's SM
+ * count.  The checkpoints are what lets the backward run its chunks in
+ * parallel instead of token by token: the method is presented as keeping
+ * training parallelisable (RWKV-7 "Goose" with Expressive Dynamic State
+ * Evolution, abstract). */
 WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
 
 /*
@@ -338,20 +341,29 @@ WKV7_API size_t wkv7_backward_workspace_size(int B, int T, int H, int N);
  * parallelisable (RWKV-7 "Goose" with Expressive Dynamic State Evolution,
  * abstract), and this call is the reverse-mode derivative of the recurrence
  * taken chunk by chunk.  Three steps: state checkpoints every 32
- * tokens, a reverse sweep of the state gradient that records dL/dS at every
- * chunk end (and ds0), then the input gradients of every chunk independently
- * (the adjoint of the chunked form of the recurrence): on the tensor cores
- * for bf16 inputs (bf16 hi/lo operands, fp32 accumulation), in fp32 on the
- * CUDA cores for fp32 inputs.  When the heads leave most SMs idle the sweep
- * runs as segments side by side: a dual pass per segment (dL/dS from 0 with
- * dy, and the segment's transposed transition product from I), a chain of
- * those for every segment's exit adjoint, and a second pass that records dS.
+ * tokens, dL/dS at every chunk end (and ds0), then the input gradients of
+ * every chunk independently (the adjoint of the chunked form of the
+ * recurrence): on the tensor cores for bf16 inputs (bf16 hi/lo operands, fp32
+ * accumulation), in fp32 on the CUDA cores for fp32 inputs.
+ * dL/dS comes, for bf16 inputs with the full workspace, from the chunks'
+ * transitions: the chunk's state map is affine, S_out = S_in M + E with
+ * y_t = S_in q_t + (terms without S_in), so dS_in = dS_out M^T + dY^T Q, one
+ * tensor-core product per chunk ([M^T; Q] exported by the checkpoint pass).
+ * Otherwise it comes from a reverse sweep of the state gradient, token by
+ * token.  When the heads leave most SMs idle that sweep runs as segments
+ * side by side: a dual pass per segment (dL/dS from 0 with dy, and the
+ * segment's transposed transition product from I), a chain of those for
+ * every segment's exit adjoint, and a second pass that records dS.  A cost
+ * model picks the chain or the sweep; the results agree within the bf16
+ * bound.
  *   r..b, s0         : the forward's inputs (s0 NULL = zeros)
  *   dy               : [B, T, H, N] of in_dtype
  *   dsT              : [B, H, N, N] fp32, or NULL for zeros
  *   dr, dw, dk, dv, da, db : [B, T, H, N] of grad_dtype, overwritten
  *   ds0              : [B, H, N, N] fp32, overwritten (required)
- *   workspace        : wkv7_backward_workspace_size() bytes
+ *   workspace        : wkv7_backward_workspace_size() bytes (at least that
+ *                      size minus the transition images; less is
+ *                      WKV7_ERR_INVALID_ARG)
  * dw is dL/dw for the decay value w itself.
  */
 WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype grad_dtype,
@@ -391,7 +403,10 @@ WKV7_API size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, in
  * wkv7_backward given the states and sT that wkv7_forward_train wrote for the
  * same inputs (s0 is not needed: states[.][.][0] is it).  Two launches: the
  * state-gradient sweep and the chunk gradients.  Same gradients, dtypes and
- * errors as wkv7_backward.
+ * errors as wkv7_backward with its workspace short of the transition images
+ * (bit for bit: dL/dS by the per-token sweep; the saved states carry no
+ * transitions, since this call cannot know whether the forward ran the
+ * chunked form).
  */
 WKV7_API wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_dtype,
                                                wkv7_dtype grad_dtype, const void *r, const void *w,
@@ -409,8 +424,8 @@ WKV7_API wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_
  * backward (an engine plugin whose enqueue path must not call the allocator,
  * or a framework whose memory pool already holds the device's memory).
  *   - Every GPU that loads the library keeps the 32 MiB array until exit.
- *   - Problems whose wkv7_backward_workspace_size() exceeds 32 MiB return
- *     WKV7_ERR_TOO_LARGE and launch nothing.
+ *   - Problems whose wkv7_backward_workspace_size() without the transition
+ *     images exceeds 32 MiB return WKV7_ERR_TOO_LARGE and launch nothing.
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it: make that first call before any
  *     stream capture.

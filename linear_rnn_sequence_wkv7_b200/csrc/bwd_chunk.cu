@@ -774,7 +774,8 @@ static double dstate_launch_ns(long long n, long long steps, int rpt, int lpr, b
 // with eight lanes (those two one-pass only), nseg = 1 or a split into
 // segments of at least two chunks.
 // need_dS: dS at every chunk end is wanted (the backward), else ds0 alone.
-DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, size_t scratch_cap) {
+DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, size_t scratch_cap,
+                       double *est_ns = nullptr) {
     const long long heads = (long long)B * H;
     const int chunks = (T + bwdc::L - 1) / bwdc::L;
     if (sms <= 0) sms = 148;
@@ -807,7 +808,19 @@ DstatePlan dstate_plan(int B, int T, int H, int sms, bool f32, bool need_dS, siz
             }
         }
     }
+    if (est_ns) *est_ns = best_ns;
     return best;
+}
+
+double bwd_dchain_ns(int B, int T, int H, int sms);   // bwd_dchain.cu
+
+// Whether the transition chain (bwd_dchain.cu) beats the per-token sweep for
+// dS at every chunk end, bf16 inputs, the sweep given scratch_cap bytes of
+// scratch.
+bool bwd_use_dchain(int B, int T, int H, int sms, size_t scratch_cap) {
+    double sweep_ns = 0.0;
+    dstate_plan(B, T, H, sms, false, true, scratch_cap, &sweep_ns);
+    return bwd_dchain_ns(B, T, H, sms) < 0.9 * sweep_ns;
 }
 
 // Scratch of the plan dstate_plan picks with room to spare, for either input
@@ -909,12 +922,21 @@ cudaError_t bwd_chunk_grads(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_
     return cudaGetLastError();
 }
 
+cudaError_t bwd_dchain(int B, int T, int H, const void *dy, const uint4 *mq, const float *dsT, float *dS_out,
+                       float *ds0, long long wait_limit, cudaStream_t st);   // bwd_dchain.cu
+
+// dS at every chunk end (the transition chain when the checkpoint pass
+// exported the chunks' transitions mq, bf16 inputs; else the sweep), then the
+// chunk gradients.
 cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r, const void *w,
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
                         void *dw, void *dk, void *dv, void *da, void *db, float *ds0, float *scratch,
-                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st) {
-    cudaError_t e = bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, dS_out, ds0, scratch, scratch_bytes, sms, st);
+                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st,
+                        const uint4 *mq) {
+    cudaError_t e = (mq != nullptr && in_dt == WKV7_BF16)
+                        ? bwd_dchain(B, T, H, dy, mq, dsT, dS_out, ds0, wait_limit, st)
+                        : bwd_dstate(B, T, H, in_dt, r, w, a, b, dy, dsT, dS_out, ds0, scratch, scratch_bytes, sms, st);
     if (e != cudaSuccess) return e;
     return bwd_chunk_grads(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, ckpt, sfin, dS_out, dr, dw, dk, dv, da, db,
                            wait_limit, st);

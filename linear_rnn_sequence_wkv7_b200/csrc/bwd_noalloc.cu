@@ -12,8 +12,10 @@
 // Limits and rules:
 //  - The array holds kNoAllocScratchBytes (32 MiB).  Every GPU that loads the
 //    library keeps it resident until the process exits.  A problem whose
-//    scratch need (wkv7_backward_workspace_size) exceeds it is rejected with
-//    WKV7_ERR_TOO_LARGE before anything is launched.
+//    minimum scratch (wkv7_backward_workspace_size without the chunks'
+//    transition images) exceeds it is rejected with WKV7_ERR_TOO_LARGE before
+//    anything is launched; one whose full size fits also takes the transition
+//    chain for dS.
 //  - Host code cannot pass the array's name to a kernel (on the host it is
 //    only a stand-in symbol).  The first call on each device looks up the
 //    array's device address with cudaGetSymbolAddress, with that device
@@ -63,7 +65,8 @@ extern "C" wkv7_status wkv7_backward_noalloc(int B, int T, int H, int N, wkv7_dt
                                              const void *dy, const float *dsT, void *dr, void *dw, void *dk,
                                              void *dv, void *da, void *db, float *ds0, cudaStream_t stream) {
     using namespace wkv7;
-    if (wkv7_backward_workspace_size(B, T, H, N) > kNoAllocScratchBytes) return WKV7_ERR_TOO_LARGE;
+    if (B > 0 && T > 0 && H > 0 && N == kN && bwd_workspace_min(B, T, H) > kNoAllocScratchBytes)
+        return WKV7_ERR_TOO_LARGE;
     void *scratch = nullptr;
     const wkv7_status s = noalloc_scratch(&scratch);
     if (s != WKV7_OK) return s;

@@ -11,6 +11,13 @@ namespace wkv7 {
 
 constexpr int kN = 64;  // head size the kernels implement
 
+// A 32-token chunk's transition [M^T; Q] (S_out = S_in M + E, y_t = S_in q_t +
+// terms without S_in; row m of M^T is column m of M, row t of Q is q_t) as the
+// checkpoint pass of the chunked forward exports it for the backward: the bf16
+// hi image of a 96 x 64 tile in core-matrix layout (rows m = 0..63, then t),
+// then the lo image; counted in 16-byte words.
+constexpr int kMqChunkVec = 2 * 96 * kN * 2 / 16;
+
 // Sticky device-side status word (one per device): kernels that detect a
 // bounded wait running out or an out-of-domain chunk set it with atomicMax;
 // wkv7_get_device_status reads and clears it.  Defined here because the

@@ -136,14 +136,16 @@ constexpr uint32_t BAR_READY = 2, BAR_DONE = 6;
 // state round R4 and its read-out are done twice.  No y.  It needs a second S
 // operand and 64 more TMEM columns, so these CTAs run one per SM.
 // EPI: the time-mix output epilogue (EpiArgs) replaces the y store.
-template <typename OutT, bool DUAL, bool EPI>
+// MQX: the checkpoint pass also exports every chunk's transition [M^T; Q] to mq.
+template <typename OutT, bool DUAL, bool EPI, bool MQX = false>
 __global__ void __launch_bounds__(chunk::NT, DUAL ? 1 : 2)
 fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *__restrict__ r,
                  const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
                  const __nv_bfloat16 *__restrict__ b, const float *s0, long long s0_zstride, OutT *__restrict__ y,
                  float *sT, long long sT_zstride, int st_only_z, long long wait_limit, float *ckpt,
-                 float *m_out, long long m_zstride, int seg0, int first_out, EpiArgs epi, float *y0q) {
+                 float *m_out, long long m_zstride, int seg0, int first_out, EpiArgs epi, float *y0q,
+                 uint4 *mq) {
     using namespace chunk;
     using namespace umma;
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -545,7 +547,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             store8_split(sm + WU_HI, sm + WU_LO, cm_off(rho, 16 * hc + 8, L), x + 8);
         };
 
-        auto P3 = [&]() {                         // rows of [M^T; Q] -> TMEM A operand of R4
+        auto P3 = [&](int c) {                    // rows of [M^T; Q] -> TMEM A operand of R4
             if (q4 == 3) return;
             uint32_t r0[16], r1[16];
             tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc, r0);
@@ -598,6 +600,22 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             }
             tmem_st16(tmem + quad + COL_MQ + 16 * hc, ph);
             tmem_st16(tmem + quad + COL_MQ + 32 + 16 * hc, pl);
+            if (MQX && out_run) {
+                // optional chunk transitions, written with the checkpoints: the
+                // same hi / lo pairs as row rho of chunk c's image (kMqChunkVec
+                // 16-byte words per chunk, indexed like ckpt); the address is
+                // formed here from the launch parameters so that it holds no
+                // register over the rest of the chunk
+                uint4 *dst = mq + ((((size_t)blockIdx.y * H + blockIdx.x) * ((T_total + L - 1) / L) +
+                                    (size_t)(seg0 + blockIdx.z % nseg) * (t_seg / L) + c) *
+                                   kMqChunkVec);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t o = cm_off(rho, 32 * hc + 8 * u, kN) >> 4;
+                    dst[o] = make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
+                    dst[kMqChunkVec / 2 + o] = make_uint4(pl[4 * u], pl[4 * u + 1], pl[4 * u + 2], pl[4 * u + 3]);
+                }
+            }
             tmem_st_wait();
         };
 
@@ -749,7 +767,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             ready_arrive(2);                               // R3(c)
             done_wait(2, c);
             issue_v(c + 1);                                // v(c) is no longer read
-            P3();
+            P3(c);
             ready_arrive(3);                               // R4(c)
             if (c + 1 < nchunks) {                         // next chunk's operands under R4(c)
                 cp_async_wait<1>();                        // tile c+1 is in place
@@ -783,26 +801,29 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
                                 const void *w, const void *k, const void *v, const void *a, const void *b,
                                 const float *s0, long long s0_zstride, void *y, float *sT, long long sT_zstride,
                                 int st_only_z, long long wait_limit, cudaStream_t st, float *ckpt = nullptr,
-                                int seg0 = 0, EpiArgs epi = EpiArgs{}) {
+                                int seg0 = 0, EpiArgs epi = EpiArgs{}, uint4 *mq = nullptr) {
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES;
-#define WKV7_CHUNK_LAUNCH(O, E)                                                                               \
+#define WKV7_CHUNK_LAUNCH(O, E, X)                                                                            \
     do {                                                                                                      \
-        auto kern = fwd_chunk_kernel<O, false, E>;                                                            \
+        auto kern = fwd_chunk_kernel<O, false, E, X>;                                                         \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
         if (e != cudaSuccess) return e;                                                                       \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nseg, (const __nv_bfloat16 *)r, (const __nv_bfloat16 *)w, \
                                             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,               \
                                             (const __nv_bfloat16 *)a, (const __nv_bfloat16 *)b, s0, s0_zstride,   \
                                             (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0,  \
-                                            seg0, 0, epi, nullptr);                                           \
+                                            seg0, 0, epi, nullptr, mq);                                       \
     } while (0)
-    if (epi.rho) {
-        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, true);
-        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, true);
+    if (mq) {                                     // the backward's checkpoint pass (no y, no epilogue)
+        if (epi.rho || y) return cudaErrorInvalidValue;
+        WKV7_CHUNK_LAUNCH(__nv_bfloat16, false, true);
+    } else if (epi.rho) {
+        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, true, false);
+        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, true, false);
     } else {
-        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, false);
-        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, false);
+        if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, false, false);
+        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, false, false);
     }
 #undef WKV7_CHUNK_LAUNCH
     return cudaGetLastError();
@@ -816,28 +837,32 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
                                const void *v, const void *a, const void *b, float *e_out, long long e_zstride,
                                float *m_out, long long m_zstride, long long wait_limit, cudaStream_t st,
                                void *y = nullptr, wkv7_dtype y_dt = WKV7_F32, const float *s0 = nullptr,
-                               float *ckpt = nullptr, EpiArgs epi = EpiArgs{}, float *y0q = nullptr) {
+                               float *ckpt = nullptr, EpiArgs epi = EpiArgs{}, float *y0q = nullptr,
+                               uint4 *mq = nullptr) {
     static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
     dim3 grid(H, B, nz);
     const size_t smem = chunk::SMEM_BYTES_DUAL;
     const int first_out = (y != nullptr || ckpt != nullptr) ? 1 : 0;
     using bf = __nv_bfloat16;
-#define WKV7_DUAL_LAUNCH(O, E)                                                                                 \
+#define WKV7_DUAL_LAUNCH(O, E, X)                                                                              \
     do {                                                                                                       \
-        auto kern = fwd_chunk_kernel<O, true, E>;                                                              \
+        auto kern = fwd_chunk_kernel<O, true, E, X>;                                                           \
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
         if (e != cudaSuccess) return e;                                                                        \
         kern<<<grid, chunk::NT, smem, st>>>(T, H, t_seg, nz, (const bf *)r, (const bf *)w, (const bf *)k,      \
                                             (const bf *)v, (const bf *)a, (const bf *)b, s0, 0, (O *)y, e_out, \
                                             e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out,   \
-                                            epi, y0q);                                                         \
+                                            epi, y0q, mq);                                                     \
     } while (0)
-    if (epi.rho && first_out) {
-        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, true);
-        else WKV7_DUAL_LAUNCH(float, true);
+    if (mq) {                                     // the backward's segmented checkpoint pass
+        if (epi.rho || y) return cudaErrorInvalidValue;
+        WKV7_DUAL_LAUNCH(bf, false, true);
+    } else if (epi.rho && first_out) {
+        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, true, false);
+        else WKV7_DUAL_LAUNCH(float, true, false);
     } else {
-        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, false);
-        else WKV7_DUAL_LAUNCH(float, false);
+        if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, false, false);
+        else WKV7_DUAL_LAUNCH(float, false, false);
     }
 #undef WKV7_DUAL_LAUNCH
     return cudaGetLastError();
@@ -1203,17 +1228,17 @@ static cudaError_t fwd_chunk_fixup(int B, int T, int H, wkv7_dtype y_dt, const v
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
-                      const EpiArgs &epi, bool fixup) {
+                      const EpiArgs &epi, bool fixup, uint4 *mq) {
     if (fixup && nseg > 1 && ckpt == nullptr && epi.rho == nullptr && y != nullptr)
         return fwd_chunk_fixup(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace, wait_limit, st);
     if (nseg <= 1)
         return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt, 0,
-                            epi);
+                            epi, mq);
     int t_seg;
     seg_split(T, nseg, t_seg, nseg);
     if (nseg <= 1)
         return launch_chunk(B, T, H, T, 1, 1, y_dt, r, w, k, v, a, b, s0, 0, y, sT, 0, -1, wait_limit, st, ckpt, 0,
-                            epi);
+                            epi, mq);
     const long long zst = (long long)B * H * kN * kN;
     float *em = static_cast<float *>(workspace);                // [2 (nseg-1)][B][H][64][64]
     float *sin = em + (size_t)2 * (nseg - 1) * zst;             // [nseg - 1][B][H][64][64]
@@ -1221,14 +1246,14 @@ cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const
     // from s0 and writes its y (and checkpoints): its E is the entry state of
     // segment 1.  Segments k >= 1 give E_k (from 0) and M_k (from I, v = 0).
     cudaError_t e = launch_dual(B, T, H, t_seg, nseg - 1, r, w, k, v, a, b, em, zst, em + (size_t)(nseg - 1) * zst,
-                                zst, wait_limit, st, y, y_dt, s0, ckpt, epi);
+                                zst, wait_limit, st, y, y_dt, s0, ckpt, epi, nullptr, mq);
     if (e != cudaSuccess) return e;
     // pass 2: entry states of segments 1..nseg-1, from segment 1's
     e = launch_combine(B, H, nseg - 2, em, false, em + zst, zst, em + (size_t)nseg * zst, zst, sin, zst, st);
     if (e != cudaSuccess) return e;
     // pass 3: segments 1..nseg-1 from their true entry states; the last one writes sT
     return launch_chunk(B, T, H, t_seg, nseg - 1, nseg - 1, y_dt, r, w, k, v, a, b, sin, zst, y, sT, 0, nseg - 2,
-                        wait_limit, st, ckpt, 1, epi);
+                        wait_limit, st, ckpt, 1, epi, mq);
 }
 
 }  // namespace wkv7

@@ -6,6 +6,7 @@
 #include "step.cu"
 #include "bwd_chunk.cu"
 #include "bwd_chunk_tc.cu"
+#include "bwd_dchain.cu"
 #include "fwd_chunk.cu"
 #include "bwd_noalloc.cu"
 #include "fwd_host.cu"

@@ -24,8 +24,11 @@ cudaError_t bwd_chunked(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype g_dt, 
                         const void *k, const void *v, const void *a, const void *b, const void *dy,
                         const float *dsT, const float *ckpt, const float *sfin, float *dS_out, void *dr,
                         void *dw, void *dk, void *dv, void *da, void *db, float *ds0, float *scratch,
-                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st);
+                        size_t scratch_bytes, int sms, long long wait_limit, cudaStream_t st,
+                        const uint4 *mq = nullptr);
 size_t bwd_chunk_ckpt_bytes(int B, int T, int H);
+size_t bwd_mq_bytes(int B, int T, int H);
+bool bwd_use_dchain(int B, int T, int H, int sms, size_t scratch_cap);
 cudaError_t bwd_dstate(int B, int T, int H, wkv7_dtype in_dt, const void *r, const void *w, const void *a,
                        const void *b, const void *dy, const float *dsT, float *dS_out, float *ds0, float *scratch,
                        size_t scratch_bytes, int sms, cudaStream_t st);
@@ -35,7 +38,7 @@ cudaError_t compose_adjoints(int B, int H, int nseg, const float *dsT, const flo
 cudaError_t fwd_chunk(int B, int T, int H, wkv7_dtype y_dt, const void *r, const void *w, const void *k,
                       const void *v, const void *a, const void *b, const float *s0, void *y, float *sT,
                       int nseg, void *workspace, long long wait_limit, cudaStream_t st, float *ckpt,
-                      const EpiArgs &epi = EpiArgs{}, bool fixup = false);
+                      const EpiArgs &epi = EpiArgs{}, bool fixup = false, uint4 *mq = nullptr);
 int chunk_segments_fixup(int B, int T, int H, int sm_count);
 size_t chunk_fixup_workspace_bytes(int B, int T, int H, int nseg);
 cudaError_t fwd_seq_train(int B, int T, int H, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r, const void *w,
@@ -122,6 +125,14 @@ size_t bwd_scratch_bytes(int B, int T, int H) {
                     round_up(dstate_scratch_for(B, T, H, sms, true)));
 }
 size_t state_bytes(int B, int H) { return (size_t)B * H * kN * kN * sizeof(float); }
+
+// wkv7_backward's workspace without the chunks' transition images: the state
+// before every chunk, dL/dS at every chunk end, the final state and the
+// segmented passes' scratch.  With the images too (wkv7_backward_workspace_size)
+// dS can come from the transition chain.
+size_t bwd_workspace_min(int B, int T, int H) {
+    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H)) + bwd_scratch_bytes(B, T, H);
+}
 
 }  // namespace
 }  // namespace wkv7
@@ -350,8 +361,8 @@ wkv7_status wkv7_step(int B, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, co
 size_t wkv7_backward_workspace_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
     // state before every chunk, dL/dS at every chunk end, the final state, the
-    // segmented passes' scratch
-    return 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H)) + bwd_scratch_bytes(B, T, H);
+    // segmented passes' scratch, the chunks' transition images
+    return bwd_workspace_min(B, T, H) + round_up(bwd_mq_bytes(B, T, H));
 }
 
 wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype g_dt, const void *r,
@@ -368,16 +379,23 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     for (const void *p : {r, w, k, v, a, b, dy, (const void *)dr, (const void *)dw, (const void *)dk,
                           (const void *)dv, (const void *)da, (const void *)db})
         if (!ptr_ok(p)) return WKV7_ERR_INVALID_ARG;
-    const size_t need = wkv7_backward_workspace_size(B, T, H, N);
-    if (workspace_bytes < need || !ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
+    if (workspace_bytes < bwd_workspace_min(B, T, H) || !ptr_ok(workspace)) return WKV7_ERR_INVALID_ARG;
     char *ws = static_cast<char *>(workspace);
     float *ckpt = reinterpret_cast<float *>(ws);
     float *dSo = reinterpret_cast<float *>(ws + round_up(bwd_ckpt_bytes(B, T, H)));
     float *sfin = reinterpret_cast<float *>(ws + 2 * round_up(bwd_ckpt_bytes(B, T, H)));
-    const size_t used = 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
+    size_t used = 2 * round_up(bwd_ckpt_bytes(B, T, H)) + round_up(state_bytes(B, H));
+    const int sms = current_sm_count();
+    // the chunks' transitions for the dS chain: bf16 inputs, room for them
+    // next to the scratch, and the chain estimated faster than the sweep
+    uint4 *mq = nullptr;
+    if (in_dt == WKV7_BF16 && workspace_bytes >= bwd_workspace_min(B, T, H) + round_up(bwd_mq_bytes(B, T, H)) &&
+        bwd_use_dchain(B, T, H, sms, workspace_bytes - used - round_up(bwd_mq_bytes(B, T, H)))) {
+        mq = reinterpret_cast<uint4 *>(ws + used);
+        used += round_up(bwd_mq_bytes(B, T, H));
+    }
     char *scratch = ws + used;
     const size_t scratch_bytes = workspace_bytes - used;
-    const int sms = current_sm_count();
     // checkpoints: the chunked tensor-core forward without y for bf16 inputs
     // (its chunk is the backward's; sequence segments side by side when the
     // heads are few), the sequential scan for fp32 inputs
@@ -387,7 +405,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
         const int want = bwd_ckpt_segments(B, T, H, sms);
         const int nseg = (want > 1 && scratch_bytes >= chunk_workspace_bytes(B, T, H, want)) ? want : 1;
         e = fwd_chunk(B, T, H, WKV7_BF16, r, w, k, v, a, b, s0, nullptr, sfin, nseg, scratch,
-                      lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt);
+                      lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, EpiArgs{}, false, mq);
     } else {
         e = fwd_checkpoints(B, T, H, in_dt, r, w, k, v, a, b, s0, ckpt, kBwdChunk, sfin,
                             lim > 0 ? lim : kDefaultWaitCycles, stream);
@@ -395,7 +413,7 @@ wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dty
     if (e != cudaSuccess) return WKV7_ERR_CUDA;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, ckpt, sfin, dSo, dr, dw, dk,
                                  dv, da, db, ds0, reinterpret_cast<float *>(scratch), scratch_bytes, sms,
-                                 lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                 lim > 0 ? lim : kDefaultWaitCycles, stream, mq));
 }
 
 size_t wkv7_state_gradient_workspace_size(int B, int T, int H, int N) {

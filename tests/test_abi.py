@@ -48,8 +48,9 @@ def test_version_and_status_strings(lib):
 def test_workspace_sizes(lib):
     assert lib.wkv7_forward_workspace_size(1, 64, 2, 64, wkv7.F32, wkv7.ALGO_SEQ, 0) == 0
     ws = lib.wkv7_backward_workspace_size(8, 4096, 32, 64)
-    # per head: the state before every 32-token chunk, dL/dS at every chunk end, the final state
-    assert ws >= 8 * 32 * (2 * (4096 // 32) + 1) * 64 * 64 * 4
+    # per head: the state before every 32-token chunk, dL/dS at every chunk end, the final state,
+    # and every chunk's transition image ([M^T; Q], bf16 hi and lo: 24 KiB)
+    assert ws >= 8 * 32 * ((2 * (4096 // 32) + 1) * 64 * 64 * 4 + (4096 // 32) * 24576)
     assert lib.wkv7_backward_workspace_size(0, 10, 1, 64) == 0
 
 

@@ -185,6 +185,54 @@ def test_training_workload_sampled_heads(cuda_device):
         assert_close(g, r, TAU_BF16, name)
 
 
+def _transition_bytes(B, T, H):
+    """Bytes of the chunks' transition images ([M^T; Q] per 32-token chunk,
+    bf16 hi and lo: 24 KiB) that the backward's workspace holds on top of its
+    minimum."""
+    return B * H * ((T + 31) // 32) * 24576
+
+
+def _kernel_names(fn):
+    """Names of the CUDA kernels fn launches (empty when the profiler
+    records no device activity on this build)."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return {e.name for e in prof.events()}
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 40, 3), (2, 333, 3), (1, 4096, 40)])
+def test_bf16_dS_by_transition_chain_and_by_sweep(cuda_device, B, T, H):
+    """With the full workspace the checkpoint pass exports every chunk's
+    transition and dS at the chunk ends comes from the tensor-core chain
+    dS_in = dS_out M^T + dY^T Q; a workspace without room for the images takes
+    the per-token sweep.  Both vs the oracle (sampled heads for the larger
+    case), and the kernels each one launches."""
+    d = _case(B, T, H, 480 + T, "bf16")
+    full = wkv7.backward_workspace_size(B, T, H, 64)
+    heads = None if H <= 3 else [0, 17, 39]
+    ref = _ref(d, heads=heads)
+    args = [to_dev(d[n]) for n in inputs.INPUT_NAMES]
+    s0, dy, dsT = to_dev(d["s0"]), to_dev(d["dy"]), to_dev(d["dsT"])
+    for ws, kernel in ((full, "bwd_dchain_kernel"), (full - _transition_bytes(B, T, H), "bwd_dstate_kernel")):
+        buf = torch.empty(ws, dtype=torch.uint8, device="cuda")
+        out = []
+        names = _kernel_names(lambda: out.append(wkv7.backward(*args, s0, dy, dsT, workspace=buf)))
+        assert wkv7.last_status() == wkv7.OK
+        if names:
+            assert any(kernel in n for n in names), (ws, sorted(names))
+        got = out[0]
+        if heads is not None:
+            got = [x[:, :, heads] for x in got[:6]] + [got[6][:, heads]]
+        for name, g, r in zip(GRAD_NAMES, [to_f64(x) for x in got], ref):
+            assert_close(g, r, TAU_BF16, f"{name} ({kernel})")
+    # below the minimum the call is rejected before any launch
+    buf = torch.empty(full - _transition_bytes(B, T, H) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError):
+        wkv7.backward(*args, s0, dy, dsT, workspace=buf)
+
+
 def test_bf16_wait_timeout_reports_and_recovers(cuda_device):
     """Device-side waits forced to run out (limit 1 cycle): the backward's
     tensor-core kernels report WKV7_ERR_TIMEOUT without a fault, and the next
