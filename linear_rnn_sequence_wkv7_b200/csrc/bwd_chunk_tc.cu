@@ -100,6 +100,11 @@ constexpr uint32_t SMEM_BYTES = CPART + 8 * 64 * 4;
 // chunk into the halves of VYZ that nothing reads before P3
 constexpr uint32_t ST_SIN = SGD_HI, ST_DS = SGD_LO;
 constexpr uint32_t ST_SOUT0 = VYZ_HI + 8192, ST_SOUT1 = VYZ_LO + 8192;
+// A staged state row (64 floats, 16 chunks of 16 bytes) keeps chunk g at
+// position g ^ (row % 8): the readers take four chunks of 8 rows per warp,
+// which then fall on distinct banks (unswizzled, the 256-byte rows put all 8
+// rows on the same banks).
+__device__ __forceinline__ uint32_t st_off(int row, int g) { return (uint32_t)(row * 256 + ((g ^ (row & 7)) << 4)); }
 
 constexpr uint32_t BAR_READY = 2, BAR_DONE = 7;      // named barriers 2-6, 7-11
 constexpr long long kDrainCycles = 200000000LL;
@@ -200,8 +205,8 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
     // S_out of a chunk into ST_SOUT0 / ST_SOUT1 (compute threads, 4 x 16 B each)
     auto issue_sout = [&](int id) {
         const float *src = s_out_of(id);
-        for (int x = tid; x < 1024; x += NC)
-            cp_async16(sm + (x < 512 ? ST_SOUT0 : ST_SOUT1) + 16 * (x & 511), src + 4 * x);
+        for (int x = tid; x < 1024; x += NC)   // chunk x: row x / 16, chunk x % 16
+            cp_async16(sm + (x < 512 ? ST_SOUT0 : ST_SOUT1) + st_off((x >> 4) & 31, x & 15), src + 4 * x);
         cp_async_commit();
     };
     // S_in and dS of a chunk into ST_SIN / ST_DS (compute threads, 8 x 16 B each)
@@ -210,7 +215,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             for (int x = tid; x < 2048; x += NC) {
                 const int which = x >> 10, o4 = 4 * (x & 1023);
                 const float *src = (which ? dS_out : ckpt) + (size_t)id * kN * kN + o4;
-                cp_async16(sm + (which ? ST_DS : ST_SIN) + 4 * o4, src);
+                cp_async16(sm + (which ? ST_DS : ST_SIN) + st_off(o4 >> 6, (o4 & 63) >> 2), src);
             }
         }
         cp_async_commit();
@@ -409,12 +414,11 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             {
                 const int i = tid >> 2, c0 = 16 * (tid & 3);
                 float sg[16], dsv[16];
-                const float *sin_s = reinterpret_cast<const float *>(sm + ST_SIN) + i * kN + c0;
-                const float *ds_s = reinterpret_cast<const float *>(sm + ST_DS) + i * kN + c0;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 s4 = *reinterpret_cast<const float4 *>(sin_s + 4 * u);
-                    const float4 d4 = *reinterpret_cast<const float4 *>(ds_s + 4 * u);
+                    const uint32_t so4 = st_off(i, (c0 >> 2) + u);
+                    const float4 s4 = *reinterpret_cast<const float4 *>(sm + ST_SIN + so4);
+                    const float4 d4 = *reinterpret_cast<const float4 *>(sm + ST_DS + so4);
                     const int j = c0 + 4 * u;
                     sg[4 * u] = s4.x * psm[j]; sg[4 * u + 1] = s4.y * psm[j + 1];
                     sg[4 * u + 2] = s4.z * psm[j + 2]; sg[4 * u + 3] = s4.w * psm[j + 3];
@@ -429,10 +433,10 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 // the chunk's last token also scales S_out: q_{Lc-1} += sum_i S_out dS
                 // (the 8 rows of a warp summed by shuffles, then per-warp partial sums)
                 float cs[16];
-                const float *so = reinterpret_cast<const float *>(sm + (i < 32 ? ST_SOUT0 : ST_SOUT1)) + (i & 31) * kN + c0;
+                const uint32_t so = i < 32 ? ST_SOUT0 : ST_SOUT1;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 s4 = *reinterpret_cast<const float4 *>(so + 4 * u);
+                    const float4 s4 = *reinterpret_cast<const float4 *>(sm + so + st_off(i & 31, (c0 >> 2) + u));
                     cs[4 * u] = s4.x * dsv[4 * u]; cs[4 * u + 1] = s4.y * dsv[4 * u + 1];
                     cs[4 * u + 2] = s4.z * dsv[4 * u + 2]; cs[4 * u + 3] = s4.w * dsv[4 * u + 3];
                 }
