@@ -34,8 +34,11 @@
 // the operands, invert the 32 x 32 unit lower triangular I - L_ab by 16 x 16
 // blocks, move results between rounds and finish the gradients.
 //
-// A persistent grid, one CTA per SM walking the chunks: warps 0-7 compute,
-// warp 8 issues the tensor-core rounds; hand-offs through named barriers
+// A persistent grid, one CTA per SM walking the chunks: warps 0-15 compute
+// (four per TMEM lane quadrant, each taking 16 of an accumulator's columns:
+// the chunk's phases are short dependent sequences, and two warps per
+// scheduler left most issue slots idle), warp 16 issues the tensor-core
+// rounds; hand-offs through named barriers
 // (ready: compute -> issuer, done: issuer -> compute), every wait of the issuer
 // bounded.  The next chunk's token tiles arrive by cp.async into the raw tile
 // buffer (read only in the first phase), issued while the compute warps wait
@@ -49,7 +52,8 @@ namespace wkv7 {
 namespace bwtc {
 
 constexpr int L = 32;
-constexpr int NC = 256, NT = NC + 32;
+constexpr int NCW = 16;                  // compute warps: four per TMEM lane quadrant
+constexpr int NC = 32 * NCW, NT = NC + 32;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns
 constexpr uint32_t CA = 0;       // round A (128), later round D's dL block (128)
@@ -86,13 +90,13 @@ constexpr uint32_t X1C_HI = VYZ_HI, X1C_LO = VYZ_LO;             // [64][128]: r
 // after round E: fp32 scratch of the q and dw sums
 constexpr int LDQ = 68;
 constexpr uint32_t CQ = VYZ_HI;                       // fp32 [4][32][68]: q terms of dr, da, db, dk
-constexpr uint32_t DWTOT = CQ + 4 * 32 * LDQ * 4;     // fp32 [4][64]: token-block sums of q
-constexpr uint32_t GSTG = DWTOT + 4 * 64 * 4;         // the four gradient tiles, rows padded by 16 B (<= 34816 B)
+constexpr uint32_t DWTOT = CQ + 4 * 32 * LDQ * 4;     // fp32 [8][64]: token-block sums of q
+constexpr uint32_t GSTG = DWTOT + 8 * 64 * 4;         // the four gradient tiles, rows padded by 16 B (<= 34816 B)
 static_assert(GSTG + 4 * 32 * (64 * 4 + 16) <= RAW, "gradient staging ends before the token tiles");
 constexpr uint32_t BAR = ZSM + 1024;                  // 6 mbarriers: rounds A..E, round E's first half
 constexpr uint32_t TMEM_SLOT = BAR + 48;
 constexpr uint32_t FLAG = BAR + 52;
-constexpr uint32_t CPART = BAR + 64;                  // fp32 [8][64]: per-warp sums of S_out dS (P0b -> P5)
+constexpr uint32_t CPART = BAR + 64;                  // fp32 [8][64]: sums of S_out dS per 8 rows (P0b -> P5)
 constexpr uint32_t SMEM_BYTES = CPART + 8 * 64 * 4;
 // staged states (fp32, row-major) arriving by cp.async: the chunk's S_in and
 // dS into the [SG; dS] tiles' space, issued under the previous chunk's round
@@ -118,13 +122,6 @@ __device__ __forceinline__ void csync() { umma::named_sync(1, NC); }
 
 __device__ __forceinline__ void bwtc_prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// store one value as bf16 hi / lo into two tiles at byte offset off
-__device__ __forceinline__ void bwtc_put1(unsigned char *sm, uint32_t hi, uint32_t lo, uint32_t off, float x) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    *reinterpret_cast<__nv_bfloat16 *>(sm + hi + off) = h;
-    *reinterpret_cast<__nv_bfloat16 *>(sm + lo + off) = __float2bfloat16_rn(x - __bfloat162float(h));
 }
 
 // 16 fp32 values -> 8 bf16 pairs (hi) and 8 (lo), packed per 32-bit word (even index in the low half)
@@ -174,7 +171,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
     // channels 8 (tid % 8) ..).  Rows past the end are no-op tokens (w = 1,
     // the rest 0), written directly.
     auto issue_tiles = [&](int id) {
-        if (id < total) {
+        if (id < total && tid < 256) {
             const int t = tid >> 3, ch = tid & 7;
             unsigned char *dst = sm + RAW + (t * RAWP + 8 * ch) * 2;
             constexpr uint32_t TEN = L * RAWP * 2;           // bytes per tensor tile
@@ -202,14 +199,14 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
     auto s_out_of = [&](int id) {
         return (id % nck) + 1 < nck ? ckpt + (size_t)(id + 1) * kN * kN : sfin + (size_t)(id / nck) * kN * kN;
     };
-    // S_out of a chunk into ST_SOUT0 / ST_SOUT1 (compute threads, 4 x 16 B each)
+    // S_out of a chunk into ST_SOUT0 / ST_SOUT1 (compute threads, 2 x 16 B each)
     auto issue_sout = [&](int id) {
         const float *src = s_out_of(id);
         for (int x = tid; x < 1024; x += NC)   // chunk x: row x / 16, chunk x % 16
             cp_async16(sm + (x < 512 ? ST_SOUT0 : ST_SOUT1) + st_off((x >> 4) & 31, x & 15), src + 4 * x);
         cp_async_commit();
     };
-    // S_in and dS of a chunk into ST_SIN / ST_DS (compute threads, 8 x 16 B each)
+    // S_in and dS of a chunk into ST_SIN / ST_DS (compute threads, 4 x 16 B each)
     auto issue_states = [&](int id) {
         if (id < total) {
             for (int x = tid; x < 2048; x += NC) {
@@ -231,7 +228,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         for (int rd = 0; rd < 6; ++rd) mbar_init(done_bar(rd), 1);
         *abort_flag = 0;
     }
-    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
+    if (warp == NCW) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if (tid < NC) {
         issue_tiles(blockIdx.x);
         issue_states(blockIdx.x);
@@ -247,7 +244,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
     fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + TMEM_SLOT);
 
-    if (warp == 8) {
+    if (warp == NCW) {
         // ================= MMA issuer =================
         const uint32_t id_a = idesc_bf16(128, 128, 0, 0);
         const uint32_t id_b1 = idesc_bf16(128, 96, 0, 0);
@@ -315,7 +312,9 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         __syncwarp();
     } else {
         // ================= compute warps =================
-        const int q4 = warp & 3, hc = warp >> 2;     // TMEM lane quadrant, column half
+        // TMEM lane quadrant, column half, and which half of that half (the
+        // four warps of a quadrant split an accumulator's columns)
+        const int q4 = warp & 3, hc = (warp >> 2) & 1, part = warp >> 3;
         const uint32_t quad = (uint32_t)(32 * q4) << 16;
         auto ready_arrive = [&](int rd) {
             fence_smem_to_async();
@@ -326,18 +325,6 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             named_sync(BAR_DONE + rd, NT);
             fence_after_sync();
         };
-        // 32 consecutive accumulator columns of this thread's lane
-        auto tld32 = [&](uint32_t col, float *x) {
-            uint32_t r0[16], r1[16];
-            tmem_ld16_nowait(tmem + quad + col, r0);
-            tmem_ld16_nowait(tmem + quad + col + 16, r1);
-            tmem_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                x[e] = __uint_as_float(r0[e]);
-                x[16 + e] = __uint_as_float(r1[e]);
-            }
-        };
         float *psm = reinterpret_cast<float *>(sm + PSM);
         for (int id = blockIdx.x; id < total; id += gridDim.x) {
             const int Lc = chunk_len(id);
@@ -347,17 +334,17 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             // zero the lo copy of dY in VYZ (rows 0-31, columns 64-127; dY is
             // exact), which round D reads; columns 0-63 of VYZ feed only
             // accumulator lanes that are never read, and rows 32-63 take dZ
-            {
-                const int t = tid >> 3, ch = tid & 7;
+            if (tid < 256) {                             // lane -> row: a quarter-warp fills one core matrix
+                const int t = tid & 31, ch = tid >> 5;
                 *reinterpret_cast<uint4 *>(sm + VYZ_LO + cm_off(t, 64 + 8 * ch, 128)) = make_uint4(0, 0, 0, 0);
             }
             cp_async_wait<1>();                      // this chunk's token tiles, S_in and dS (not yet S_out)
             csync();
-            // ---- P0a: suffix decay products and the decayed operands (warp -> 8
-            //      channels, lane -> token) ----
-            {
+            // ---- P0a: suffix decay products and the decayed operands (warps 0-7:
+            //      warp -> 8 channels, lane -> token; 16-byte accesses, so that a
+            //      quarter-warp's 8 tokens fall on distinct banks) ----
+            if (warp < 8) {
                 const int g = warp, t = lane;
-                float wv[8], rv[8], kv[8], av[8], bv[8];
                 auto ld8 = [&](int ten, float *o) {
                     const uint4 u = *reinterpret_cast<const uint4 *>(sm + RAW + ((ten * L + t) * RAWP + 8 * g) * 2);
                     const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
@@ -367,10 +354,8 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                         o[2 * q + 1] = __uint_as_float(uu[q] & 0xffff0000u);
                     }
                 };
-                ld8(TW, wv); ld8(TR, rv); ld8(TK, kv); ld8(TA, av); ld8(TB, bv);
                 float inc[8];                            // p_t = prod_{m >= t} w_m
-#pragma unroll
-                for (int e = 0; e < 8; ++e) inc[e] = wv[e];
+                ld8(TW, inc);
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1)
 #pragma unroll
@@ -384,21 +369,33 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     *reinterpret_cast<float4 *>(psm + L * LDP + 8 * g) = make_float4(1.f, 1.f, 1.f, 1.f);
                     *reinterpret_cast<float4 *>(psm + L * LDP + 8 * g + 4) = make_float4(1.f, 1.f, 1.f, 1.f);
                 }
-                float xa[8], xr[8], xb[8], xk[8];
+                float nxt[8];                            // p_{t+1}
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float n1 = __shfl_down_sync(0xffffffffu, inc[e], 1);
-                    const float nxt = lane == 31 ? 1.f : n1;           // p_{t+1}
+                    nxt[e] = lane == 31 ? 1.f : n1;
                     if (lane == 0 && inc[e] < kMinDecay) raise_status(WKV7_ERR_RANGE);
-                    xa[e] = __fdividef(av[e], inc[e]);
-                    xr[e] = __fdividef(rv[e], nxt);
-                    xb[e] = bv[e] * nxt;
-                    xk[e] = kv[e] * nxt;
                 }
-                store8_split(sm + X1_HI, sm + X1_LO, cm_off(t, 8 * g, 64), xr);
-                store8_split(sm + X1_HI, sm + X1_LO, cm_off(32 + t, 8 * g, 64), xa);
-                store8_split(sm + X1_HI, sm + X1_LO, cm_off(64 + t, 8 * g, 64), xb);
-                store8_split(sm + X1_HI, sm + X1_LO, cm_off(96 + t, 8 * g, 64), xk);
+                // one operand at a time (loaded just before use: fewer live registers)
+                {
+                    float v[8], x[8];
+                    ld8(TR, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = __fdividef(v[e], nxt[e]);
+                    store8_split(sm + X1_HI, sm + X1_LO, cm_off(t, 8 * g, 64), x);
+                    ld8(TA, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = __fdividef(v[e], inc[e]);
+                    store8_split(sm + X1_HI, sm + X1_LO, cm_off(32 + t, 8 * g, 64), x);
+                    ld8(TB, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = v[e] * nxt[e];
+                    store8_split(sm + X1_HI, sm + X1_LO, cm_off(64 + t, 8 * g, 64), x);
+                    ld8(TK, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = v[e] * nxt[e];
+                    store8_split(sm + X1_HI, sm + X1_LO, cm_off(96 + t, 8 * g, 64), x);
+                }
                 // exact bf16 operands: V, dY into VYZ rows t ([V | dY]) and ZYUV rows t (dY), 96 + t (V)
                 const uint4 vraw = *reinterpret_cast<const uint4 *>(sm + RAW + ((TV * L + t) * RAWP + 8 * g) * 2);
                 const uint4 yraw = *reinterpret_cast<const uint4 *>(sm + RAW + ((TDY * L + t) * RAWP + 8 * g) * 2);
@@ -410,87 +407,91 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             ready_arrive(0);                                     // round A: X1
             csync();                                             // p_t visible; RAW no longer read
             // ---- P0b: SG = S_in diag(G) (rows 0-63) and dS (rows 64-127); thread ->
-            //      row tid / 4, columns 16 (tid % 4) .. ----
+            //      row 8 (tid / 64) + tid % 8, columns 8 ((tid / 8) % 8) ..: a quarter-warp
+            //      takes 8 rows of one column group, 16-byte accesses on distinct banks ----
             {
-                const int i = tid >> 2, c0 = 16 * (tid & 3);
-                float sg[16], dsv[16];
+                const int rb = tid >> 6, i = 8 * rb + (tid & 7), c0 = 8 * ((tid >> 3) & 7);
+                float sg[8], dsv[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const uint32_t so4 = st_off(i, (c0 >> 2) + u);
                     const float4 s4 = *reinterpret_cast<const float4 *>(sm + ST_SIN + so4);
                     const float4 d4 = *reinterpret_cast<const float4 *>(sm + ST_DS + so4);
-                    const int j = c0 + 4 * u;
-                    sg[4 * u] = s4.x * psm[j]; sg[4 * u + 1] = s4.y * psm[j + 1];
-                    sg[4 * u + 2] = s4.z * psm[j + 2]; sg[4 * u + 3] = s4.w * psm[j + 3];
+                    const float4 p4 = *reinterpret_cast<const float4 *>(psm + c0 + 4 * u);   // G = p_0
+                    sg[4 * u] = s4.x * p4.x; sg[4 * u + 1] = s4.y * p4.y;
+                    sg[4 * u + 2] = s4.z * p4.z; sg[4 * u + 3] = s4.w * p4.w;
                     dsv[4 * u] = d4.x; dsv[4 * u + 1] = d4.y; dsv[4 * u + 2] = d4.z; dsv[4 * u + 3] = d4.w;
                 }
                 cp_async_wait<0>();                      // S_out
                 csync();                                 // the staged states are read before SGD replaces them
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0, 64), sg);
-                store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(i, c0 + 8, 64), sg + 8);
                 store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(64 + i, c0, 64), dsv);
-                store8_split(sm + SGD_HI, sm + SGD_LO, cm_off(64 + i, c0 + 8, 64), dsv + 8);
                 // the chunk's last token also scales S_out: q_{Lc-1} += sum_i S_out dS
-                // (the 8 rows of a warp summed by shuffles, then per-warp partial sums)
-                float cs[16];
+                // (the 8 rows of a quarter-warp summed by shuffles, then partial sums
+                // per block of 8 rows)
+                float cs[8];
                 const uint32_t so = i < 32 ? ST_SOUT0 : ST_SOUT1;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const float4 s4 = *reinterpret_cast<const float4 *>(sm + so + st_off(i & 31, (c0 >> 2) + u));
                     cs[4 * u] = s4.x * dsv[4 * u]; cs[4 * u + 1] = s4.y * dsv[4 * u + 1];
                     cs[4 * u + 2] = s4.z * dsv[4 * u + 2]; cs[4 * u + 3] = s4.w * dsv[4 * u + 3];
                 }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
+                for (int e = 0; e < 8; ++e) {
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 1);
+                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 2);
                     cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 4);
-                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 8);
-                    cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 16);
                 }
-                if (lane < 4) {
-                    float *cp = reinterpret_cast<float *>(sm + CPART) + warp * kN + c0;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) cp[e] = cs[e];
+                if ((lane & 7) == 0) {
+                    float *cp = reinterpret_cast<float *>(sm + CPART) + rb * kN + c0;
+                    *reinterpret_cast<float4 *>(cp) = make_float4(cs[0], cs[1], cs[2], cs[3]);
+                    *reinterpret_cast<float4 *>(cp + 4) = make_float4(cs[4], cs[5], cs[6], cs[7]);
                 }
             }
 
-            // ---- P1: Gram rows -> L tiles (lane = row of X X^T) ----
+            // ---- P1: Gram rows -> L tiles (lane = row of X X^T; the two warps of a
+            //      role take 16 of its 32 columns each) ----
             done_wait(0);
             {
-                const int lr = lane;                     // token t (quadrants 0, 1) or s (quadrant 2)
+                const int lr = lane, e0 = 16 * part;     // token t (quadrants 0, 1) or s (quadrant 2)
                 if (q4 == 0 && hc == 1) {                // r'_t . k-_s: L_rk rows t (s <= t)
-                    float x[32];
-                    tld32(CA + 96, x);
+                    float x[16];
+                    tmem_ld16(tmem + quad + CA + 96 + e0, x);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = e <= lr ? x[e] : 0.f;
+                    for (int e = 0; e < 16; ++e) x[e] = e0 + e <= lr ? x[e] : 0.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) store8_split(sm + LRK_HI, sm + LRK_LO, cm_off(lr, 8 * u, 32), x + 8 * u);
+                    for (int u = 0; u < 2; ++u)
+                        store8_split(sm + LRK_HI, sm + LRK_LO, cm_off(lr, e0 + 8 * u, 32), x + 8 * u);
                 } else if (q4 == 1 && hc == 1) {         // a'_t . k-_s: L_ak rows t (s < t)
-                    float x[32];
-                    tld32(CA + 96, x);
+                    float x[16];
+                    tmem_ld16(tmem + quad + CA + 96 + e0, x);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = e < lr ? x[e] : 0.f;
+                    for (int e = 0; e < 16; ++e) x[e] = e0 + e < lr ? x[e] : 0.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        store8_split(sm + LB2_HI, sm + LB2_LO, cm_off(lr, 8 * u, 32), x + 8 * u);
-                        store8_split(sm + LRK_HI, sm + LRK_LO, cm_off(32 + lr, 8 * u, 32), x + 8 * u);
+                    for (int u = 0; u < 2; ++u) {
+                        store8_split(sm + LB2_HI, sm + LB2_LO, cm_off(lr, e0 + 8 * u, 32), x + 8 * u);
+                        store8_split(sm + LRK_HI, sm + LRK_LO, cm_off(32 + lr, e0 + 8 * u, 32), x + 8 * u);
                     }
                 } else if (q4 == 2 && hc == 0) {         // b-_s . r'_t: L_rb^T rows s (t >= s)
-                    float x[32];
-                    tld32(CA + 0, x);
+                    float x[16];
+                    tmem_ld16(tmem + quad + CA + 0 + e0, x);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = e >= lr ? x[e] : 0.f;
+                    for (int e = 0; e < 16; ++e) x[e] = e0 + e >= lr ? x[e] : 0.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        store8_split(sm + LB2_HI, sm + LB2_LO, cm_off(32 + lr, 8 * u, 32), x + 8 * u);
+                    for (int u = 0; u < 2; ++u)
+                        store8_split(sm + LB2_HI, sm + LB2_LO, cm_off(32 + lr, e0 + 8 * u, 32), x + 8 * u);
                 } else if (q4 == 2 && hc == 1) {         // b-_s . a'_t: L_ab^T rows s (t > s), fp32
-                    float x[32];
-                    tld32(CA + 32, x);
-                    float *dst = reinterpret_cast<float *>(sm + LABT) + lr * LDT;
+                    float x[16];
+                    tmem_ld16(tmem + quad + CA + 32 + e0, x);
+                    float *dst = reinterpret_cast<float *>(sm + LABT) + lr * LDT + e0;
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4)
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int t0 = e0 + 4 * e4;
                         *reinterpret_cast<float4 *>(dst + 4 * e4) =
-                            make_float4(4 * e4 + 0 > lr ? x[4 * e4 + 0] : 0.f, 4 * e4 + 1 > lr ? x[4 * e4 + 1] : 0.f,
-                                        4 * e4 + 2 > lr ? x[4 * e4 + 2] : 0.f, 4 * e4 + 3 > lr ? x[4 * e4 + 3] : 0.f);
+                            make_float4(t0 + 0 > lr ? x[4 * e4 + 0] : 0.f, t0 + 1 > lr ? x[4 * e4 + 1] : 0.f,
+                                        t0 + 2 > lr ? x[4 * e4 + 2] : 0.f, t0 + 3 > lr ? x[4 * e4 + 3] : 0.f);
+                    }
                 }
             }
             ready_arrive(1);                             // round B: SG, dS, a', b-, k-, V, dY, L_ak, L_rb^T
@@ -522,7 +523,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     }
                 }
                 csync();
-                {                                        // Z = L21 T11
+                if (tid < 256) {                         // Z = L21 T11
                     const int t = tid >> 4, s = tid & 15;
                     float acc = 0.f;
 #pragma unroll
@@ -530,7 +531,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     zs[t * 16 + s] = acc;
                 }
                 csync();
-                {                                        // T21 = T22 Z
+                if (tid < 256) {                         // T21 = T22 Z
                     const int t = tid >> 4, s = tid & 15;
                     float acc = 0.f;
 #pragma unroll
@@ -538,20 +539,26 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     ts[(16 + t) * LDTS + s] = acc;
                 }
                 csync();
-                {                                        // T rows t and T^T rows 32 + s of TT
-                    const int t = tid >> 3, s0 = 4 * (tid & 7);
+                if (tid < 256) {                         // T rows t and T^T rows 32 + s of TT
+                    // thread -> row (lane) and 8 columns (warp % 4) of T (warps 0-3)
+                    // or of T^T (warps 4-7): a quarter-warp stores 8 rows of one
+                    // core-matrix column, the fp32 reads spread over the banks
+                    const int r = tid & 31, u = (tid >> 5) & 3;
+                    float x[8];
+                    if (tid < 128) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = s0 + e;
-                        const float x = ts[t * LDTS + s];
-                        bwtc_put1(sm, TT_HI, TT_LO, cm_off(t, s, 32), x);
-                        bwtc_put1(sm, TT_HI, TT_LO, cm_off(32 + s, t, 32), x);
+                        for (int k = 0; k < 8; ++k) x[k] = ts[r * LDTS + 8 * u + k];
+                        store8_split(sm + TT_HI, sm + TT_LO, cm_off(r, 8 * u, 32), x);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) x[k] = ts[(8 * u + k) * LDTS + r];
+                        store8_split(sm + TT_HI, sm + TT_LO, cm_off(32 + r, 8 * u, 32), x);
                     }
                 }
             }
             // ---- P2: Z^T (lanes 0-63) and dU^T (lanes 64-127) -> ZDU rows ----
             done_wait(1);
-            {
+            if (part == 0) {                             // 8 warps: 16 columns each
                 const int row = 32 * q4 + lane;
                 const uint32_t col = CB + (q4 < 2 ? 0u : 32u) + 16u * (uint32_t)hc;
                 uint32_t r0[16];
@@ -569,23 +576,23 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             // ---- P3: U rows (lanes 0-31), dZ rows (lanes 32-63) -> ZYUV, VYZ ----
             done_wait(2);
             if (q4 < 2) {
-                const int t = lane;
-                float x[32];
-                tld32(CC + (q4 == 0 ? 0u : 64u) + 32u * (uint32_t)hc, x);
+                const int t = lane, cb = 32 * hc + 16 * part;
+                float x[16];
+                tmem_ld16(tmem + quad + CC + (q4 == 0 ? 0u : 64u) + (uint32_t)cb, x);
                 if (q4 == 0) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        store8_split(sm + ZY_HI, sm + ZY_LO, cm_off(64 + t, 32 * hc + 8 * u, 64), x + 8 * u);
+                    for (int u = 0; u < 2; ++u)
+                        store8_split(sm + ZY_HI, sm + ZY_LO, cm_off(64 + t, cb + 8 * u, 64), x + 8 * u);
                 } else {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        store8_split(sm + ZY_HI, sm + ZY_LO, cm_off(32 + t, 32 * hc + 8 * u, 64), x + 8 * u);
-                        store8_split(sm + VYZ_HI, sm + VYZ_LO, cm_off(32 + t, 64 + 32 * hc + 8 * u, 128), x + 8 * u);
+                    for (int u = 0; u < 2; ++u) {
+                        store8_split(sm + ZY_HI, sm + ZY_LO, cm_off(32 + t, cb + 8 * u, 64), x + 8 * u);
+                        store8_split(sm + VYZ_HI, sm + VYZ_LO, cm_off(32 + t, 64 + cb + 8 * u, 128), x + 8 * u);
                     }
                 }
-            } else {                                     // the other four warps: [SG | dS] side by side
-                const int u = (2 * hc + q4 - 2) * 32 + lane;   // 0 .. 127; SG rows to columns 0-63, dS to 64-127
-                for (int x = u; x < 2048; x += 128) {
+            } else {                                     // the other eight warps: [SG | dS] side by side
+                const int u = ((2 * hc + q4 - 2) + 4 * part) * 32 + lane;   // 0 .. 255; SG rows to columns 0-63, dS to 64-127
+                for (int x = u; x < 2048; x += 256) {
                     const int blk = x >> 6, hl = (blk >> 4) & 1, G = blk & 15;
                     const uint32_t src = (hl ? SGD_LO : SGD_HI) + G * 1024;
                     const uint32_t dst = (hl ? SGDC_LO : SGDC_HI) + ((G & 7) * 16 + (G < 8 ? 0 : 8)) * 128;
@@ -610,7 +617,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 *reinterpret_cast<uint4 *>(sm + dst + 16 * (x & 63)) =
                     *reinterpret_cast<const uint4 *>(sm + src + 16 * (x & 63));
             }
-            if (q4 >= 2) {                               // dV^T rows i, columns s = 16 hc ..
+            if (q4 >= 2 && part == 0) {                  // dV^T rows i, columns s = 16 hc ..
                 const int i = 32 * (q4 - 2) + lane;
                 uint32_t r0[16];
                 tmem_ld16_nowait(tmem + quad + CB + 64 + 16 * hc, r0);
@@ -622,24 +629,24 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 }
             }
             {
-                // lanes 0-63: dL rows t' (columns s' = 32 hc + e at CA + 64 + s');
-                // lanes 64-127: dL^T rows s' (columns t' = 32 hc + e at CA + t').
+                // lanes 0-63: dL rows t' (columns s' = 32 hc + 16 part + e at CA + 64 + s');
+                // lanes 64-127: dL^T rows s' (columns t' = 32 hc + 16 part + e at CA + t').
                 // Mask: t' < 32 (r' rows) keeps s <= t, t' >= 32 (a' rows) keeps s < t.
-                float x[32];
-                tld32(CA + (q4 < 2 ? 64u : 0u) + 32u * (uint32_t)hc, x);
+                const int e0 = 32 * hc + 16 * part;
+                float x[16];
+                tmem_ld16(tmem + quad + CA + (q4 < 2 ? 64u : 0u) + (uint32_t)e0, x);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
+                for (int e = 0; e < 16; ++e) {
                     int tp, t_, s_;
-                    if (q4 < 2) { tp = 32 * q4 + lane; t_ = lane; s_ = e; }
-                    else { tp = 32 * hc + e; t_ = e; s_ = lane; }
+                    if (q4 < 2) { tp = 32 * q4 + lane; t_ = lane; s_ = (e0 + e) & 31; }
+                    else { tp = e0 + e; t_ = (e0 + e) & 31; s_ = lane; }
                     const bool keep = tp < 32 ? s_ <= t_ : s_ < t_;
                     x[e] = keep ? x[e] : 0.f;
                 }
-                uint32_t ph[16], pl[16];
+                uint32_t ph[8], pl[8];
                 bwtc_pack16(x, ph, pl);
-                bwtc_pack16(x + 16, ph + 8, pl + 8);
-                tmem_st16(tmem + quad + ADL_HI + 16 * hc, ph);
-                tmem_st16(tmem + quad + ADL_LO + 16 * hc, pl);
+                tmem_st8(tmem + quad + ADL_HI + (uint32_t)(e0 >> 1), ph);
+                tmem_st8(tmem + quad + ADL_LO + (uint32_t)(e0 >> 1), pl);
                 tmem_st_wait();
             }
             ready_arrive(4);                             // round E
@@ -647,9 +654,9 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
             done_wait(4);
             {
                 const int rrow = lane;                   // token t (q4 0, 1) or s (q4 2, 3)
-                float x[32];
-                tld32(CE + (q4 < 2 ? 0u : 64u) + 32u * (uint32_t)hc, x);
-                const int j0 = 32 * hc;
+                const int j0 = 32 * hc + 16 * part;      // this warp's 16 channels
+                float x[16];
+                tmem_ld16(tmem + quad + CE + (q4 < 2 ? 0u : 64u) + (uint32_t)j0, x);
                 // q terms, from the unscaled gradients and the decayed operands:
                 // dr r = dr' r', da a = da' a', db b = db' b-, dk k = dk' k-
                 // (X1 row 32 q4 + lane holds r', a', b-, k- for q4 = 0 .. 3);
@@ -659,7 +666,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                     float *cq = reinterpret_cast<float *>(sm + CQ) + (q4 * L + rrow) * LDQ + j0;
                     const float sign = q4 >= 2 ? -1.f : 1.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 2; ++u) {
                         const uint32_t off = cm_off(32 * q4 + rrow, j0 + 8 * u, 64);
                         const uint4 h8 = *reinterpret_cast<const uint4 *>(sm + X1_HI + off);
                         const uint4 l8 = *reinterpret_cast<const uint4 *>(sm + X1_LO + off);
@@ -676,29 +683,25 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                         *reinterpret_cast<float4 *>(cq + 8 * u + 4) = make_float4(o8[4], o8[5], o8[6], o8[7]);
                     }
                 }
-                GradT *dst;
                 const float *prow = psm + (q4 == 1 ? rrow : rrow + 1) * LDP + j0;   // p_t for da, p_{t+1} else
-                float pv[32];
+                float pv[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const float4 p4 = *reinterpret_cast<const float4 *>(prow + 4 * u);
                     pv[4 * u] = p4.x; pv[4 * u + 1] = p4.y; pv[4 * u + 2] = p4.z; pv[4 * u + 3] = p4.w;
                 }
                 if (q4 < 2) {                            // dr = dr' / p_{t+1},  da = da' / p_t
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = __fdividef(x[e], pv[e]);
-                    dst = q4 == 0 ? dr : da;
+                    for (int e = 0; e < 16; ++e) x[e] = __fdividef(x[e], pv[e]);
                 } else {                                 // db, dk = (db', dk') p_{s+1}
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = x[e] * pv[e];
-                    dst = q4 == 2 ? db : dk;
+                    for (int e = 0; e < 16; ++e) x[e] = x[e] * pv[e];
                 }
-                (void)dst;
                 {   // into the staging tile of this gradient (row rrow, columns j0 ..); written out coalesced below
                     constexpr int PITCH = kN * (int)sizeof(GradT) + 16;
                     GradT *o = reinterpret_cast<GradT *>(sm + GSTG + (q4 * L + rrow) * PITCH) + j0;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
+                    for (int u = 0; u < 4; ++u)
                         store4(o + 4 * u, make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]));
                 }
             }
@@ -714,18 +717,18 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                             *reinterpret_cast<const uint4 *>(sm + GSTG + (tile * L + row) * PITCH + 16 * ch);
                 }
             }
-            {   // dw_m = sum_{t >= m} q_t / w_m: thread -> column j, block of 8 tokens
+            {   // dw_m = sum_{t >= m} q_t / w_m: thread -> column j, block of 4 tokens
                 const float *cq = reinterpret_cast<const float *>(sm + CQ);
                 const float *cp = reinterpret_cast<const float *>(sm + CPART);
                 float *tot = reinterpret_cast<float *>(sm + DWTOT);
                 const int j = tid & 63, blk = tid >> 6;
                 float colsum = 0.f;
 #pragma unroll
-                for (int wv = 0; wv < 8; ++wv) colsum += cp[wv * kN + j];
-                float loc[8], run = 0.f;
+                for (int rb = 0; rb < 8; ++rb) colsum += cp[rb * kN + j];
+                float loc[4], run = 0.f;
 #pragma unroll
-                for (int e = 7; e >= 0; --e) {
-                    const int t = 8 * blk + e;
+                for (int e = 3; e >= 0; --e) {
+                    const int t = 4 * blk + e;
                     float q = cq[t * LDQ + j] + cq[(2 * L + t) * LDQ + j] + cq[(3 * L + t) * LDQ + j];
                     if (t + 1 < L) q += cq[(L + t + 1) * LDQ + j];
                     if (t == Lc - 1) q += colsum;
@@ -735,10 +738,10 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 tot[blk * kN + j] = run;
                 csync();
                 float later = 0.f;
-                for (int b2 = blk + 1; b2 < 4; ++b2) later += tot[b2 * kN + j];
+                for (int b2 = blk + 1; b2 < 8; ++b2) later += tot[b2 * kN + j];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = 8 * blk + e;
+                for (int e = 0; e < 4; ++e) {
+                    const int t = 4 * blk + e;
                     if (t < Lc)
                         dw[base + (size_t)t * tok_stride + j] =
                             from_f32<GradT>(__fdividef((loc[e] + later) * psm[(t + 1) * LDP + j], psm[t * LDP + j]));
@@ -757,7 +760,7 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
         __syncthreads();
     }
     fence_after_sync();
-    if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == NCW) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 template <typename GradT>
