@@ -378,7 +378,9 @@ def bench_train(args, dist, peaks, device, d):
     dy = to_dev(inputs.gen_dy(B, T, H, N, seed=shard_seed(cfg["seed"], dist.rank), dtype="bf16"), device)
     y = torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device)
     sT = torch.empty(B, H, N, N, dtype=torch.float32, device=device)
-    states = torch.empty(B, H, (T + 31) // 32, N, N, dtype=torch.float32, device=device)
+    # the saved states (the state before every chunk), then the chunks' transitions
+    states_buf = torch.empty(wkv7.saved_states_size(B, T, H, N) // 4, dtype=torch.float32, device=device)
+    states = states_buf[: B * H * ((T + 31) // 32) * N * N].view(B, H, (T + 31) // 32, N, N)
     grads = [torch.empty(B, T, H, N, dtype=torch.bfloat16, device=device) for _ in range(6)]
     grads.append(torch.empty(B, H, N, N, dtype=torch.float32, device=device))
     ws_b = torch.empty(wkv7.backward_from_states_workspace_size(B, T, H, N), dtype=torch.uint8, device=device)
@@ -400,8 +402,8 @@ def bench_train(args, dist, peaks, device, d):
     return {"value": aggregate_throughput(B * T * H, per, dist.world), "unit": "head-tokens/s",
             "ms_per_step": per * 1e3, "steps": steps, "launches": 4 * steps,
             "separate_ms_per_step": per_sep * 1e3,
-            "note": "wkv7_forward_train + wkv7_backward_from_states; separate = wkv7_forward + wkv7_backward "
-                    "(which recomputes the chunk states)",
+            "note": "wkv7_forward_train (states and chunk transitions kept) + wkv7_backward_from_states; "
+                    "separate = wkv7_forward + wkv7_backward (which recomputes the chunk states)",
             "config": {"workload": "train_bwd_b8_t4096_h32", "B": B, "T": T, "H": H, "N": N,
                        "y_dtype": "bf16", "grad_dtype": "bf16", "dsT": "zero"}}
 

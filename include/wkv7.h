@@ -376,18 +376,25 @@ WKV7_API wkv7_status wkv7_backward(int B, int T, int H, int N, wkv7_dtype in_dty
 /*
  * Training pair: a forward that also keeps what the backward needs, and a
  * backward that starts from it instead of recomputing the states (saves the
- * checkpoint pass, about a sixth of wkv7_backward on the training workload).
+ * checkpoint pass, about a quarter of wkv7_backward on the training workload).
  *
  * Bytes of the saved states: the state before every 32-token chunk,
- * [B, H, ceil(T / 32), N, N] fp32 (512 B per head-token at N = 64).
+ * [B, H, ceil(T / 32), N, N] fp32 (512 B per head-token at N = 64), then,
+ * from the next multiple of 256 bytes on, every chunk's transition image
+ * (24 KiB per chunk: 768 B per head-token; written for bf16 inputs, opaque).
  */
 WKV7_API size_t wkv7_saved_states_size(int B, int T, int H, int N);
 
 /*
  * wkv7_forward that also writes `states` (wkv7_saved_states_size() bytes,
- * device, overwritten; states[b][h][c] = the state before token 32 c).  sT is
- * required here (the backward reads it as the state after the last chunk).
- * Same arguments, algorithms, results and errors as wkv7_forward otherwise.
+ * device, overwritten; states[b][h][c] = the state before token 32 c, then
+ * the chunks' transitions).  sT is required here (the backward reads it as
+ * the state after the last chunk).  Same arguments, algorithms, results and
+ * errors as wkv7_forward otherwise.  For bf16 inputs the states and the
+ * transitions always come from the chunked form (the backward's dS chain
+ * needs the transitions): when the call runs the scan (WKV7_ALGO_SEQ, or
+ * AUTO below 64 tokens) y and sT come from the scan and one chunked pass
+ * without y writes the states and transitions.
  */
 WKV7_API wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dtype, wkv7_dtype y_dtype,
                                         const void *r, const void *w, const void *k, const void *v,
@@ -401,11 +408,11 @@ WKV7_API size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, in
 
 /*
  * wkv7_backward given the states and sT that wkv7_forward_train wrote for the
- * same inputs (s0 is not needed: states[.][.][0] is it).  Two launches: the
- * state-gradient sweep and the chunk gradients.  Same gradients, dtypes and
- * errors as wkv7_backward with its workspace short of the transition images
- * (bit for bit: dL/dS by the per-token sweep; the saved states carry no
- * transitions, since this call cannot know whether the forward ran the
+ * same inputs (s0 is not needed: states[.][.][0] is it).  Two launches:
+ * dL/dS at every chunk end (bf16 inputs: the transition chain over the saved
+ * transitions; fp32: the per-token sweep) and the chunk gradients.  Same
+ * gradients, dtypes and errors as wkv7_backward (for bf16 inputs bit for bit
+ * with wkv7_backward given its full workspace when the forward ran the
  * chunked form).
  */
 WKV7_API wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_dtype,

@@ -815,9 +815,10 @@ static cudaError_t launch_chunk(int B, int T, int H, int t_seg, int nseg, int nz
                                             (O *)y, sT, sT_zstride, st_only_z, wait_limit, ckpt, nullptr, 0,  \
                                             seg0, 0, epi, nullptr, mq);                                       \
     } while (0)
-    if (mq) {                                     // the backward's checkpoint pass (no y, no epilogue)
-        if (epi.rho || y) return cudaErrorInvalidValue;
-        WKV7_CHUNK_LAUNCH(__nv_bfloat16, false, true);
+    if (mq) {                                     // checkpoints with the transitions (no epilogue)
+        if (epi.rho) return cudaErrorInvalidValue;
+        if (y && y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, false, true);
+        else WKV7_CHUNK_LAUNCH(__nv_bfloat16, false, true);
     } else if (epi.rho) {
         if (y_dt == WKV7_F32) WKV7_CHUNK_LAUNCH(float, true, false);
         else WKV7_CHUNK_LAUNCH(__nv_bfloat16, true, false);
@@ -854,9 +855,10 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
                                             e_zstride, -1, wait_limit, ckpt, m_out, m_zstride, 0, first_out,   \
                                             epi, y0q, mq);                                                     \
     } while (0)
-    if (mq) {                                     // the backward's segmented checkpoint pass
-        if (epi.rho || y) return cudaErrorInvalidValue;
-        WKV7_DUAL_LAUNCH(bf, false, true);
+    if (mq) {                                     // segmented checkpoints with the transitions
+        if (epi.rho) return cudaErrorInvalidValue;
+        if (y && y_dt == WKV7_F32) WKV7_DUAL_LAUNCH(float, false, true);
+        else WKV7_DUAL_LAUNCH(bf, false, true);
     } else if (epi.rho && first_out) {
         if (y_dt == WKV7_BF16) WKV7_DUAL_LAUNCH(bf, true, false);
         else WKV7_DUAL_LAUNCH(float, true, false);

@@ -181,7 +181,7 @@ wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
                          const void *w, const void *k, const void *v, const void *a, const void *b,
                          const float *s0, void *y, float *sT, wkv7_algo algo, int chunk_len, void *workspace,
                          size_t workspace_bytes, cudaStream_t stream, float *ckpt,
-                         const EpiArgs &epi = EpiArgs{}) {
+                         const EpiArgs &epi = EpiArgs{}, uint4 *mq = nullptr) {
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if (!dtype_ok(in_dt) || !dtype_ok(y_dt)) return WKV7_ERR_INVALID_ARG;
@@ -215,7 +215,7 @@ wkv7_status forward_impl(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
             if (want > 1 && workspace_bytes >= chunk_workspace_bytes(B, T, H, want)) nseg = want;
         }
         return from_cuda(fwd_chunk(B, T, H, y_dt, r, w, k, v, a, b, s0, y, sT, nseg, workspace,
-                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, epi, fixup));
+                                   lim > 0 ? lim : kDefaultWaitCycles, stream, ckpt, epi, fixup, mq));
     }
     if (epi.rho) return WKV7_ERR_UNSUPPORTED;      // the scan's epilogue is a separate pass (timemix.cu)
     const long long lim = g_wait_limit.load() > 0 ? g_wait_limit.load() : kDefaultWaitCycles;
@@ -239,7 +239,8 @@ wkv7_status wkv7_forward(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtyp
 
 size_t wkv7_saved_states_size(int B, int T, int H, int N) {
     if (B <= 0 || T <= 0 || H <= 0 || N != kN) return 0;
-    return bwd_ckpt_bytes(B, T, H);
+    // the state before every chunk, then every chunk's transition image
+    return round_up(bwd_ckpt_bytes(B, T, H)) + round_up(bwd_mq_bytes(B, T, H));
 }
 
 wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dt, wkv7_dtype y_dt, const void *r,
@@ -249,8 +250,22 @@ wkv7_status wkv7_forward_train(int B, int T, int H, int N, wkv7_dtype in_dt, wkv
     wkv7_status s = check_dims(B, T, H, N);
     if (s != WKV7_OK) return s;
     if ((size_t)B * H > 0 && (!ptr_ok(sT) || (T > 0 && !ptr_ok(states)))) return WKV7_ERR_INVALID_ARG;
-    return forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
-                        workspace_bytes, stream, states);
+    if (in_dt != WKV7_BF16 || (size_t)B * H == 0 || T == 0)
+        return forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
+                            workspace_bytes, stream, states);
+    // bf16 inputs: the states and every chunk's transition come from the
+    // chunked form (the backward's dS chain reads the transitions)
+    uint4 *mq = reinterpret_cast<uint4 *>(reinterpret_cast<char *>(states) + round_up(bwd_ckpt_bytes(B, T, H)));
+    if (resolve_algo(T, in_dt, algo) == WKV7_ALGO_CHUNK)
+        return forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
+                            workspace_bytes, stream, states, EpiArgs{}, mq);
+    // the scan for y and sT, then a chunked checkpoint pass (no y) for the states and transitions
+    s = forward_impl(B, T, H, N, in_dt, y_dt, r, w, k, v, a, b, s0, y, sT, algo, chunk_len, workspace,
+                     workspace_bytes, stream, nullptr);
+    if (s != WKV7_OK) return s;
+    const long long lim = g_wait_limit.load();
+    return from_cuda(fwd_chunk(B, T, H, WKV7_BF16, r, w, k, v, a, b, s0, nullptr, nullptr, 1, nullptr,
+                               lim > 0 ? lim : kDefaultWaitCycles, stream, states, EpiArgs{}, false, mq));
 }
 
 size_t wkv7_backward_from_states_workspace_size(int B, int T, int H, int N) {
@@ -279,10 +294,16 @@ wkv7_status wkv7_backward_from_states(int B, int T, int H, int N, wkv7_dtype in_
     const long long lim = g_wait_limit.load();
     const size_t ds_bytes = round_up(bwd_ckpt_bytes(B, T, H));
     char *ws = static_cast<char *>(workspace);
+    // bf16 inputs: dS by the transition chain from the transitions the
+    // training forward saved after the states; fp32: the per-token sweep
+    const uint4 *mq = in_dt == WKV7_BF16
+                          ? reinterpret_cast<const uint4 *>(reinterpret_cast<const char *>(states) +
+                                                            round_up(bwd_ckpt_bytes(B, T, H)))
+                          : nullptr;
     return from_cuda(bwd_chunked(B, T, H, in_dt, g_dt, r, w, k, v, a, b, dy, dsT, states, sT,
                                  reinterpret_cast<float *>(ws), dr, dw, dk, dv, da, db, ds0,
                                  reinterpret_cast<float *>(ws + ds_bytes), workspace_bytes - ds_bytes,
-                                 current_sm_count(), lim > 0 ? lim : kDefaultWaitCycles, stream));
+                                 current_sm_count(), lim > 0 ? lim : kDefaultWaitCycles, stream, mq));
 }
 
 size_t wkv7_forward_summary_workspace_size(int B, int T, int H, int N) {

@@ -436,10 +436,21 @@ def backward_from_states_workspace_size(B, T, H, N) -> int:
     return load_library().wkv7_backward_from_states_workspace_size(B, T, H, N)
 
 
+def _saved_states_capacity_ok(states, B, T, H, N):
+    """The saved-states buffer holds wkv7_saved_states_size bytes from the
+    tensor's first element on (the states, then the chunks' transitions)."""
+    need = load_library().wkv7_saved_states_size(B, T, H, N)
+    have = states.untyped_storage().nbytes() - states.storage_offset() * states.element_size()
+    return states.is_contiguous() and have >= need
+
+
 def forward_train(r, w, k, v, a, b, s0=None, *, y=None, sT=None, states=None, y_dtype=None, algo="auto",
                   chunk_len=0, workspace=None, stream=None):
     """(y, sT, states): the forward plus the state before every 32-token chunk,
-    [B, H, ceil(T/32), N, N] fp32, for ``backward_from_states``."""
+    [B, H, ceil(T/32), N, N] fp32, for ``backward_from_states``.  ``states`` is
+    a view of the first part of a buffer of ``saved_states_size`` bytes whose
+    remainder holds every chunk's transition (bf16 inputs); pass it to
+    ``backward_from_states`` as returned."""
     lib = load_library()
     B, T, H, N = r.shape
     _same((w, k, v, a, b), r.shape, r.dtype)
@@ -449,7 +460,12 @@ def forward_train(r, w, k, v, a, b, s0=None, *, y=None, sT=None, states=None, y_
     if sT is None:
         sT = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
     if states is None:
-        states = torch.empty((B, H, (T + 31) // 32, N, N), dtype=torch.float32, device=r.device)
+        nck = (T + 31) // 32
+        buf = torch.empty(max(lib.wkv7_saved_states_size(B, T, H, N), 4) // 4, dtype=torch.float32,
+                          device=r.device)
+        states = buf[: B * H * nck * N * N].view(B, H, nck, N, N)
+    elif T > 0 and not _saved_states_capacity_ok(states, B, T, H, N):
+        raise ValueError("states: needs saved_states_size(B, T, H, N) bytes of contiguous storage")
     if s0 is not None:
         _same((s0,), (B, H, N, N), torch.float32)
     ws_bytes = lib.wkv7_forward_workspace_size(B, T, H, N, _dt(r), ALGOS[algo], chunk_len)
@@ -468,6 +484,8 @@ def backward_from_states(r, w, k, v, a, b, states, sT, dy, dsT=None, *, grad_dty
     lib = load_library()
     B, T, H, N = r.shape
     _same((w, k, v, a, b, dy), r.shape, r.dtype)
+    if T > 0 and not _saved_states_capacity_ok(states, B, T, H, N):
+        raise ValueError("states: pass the tensor forward_train returned (saved_states_size bytes)")
     gcode = F32 if grad_dtype == torch.float32 else BF16
     if out is None:
         out = [torch.empty((B, T, H, N), dtype=grad_dtype, device=r.device) for _ in range(6)]

@@ -171,7 +171,8 @@ def test_training_pair_rejects_invalid_arguments(lib):
     bad = [P] * 17
     bad[16] = None                                       # ds0 is required
     assert bs(ptrs=bad) == wkv7.ERR_INVALID_ARG
-    assert lib.wkv7_saved_states_size(2, 100, 3, 64) == 2 * 3 * 4 * 64 * 64 * 4
+    # the state before every chunk, then every chunk's transition image (24 KiB)
+    assert lib.wkv7_saved_states_size(2, 100, 3, 64) == 2 * 3 * 4 * 64 * 64 * 4 + 2 * 3 * 4 * 24576
     assert lib.wkv7_backward_from_states_workspace_size(2, 100, 3, 64) >= 2 * 3 * 4 * 64 * 64 * 4
 
 

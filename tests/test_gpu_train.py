@@ -86,12 +86,12 @@ def test_backward_from_states_matches_oracle(cuda_device, dtype, B, T, H):
 
 def test_training_workload_equals_backward(cuda_device):
     """B=8, T=4096, H=32 bf16 (the training workload): the forward's saved
-    states are the backward's own checkpoints bit for bit, so every gradient
-    equals that of wkv7_backward given its minimum workspace, which takes dS
-    from the same per-token sweep.  With its full workspace wkv7_backward
-    takes dS from the chunks' transitions instead: the same gradients within
-    the bf16 tolerance (its fp32 gradients against the bf16 ones, so that one
-    rounding separates them)."""
+    states and chunk transitions are the backward's own checkpoint pass bit
+    for bit, so every gradient equals that of wkv7_backward given its full
+    workspace (dS by the transition chain in both).  wkv7_backward given its
+    minimum workspace takes dS from the per-token sweep instead: the same
+    gradients within the bf16 bound (its fp32 gradients against these bf16
+    ones, so that one rounding separates them)."""
     cfg = inputs.WORKLOADS["train_bwd_b8_t4096_h32"]
     B, T, H = cfg["B"], cfg["T"], cfg["H"]
     d = inputs.gen_sequence(B, T, H, cfg["N"], seed=cfg["seed"], dtype="bf16", s0_std=cfg["s0_std"])
@@ -100,18 +100,30 @@ def test_training_workload_equals_backward(cuda_device):
     dy = to_dev(inputs.gen_dy(B, T, H, cfg["N"], seed=cfg["seed"], dtype="bf16"))
     _, sT, states = wkv7.forward_train(*x, s0)
     a = wkv7.backward_from_states(*x, states, sT, dy, None, grad_dtype=torch.bfloat16)
+    b = wkv7.backward(*x, s0, dy, None, grad_dtype=torch.bfloat16)
     transitions = B * H * ((T + 31) // 32) * 24576
     ws_min = torch.empty(wkv7.backward_workspace_size(B, T, H, 64) - transitions, dtype=torch.uint8, device="cuda")
-    b = wkv7.backward(*x, s0, dy, None, grad_dtype=torch.bfloat16, workspace=ws_min)
-    c = wkv7.backward(*x, s0, dy, None, grad_dtype=torch.float32)
+    c = wkv7.backward(*x, s0, dy, None, grad_dtype=torch.float32, workspace=ws_min)
     torch.cuda.synchronize()
     assert wkv7.device_status() == wkv7.OK
     for name, g1, g2 in zip(GRAD_NAMES, a, b):
         assert torch.equal(g1, g2), name
-    # fp32 gradients by the chain vs bf16 gradients by the sweep: the bf16 bound
-    # of tests/_tol.py (one bf16 rounding), on the device
-    for name, g1, g3 in zip(GRAD_NAMES, a, c):
+    for name, g1, g3 in zip(GRAD_NAMES, a, c):      # the bf16 bound of tests/_tol.py, on the device
         r = g1.double()
         bound = TAU_BF16 * r.pow(2).mean().sqrt() + (2.0 ** -8 if name != "ds0" else 0.0) * r.abs()
         excess = ((g3.double() - r).abs() - bound).max().item()
-        assert excess <= 0.0, f"{name} (transition chain): excess over the bound {excess:.3e}"
+        assert excess <= 0.0, f"{name} (per-token sweep): excess over the bound {excess:.3e}"
+
+
+def test_saved_states_buffer_size_is_checked(cuda_device):
+    """The saved states carry the chunks' transitions after the states: a
+    states tensor of the states' size alone is refused before any launch."""
+    d = _case(1, 100, 2, 995, "bf16")
+    x, s0, dy, _ = _dev(d)
+    small = torch.empty(1, 2, 4, 64, 64, device="cuda")
+    with pytest.raises(ValueError):
+        wkv7.forward_train(*x, s0, states=small)
+    _, sT, states = wkv7.forward_train(*x, s0)
+    with pytest.raises(ValueError):
+        wkv7.backward_from_states(*x, small, sT, dy)
+    assert states.shape == (1, 2, 4, 64, 64)
