@@ -70,7 +70,10 @@ constexpr int NC = 256;            // compute threads (warps 0-7)
 constexpr int NT = NC + 32;        // + the MMA warp
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_X = 0, COL_Z = 64, COL_MQ = 192;
-constexpr uint32_t TMEM_COLS_DUAL = 512, COL_S2 = 256;   // dual runs: the second state's [S_out^T; .]
+// dual runs: the second state's [S2_out^T; q] goes to [M''^T; Q'']'s columns
+// (P3 has read them before R4 is issued); P4 parks S2_out in the [M^T; Q]
+// columns until the next chunk's P3 turns it into the S2^T operand
+constexpr uint32_t COL_S2 = COL_Z;
 
 // shared memory map (bytes)
 constexpr uint32_t IN_W = 0, IN_R = 4096, IN_K = 8192, IN_A = 12288, IN_B = 16384;   // [32][128 B], rotated
@@ -87,8 +90,10 @@ constexpr uint32_t LABT = R + 8192;                 //   P1: fp32 L_ab^T [32][36
 constexpr uint32_t LAK = R + 12800;                 //   P1: fp32 L_ak [32][33] (padded)
 constexpr uint32_t WU_HI = R, WU_LO = R + 8192;     //   P2..R3: [128][32] = W'^T rows, U~^T rows
 constexpr uint32_t SMEM_BYTES = R + 17024;
-constexpr uint32_t S2_HI = SMEM_BYTES, S2_LO = S2_HI + 8192;   // dual runs: S^T of the second state
-constexpr uint32_t SMEM_BYTES_DUAL = S2_LO + 8192;
+// dual runs: S2^T operand [64 j][64 i], in the short-lived buffers: staged
+// in P3 (R3 has read [W' | U~]), read by R4, overwritten by the next P1
+constexpr uint32_t S2_HI = R, S2_LO = R + 8192;
+static_assert(S2_LO + 8192 <= SMEM_BYTES, "S2^T fits in the short-lived buffers");
 // in the free halves of RZ (bytes [1024, 2048) of each 2 KB group)
 constexpr uint32_t TSM = RZ_HI + 1024;              // fp32 T, row t at TSM + (t/8)*2048 + (t%8)*128
 constexpr uint32_t ZSM = RZ_LO + 1024;              // fp32 [16][16]
@@ -133,12 +138,15 @@ constexpr uint32_t BAR_READY = 2, BAR_DONE = 6;
 // DUAL: a summary run that carries two states through the same chunk algebra,
 // S from S_in (here 0, giving the segment's E) and S2 from I (giving M): the
 // chunk's operands, T, W', M and Q do not depend on the state, so only the
-// state round R4 and its read-out are done twice.  No y.  It needs a second S
-// operand and 64 more TMEM columns, so these CTAs run one per SM.
+// state round R4 and its read-out are done twice.  No y.  The second state
+// needs no room of its own: R4 writes it into [M''^T; Q'']'s TMEM columns (P3
+// has read them), P4 parks it in the [M^T; Q] columns (R4 has read them), and
+// the next P3 turns it into its S2^T operand in the short-lived buffers (R3
+// has read [W' | U~]).  So dual CTAs run two per SM, like the plain ones.
 // EPI: the time-mix output epilogue (EpiArgs) replaces the y store.
 // MQX: the checkpoint pass also exports every chunk's transition [M^T; Q] to mq.
 template <typename OutT, bool DUAL, bool EPI, bool MQX = false>
-__global__ void __launch_bounds__(chunk::NT, DUAL ? 1 : 2)
+__global__ void __launch_bounds__(chunk::NT, 2)
 fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *__restrict__ r,
                  const __nv_bfloat16 *__restrict__ w, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ a,
@@ -213,7 +221,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         }
         *abort_flag = 0;
     }
-    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
+    if (warp == 8) tmem_alloc(sbase + TMEM_SLOT, TMEM_COLS);
     if constexpr (EPI) {
         if (tid < kN)
             reinterpret_cast<float2 *>(sm + GAMBET)[tid] =
@@ -240,12 +248,6 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         if (ckp) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) ckp[(size_t)(16 * part + e) * kN + j] = x[e];
-        }
-        if constexpr (DUAL) {                         // the second state starts at I
-#pragma unroll
-            for (int e = 0; e < 16; ++e) x[e] = (16 * part + e == j) ? 1.f : 0.f;
-            store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part, 64), x);
-            store8_split(sm + S2_HI, sm + S2_LO, cm_off(j, 16 * part + 8, 64), x + 8);
         }
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -316,6 +318,19 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         const int sub = lane & 15;                   // row within the quadrant's 16 (M=64 layout)
         const bool upper = lane >= 16;
         const int rho = 32 * q4 + lane;              // row of an M=128 accumulator
+        if constexpr (DUAL) {                        // the second state starts at I: S2^T rows, parked in
+            if (q4 < 2) {                            // the [M^T; Q] columns until P3 of the first chunk
+                uint32_t id0[16], id1[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    id0[e] = __float_as_uint(32 * hc + e == rho ? 1.f : 0.f);
+                    id1[e] = __float_as_uint(32 * hc + 16 + e == rho ? 1.f : 0.f);
+                }
+                tmem_st16(tmem + quad + COL_MQ + 16 * hc, id0);          // the columns that this
+                tmem_st16(tmem + quad + COL_MQ + 32 + 16 * hc, id1);     // warp's P3 overwrites
+                tmem_st_wait();
+            }
+        }
 
         // Hand-offs with the issuer warp.  Waiting warps park at a hardware
         // barrier (no issue slots taken from the other CTA on the SM).  The
@@ -549,6 +564,23 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 
         auto P3 = [&](int c) {                    // rows of [M^T; Q] -> TMEM A operand of R4
             if (q4 == 3) return;
+            if constexpr (DUAL) {                 // S2^T row rho (parked by the last P4) -> its operand
+                if (q4 < 2) {
+                    uint32_t s0[16], s1[16];
+                    tmem_ld16_nowait(tmem + quad + COL_MQ + 16 * hc, s0);
+                    tmem_ld16_nowait(tmem + quad + COL_MQ + 32 + 16 * hc, s1);
+                    tmem_wait();
+                    float x2[32];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        x2[e] = __uint_as_float(s0[e]);
+                        x2[16 + e] = __uint_as_float(s1[e]);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        store8_split(sm + S2_HI, sm + S2_LO, cm_off(rho, 32 * hc + 8 * u, 64), x2 + 8 * u);
+                }
+            }
             uint32_t r0[16], r1[16];
             tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc, r0);
             tmem_ld16_nowait(tmem + quad + COL_Z + 32 * hc + 16, r1);
@@ -644,23 +676,24 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dst[(size_t)(32 * hc + e) * kN] = x[e];
                 }
-                if constexpr (DUAL) {             // the same for the second state
+                if constexpr (DUAL) {             // the second state: parked in the [M^T; Q] columns
                     tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc, r0);
                     tmem_ld16_nowait(tmem + quad + COL_S2 + 32 * hc + 16, r1);
                     tmem_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        x[e] = __uint_as_float(r0[e]);
-                        x[16 + e] = __uint_as_float(r1[e]);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        store8_split(sm + S2_HI, sm + S2_LO, cm_off(rho, 32 * hc + 8 * u, 64), x + 8 * u);
+                    // R4 has read [M^T; Q]; the parked row goes to the columns that
+                    // this warp's next P3 reads it from and then overwrites (its hi
+                    // and lo words), so no other warp's P3 store can land on it first
+                    tmem_st16(tmem + quad + COL_MQ + 16 * hc, r0);
+                    tmem_st16(tmem + quad + COL_MQ + 32 + 16 * hc, r1);
                     if (c == nchunks - 1 && m_out != nullptr) {
                         float *mp = m_out + (size_t)z * m_zstride + st_base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) mp[(size_t)(32 * hc + e) * kN + rho] = x[e];
+                        for (int e = 0; e < 16; ++e) {
+                            mp[(size_t)(32 * hc + e) * kN + rho] = __uint_as_float(r0[e]);
+                            mp[(size_t)(32 * hc + 16 + e) * kN + rho] = __uint_as_float(r1[e]);
+                        }
                     }
+                    tmem_st_wait();
                 }
             } else if (DUAL && !yo && y0q != nullptr) {
                 // a summary run's y rows: y0 (its output from S = 0) and q = M_{<=t} r_t
@@ -793,7 +826,7 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         __syncthreads();
     }
     fence_after_sync();
-    if (warp == 8) tmem_dealloc(tmem, DUAL ? TMEM_COLS_DUAL : TMEM_COLS);
+    if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // One launch of the chunked kernel over nz = gridDim.z segment runs.
@@ -840,9 +873,9 @@ static cudaError_t launch_dual(int B, int T, int H, int t_seg, int nz, const voi
                                void *y = nullptr, wkv7_dtype y_dt = WKV7_F32, const float *s0 = nullptr,
                                float *ckpt = nullptr, EpiArgs epi = EpiArgs{}, float *y0q = nullptr,
                                uint4 *mq = nullptr) {
-    static_assert(chunk::SMEM_BYTES_DUAL <= 227 * 1024, "dual-run shared memory");
+
     dim3 grid(H, B, nz);
-    const size_t smem = chunk::SMEM_BYTES_DUAL;
+    const size_t smem = chunk::SMEM_BYTES;
     const int first_out = (y != nullptr || ckpt != nullptr) ? 1 : 0;
     using bf = __nv_bfloat16;
 #define WKV7_DUAL_LAUNCH(O, E, X)                                                                              \
@@ -1034,12 +1067,13 @@ static double launch_rounds(long long n, int sms) {
     return t;
 }
 
-// Relative time of one launch of n dual summary runs (one CTA per SM, each
-// about kDualCost times a plain run alone on its SM; measured on the
-// long-context shape).
-constexpr double kDualCost = 1.15;
+// Relative time of one launch of n dual summary runs: they fit two per SM
+// like the plain runs, each chunk step about kDualCost times a plain one at
+// the same co-residency (measured on the long-context shape: 8.64 vs 7.66 us
+// per chunk step with two CTAs per SM).
+constexpr double kDualCost = 1.13;
 static double dual_rounds(long long n, int sms) {
-    return n > 0 ? kDualCost * (double)((n + sms - 1) / sms) : 0.0;
+    return n > 0 ? kDualCost * launch_rounds(n, sms) : 0.0;
 }
 
 // Number of sequence segments for a chunked forward over B*H heads.  The
