@@ -606,29 +606,10 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
 
             // ---- P4: dV out; the masked dL block as round E's A operand in TMEM ----
             done_wait(3);
-            // side-by-side copy for round E's second half: [[b-; k-] | [r'; a']]
-            // from the X1 rows.  A group of 8 rows is 1 KB in both layouts (8
-            // column chunks of 8 rows), so each moves as one contiguous block;
-            // consecutive lanes move consecutive 16 bytes.
-            for (int x = tid; x < 2048; x += NC) {
-                const int blk = x >> 6, hl = (blk >> 4) & 1, G = blk & 15;
-                const uint32_t src = (hl ? X1_LO : X1_HI) + G * 1024;
-                const uint32_t dst = (hl ? X1C_LO : X1C_HI) + ((G & 7) * 16 + (G < 8 ? 8 : 0)) * 128;
-                *reinterpret_cast<uint4 *>(sm + dst + 16 * (x & 63)) =
-                    *reinterpret_cast<const uint4 *>(sm + src + 16 * (x & 63));
-            }
-            if (q4 >= 2 && part == 0) {                  // dV^T rows i, columns s = 16 hc ..
-                const int i = 32 * (q4 - 2) + lane;
-                uint32_t r0[16];
-                tmem_ld16_nowait(tmem + quad + CB + 64 + 16 * hc, r0);
-                tmem_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int s_ = 16 * hc + e;
-                    if (s_ < Lc) dv[base + (size_t)s_ * tok_stride + i] = from_f32<GradT>(__uint_as_float(r0[e]));
-                }
-            }
             {
+                // first the TMEM traffic (round E's first half is starting up on the
+                // tensor pipe; these loads and stores then wait less for it), then
+                // dV out and the side-by-side copy.
                 // lanes 0-63: dL rows t' (columns s' = 32 hc + 16 part + e at CA + 64 + s');
                 // lanes 64-127: dL^T rows s' (columns t' = 32 hc + 16 part + e at CA + t').
                 // Mask: t' < 32 (r' rows) keeps s <= t, t' >= 32 (a' rows) keeps s < t.
@@ -648,6 +629,28 @@ bwd_chunk_tc_kernel(int T, int H, const __nv_bfloat16 *__restrict__ r, const __n
                 tmem_st8(tmem + quad + ADL_HI + (uint32_t)(e0 >> 1), ph);
                 tmem_st8(tmem + quad + ADL_LO + (uint32_t)(e0 >> 1), pl);
                 tmem_st_wait();
+            }
+            if (q4 >= 2 && part == 0) {                  // dV^T rows i, columns s = 16 hc ..
+                const int i = 32 * (q4 - 2) + lane;
+                uint32_t r0[16];
+                tmem_ld16_nowait(tmem + quad + CB + 64 + 16 * hc, r0);
+                tmem_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int s_ = 16 * hc + e;
+                    if (s_ < Lc) dv[base + (size_t)s_ * tok_stride + i] = from_f32<GradT>(__uint_as_float(r0[e]));
+                }
+            }
+            // side-by-side copy for round E's second half: [[b-; k-] | [r'; a']]
+            // from the X1 rows.  A group of 8 rows is 1 KB in both layouts (8
+            // column chunks of 8 rows), so each moves as one contiguous block;
+            // consecutive lanes move consecutive 16 bytes.
+            for (int x = tid; x < 2048; x += NC) {
+                const int blk = x >> 6, hl = (blk >> 4) & 1, G = blk & 15;
+                const uint32_t src = (hl ? X1_LO : X1_HI) + G * 1024;
+                const uint32_t dst = (hl ? X1C_LO : X1C_HI) + ((G & 7) * 16 + (G < 8 ? 8 : 0)) * 128;
+                *reinterpret_cast<uint4 *>(sm + dst + 16 * (x & 63)) =
+                    *reinterpret_cast<const uint4 *>(sm + src + 16 * (x & 63));
             }
             ready_arrive(4);                             // round E
             // ---- P5: the four gradients, q, dw ----
