@@ -356,8 +356,9 @@ def bench_backward(args, dist, peaks, device, d):
                          "frac": ach / peaks["hbm_gbs"], "peak_source": peaks["source"],
                          "per_unit": "1664 B per head-token (6 inputs + dy read, 6 bf16 gradients written) "
                                      "+ 32 KiB state per head", "bytes_per_launch": nbytes,
-                         "kernels": "checkpoints (chunked forward), dS chain, per-chunk gradients "
-                                    "(tcgen05, bf16 hi/lo operands, fp32 accumulation)",
+                         "kernels": "checkpoints with every chunk's transition (chunked forward), dS by the "
+                                    "transition chain (tcgen05), per-chunk gradients (tcgen05, bf16 hi/lo "
+                                    "operands, fp32 accumulation)",
                          "fp32_alu": {"achieved": ach_flops, "peak": pk, "unit": "TFLOP/s", "frac": ach_flops / pk,
                                       "per_unit": "28*N^2 flop per head-token (the sequential scan's algebra)"},
                          "tensor_frac": ach_flops / peaks["bf16_tflops"]},
