@@ -87,9 +87,9 @@ constexpr uint32_t R = 94208;                       // short-lived buffers:
 constexpr uint32_t TP_HI = R, TP_LO = R + 4096;     //   P1..R2: [64][32] = T rows 0-31, P rows 32-63
 constexpr int LDT = 36;                             //   row pitch of L_ab^T (floats; bank spread)
 constexpr uint32_t LABT = R + 8192;                 //   P1: fp32 L_ab^T [32][36]
-constexpr uint32_t LAK = R + 12800;                 //   P1: fp32 L_ak [32][33] (padded)
+constexpr uint32_t LAKT = R + 12800;                //   P1: fp32 L_ak^T [32][36]
 constexpr uint32_t WU_HI = R, WU_LO = R + 8192;     //   P2..R3: [128][32] = W'^T rows, U~^T rows
-constexpr uint32_t SMEM_BYTES = R + 17024;
+constexpr uint32_t SMEM_BYTES = R + 17408;
 // dual runs: S2^T operand [64 j][64 i], in the short-lived buffers: staged
 // in P3 (R3 has read [W' | U~]), read by R4, overwritten by the next P1
 constexpr uint32_t S2_HI = R, S2_LO = R + 8192;
@@ -110,6 +110,7 @@ constexpr uint32_t GAMBET = RZ_LO + 7680;           // float2 [64]: (gamma, beta
 // the gate rows of the chunk, bf16 [32][64], arrive by cp.async in TSM's rows
 // (free from the end of P1 to the next P1)
 constexpr uint32_t BAR_EPI = 10;                    // named barrier of warps 2 and 6 (the y rows)
+constexpr uint32_t BAR_T = 11;                      // named barrier of warps 0 and 1 (the inverse T)
 
 constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
 constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (prod of 32 w)
@@ -203,13 +204,19 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         cp_async_commit();
     };
     // v of chunk c straight into its operand (AV columns 64-127); rows past the
-    // end keep the zeros P0 writes.  Transition runs keep v = 0.
+    // end keep the zeros P0 writes.  Transition runs keep v = 0.  The copies
+    // are issued by warps 3 and 7, which have no rows in P3 (every compute
+    // thread still commits a group, empty for the others).
     auto issue_v = [&](int c) {
-        if (c < nchunks) {
+        if (c < nchunks && (warp & 3) == 3) {
             const int t0 = c * L;
-            const int t = tid >> 3, ch = tid & 7;
-            if (t0 + t < T)
-                cp_async16(sm + AV_HI + cm_off(t, 64 + 8 * ch, 128), v + base + (size_t)(t0 + t) * tok_stride + ch * 8);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int x = 32 * (warp >> 2) + lane + 64 * u;
+                const int t = x >> 3, ch = x & 7;
+                if (t0 + t < T)
+                    cp_async16(sm + AV_HI + cm_off(t, 64 + 8 * ch, 128), v + base + (size_t)(t0 + t) * tok_stride + ch * 8);
+            }
         }
         cp_async_commit();
     };
@@ -380,15 +387,18 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
             for (int e = 0; e < 8; ++e) {
                 const float n1 = __shfl_down_sync(0xffffffffu, inc[e], 1);
                 const float nxt = lane == 31 ? 1.f : n1;
-                const float G = __shfl_sync(0xffffffffu, inc[e], 0);
-                if (lane == 0) {
-                    reinterpret_cast<float *>(sm + GAML)[8 * g + e] = G;
-                    if (G < kMinDecay) raise_status(WKV7_ERR_RANGE);
-                }
                 xa[e] = __fdividef(av[e], inc[e]);
                 xr[e] = __fdividef(rv[e], nxt);
                 xb[e] = bv[e] * nxt;
                 xk[e] = kv[e] * nxt;
+            }
+            if (lane == 0) {                      // G = p_0 of the warp's channels
+                float4 *gp = reinterpret_cast<float4 *>(sm + GAML) + 2 * g;
+                gp[0] = make_float4(inc[0], inc[1], inc[2], inc[3]);
+                gp[1] = make_float4(inc[4], inc[5], inc[6], inc[7]);
+                const float mn = fminf(fminf(fminf(inc[0], inc[1]), fminf(inc[2], inc[3])),
+                                       fminf(fminf(inc[4], inc[5]), fminf(inc[6], inc[7])));
+                if (mn < kMinDecay) raise_status(WKV7_ERR_RANGE);
             }
             if constexpr (EPI) {                  // part of u_t over this warp's 8 channels
                 const float4 *rp = reinterpret_cast<const float4 *>(epi.rho + (size_t)h * kN + 8 * g);
@@ -420,8 +430,8 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                         g[16 + e] = __uint_as_float(r1[e]);
                     }
                     const int s = row & 31;
-                    if (row < L && hc == 0) {         // column s of L_ab -> row s of L_ab^T
-                        float *dst = reinterpret_cast<float *>(sm + LABT) + s * LDT;
+                    if (hc == 0) {                    // column s of L_ab / L_ak -> row s of L_ab^T / L_ak^T
+                        float *dst = reinterpret_cast<float *>(sm + (row < L ? LABT : LAKT)) + s * LDT;
 #pragma unroll
                         for (int t4 = 0; t4 < 8; ++t4) {
                             float4 o;
@@ -431,10 +441,6 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                             o.w = 4 * t4 + 3 > s ? g[4 * t4 + 3] : 0.f;
                             *reinterpret_cast<float4 *>(dst + 4 * t4) = o;
                         }
-                    } else if (row >= L && hc == 0) { // column s of L_ak (rows padded to 33)
-                        float *dst = reinterpret_cast<float *>(sm + LAK) + s;
-#pragma unroll
-                        for (int t = 0; t < L; ++t) dst[t * 33] = t > s ? g[t] : 0.f;
                     } else {                          // column s of L_rb / L_rk -> columns 64.. of row s / 32+s
                         float u = 0.f;            // epilogue: u_s on the diagonal of L_rk
                         if (EPI && row >= L) {
@@ -453,12 +459,11 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                     }
                 }
             }
-            fence_before_sync();
-            csync();
             const float *labt = reinterpret_cast<const float *>(sm + LABT);
             auto trow = [&](int t) { return reinterpret_cast<float *>(sm + tsm_row(t)); };
-            if (warp == 0) {                      // diagonal 16x16 blocks of T, one column per lane
-                const int blk = lane >> 4, s = 16 * blk + sub;
+            if (warp < 2) {                       // diagonal 16x16 block 'warp' of T, one column per lane
+                __syncwarp();                     // (its rows of L_ab^T are this warp's own)
+                const int blk = warp, s = 16 * blk + sub;
                 float acc[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) acc[e] = (e == sub) ? 1.f : 0.f;
@@ -475,62 +480,87 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
                             if (4 * e4 + c4 > m) acc[4 * e4 + c4] = fmaf(lv[c4], x, acc[4 * e4 + c4]);
                     }
                 }
+                if (!upper) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) trow(16 * blk + e)[s] = acc[e];
-            } else if (warp == 1) {               // upper-right block of T is zero
+                    for (int e = 0; e < 16; ++e) trow(16 * blk + e)[s] = acc[e];
+                }
+            } else if (warp == 4) {               // upper-right block of T is zero
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int x = lane + 32 * e;
                     trow(x >> 4)[16 + (x & 15)] = 0.f;
                 }
             }
-            csync();
             float *zsm = reinterpret_cast<float *>(sm + ZSM);
-            {                                     // Z = L21 T11 (16 x 16), one entry per thread
-                const int t = tid >> 4, s = tid & 15;
-                float acc = 0.f;
+            if (warp < 2) named_sync(BAR_T, 64);  // both diagonal blocks are in place
+            if (tid < 64) {                       // Z = L21 T11 (16 x 16), four entries of a row per thread
+                const int t = tid >> 2, s0 = 4 * (tid & 3);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(labt[m * LDT + 16 + t], trow(m)[s], acc);
-                zsm[t * 16 + s] = acc;
+                for (int m = 0; m < 16; ++m) {
+                    const float l = labt[m * LDT + 16 + t];
+                    const float4 tv = *reinterpret_cast<const float4 *>(trow(m) + s0);
+                    acc[0] = fmaf(l, tv.x, acc[0]);
+                    acc[1] = fmaf(l, tv.y, acc[1]);
+                    acc[2] = fmaf(l, tv.z, acc[2]);
+                    acc[3] = fmaf(l, tv.w, acc[3]);
+                }
+                *reinterpret_cast<float4 *>(zsm + t * 16 + s0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                named_sync(BAR_T, 64);
             }
-            csync();
-            {                                     // T21 = T22 Z
-                const int t = tid >> 4, s = tid & 15;
-                float acc = 0.f;
+            if (tid < 64) {                       // T21 = T22 Z
+                const int t = tid >> 2, s0 = 4 * (tid & 3);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(trow(16 + t)[16 + m], zsm[m * 16 + s], acc);
-                trow(16 + t)[s] = acc;
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(trow(16 + t) + 16 + 4 * m4);
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float4 zv = *reinterpret_cast<const float4 *>(zsm + (4 * m4 + c4) * 16 + s0);
+                        acc[0] = fmaf(av[c4], zv.x, acc[0]);
+                        acc[1] = fmaf(av[c4], zv.y, acc[1]);
+                        acc[2] = fmaf(av[c4], zv.z, acc[2]);
+                        acc[3] = fmaf(av[c4], zv.w, acc[3]);
+                    }
+                }
+                *reinterpret_cast<float4 *>(trow(16 + t) + s0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
-            csync();
+            fence_before_sync();
+            csync();                              // T, L_ak (warps 2-3) and the zero block are in place
             {   // P = T L_ak, skipping the zero 16x16 blocks: P11 = T11 L11,
                 // P21 = T21 L11 + T22 L21, P22 = T22 L22, P12 = 0.  Half-warp
                 // kk (0..15), lane column s: row kk (cols < 16, m < 16), row
                 // 16 + kk (cols < 16, all m; cols >= 16, m >= 16).
-                const float *lak = reinterpret_cast<const float *>(sm + LAK);
+                const float *lakt = reinterpret_cast<const float *>(sm + LAKT);
                 const int kk = 2 * warp + (lane >> 4), s = lane & 15;
                 const float *ta = trow(kk), *tb = trow(16 + kk);
+                const float *la = lakt + s * LDT, *lc = lakt + (16 + s) * LDT;   // columns s, 16 + s of L_ak
                 float pa = 0.f, pb = 0.f, pc = 0.f;
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
                     const float4 xa = *reinterpret_cast<const float4 *>(ta + 4 * m4);
                     const float4 xb = *reinterpret_cast<const float4 *>(tb + 4 * m4);
+                    const float4 l4 = *reinterpret_cast<const float4 *>(la + 4 * m4);
                     const float va[4] = {xa.x, xa.y, xa.z, xa.w}, vb[4] = {xb.x, xb.y, xb.z, xb.w};
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const float lv = lak[(4 * m4 + c4) * 33 + s];
-                        pa = fmaf(va[c4], lv, pa);
-                        pb = fmaf(vb[c4], lv, pb);
+                        pa = fmaf(va[c4], lv[c4], pa);
+                        pb = fmaf(vb[c4], lv[c4], pb);
                     }
                 }
 #pragma unroll
                 for (int m4 = 4; m4 < 8; ++m4) {
                     const float4 xb = *reinterpret_cast<const float4 *>(tb + 4 * m4);
+                    const float4 l4 = *reinterpret_cast<const float4 *>(la + 4 * m4);
+                    const float4 c4v = *reinterpret_cast<const float4 *>(lc + 4 * m4);
                     const float vb[4] = {xb.x, xb.y, xb.z, xb.w};
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, cv[4] = {c4v.x, c4v.y, c4v.z, c4v.w};
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const float* lrow = lak + (4 * m4 + c4) * 33;
-                        pb = fmaf(vb[c4], lrow[s], pb);
-                        pc = fmaf(vb[c4], lrow[16 + s], pc);
+                        pb = fmaf(vb[c4], lv[c4], pb);
+                        pc = fmaf(vb[c4], cv[c4], pc);
                     }
                 }
                 auto put = [&](uint32_t hi_base, uint32_t lo_base, int row, int col, float x) {
@@ -769,20 +799,20 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         };
 
         // ---- compute schedule ----
-        // cp.async groups are committed in a fixed order: [w r k a b](c+1) at
-        // the start of P1(c), [v](c+1) at the start of P3(c) (both possibly
-        // empty).  Gram(c) done means every warp has finished P0(c), so the
-        // staging tile is free for the next chunk.
+        // cp.async groups are committed in a fixed order: [w r k a b](c+1)
+        // while R2(c) runs (the warps wait for it anyway; Gram(c) done means
+        // every warp has finished P0(c), so the staging tile is free), [v](c+1)
+        // at the start of P3(c) (both possibly empty).
         cp_async_wait<0>();
         csync();
         P0(min(L, T));
         ready_arrive(0);                                   // R1(0)
         for (int c = 0; c < nchunks; ++c) {
             done_wait(0, c);                               // Gram(c)
-            issue_in(c + 1);
             P1();
-            cp_async_wait<1>();                            // v(c) is in place
+            cp_async_wait<0>();                            // v(c) is in place
             ready_arrive(1);                               // R2(c)
+            issue_in(c + 1);                               // under R2(c)
             done_wait(1, c);
             if constexpr (EPI) {                           // gate rows of chunk c (P1's T rows are dead)
                 if (yo && epi.g && warp % 4 == 2) {
