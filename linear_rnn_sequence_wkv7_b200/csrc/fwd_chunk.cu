@@ -111,6 +111,7 @@ constexpr uint32_t GAMBET = RZ_LO + 7680;           // float2 [64]: (gamma, beta
 // (free from the end of P1 to the next P1)
 constexpr uint32_t BAR_EPI = 10;                    // named barrier of warps 2 and 6 (the y rows)
 constexpr uint32_t BAR_T = 11;                      // named barrier of warps 0 and 1 (the inverse T)
+constexpr uint32_t BAR_G = 12;                      // warps 0-1 have read the Gram; warps 4-7 may read theirs
 
 constexpr long long kDrainCycles = 200000000LL;     // ~0.1 s to let committed tensor-core work finish
 constexpr float kMinDecay = 1e-30f;                 // per-chunk decay floor (prod of 32 w)
@@ -418,9 +419,11 @@ fwd_chunk_kernel(int T_total, int H, int t_seg, int nseg, const __nv_bfloat16 *_
         auto P1 = [&]() {                         // Gram -> L's; T = (I - L_ab)^{-1}; P = T L_ak
             {
                 uint32_t r0[16], r1[16];
+                if (warp >= 4) named_sync(BAR_G, 192);
                 tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc, r0);
                 tmem_ld16_nowait(tmem + quad + COL_X + 32 * hc + 16, r1);
                 tmem_wait();
+                if (warp < 2) named_arrive(BAR_G, 192);
                 if (!upper) {
                     const int row = 16 * q4 + sub;
                     float g[32];
