@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     WKV7_OK = 0,
     WKV7_ERR_INVALID_ARG = 1,  /* bad pointer / size / dtype / alignment      */
-    WKV7_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    WKV7_ERR_UNSUPPORTED = 2,  /* valid request that this library does not implement */
     WKV7_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed        */
     WKV7_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up          */
     WKV7_ERR_RANGE = 5,        /* device-side: input outside the chunked

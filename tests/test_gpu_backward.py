@@ -194,7 +194,7 @@ def _transition_bytes(B, T, H):
 
 def _kernel_names(fn):
     """Names of the CUDA kernels fn launches (empty when the profiler
-    records no device activity on this build)."""
+    records no device activity in this PyTorch installation)."""
     from torch.profiler import ProfilerActivity, profile
     with profile(activities=[ProfilerActivity.CUDA]) as prof:
         fn()
