@@ -60,3 +60,37 @@ def test_single_process_is_identity():
         assert d.max(3.5) == 3.5
         d.barrier()
         d.close()
+
+
+def _failing_rank_main(rank, world, port, out):
+    """Rank 1 fails between steps (an exception before the timing reduction);
+    rank 0 must learn of it from its own collective, as an error, not a hang."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    d = Dist("gloo").init(timeout_s=5)
+    d.barrier()
+    if rank == 1:
+        raise RuntimeError("rank 1 fails between steps")
+    try:
+        d.max(1.0)
+        out.put(("no error", ""))
+    except Exception as e:          # a closed connection or the process-group timeout
+        out.put(("error", type(e).__name__))
+    out.close()
+    out.join_thread()
+    os._exit(0)                     # no teardown collective with a dead peer
+
+
+def test_a_failed_rank_ends_the_others_collective_with_an_error():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    status, _ = out.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert status == "error"
+    assert procs[0].exitcode == 0
+    assert procs[1].exitcode != 0
